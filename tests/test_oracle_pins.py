@@ -1,0 +1,347 @@
+"""Pins of the fp64 oracle to facts the pages and the mathematics fix (CPU only).
+
+Each test checks the oracle against something other than itself: a worked
+example derived by hand (tests/golden), a closed form, a library routine the
+case reduces to (torch's scaled_dot_product_attention in float64), or an
+invariant the pages state (packing, paging, masked pairs contributing nothing).
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(shape, dtype=torch.float32, seed=0, sigma=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(shape, generator=g) * sigma).to(dtype)
+
+
+def _seq_case(L, Lkv, H, Hkv, d, mask_type, dtype=torch.float32, seed=0, slopes=None, dv=None):
+    q = _rand((L, H, d), dtype, seed)
+    k = _rand((Lkv, Hkv, d), dtype, seed + 1)
+    v = _rand((Lkv, Hkv, dv or d), dtype, seed + 2)
+    return q, k, v
+
+
+# --------------------------------------------------------------------------
+# hand-derived worked examples
+# --------------------------------------------------------------------------
+
+def _read_kv(path):
+    vals = {}
+    for line in open(path):
+        if line.startswith("#") or not line.strip():
+            continue
+        key, *rest = line.split()
+        vals[key] = [float(x) for x in rest]
+    return vals
+
+
+def test_two_key_worked_example():
+    g = _read_kv(os.path.join(GOLDEN, "two_key_softmax.txt"))
+    q = torch.tensor(g["q"], dtype=torch.float32).view(1, 1, 1)
+    k = torch.tensor(g["k"], dtype=torch.float32).view(2, 1, 1)
+    v = torch.tensor(g["v"], dtype=torch.float32).view(2, 1, 1)
+    out, lse = oracle.attention(q, k, v, [1], [2], oracle.MASK_NONE, 1, 1, g["qk_scale"][0])
+    assert abs(out[0, 0] - g["out"][0]) < 1e-6
+    assert abs(lse[0] - g["lse"][0]) < 1e-6
+
+
+def test_mask_rule_matches_hand_derived_masks():
+    rows = {}
+    for line in open(os.path.join(GOLDEN, "alibi_masks_L2_Lkv4.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        parts = line.split()
+        rows[(int(parts[0]), int(parts[1]))] = [float(x) for x in parts[2:]]
+    for mt in (0, 3, 4, 5, 9):
+        m = oracle.build_mask(mt, np.array([0.5], np.float32), 1, 2, 4)
+        for i in range(2):
+            np.testing.assert_allclose(m[0, i], rows[(mt, i)], rtol=0, atol=1e-15)
+
+
+# --------------------------------------------------------------------------
+# closed forms
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mask_type", [0, 3, 4, 5, 9])
+def test_single_key_returns_v0(mask_type):
+    q, k, v = _seq_case(1, 1, 2, 1, 8, mask_type, seed=3)
+    slopes = np.array([0.25, 0.5], np.float32)
+    out, lse = oracle.attention(q, k, v, [1], [1], mask_type, 2, 1, 0.3, slopes=slopes)
+    for h in range(2):
+        np.testing.assert_array_equal(out[h], v[0, 0].double().numpy())
+        dot = float((q[0, h].double() * k[0, 0].double()).sum())
+        assert abs(lse[h] - 0.3 * dot) < 1e-12  # bias is 0 at distance 0 for 3/4; j=0 for 5
+
+
+@pytest.mark.parametrize("mask_type", [0, 9])
+def test_zero_query_gives_mean_of_allowed_values(mask_type):
+    L, Lkv = 5, 9  # prefix of 4 tokens
+    q = torch.zeros((L, 2, 4))
+    _, k, v = _seq_case(L, Lkv, 2, 2, 4, mask_type, seed=5)
+    out, lse = oracle.attention(q, k, v, [L], [Lkv], mask_type, 2, 2, 0.7)
+    out = out.reshape(L, 2, 4)
+    lse = lse.reshape(L, 2)
+    for i in range(L):
+        n_allowed = Lkv if mask_type == 0 else i + (Lkv - L) + 1
+        for h in range(2):
+            np.testing.assert_allclose(out[i, h], v[:n_allowed, h].double().mean(0).numpy(), rtol=0, atol=1e-12)
+            assert abs(lse[i, h] - math.log(n_allowed)) < 1e-12
+
+
+@pytest.mark.parametrize("mask_type", [0, 3, 4, 5, 9])
+def test_constant_values_give_that_constant(mask_type):
+    L, Lkv = 6, 10
+    q, k, _ = _seq_case(L, Lkv, 4, 2, 8, mask_type, seed=7)
+    c = torch.linspace(-2.0, 3.0, 8)
+    v = c.expand(Lkv, 2, 8).contiguous()
+    out, _ = oracle.attention(q, k, v, [L], [Lkv], mask_type, 4, 2, 0.35,
+                              slopes=synth.alibi_slopes(4))
+    np.testing.assert_allclose(out, np.broadcast_to(c.double().numpy(), out.shape), rtol=0, atol=1e-12)
+
+
+def test_right_aligned_alibi_geometric_closed_form():
+    """q = 0, d = 1, v_j = j: weights r^(iabs-j) with r = exp(-slope) -> a geometric-series mean."""
+    L, Lkv, slope = 4, 11, 0.37
+    q = torch.zeros((L, 1, 1))
+    k = _rand((Lkv, 1, 1), seed=11)
+    v = torch.arange(Lkv, dtype=torch.float32).view(Lkv, 1, 1)
+    out, lse = oracle.attention(q, k, v, [L], [Lkv], oracle.MASK_ALIBI, 1, 1, 1.0,
+                                slopes=np.array([slope], np.float32))
+    s = float(np.float32(slope))
+    r = math.exp(-s)
+    for i in range(L):
+        n = i + (Lkv - L)  # iabs; keys 0..n allowed
+        s0 = (1 - r ** (n + 1)) / (1 - r)                                     # sum_k r^k
+        s1 = r * (1 - (n + 1) * r ** n + n * r ** (n + 1)) / (1 - r) ** 2     # sum_k k r^k
+        assert abs(out[i, 0] - (n * s0 - s1) / s0) < 1e-12                  # sum_j j r^(n-j) / s0
+        assert abs(lse[i] - math.log(s0)) < 1e-12
+
+
+# --------------------------------------------------------------------------
+# library routine the cases reduce to: torch SDPA (math path, float64)
+# --------------------------------------------------------------------------
+
+def _sdpa(q, k, v, scale, attn_mask=None, is_causal=False):
+    qq = q.double().permute(1, 0, 2).unsqueeze(0)
+    kk = k.double().permute(1, 0, 2).unsqueeze(0)
+    vv = v.double().permute(1, 0, 2).unsqueeze(0)
+    o = F.scaled_dot_product_attention(qq, kk, vv, attn_mask=attn_mask, is_causal=is_causal, scale=scale,
+                                       enable_gqa=True)
+    return o.squeeze(0).permute(1, 0, 2).reshape(-1, v.shape[-1]).numpy()
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
+def test_no_mask_and_causal_match_sdpa_with_gqa(dtype):
+    L, H, Hkv, d = 37, 8, 2, 16
+    q, k, v = _seq_case(L, L, H, Hkv, d, 0, dtype=dtype, seed=13)
+    for mt, causal in ((oracle.MASK_NONE, False), (oracle.MASK_CAUSAL, True)):
+        out, _ = oracle.attention(q, k, v, [L], [L], mt, H, Hkv, 0.25)
+        ref = _sdpa(q, k, v, 0.25, is_causal=causal)
+        np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("mask_type", [3, 4, 5, 9])
+def test_prefix_offset_masks_match_sdpa_with_additive_bias(mask_type):
+    """Bias built from the page rules as a float mask; SDPA adds it after scaling."""
+    L, Lkv, H, Hkv, d = 7, 19, 4, 4, 8
+    q, k, v = _seq_case(L, Lkv, H, Hkv, d, mask_type, seed=17)
+    slopes = synth.alibi_slopes(H)
+    out, _ = oracle.attention(q, k, v, [L], [Lkv], mask_type, H, Hkv, 0.5, slopes=slopes)
+    bias = torch.full((H, L, Lkv), float("-inf"), dtype=torch.float64)
+    for h in range(H):
+        sl = float(slopes[h])
+        for i in range(L):
+            iabs = i + Lkv - L
+            for j in range(iabs + 1):
+                bias[h, i, j] = {3: sl * (j - iabs), 4: -sl * math.sqrt(iabs - j), 5: sl * j, 9: 0.0}[mask_type]
+    ref = _sdpa(q, k, v, 0.5, attn_mask=bias.unsqueeze(0))
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# invariants the pages state
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mask_type", [0, 3, 4, 5, 9])
+def test_rule_equals_explicit_full_mask(mask_type):
+    L, Lkv, H, Hkv, d = 9, 14, 4, 2, 8
+    q, k, v = _seq_case(L, Lkv, H, Hkv, d, mask_type, seed=19)
+    slopes = synth.alibi_slopes(H)
+    out, lse = oracle.attention(q, k, v, [L], [Lkv], mask_type, H, Hkv, 0.4, slopes=slopes)
+    m = oracle.build_mask(mask_type, slopes, H, L, Lkv)
+    out2, lse2 = oracle.attention_explicit(q, k, v, m, H, Hkv, 0.4)
+    np.testing.assert_allclose(out, out2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lse2, rtol=0, atol=1e-12)
+
+
+def test_compressed_causal_triangle_expands_to_rule():
+    tri = np.where(np.arange(128)[None, :] > np.arange(128)[:, None], -np.inf, 0.0)
+    for L, Lkv in ((5, 5), (40, 300), (200, 200), (130, 400)):
+        m = oracle.expand_causal_compressed(tri, L, Lkv)
+        ref = oracle.build_mask(oracle.MASK_CAUSAL, None, 1, L, Lkv)[0]
+        np.testing.assert_array_equal(m, ref)
+
+
+def test_zero_slopes_equal_causal():
+    L, Lkv, H = 8, 13, 3
+    q, k, v = _seq_case(L, Lkv, H, H, 8, 3, seed=23)
+    ref, lref = oracle.attention(q, k, v, [L], [Lkv], oracle.MASK_CAUSAL, H, H, 0.5)
+    for mt in (3, 4, 5):
+        out, lse = oracle.attention(q, k, v, [L], [Lkv], mt, H, H, 0.5, slopes=np.zeros(H, np.float32))
+        np.testing.assert_array_equal(out, ref)
+        np.testing.assert_array_equal(lse, lref)
+
+
+def test_left_aligned_equals_right_aligned_up_to_row_shift():
+    L, Lkv, H = 6, 15, 4
+    q, k, v = _seq_case(L, Lkv, H, H, 8, 3, seed=29)
+    slopes = synth.alibi_slopes(H)
+    o3, l3 = oracle.attention(q, k, v, [L], [Lkv], 3, H, H, 0.5, slopes=slopes)
+    o5, l5 = oracle.attention(q, k, v, [L], [Lkv], 5, H, H, 0.5, slopes=slopes)
+    np.testing.assert_allclose(o3, o5, rtol=0, atol=1e-12)
+    for i in range(L):
+        for h in range(H):
+            iabs = i + Lkv - L
+            assert abs(l5[i * H + h] - l3[i * H + h] - float(slopes[h]) * iabs) < 1e-12
+
+
+def test_sqrt_equals_linear_on_unit_distances():
+    q, k, v = _seq_case(2, 2, 2, 2, 8, 4, seed=31)
+    slopes = synth.alibi_slopes(2)
+    o3, l3 = oracle.attention(q, k, v, [2], [2], 3, 2, 2, 0.5, slopes=slopes)
+    o4, l4 = oracle.attention(q, k, v, [2], [2], 4, 2, 2, 0.5, slopes=slopes)
+    np.testing.assert_allclose(o3, o4, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(l3, l4, rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("mask_type", [0, 4, 9])
+def test_packed_equals_each_sequence_alone(mask_type):
+    rng = np.random.Generator(np.random.PCG64(37))
+    L = rng.integers(1, 40, size=4).astype(np.int32)
+    pre = rng.integers(0, 30, size=4).astype(np.int32)
+    case = synth.make_prefill("t", L, L + pre, 4, 2, 8, torch.bfloat16, mask_type, 37)
+    out, lse = oracle.attention(case.q, case.k, case.v, case.seq_len, case.kv_seq_len, mask_type, 4, 2, 0.3,
+                                slopes=case.slopes)
+    qo = ko = 0
+    for b in range(4):
+        Lb, Lkvb = int(L[b]), int(L[b] + pre[b])
+        o1, l1 = oracle.attention(case.q[qo:qo + Lb], case.k[ko:ko + Lkvb], case.v[ko:ko + Lkvb], [Lb], [Lkvb],
+                                  mask_type, 4, 2, 0.3, slopes=case.slopes)
+        np.testing.assert_array_equal(out[qo * 4:(qo + Lb) * 4], o1)
+        np.testing.assert_array_equal(lse[qo * 4:(qo + Lb) * 4], l1)
+        qo += Lb
+        ko += Lkvb
+
+
+def test_packed_equals_padded_layout_on_valid_rows():
+    case = synth.varlen_causal_bf16(seed=41, batch=3, lo=5, hi=30)
+    case.heads, case.kv_heads = 32, 8
+    pad = synth.padded_from(case)
+    out, _ = oracle.attention(case.q, case.k, case.v, case.seq_len, case.kv_seq_len, 9, 32, 8, case.qk_scale)
+    outp, _ = oracle.attention(pad.q, pad.k, pad.v, pad.seq_len, pad.kv_seq_len, 9, 32, 8, pad.qk_scale)
+    Lmax = pad.meta["Lmax"]
+    pos = 0
+    for b, L in enumerate(case.seq_len.tolist()):
+        np.testing.assert_array_equal(out[pos * 32:(pos + L) * 32], outp[b * Lmax * 32:(b * Lmax + L) * 32])
+        pos += L
+    assert pad.meta["padding_positions"] == 3 * Lmax - int(case.seq_len.sum())
+
+
+@pytest.mark.parametrize("block_size", [16, 64, 128])
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_paged_equals_contiguous(block_size, dtype):
+    rng = np.random.Generator(np.random.PCG64(43 + block_size))
+    L = rng.integers(1, 50, size=3).astype(np.int32)
+    Lkv = L + rng.integers(0, 300, size=3).astype(np.int32)
+    contig = synth.make_prefill("c", L, Lkv, 4, 2, 16, dtype, 3, 43)
+    paged = synth.make_prefill("p", L, Lkv, 4, 2, 16, dtype, 3, 43, paged=True, block_size=block_size)
+    assert (paged.block_tables >= -1).all()
+    o1, l1 = oracle.attention(contig.q, contig.k, contig.v, L, Lkv, 3, 4, 2, 0.25, slopes=contig.slopes)
+    o2, l2 = oracle.attention(paged.q, paged.k, paged.v, L, Lkv, 3, 4, 2, 0.25, slopes=paged.slopes,
+                              block_tables=paged.block_tables, block_size=block_size)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+
+
+def test_masked_keys_and_values_do_not_contribute():
+    L, Lkv, H = 6, 10, 2
+    q, k, v = _seq_case(L, Lkv, H, H, 8, 9, seed=47)
+    out, lse = oracle.attention(q, k, v, [L], [Lkv], 9, H, H, 0.5)
+    # row 0 sits at iabs 4: keys 5.. are masked for it; row L-1 sees all
+    k2, v2 = k.clone(), v.clone()
+    k2[5:] = 1e4
+    v2[5:] = -1e4
+    out2, lse2 = oracle.attention(q, k2, v2, [L], [Lkv], 9, H, H, 0.5)
+    np.testing.assert_array_equal(out[:H], out2[:H])
+    np.testing.assert_array_equal(lse[:H], lse2[:H])
+    assert not np.allclose(out[-H:], out2[-H:])
+
+
+def test_lse_merge_of_disjoint_key_ranges_equals_whole():
+    """Split the keys in two ranges, attend to each alone, merge by lse: equals attending to all."""
+    L, Lkv, H, d = 3, 50, 2, 8
+    q, k, v = _seq_case(L, Lkv, H, H, d, 0, seed=53)
+    whole, lw = oracle.attention(q, k, v, [L], [Lkv], 0, H, H, 0.3)
+    a = 21
+    o1, l1 = oracle.attention(q, k[:a], v[:a], [L], [a], 0, H, H, 0.3)
+    o2, l2 = oracle.attention(q, k[a:], v[a:], [L], [Lkv - a], 0, H, H, 0.3)
+    mo, ml = oracle.lse_merge(np.stack([o1, o2]), np.stack([l1, l2]))
+    np.testing.assert_allclose(mo, whole, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(ml, lw, rtol=0, atol=1e-12)
+    # lse normalises the weights: sum_j exp(s_j - lse) = 1 with s_j from an independent dot product
+    s = 0.3 * torch.einsum("lhd,jhd->lhj", q.double(), k.double())
+    np.testing.assert_allclose(torch.exp(s - torch.tensor(lw).view(L, H, 1)).sum(-1).numpy(), 1.0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# MLA entry point
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("qs", [1, 4])
+def test_mla_equals_generic_with_concatenated_key(qs):
+    rng = np.random.Generator(np.random.PCG64(59))
+    ctx = rng.integers(qs, 300, size=3).astype(np.int32)
+    case = synth.make_mla("m", ctx, qs, 4, 59, rng=rng, block_size=64, d_nope=32, d_rope=8)
+    out, lse = oracle.mla(case.q_nope, case.q_rope, case.ct_kv, case.k_rope, case.block_tables, 64,
+                          case.context_lens, case.q_seq_len, 4, case.qk_scale)
+    q = torch.cat([case.q_nope, case.q_rope], dim=-1)
+    kcat = torch.cat([case.ct_kv, case.k_rope], dim=-1)
+    o2, l2 = oracle.attention(q, kcat, case.ct_kv, case.q_seq_len, case.context_lens, oracle.MASK_CAUSAL, 4, 1,
+                              case.qk_scale, block_tables=case.block_tables, block_size=64)
+    np.testing.assert_allclose(out, o2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, l2, rtol=0, atol=1e-12)
+
+
+def test_mla_spec_last_token_equals_decode_over_full_context():
+    rng = np.random.Generator(np.random.PCG64(61))
+    ctx = rng.integers(8, 200, size=2).astype(np.int32)
+    case = synth.make_mla("m", ctx, 4, 2, 61, rng=rng, block_size=16, d_nope=16, d_rope=8)
+    out, lse = oracle.mla(case.q_nope, case.q_rope, case.ct_kv, case.k_rope, case.block_tables, 16,
+                          case.context_lens, case.q_seq_len, 2, case.qk_scale)
+    for b in range(2):
+        t = b * 4 + 3
+        o1, l1 = oracle.mla(case.q_nope[t:t + 1], case.q_rope[t:t + 1], case.ct_kv, case.k_rope,
+                            case.block_tables[b:b + 1], 16, case.context_lens[b:b + 1], [1], 2, case.qk_scale)
+        np.testing.assert_array_equal(out[t * 2:t * 2 + 2], o1)
+        np.testing.assert_array_equal(lse[t * 2:t * 2 + 2], l1)
+
+
+def test_row_subset_equals_full_run():
+    case = synth.make_prefill("r", [20, 33], [50, 33], 4, 2, 16, torch.bfloat16, 4, 67)
+    full, lf = oracle.attention(case.q, case.k, case.v, case.seq_len, case.kv_seq_len, 4, 4, 2, 0.25,
+                                slopes=case.slopes)
+    rows = np.array([0, 5, 79, 80, 150, 211], dtype=np.int64)
+    sub, ls = oracle.attention(case.q, case.k, case.v, case.seq_len, case.kv_seq_len, 4, 4, 2, 0.25,
+                               slopes=case.slopes, rows=rows)
+    np.testing.assert_array_equal(sub, full[rows])
+    np.testing.assert_array_equal(ls, lf[rows])
