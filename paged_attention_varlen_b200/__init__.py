@@ -1,0 +1,228 @@
+"""Python binding of libala.so: packed-varlen / paged attention on B200 (sm_100a).
+
+Argument marshalling only.  Every step of the computation runs in the CUDA
+kernels behind the C ABI declared in ``include/ala.h``; there is no CPU or
+PyTorch fallback.  If the shared library is missing the calls raise.
+
+Entry points (names as in the C ABI):
+  * ``varlen_attention``         contiguous packed K/V, mask types 0/3/4/5/9
+  * ``atb_like_prefix_encoder``  paged K/V through blockTables, mask types 3/4/5/9
+  * ``atb_like_mla``             MLA decode / speculative decode over a paged latent cache
+
+Each returns an ``Op`` that owns the workspace and can be executed again on
+the current CUDA stream (``op()``), which is what the bench does.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libala.so")
+
+F16, BF16, F32, I32 = 0, 1, 2, 3
+MASK_NONE, MASK_ALIBI, MASK_ALIBI_SQRT, MASK_ALIBI_LEFT, MASK_CAUSAL = 0, 3, 4, 5, 9
+MLA_MASK_UNDEFINED, MLA_MASK_SPEC, MLA_MASK_FREE = 0, 1, 2
+MLA_CALC_UNDEFINED, MLA_CALC_SPEC, MLA_CALC_RING, MLA_CALC_PREFILL = 0, 1, 2, 3
+MLA_CACHE_KVCACHE, MLA_CACHE_KROPE_CTKV, MLA_CACHE_INT8_NZ, MLA_CACHE_NZ = 0, 1, 2, 3
+
+STATUS = {0: "OK", 1: "NULL_REQUIRED", 2: "INVALID_SHAPE", 3: "INVALID_DTYPE", 4: "INVALID_PARAM",
+          5: "UNSUPPORTED", 6: "WORKSPACE_TOO_SMALL", 7: "CUDA_ERROR", 8: "DEVICE_TIMEOUT"}
+
+_TORCH_DTYPE = {torch.float16: F16, torch.bfloat16: BF16, torch.float32: F32, torch.int32: I32}
+_NP_DTYPE = {np.dtype(np.int32): I32, np.dtype(np.float32): F32}
+
+
+class AlaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class AlaTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("dims", ctypes.c_int64 * 4)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libala.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m paged_attention_varlen_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.c_void_p
+        T = ctypes.POINTER(AlaTensor)
+        OPP = ctypes.POINTER(ctypes.c_void_p)
+        U64P = ctypes.POINTER(ctypes.c_uint64)
+        L.ala_last_error.restype = ctypes.c_char_p
+        L.ala_op_destroy.argtypes = [P]
+        L.ala_op_destroy.restype = None
+        L.ala_workspace_status.argtypes = [P, P, P, ctypes.POINTER(ctypes.c_int32)]
+        L.atb_like_prefix_encoder_get_workspace_size.argtypes = [T, T, T, T, T, T, T, T, ctypes.c_int, ctypes.c_int32,
+                                                                 ctypes.c_int32, ctypes.c_float, T, U64P, OPP]
+        L.varlen_attention_get_workspace_size.argtypes = [T, T, T, T, T, T, ctypes.c_int, ctypes.c_int32,
+                                                          ctypes.c_int32, ctypes.c_float, T, T, U64P, OPP]
+        L.atb_like_mla_get_workspace_size.argtypes = [T, T, T, T, T, T, T, T, T, T, ctypes.c_int32, ctypes.c_float,
+                                                      ctypes.c_int32, ctypes.c_int, ctypes.c_int, ctypes.c_uint8, T, T,
+                                                      U64P, OPP]
+        for f in ("atb_like_prefix_encoder", "varlen_attention", "atb_like_mla"):
+            getattr(L, f).argtypes = [P, ctypes.c_uint64, P, P]
+        for f in ("ala_workspace_status", "atb_like_prefix_encoder_get_workspace_size",
+                  "varlen_attention_get_workspace_size", "atb_like_mla_get_workspace_size",
+                  "atb_like_prefix_encoder", "varlen_attention", "atb_like_mla"):
+            getattr(L, f).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(status: int):
+    if status != 0:
+        raise AlaError(status, lib().ala_last_error().decode())
+
+
+def tensor(x) -> AlaTensor | None:
+    """Describe a torch tensor or numpy array (contiguous) as an ala_tensor; None -> NULL."""
+    if x is None:
+        return None
+    if isinstance(x, np.ndarray):
+        assert x.flags["C_CONTIGUOUS"]
+        dt, ptr, shape = _NP_DTYPE[x.dtype], x.ctypes.data, x.shape
+    else:
+        assert x.is_contiguous(), "tensors passed to libala must be contiguous"
+        dt, ptr, shape = _TORCH_DTYPE[x.dtype], x.data_ptr(), tuple(x.shape)
+    assert 1 <= len(shape) <= 4
+    t = AlaTensor()
+    t.data = ptr
+    t.dtype = dt
+    t.ndim = len(shape)
+    for i, s in enumerate(shape):
+        t.dims[i] = s
+    return t
+
+
+def _ref(t):
+    return None if t is None else ctypes.byref(t)
+
+
+def _host_i32(x) -> np.ndarray:
+    if isinstance(x, torch.Tensor):
+        x = x.cpu().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.int32))
+
+
+class Op:
+    """A planned call: owns the op handle, its workspace and references to its tensors."""
+
+    def __init__(self, handle, ws_size, execute_fn, device, keep):
+        self._handle = handle
+        self._execute = execute_fn
+        self.workspace = torch.empty(max(int(ws_size), 16), dtype=torch.uint8, device=device)
+        self.workspace_size = int(ws_size)
+        self._keep = keep
+
+    def __call__(self, stream: torch.cuda.Stream | None = None):
+        s = stream if stream is not None else torch.cuda.current_stream(self.workspace.device)
+        _check(self._execute(ctypes.c_void_p(self.workspace.data_ptr()), self.workspace_size, self._handle,
+                             ctypes.c_void_p(s.cuda_stream)))
+        return self
+
+    def device_status(self) -> int:
+        code = ctypes.c_int32(0)
+        s = torch.cuda.current_stream(self.workspace.device)
+        _check(lib().ala_workspace_status(self._handle, ctypes.c_void_p(self.workspace.data_ptr()),
+                                          ctypes.c_void_p(s.cuda_stream), ctypes.byref(code)))
+        return code.value
+
+    def __del__(self):
+        if getattr(self, "_handle", None) and _lib is not None:
+            _lib.ala_op_destroy(self._handle)
+            self._handle = None
+
+
+def plan_varlen_attention(q, k, v, seq_len, kv_seq_len, mask_type, heads, kv_heads, qk_scale, slopes=None,
+                          out=None, lse=None) -> tuple[Op, torch.Tensor]:
+    """Plan contiguous packed-varlen attention; returns (op, out).  Call op() to run."""
+    L = lib()
+    out = torch.empty_like(q) if out is None else out
+    sl, kl = _host_i32(seq_len), _host_i32(kv_seq_len)
+    ts = [tensor(q), tensor(k), tensor(v), tensor(sl), tensor(kl), tensor(slopes)]
+    to, tl = tensor(out), tensor(lse)
+    ws = ctypes.c_uint64(0)
+    h = ctypes.c_void_p(0)
+    _check(L.varlen_attention_get_workspace_size(*[_ref(t) for t in ts], int(mask_type), int(heads), int(kv_heads),
+                                                 float(qk_scale), _ref(to), _ref(tl), ctypes.byref(ws),
+                                                 ctypes.byref(h)))
+    return Op(h, ws.value, L.varlen_attention, q.device, (q, k, v, sl, kl, slopes, out, lse)), out
+
+
+def varlen_attention(q, k, v, seq_len, kv_seq_len, mask_type, heads, kv_heads, qk_scale, slopes=None,
+                     return_lse=False):
+    """O (and optionally the fp32 lse [nTokens, heads]) for contiguous packed K/V."""
+    lse = torch.empty((q.shape[0], heads), dtype=torch.float32, device=q.device) if return_lse else None
+    op, out = plan_varlen_attention(q, k, v, seq_len, kv_seq_len, mask_type, heads, kv_heads, qk_scale, slopes,
+                                    lse=lse)
+    op()
+    return (out, lse) if return_lse else out
+
+
+def plan_prefix_encoder(q, k, v, block_tables, seq_len, kv_seq_len, mask_type, heads, kv_heads, qk_scale,
+                        slopes=None, mask=None, out=None) -> tuple[Op, torch.Tensor]:
+    """Plan the paged PrefixEncoder call; returns (op, out)."""
+    L = lib()
+    out = torch.empty_like(q) if out is None else out
+    sl, kl = _host_i32(seq_len), _host_i32(kv_seq_len)
+    ts = [tensor(q), tensor(k), tensor(v), tensor(block_tables), tensor(mask), tensor(sl), tensor(kl),
+          tensor(slopes)]
+    to = tensor(out)
+    ws = ctypes.c_uint64(0)
+    h = ctypes.c_void_p(0)
+    _check(L.atb_like_prefix_encoder_get_workspace_size(*[_ref(t) for t in ts], int(mask_type), int(heads),
+                                                        int(kv_heads), float(qk_scale), _ref(to), ctypes.byref(ws),
+                                                        ctypes.byref(h)))
+    return Op(h, ws.value, L.atb_like_prefix_encoder, q.device,
+              (q, k, v, block_tables, mask, sl, kl, slopes, out)), out
+
+
+def atb_like_prefix_encoder(q, k, v, block_tables, seq_len, kv_seq_len, mask_type, heads, kv_heads, qk_scale,
+                            slopes=None, mask=None):
+    op, out = plan_prefix_encoder(q, k, v, block_tables, seq_len, kv_seq_len, mask_type, heads, kv_heads,
+                                  qk_scale, slopes, mask)
+    op()
+    return out
+
+
+def plan_mla(q_nope, q_rope, ct_kv, k_rope, block_tables, context_lens, q_seq_len, heads, qk_scale,
+             mask_type=MLA_MASK_UNDEFINED, calc_type=MLA_CALC_UNDEFINED, cache_mode=MLA_CACHE_KROPE_CTKV,
+             lse=None, out=None, kv_heads=1) -> tuple[Op, torch.Tensor]:
+    """Plan the MLA decode/spec call; returns (op, attenOut)."""
+    L = lib()
+    out = torch.empty_like(q_nope) if out is None else out
+    cl = _host_i32(context_lens)
+    qs = None if q_seq_len is None else _host_i32(q_seq_len)
+    ts = [tensor(q_nope), tensor(q_rope), tensor(ct_kv), tensor(k_rope), tensor(block_tables), tensor(cl), None,
+          tensor(qs), None, None]
+    to, tl = tensor(out), tensor(lse)
+    ws = ctypes.c_uint64(0)
+    h = ctypes.c_void_p(0)
+    _check(L.atb_like_mla_get_workspace_size(*[_ref(t) for t in ts], int(heads), float(qk_scale), int(kv_heads),
+                                             int(mask_type), int(calc_type), int(cache_mode), _ref(to), _ref(tl),
+                                             ctypes.byref(ws), ctypes.byref(h)))
+    return Op(h, ws.value, L.atb_like_mla, q_nope.device,
+              (q_nope, q_rope, ct_kv, k_rope, block_tables, cl, qs, out, lse)), out
+
+
+def atb_like_mla(q_nope, q_rope, ct_kv, k_rope, block_tables, context_lens, q_seq_len, heads, qk_scale,
+                 mask_type=MLA_MASK_UNDEFINED, calc_type=MLA_CALC_UNDEFINED, return_lse=False):
+    lse = (torch.empty((q_nope.shape[0], heads, 1), dtype=torch.float32, device=q_nope.device)
+           if return_lse else None)
+    op, out = plan_mla(q_nope, q_rope, ct_kv, k_rope, block_tables, context_lens, q_seq_len, heads, qk_scale,
+                       mask_type, calc_type, lse=lse)
+    op()
+    return (out, lse) if return_lse else out

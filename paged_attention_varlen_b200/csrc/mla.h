@@ -1,0 +1,38 @@
+// mla.h -- host plan for the MLA decode / speculative-decode path.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "../../include/ala.h"
+
+namespace ala {
+
+struct MlaPlan {
+  int32_t dtype = 0, heads = 0, batch = 0, block_size = 0, max_blocks = 0;
+  int32_t calc_type = 0, mask_type = 0;
+  float qk_scale = 1.f;
+  int64_t tokens = 0, num_blocks = 0;
+  void *q_nope = nullptr, *q_rope = nullptr, *ct_kv = nullptr, *k_rope = nullptr, *out = nullptr;
+  float* lse = nullptr;
+  const int32_t* block_tables = nullptr;
+  std::vector<int32_t> ctx, qs;
+  // schedule and workspace
+  int32_t n_work = 0, n_splits_total = 0;
+  uint64_t ws_size = 0, off_work = 0, off_rows = 0, off_part_o = 0, off_part_lse = 0;
+  std::vector<uint8_t> image;
+  bool maps_ready = false;
+  CUtensorMap tmQn, tmQr, tmKV, tmKR;
+};
+
+int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, const ala_tensor* ctKV,
+             const ala_tensor* kRope, const ala_tensor* blockTables, const ala_tensor* contextLens,
+             const ala_tensor* mask, const ala_tensor* qSeqLen, const ala_tensor* qkDescale,
+             const ala_tensor* pvDescale, int32_t headNum, float qkScale, int32_t kvHeadNum, int maskType,
+             int calcType, uint8_t cacheMode, ala_tensor* attenOut, ala_tensor* lse, char* err, size_t errlen);
+
+int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size_t errlen);
+
+}  // namespace ala

@@ -1,0 +1,159 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol, and
+rejects bad arguments with the documented status before touching the device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import paged_attention_varlen_b200 as ala
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from paged_attention_varlen_b200 import build
+    build.build()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "ala.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:ALA_API\s+)?(?:const\s+)?\w+\*?\s+\**(\w+)\s*\(", text, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert {"atb_like_prefix_encoder", "atb_like_mla", "varlen_attention", "ala_last_error"} <= set(names)
+    L = ctypes.CDLL(ala.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/ala.h but not exported"
+
+
+def _varlen_args(**over):
+    a = dict(q=torch.zeros(10, 4, 128, dtype=torch.bfloat16), k=torch.zeros(14, 2, 128, dtype=torch.bfloat16),
+             v=torch.zeros(14, 2, 128, dtype=torch.bfloat16), seq_len=[4, 6], kv_seq_len=[6, 8], mask_type=9,
+             heads=4, kv_heads=2, qk_scale=0.1, slopes=None)
+    a.update(over)
+    return a
+
+
+def _plan_varlen(**over):
+    a = _varlen_args(**over)
+    return ala.plan_varlen_attention(a["q"], a["k"], a["v"], a["seq_len"], a["kv_seq_len"], a["mask_type"],
+                                     a["heads"], a["kv_heads"], a["qk_scale"], a["slopes"])
+
+
+def test_valid_plan_needs_no_gpu():
+    op, out = _plan_varlen()
+    assert op.workspace_size > 0 and out.shape == (10, 4, 128)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(heads=0), 4),                                          # headNum must be > 0
+    (dict(kv_heads=3), 4),                                       # kvHeadNum must divide headNum
+    (dict(mask_type=7), 4),                                      # maskType not in {0,3,4,5,9}
+    (dict(kv_seq_len=[3, 8]), 4),                                # kvSeqLen < seqLen
+    (dict(seq_len=[4, 5], kv_seq_len=[6, 8]), 2),                # sum(seqLen) != nTokens
+    (dict(kv_seq_len=[6, 9]), 2),                                # sum(kvSeqLen) != nKvTokens
+    (dict(mask_type=3), 1),                                      # ALiBi needs slopes
+    (dict(slopes=np.ones(4, np.float32)), 4),                    # causal forbids slopes
+    (dict(mask_type=3, slopes=np.ones(3, np.float32)), 2),       # slopes must be [headNum]
+    (dict(k=torch.zeros(14, 2, 128, dtype=torch.float16)), 3),   # dtype mismatch
+    (dict(q=torch.zeros(10, 4, 256, dtype=torch.bfloat16), k=torch.zeros(14, 2, 256, dtype=torch.bfloat16),
+          v=torch.zeros(14, 2, 256, dtype=torch.bfloat16), mask_type=3, slopes=np.ones(4, np.float32)), 4),
+    (dict(q=torch.zeros(10, 4, 96, dtype=torch.bfloat16), k=torch.zeros(14, 2, 96, dtype=torch.bfloat16),
+          v=torch.zeros(14, 2, 96, dtype=torch.bfloat16)), 5),   # head size not built
+    (dict(q=torch.zeros(10, 4, 128), k=torch.zeros(14, 2, 128), v=torch.zeros(14, 2, 128)), 5),  # f32 d=128
+])
+def test_varlen_rejects(over, status):
+    with pytest.raises(ala.AlaError) as e:
+        _plan_varlen(**over)
+    assert e.value.status == status, str(e.value)
+
+
+def _prefix_args():
+    bs, nb = 16, 8
+    return dict(q=torch.zeros(10, 4, 128, dtype=torch.float16), k=torch.zeros(nb, bs, 2, 128, dtype=torch.float16),
+                v=torch.zeros(nb, bs, 2, 128, dtype=torch.float16),
+                block_tables=torch.zeros(2, 2, dtype=torch.int32), seq_len=[4, 6], kv_seq_len=[20, 30],
+                mask_type=3, heads=4, kv_heads=2, qk_scale=0.1, slopes=torch.ones(4), mask=None)
+
+
+def _plan_prefix(**over):
+    a = _prefix_args()
+    a.update(over)
+    return ala.plan_prefix_encoder(a["q"], a["k"], a["v"], a["block_tables"], a["seq_len"], a["kv_seq_len"],
+                                   a["mask_type"], a["heads"], a["kv_heads"], a["qk_scale"], a["slopes"], a["mask"])
+
+
+def test_prefix_plan_ok_and_mask_tensor_accepted():
+    _plan_prefix()
+    _plan_prefix(mask=torch.zeros(256, 256, dtype=torch.float16))
+    _plan_prefix(mask=torch.zeros(4, 4, 128, dtype=torch.float16), mask_type=4)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(mask_type=0, slopes=None), 4),                                      # PrefixEncoder: 3/4/5/9 only
+    (dict(mask_type=9), 4),                                                   # slopes must be NULL for causal
+    (dict(mask_type=5, mask=torch.zeros(256, 256, dtype=torch.float16)), 4),  # mask NULL for 5/9
+    (dict(mask=torch.zeros(128, 128, dtype=torch.float16)), 2),               # mask shape
+    (dict(kv_seq_len=[20, 40]), 4),                                           # needs 3 blocks > maxBlockNum 2
+    (dict(block_tables=torch.zeros(3, 2, dtype=torch.int32)), 2),             # rows != batch
+    (dict(k=torch.zeros(8, 24, 2, 128, dtype=torch.float16), v=torch.zeros(8, 24, 2, 128, dtype=torch.float16)), 5),
+    (dict(q=torch.zeros(10, 4, 128), k=torch.zeros(8, 16, 2, 128), v=torch.zeros(8, 16, 2, 128)), 3),  # f32
+    (dict(block_tables=None), 1),
+])
+def test_prefix_rejects(over, status):
+    with pytest.raises(ala.AlaError) as e:
+        _plan_prefix(**over)
+    assert e.value.status == status, str(e.value)
+
+
+def _mla_args():
+    nb, bs, H = 6, 64, 128
+    return dict(q_nope=torch.zeros(3, H, 512, dtype=torch.bfloat16), q_rope=torch.zeros(3, H, 64, dtype=torch.bfloat16),
+                ct_kv=torch.zeros(nb, bs, 1, 512, dtype=torch.bfloat16),
+                k_rope=torch.zeros(nb, bs, 1, 64, dtype=torch.bfloat16),
+                block_tables=torch.zeros(3, 2, dtype=torch.int32), context_lens=[5, 100, 128], q_seq_len=None,
+                heads=H, qk_scale=0.04, mask_type=0, calc_type=0, cache_mode=1, kv_heads=1)
+
+
+def _plan_mla(**over):
+    a = _mla_args()
+    a.update(over)
+    return ala.plan_mla(a["q_nope"], a["q_rope"], a["ct_kv"], a["k_rope"], a["block_tables"], a["context_lens"],
+                        a["q_seq_len"], a["heads"], a["qk_scale"], a["mask_type"], a["calc_type"], a["cache_mode"],
+                        kv_heads=a["kv_heads"])
+
+
+def test_mla_plan_ok():
+    _plan_mla()
+    _plan_mla(q_nope=torch.zeros(6, 128, 512, dtype=torch.bfloat16), q_rope=torch.zeros(6, 128, 64, dtype=torch.bfloat16),
+              q_seq_len=[2, 2, 2], mask_type=1, calc_type=1)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(cache_mode=0), 5), (dict(cache_mode=2), 5), (dict(cache_mode=3), 5),
+    (dict(calc_type=2), 5), (dict(calc_type=3), 5),
+    (dict(mask_type=3), 4),                        # ALiBi only on the encoder paths
+    (dict(kv_heads=2), 5),
+    (dict(context_lens=[5, 100, 129]), 4),         # needs 3 blocks > 2
+    (dict(calc_type=1), 1),                        # SPEC needs qseqlen
+    (dict(q_seq_len=[1, 1, 1]), 4),                # qseqlen only with SPEC
+    (dict(q_rope=torch.zeros(3, 128, 32, dtype=torch.bfloat16)), 2),
+    (dict(heads=0), 4),
+])
+def test_mla_rejects(over, status):
+    with pytest.raises(ala.AlaError) as e:
+        _plan_mla(**over)
+    assert e.value.status == status, str(e.value)
+
+
+def test_last_error_is_text():
+    with pytest.raises(ala.AlaError) as e:
+        _plan_varlen(heads=0)
+    assert "headNum" in str(e.value)

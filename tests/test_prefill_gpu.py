@@ -1,0 +1,157 @@
+"""GPU parity of the prefill kernel (varlen_attention / atb_like_prefix_encoder)
+against the fp64 oracle on the same seeded inputs.
+
+Small cases compare every output element; the full-size workloads compare
+sampled rows (each sequence's first and last rows, tile boundaries, random
+rows) that the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_attention_varlen_b200 as ala
+import synth
+from parity import check_lse, check_out, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    from paged_attention_varlen_b200 import build
+    build.build()
+
+
+def _dev(case):
+    d = "cuda"
+    return (case.q.to(d), case.k.to(d), case.v.to(d),
+            None if case.slopes is None else torch.from_numpy(case.slopes).to(d),
+            None if case.block_tables is None else torch.from_numpy(case.block_tables).to(d))
+
+
+def _run(case, want_lse=True):
+    q, k, v, slopes, bt = _dev(case)
+    lse = None
+    if case.paged:
+        op, out = ala.plan_prefix_encoder(q, k, v, bt, case.seq_len, case.kv_seq_len, case.mask_type, case.heads,
+                                          case.kv_heads, case.qk_scale, slopes)
+    else:
+        if want_lse:
+            lse = torch.empty((q.shape[0], case.heads), dtype=torch.float32, device="cuda")
+        op, out = ala.plan_varlen_attention(q, k, v, case.seq_len, case.kv_seq_len, case.mask_type, case.heads,
+                                            case.kv_heads, case.qk_scale, slopes, lse=lse)
+    op()
+    torch.cuda.synchronize()
+    assert op.device_status() == 0, f"device status {op.device_status():#x}"
+    return out, lse
+
+
+def _oracle(case, rows=None):
+    return oracle.attention(case.q, case.k, case.v, case.seq_len, case.kv_seq_len, case.mask_type, case.heads,
+                            case.kv_heads, case.qk_scale, slopes=case.slopes, block_tables=case.block_tables,
+                            block_size=case.block_size, rows=rows)
+
+
+def _full_check(case):
+    out, lse = _run(case)
+    ref, lref = _oracle(case)
+    H = case.heads
+    check_out(out.reshape(-1, out.shape[-1]), ref)
+    if lse is not None:
+        check_lse(lse.reshape(-1), lref)
+    return out
+
+
+def test_tiny_causal_fp32_tf32():
+    _full_check(synth.tiny_causal_fp32())
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_ragged_varlen_causal_gqa(d, dtype):
+    L = [1, 127, 128, 129, 300, 0, 5, 257]
+    case = synth.make_prefill("ragged", L, L, 8, 2, d, dtype, synth.MASK_CAUSAL, 7)
+    _full_check(case)
+
+
+@pytest.mark.parametrize("mask_type", [0, 3, 4, 5, 9])
+def test_prefix_offset_masks_contiguous(mask_type):
+    L = [3, 130, 64, 200]
+    pre = [0, 77, 256, 1000]
+    case = synth.make_prefill("prefix", L, [a + b for a, b in zip(L, pre)], 8, 4, 128, torch.bfloat16, mask_type, 11)
+    _full_check(case)
+
+
+@pytest.mark.parametrize("block_size", [16, 32, 64, 128, 256])
+@pytest.mark.parametrize("mask_type", [3, 4, 5, 9])
+def test_paged_prefix_encoder(block_size, mask_type):
+    L = [64, 1, 333, 129]
+    pre = [256, 40, 512, 0]
+    case = synth.make_prefill("paged", L, [a + b for a, b in zip(L, pre)], 8, 2, 128, torch.float16, mask_type, 13,
+                              paged=True, block_size=block_size)
+    _full_check(case)
+
+
+def test_paged_equals_contiguous_on_gpu():
+    L, pre = [100, 250], [300, 17]
+    kv = [a + b for a, b in zip(L, pre)]
+    c = synth.make_prefill("c", L, kv, 8, 2, 128, torch.float16, 3, 17)
+    p = synth.make_prefill("p", L, kv, 8, 2, 128, torch.float16, 3, 17, paged=True, block_size=64)
+    oc, _ = _run(c, want_lse=False)
+    op, _ = _run(p, want_lse=False)
+    assert torch.equal(oc, op)
+
+
+def test_padded_run_matches_packed_on_valid_rows():
+    case = synth.varlen_causal_bf16(seed=21, batch=4, lo=20, hi=400)
+    pad = synth.padded_from(case)
+    out, _ = _run(case, want_lse=False)
+    outp, _ = _run(pad, want_lse=False)
+    Lmax = pad.meta["Lmax"]
+    pos = 0
+    for b, L in enumerate(case.seq_len.tolist()):
+        assert torch.equal(out[pos:pos + L], outp[b * Lmax:b * Lmax + L])
+        pos += L
+
+
+def test_repeat_is_deterministic_and_status_clean():
+    case = synth.make_prefill("rep", [300, 50], [400, 50], 8, 2, 128, torch.bfloat16, 4, 23)
+    q, k, v, slopes, _ = _dev(case)
+    op, out = ala.plan_varlen_attention(q, k, v, case.seq_len, case.kv_seq_len, 4, 8, 2, case.qk_scale, slopes)
+    op()
+    first = out.clone()
+    for _ in range(3):
+        op()
+    torch.cuda.synchronize()
+    assert torch.equal(first, out)
+    assert op.device_status() == 0
+
+
+# ---------------------------------------------------------------------------- full-size workloads, sampled rows
+
+def _sampled_check(case, n=384, seed=0):
+    out, lse = _run(case)
+    H = case.heads
+    rows = sample_rows(case.seq_len, H, n, seed)
+    ref, lref = _oracle(case, rows)
+    check_out(out.reshape(-1, out.shape[-1])[torch.from_numpy(rows).cuda()], ref)
+    if lse is not None:
+        check_lse(lse.reshape(-1)[torch.from_numpy(rows).cuda()], lref)
+    # every row finite, not only the sampled ones
+    assert torch.isfinite(out.float()).all()
+
+
+def test_full_varlen_causal_bf16():
+    _sampled_check(synth.varlen_causal_bf16())
+
+
+def test_full_prefix_paged_alibi_fp16():
+    _sampled_check(synth.prefix_paged_alibi_fp16())
+
+
+@pytest.mark.parametrize("variant", [synth.MASK_ALIBI_SQRT, synth.MASK_ALIBI_LEFT])
+def test_full_long_alibi_bf16(variant):
+    _sampled_check(synth.long_alibi_bf16(variant), n=192)
