@@ -1,0 +1,388 @@
+"""Benchmark of the packed-varlen attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one call of the library's varlen_attention over the packed-varlen
+causal prefill workload (batch 8, seqLen ~ U[64, 2048] seeded, headNum 32,
+kvHeadNum 8, headSize 128, bf16, qkScale 1/sqrt(128)): host-side schedule
+upload plus one prefill kernel launch.  The metric is attention TFLOPS on
+valid tokens: 4 * headSize * headNum * (allowed query/key pairs) per step.
+
+Timing: W untimed warm-up steps, then K timed steps bracketed by a barrier
+and a device synchronise; each step is timed with CUDA events on the launch
+stream, with the L2 flushed (a 256 MiB write) before every step, outside its
+events.  Under torchrun every rank runs the same workload on its own GPU
+(independent sequences, no collective on the data path; weak scaling), and
+the per-step time is the max over ranks.
+
+Also reported on rank 0:
+  * roofline of the prefill kernel against the measured dense bf16 peak;
+  * e2e: the same metric through the public call with inputs copied from
+    pinned host memory and the output copied back inside the timed region;
+  * cpu_baseline: the fp64 oracle on the host cores over a bounded sample of
+    the same workload's rows;
+  * extra: the other workloads (paged ALiBi prefix encoder fp16, long ALiBi
+    bf16 in both variants, MLA decode/spec when built) measured the same way.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+PROFILE = os.path.join(ROOT, "profiles", "prefill_varlen_causal_bf16.md")
+KERNEL_SOURCES = ["paged_attention_varlen_b200/csrc/prefill.cu", "paged_attention_varlen_b200/csrc/ptx.cuh"]
+L2_FLUSH_BYTES = 256 << 20
+
+
+def kernel_source_hash(paths=KERNEL_SOURCES) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def profiled_traffic(path, src_hash):
+    """dram bytes per launch from the committed ncu summary, if it was taken on the current kernel source."""
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for line in open(path):
+        if ":" in line and line.strip().startswith(("traffic_bytes_per_launch", "kernel_source_sha256")):
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha256") != src_hash or "traffic_bytes_per_launch" not in vals:
+        return None
+    return float(vals["traffic_bytes_per_launch"])
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index):
+        self.samples, self.reasons, self.ok = [], set(), False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------- workloads
+
+def prefill_flops(case) -> float:
+    return 4.0 * case.head_size * case.heads * case.valid_pairs()
+
+
+def prefill_bytes(case) -> float:
+    es = case.q.element_size()
+    kv_tokens = int(case.kv_seq_len.sum())
+    return es * case.head_size * (2 * case.n_tokens * case.heads + 2 * kv_tokens * case.kv_heads)
+
+
+def mla_flops(case) -> float:
+    return case.heads * (2 * 576 + 2 * 512) * case.valid_pairs()
+
+
+def mla_bytes(case) -> float:
+    es = case.q_nope.element_size()
+    kv = int(case.context_lens.sum()) * 576 * es
+    q = case.n_tokens * case.heads * 576 * es
+    o = case.n_tokens * case.heads * 512 * es + case.n_tokens * case.heads * 4
+    return kv + q + o
+
+
+def plan_case(ala, case, device):
+    """Device copies of the inputs and a planned op; returns (op, tensors dict)."""
+    if isinstance(case, synth.MlaCase):
+        t = {"q_nope": case.q_nope.to(device), "q_rope": case.q_rope.to(device), "ct_kv": case.ct_kv.to(device),
+             "k_rope": case.k_rope.to(device), "bt": torch.from_numpy(case.block_tables).to(device)}
+        t["lse"] = torch.empty((case.n_tokens, case.heads, 1), dtype=torch.float32, device=device)
+        op, out = ala.plan_mla(t["q_nope"], t["q_rope"], t["ct_kv"], t["k_rope"], t["bt"], case.context_lens,
+                               case.q_seq_len if case.calc_type == synth.MLA_CALC_SPEC else None, case.heads,
+                               case.qk_scale, case.mask_type, case.calc_type, lse=t["lse"])
+        t["out"] = out
+        return op, t
+    t = {"q": case.q.to(device), "k": case.k.to(device), "v": case.v.to(device)}
+    slopes = None if case.slopes is None else torch.from_numpy(case.slopes).to(device)
+    if case.paged:
+        t["bt"] = torch.from_numpy(case.block_tables).to(device)
+        op, out = ala.plan_prefix_encoder(t["q"], t["k"], t["v"], t["bt"], case.seq_len, case.kv_seq_len,
+                                          case.mask_type, case.heads, case.kv_heads, case.qk_scale, slopes)
+    else:
+        op, out = ala.plan_varlen_attention(t["q"], t["k"], t["v"], case.seq_len, case.kv_seq_len, case.mask_type,
+                                            case.heads, case.kv_heads, case.qk_scale, slopes)
+    t["out"], t["slopes"] = out, slopes
+    return op, t
+
+
+def time_steps(op, steps, warmup, flush, stream, barrier=lambda: None):
+    for _ in range(warmup):
+        op(stream)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record(stream)
+        op(stream)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    assert op.device_status() == 0, "device status nonzero after the timed steps"
+    return [e0.elapsed_time(e1) for e0, e1 in ev]
+
+
+def e2e_prefill(ala, case, tens, op, steps, stream):
+    """Same metric through the public call, inputs from pinned host memory and output back to host."""
+    host = {k: case_t.pin_memory() for k, case_t in (("q", case.q), ("k", case.k), ("v", case.v))}
+    out_host = torch.empty(tens["out"].shape, dtype=tens["out"].dtype).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    times = []
+    for i in range(steps + 2):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for k in ("q", "k", "v"):
+                tens[k].copy_(host[k], non_blocking=True)
+            op(stream)
+            out_host.copy_(tens["out"], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= 2:
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.mean(times)
+    return {"value": prefill_flops(case) / (ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def cpu_baseline(case, budget_s=12.0):
+    """The fp64 oracle, as it stands, on a bounded random sample of the workload's rows."""
+    import oracle
+    cu = np.concatenate([[0], np.cumsum(case.seq_len)])
+    tok_seq = np.repeat(np.arange(len(case.seq_len)), case.seq_len)
+    rng = np.random.Generator(np.random.PCG64(7))
+    n_rows = 256
+    total_flops, total_s, rows_done = 0.0, 0.0, 0
+    while total_s < budget_s:
+        rows = rng.choice(case.n_tokens * case.heads, size=n_rows, replace=False)
+        t0 = time.perf_counter()
+        oracle.attention(case.q, case.k, case.v, case.seq_len, case.kv_seq_len, case.mask_type, case.heads,
+                         case.kv_heads, case.qk_scale, slopes=case.slopes, block_tables=case.block_tables,
+                         block_size=case.block_size, rows=rows)
+        total_s += time.perf_counter() - t0
+        tok = rows // case.heads
+        b = tok_seq[tok]
+        i = tok - cu[b]
+        allowed = np.minimum(i + (case.kv_seq_len[b] - case.seq_len[b]) + 1, case.kv_seq_len[b])
+        total_flops += float((4.0 * case.head_size * allowed).sum())
+        rows_done += n_rows
+        n_rows = min(n_rows * 2, case.n_tokens * case.heads)
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": total_flops / total_s / 1e12, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+            "sample": f"{rows_done} random (token, head) rows of the {case.name} workload, {total_s:.1f} s "
+                      f"fp64 on the host (valid FLOPs of the sampled rows / time)"}
+
+
+def base_config(case):
+    return {"workload": case.name, "global_batch": len(case.seq_len), "tokens": case.n_tokens,
+            "seq_len": "U[64,2048] per sequence", "heads": case.heads, "kv_heads": case.kv_heads,
+            "head_size": case.head_size, "mask": "causal", "parallelism": "replicas (independent sequences)",
+            "l2": "flushed before every step (256 MiB write, outside the step events)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    case = synth.varlen_causal_bf16()
+    cb = cpu_baseline(case, budget_s=max(3.0, 10.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    for _ in range(args.warmup + args.steps):
+        vals.append(cpu_baseline(case, budget_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)))["value"])
+    v = statistics.mean(vals[args.warmup:]) if len(vals) > args.warmup else vals[-1]
+    flops = prefill_flops(case)
+    line = {"impl": "reference", "metric": "attention TFLOPS on valid tokens (prefill)", "value": v,
+            "unit": "TFLOPS", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": flops / (v * 1e12) * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": base_config(case),
+            "cpu_baseline": {"value": v, "unit": "TFLOPS", "cores": cb["cores"], "kind": "oracle",
+                             "sample": "each step: a bounded random sample of rows; " + cb["sample"]},
+            "e2e": {"value": v, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import paged_attention_varlen_b200 as ala
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    barrier = (lambda: dist.barrier()) if dist else (lambda: None)
+
+    case = synth.varlen_causal_bf16()
+    op, tens = plan_case(ala, case, device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    with ClockSampler(local) as clk:
+        times = time_steps(op, args.steps, args.warmup, flush, stream, barrier)
+    ms = statistics.mean(times)
+    if dist:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    flops = prefill_flops(case)
+    value = world * flops / (ms * 1e-3) / 1e12
+
+    if rank == 0:
+        peaks = measured_peaks()
+        src = kernel_source_hash()
+        achieved = flops / (statistics.mean(times) * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": achieved / peaks["bf16_tflops"], "traffic": profiled_traffic(PROFILE, src),
+                    "algorithmic_bytes": prefill_bytes(case), "peak_source": peaks["source"] + " (burst bf16)",
+                    "kernel": "prefill_kernel<bf16,128>", "kernel_source_sha256": src}
+        line = {"metric": "attention TFLOPS on valid tokens (prefill)", "value": value, "unit": "TFLOPS",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic", "config": base_config(case), "roofline": roofline,
+                "clocks": clk.summary(), "gpu_launches": args.steps,
+                "valid_flops_per_step": flops, "padding_positions": int(len(case.seq_len) * case.seq_len.max()
+                                                                         - case.seq_len.sum())}
+        if not args.no_e2e:
+            line["e2e"] = e2e_prefill(ala, case, tens, op, min(args.steps, 10), stream)
+        if not args.no_extra:
+            line["extra"] = extra_workloads(ala, device, flush, stream, peaks, case, args)
+        if world == 1 and not args.no_cpu:
+            line["cpu_baseline"] = cpu_baseline(case)
+        print(json.dumps(line))
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def extra_workloads(ala, device, flush, stream, peaks, main_case, args):
+    out = {}
+    steps = max(5, min(args.steps, 20))
+    # padded layout of the same batch: same kernel, the work a padded batch carries
+    pad = synth.padded_from(main_case)
+    op, _ = plan_case(ala, pad, device)
+    ms = statistics.mean(time_steps(op, steps, 3, flush, stream))
+    out["varlen_causal_bf16_padded"] = {
+        "ms": ms, "padding_positions": pad.meta["padding_positions"],
+        "pairs_ratio_vs_packed": pad.valid_pairs() / main_case.valid_pairs(),
+        "valid_tflops": prefill_flops(main_case) / (ms * 1e-3) / 1e12}
+    del op
+    for case in (synth.prefix_paged_alibi_fp16(), synth.long_alibi_bf16(synth.MASK_ALIBI_SQRT),
+                 synth.long_alibi_bf16(synth.MASK_ALIBI_LEFT)):
+        op, _ = plan_case(ala, case, device)
+        ms = statistics.mean(time_steps(op, steps, 3, flush, stream))
+        tf = prefill_flops(case) / (ms * 1e-3) / 1e12
+        out[case.name] = {"ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / peaks["bf16_tflops"]}
+        del op
+    for qs in (1, 4):
+        case = synth.mla_decode_bf16(qs)
+        try:
+            op, _ = plan_case(ala, case, device)
+            ms = statistics.mean(time_steps(op, steps, 3, flush, stream))
+        except ala.AlaError as e:
+            out[case.name] = {"unavailable": str(e)}
+            continue
+        gbs = mla_bytes(case) / (ms * 1e-3) / 1e9
+        tf = mla_flops(case) / (ms * 1e-3) / 1e12
+        out[case.name] = {"ms": ms, "hbm_gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"], "tflops": tf,
+                          "frac_of_bf16_peak": tf / peaks["bf16_tflops"]}
+        del op
+    return out
+
+
+if __name__ == "__main__":
+    main()

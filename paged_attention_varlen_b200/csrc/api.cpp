@@ -103,6 +103,28 @@ bool encode_rows_heads_d(CUtensorMap* map, void* base, int32_t dtype, int64_t ro
 }  // namespace
 
 // ------------------------------------------------------------------ op
+// Page-locked copy of a host image, made on first use so the per-call upload
+// is a plain asynchronous DMA (host memory only; no device memory is allocated).
+struct PinnedImage {
+  void* ptr = nullptr;
+  size_t size = 0;
+  ~PinnedImage() {
+    if (ptr) cudaFreeHost(ptr);
+  }
+  const void* get(const std::vector<uint8_t>& img) {
+    if (!ptr && !img.empty()) {
+      if (cudaHostAlloc(&ptr, img.size(), cudaHostAllocDefault) != cudaSuccess) {
+        ptr = nullptr;
+        cudaGetLastError();
+        return img.data();  // fall back to a staged copy from pageable memory
+      }
+      std::memcpy(ptr, img.data(), img.size());
+      size = img.size();
+    }
+    return ptr ? ptr : img.data();
+  }
+};
+
 struct ala_op {
   enum Kind { kPrefill, kMla } kind = kPrefill;
   // prefill
@@ -118,6 +140,7 @@ struct ala_op {
   uint64_t off_seqs = 0, off_units = 0, ws_size = 0;
   int32_t n_units = 0;
   std::vector<uint8_t> image;  // host copy of the workspace header (status, seqs, units)
+  PinnedImage pinned;
   bool maps_ready = false;
   CUtensorMap tmQ, tmK, tmV;
   // mla
@@ -291,25 +314,46 @@ int build_prefill(ala_op* op, const ala_tensor* query, const ala_tensor* key, co
   op->slopes = alibi ? static_cast<const float*>(slopes->data) : nullptr;
   op->lse = lse ? static_cast<float*>(lse->data) : nullptr;
 
-  // schedule: one unit per (sequence, 128-row query tile, query head); key tiles up to the last allowed key
+  // schedule: units of up to two 128-row blocks that share a kv head (two query heads
+  // of one group, or two consecutive row tiles of one head when there is no grouping);
+  // each block visits key tiles up to its last allowed key.
   std::vector<SeqInfo> seqs(batch);
   std::vector<PrefillUnit> units;
+  const int32_t group = headNum / kvHeadNum;
   int32_t cq = 0, ckv = 0;
   for (int32_t b = 0; b < batch; ++b) {
     seqs[b] = SeqInfo{cq, sl[b], kl[b], ckv};
     const int32_t off = kl[b] - sl[b];
-    for (int32_t q0 = 0; q0 < sl[b]; q0 += 128) {
+    auto tiles_for = [&](int32_t q0) {
       const int32_t last_row = std::min(q0 + 127, sl[b] - 1);
       const int32_t kv_end = maskType == 0 ? kl[b] : std::min(kl[b], last_row + off + 1);
-      const int32_t n_tiles = (kv_end + 127) / 128;
-      for (int32_t h = 0; h < headNum; ++h) units.push_back(PrefillUnit{b, q0, h, n_tiles});
+      return (kv_end + 127) / 128;
+    };
+    if (group >= 2) {
+      for (int32_t q0 = 0; q0 < sl[b]; q0 += 128) {
+        const int32_t nt = tiles_for(q0);
+        for (int32_t g = 0; g < kvHeadNum; ++g)
+          for (int32_t i = 0; i < group; i += 2) {
+            const int32_t h = g * group + i;
+            const bool two = i + 1 < group;
+            units.push_back(PrefillUnit{b, two ? 2 : 1, {q0, q0}, {h, two ? h + 1 : h}, {nt, two ? nt : 0}});
+          }
+      }
+    } else {
+      for (int32_t h = 0; h < headNum; ++h)
+        for (int32_t q0 = 0; q0 < sl[b]; q0 += 256) {
+          const bool two = q0 + 128 < sl[b];
+          units.push_back(PrefillUnit{b, two ? 2 : 1, {q0, q0 + 128}, {h, h},
+                                      {tiles_for(q0), two ? tiles_for(q0 + 128) : 0}});
+        }
     }
     cq += sl[b];
     ckv += kl[b];
   }
   // longest first, so the tail of the grid is made of short units
+  auto cost = [](const PrefillUnit& u) { return u.n_tiles[0] + u.n_tiles[1]; };
   std::stable_sort(units.begin(), units.end(),
-                   [](const PrefillUnit& a, const PrefillUnit& b) { return a.n_tiles > b.n_tiles; });
+                   [&](const PrefillUnit& a, const PrefillUnit& b) { return cost(a) > cost(b); });
   op->n_units = (int32_t)units.size();
   op->off_seqs = kAlign;
   op->off_units = align_up(op->off_seqs + sizeof(SeqInfo) * std::max(batch, 1));
@@ -338,7 +382,7 @@ int run_prefill(void* workspace, uint64_t workspaceSize, ala_op* op, ala_stream_
       return fail(ALA_CUDA_ERROR, "%s: cuTensorMapEncodeTiled failed (pointers must be 16-byte aligned)", fn);
     op->maps_ready = true;
   }
-  if (cudaMemcpyAsync(workspace, op->image.data(), op->ws_size, cudaMemcpyHostToDevice, st) != cudaSuccess)
+  if (cudaMemcpyAsync(workspace, op->pinned.get(op->image), op->ws_size, cudaMemcpyHostToDevice, st) != cudaSuccess)
     return fail(ALA_CUDA_ERROR, "%s: schedule upload failed: %s", fn, cudaGetErrorString(cudaGetLastError()));
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   PrefillParams p{};

@@ -30,12 +30,16 @@ struct SeqInfo {
   int32_t cu_kv;    // first packed key row (contiguous layout only)
 };
 
-// One CTA's work: 128 query rows of one query head of one sequence.
+// One CTA's work: up to two blocks of 128 query rows of one sequence that read
+// the same kv head (two query heads of a group, or two consecutive row tiles of
+// one head), so every K/V tile the CTA loads serves both.
 struct PrefillUnit {
-  int32_t b;        // sequence
-  int32_t q0;       // first query row of the tile (within the sequence)
-  int32_t head;     // query head
-  int32_t n_tiles;  // 128-key tiles to visit: ceil(min(kv_len, last allowed key + 1) / 128)
+  int32_t b;           // sequence
+  int32_t n_blocks;    // 1 or 2
+  int32_t q0[2];       // first query row of each block (within the sequence)
+  int32_t head[2];     // query head of each block
+  int32_t n_tiles[2];  // 128-key tiles each block visits: ceil(min(kv_len, last allowed key + 1) / 128);
+                       // n_tiles[1] >= n_tiles[0] when n_blocks == 2
 };
 
 struct PrefillParams {

@@ -4,24 +4,30 @@
 // table; nalar.dev padding-mask article, sections on packing and on fused
 // kernels that apply the mask rule without materialising it).
 //
-// One CTA computes 128 query rows of one query head of one sequence:
+// One CTA computes up to two blocks of 128 query rows that read the same kv
+// head (two query heads of a GQA group, or two consecutive row tiles of one
+// head), so each K/V tile staged in shared memory serves 256 rows.
 //
-//   warp 4      TMA producer: Q tile once, then K and V tiles (128 keys each)
-//               into a STAGES-deep ring; paged K/V rows are gathered page by
-//               page through the block table.
-//   warp 5      tcgen05 issuer: S = Q K^T into one of two TMEM buffers, then
-//               O += P V into the TMEM accumulator; completion is signalled
-//               with tcgen05.commit on mbarriers.
-//   warps 0..3  softmax: thread r owns query row r (TMEM lane r).  It reads its
-//               S row from TMEM, applies qkScale, the ALiBi bias and the mask
-//               rule in registers (the mask is never materialised), keeps the
-//               online max / sum, rescales O in TMEM when the running max grows
-//               by more than 2^8, writes P to shared memory in the swizzled
-//               operand layout, and finally normalises O and stores it.
+//   warp 8       TMA producer: both Q tiles once, then K and V tiles (128 keys)
+//                into 2-deep rings; paged rows are gathered page by page
+//                through the block table.
+//   warp 9       tcgen05 issuer.  Per key tile j and block b:
+//                  S_b = Q_b K_j^T        (SS MMA into TMEM columns of S_b)
+//                  O_b += P_b V_j         (TS MMA: P_b read from TMEM)
+//                in the order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so the
+//                tensor core works on one block while the other block's
+//                softmax runs.
+//   warps 0..3,  softmax of block 0 / block 1: thread r owns row r (TMEM lane
+//   4..7         r).  It reads its S row, applies qkScale, the ALiBi bias and
+//                the causal / prefix-offset rule in registers (the mask is
+//                never materialised), updates the running max and sum, rescales
+//                O_b in TMEM only when the max grew by more than 2^8, and writes
+//                P_b (16-bit, or fp32 for tf32) over S_b in TMEM.  At the end it
+//                normalises O_b and stores it.
 //
 // Key tiles wholly above the prefix-shifted causal diagonal, or past the
-// sequence's kvSeqLen, are never visited: the host gives each unit the
-// number of tiles up to its last allowed key.
+// sequence's kvSeqLen, are never visited: the host gives each block the number
+// of tiles up to its last allowed key.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -51,25 +57,25 @@ struct ElemFmt<float> {
   static constexpr uint32_t fmt = 2;  // tf32 tensor-core inputs
 };
 
-template <typename T, int D, int STAGES>
+template <typename T, int D>
 struct Cfg {
   static constexpr int ES = sizeof(T);
   static constexpr int AW = 128 / ES;    // elements in one 128-byte swizzled row
   static constexpr int UK = 32 / ES;     // K extent of one MMA instruction
-  static constexpr int BM = 128;         // query rows per CTA
-  static constexpr int BN = 128;         // keys per tile
   static constexpr int BLK = 128 * 128;  // bytes of one 128-row x 128-byte swizzle column block
-  static constexpr int Q_BYTES = BM * D * ES;
-  static constexpr int KV_BYTES = BN * D * ES;
-  static constexpr int P_BYTES = BM * BN * ES;
-  static constexpr int N_BARS = 1 + 4 * STAGES + 7;
-  static constexpr int SMEM = 1024 + Q_BYTES + 2 * STAGES * KV_BYTES + P_BYTES + N_BARS * 8 + 16;
+  static constexpr int STAGES = 2;
+  static constexpr int Q_BYTES = 128 * D * ES;
+  static constexpr int KV_BYTES = 128 * D * ES;
+  static constexpr int TBL_FLOATS = 160;  // per-warp sqrt-bias table: lane - column + 127 in [0, 159)
+  static constexpr int TBL_BYTES = 8 * 2 * TBL_FLOATS * 4;
+  static constexpr int N_BARS = 18;
+  static constexpr int SMEM = 1024 + 2 * Q_BYTES + 2 * STAGES * KV_BYTES + TBL_BYTES + N_BARS * 8 + 16;
   static constexpr uint32_t IDESC_QK = instr_desc(ElemFmt<T>::fmt, false, false, 128, 128);
   static constexpr uint32_t IDESC_PV = instr_desc(ElemFmt<T>::fmt, false, true, 128, D);
-  static constexpr uint32_t TMEM_COLS = 512;  // S0 [0,128) S1 [128,256) O [256, 256+D)
-  static constexpr uint32_t O_COL = 256;
+  static constexpr uint32_t TMEM_COLS = 512;  // S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D, 256+2D)
   static_assert(D % AW == 0, "head size must fill whole swizzle rows");
   static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(256 + 2 * D <= 512, "tensor memory budget");
 };
 
 __device__ __forceinline__ uint32_t pack2(float a, float b, __nv_bfloat16*) {
@@ -81,61 +87,79 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, __half*) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Write 16 bytes of row r's operand data into a 128B-swizzled K-major block.
-__device__ __forceinline__ void st_swizzled16(uint8_t* block, int r, int chunk, uint4 v) {
-  uint8_t* dst = block + r * 128 + ((chunk ^ (r & 7)) << 4);
-  *reinterpret_cast<uint4*>(dst) = v;
+template <typename T, int D>
+__device__ __forceinline__ void load_kv_tile(const CUtensorMap* map, uint8_t* dst, uint64_t* full, int j,
+                                             const SeqInfo& si, const PrefillParams& p, const int32_t* bt,
+                                             int n_pages, int kvh) {
+  using C = Cfg<T, D>;
+  const bool paged = bt != nullptr;
+  const int bs = p.block_size;
+  const int box_rows = paged ? (bs < 128 ? bs : 128) : 128;
+  const int j0 = j * 128;
+  for (int r0 = 0; r0 < 128; r0 += box_rows) {
+    int row;
+    if (!paged) {
+      row = si.cu_kv + j0 + r0;
+    } else {
+      const int pos = j0 + r0;
+      const int pg = pos / bs;
+      row = pg < n_pages ? bt[pg] * bs + (pos % bs) : p.oob_row;  // past the last page: zero fill
+    }
+#pragma unroll
+    for (int cb = 0; cb < D / C::AW; ++cb) tma_load_3d(dst + cb * C::BLK + r0 * 128, map, full, cb * C::AW, kvh, row);
+  }
 }
 
-template <typename T, int D, int STAGES>
-__global__ void __launch_bounds__(192, 1)
+template <typename T, int D>
+__global__ void __launch_bounds__(384, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
-  using C = Cfg<T, D, STAGES>;
+  using C = Cfg<T, D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + C::Q_BYTES;
-  uint8_t* sV = sK + STAGES * C::KV_BYTES;
-  uint8_t* sP = sV + STAGES * C::KV_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + C::P_BYTES);
+  uint8_t* sQ = smem;                        // [2][Q_BYTES]
+  uint8_t* sK = sQ + 2 * C::Q_BYTES;         // [STAGES][KV_BYTES]
+  uint8_t* sV = sK + C::STAGES * C::KV_BYTES;
+  float* sTbl = reinterpret_cast<float*>(sV + C::STAGES * C::KV_BYTES);  // [8 warps][2][TBL_FLOATS]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sTbl) + C::TBL_BYTES);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;
-  uint64_t* v_full = bars + 1 + STAGES;
-  uint64_t* k_empty = bars + 1 + 2 * STAGES;
-  uint64_t* v_empty = bars + 1 + 3 * STAGES;
-  uint64_t* s_full = bars + 1 + 4 * STAGES;  // [2]
-  uint64_t* s_free = s_full + 2;             // [2]
-  uint64_t* p_full = s_full + 4;
-  uint64_t* o_done = s_full + 5;
-  uint64_t* fin = s_full + 6;
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* v_full = bars + 3;    // [2]
+  uint64_t* k_empty = bars + 5;   // [2]
+  uint64_t* v_empty = bars + 7;   // [2]
+  uint64_t* s_full = bars + 9;    // [2] per block
+  uint64_t* p_full = bars + 11;   // [2] per block
+  uint64_t* pv_done = bars + 13;  // [2] per block
+  uint64_t* o_done = bars + 15;   // [2] per block
+  uint64_t* fin = bars + 17;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::N_BARS);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const PrefillUnit u = p.units[blockIdx.x];
   const SeqInfo si = p.seqs[u.b];
-  const int n = u.n_tiles;
+  const int nb = u.n_blocks;
+  const int n0 = u.n_tiles[0];
+  const int n1 = nb > 1 ? u.n_tiles[1] : 0;
+  const int nmax = n0 > n1 ? n0 : n1;
   int* status = p.status;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < 2; ++s) {
       mbar_init(k_full + s, 1);
       mbar_init(v_full + s, 1);
       mbar_init(k_empty + s, 1);
       mbar_init(v_empty + s, 1);
+      mbar_init(s_full + s, 1);
+      mbar_init(p_full + s, 128);
+      mbar_init(pv_done + s, 1);
+      mbar_init(o_done + s, 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(s_full + i, 1);
-      mbar_init(s_free + i, 128);
-    }
-    mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
     mbar_init(fin, 1);
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -144,105 +168,126 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  // register split: the softmax warpgroups take 216 per thread, warps 8..11 keep 56
+  // (256*216 + 128*56 = 62464 <= 384*168, the registers the block is launched with)
+  if (warp >= 8) {
+    regs_decrease<56>();
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      const int kvh = u.head / p.group;
-      mbar_expect_tx(q_full, C::Q_BYTES);
-      for (int cb = 0; cb < D / C::AW; ++cb)
-        tma_load_3d(sQ + cb * C::BLK, &tmQ, q_full, cb * C::AW, u.head, si.cu_q + u.q0);
-
-      const bool paged = p.block_tables != nullptr;
-      const int bs = p.block_size;
-      const int box_rows = paged ? (bs < 128 ? bs : 128) : 128;
-      const int n_pages = paged ? (si.kv_len + bs - 1) / bs : 0;
-      const int32_t* bt = paged ? p.block_tables + (size_t)u.b * p.max_blocks : nullptr;
+      const int kvh = u.head[0] / p.group;
+      mbar_expect_tx(q_full, nb * C::Q_BYTES);
+      for (int b = 0; b < nb; ++b)
+        for (int cb = 0; cb < D / C::AW; ++cb)
+          tma_load_3d(sQ + b * C::Q_BYTES + cb * C::BLK, &tmQ, q_full, cb * C::AW, u.head[b], si.cu_q + u.q0[b]);
+      const int32_t* bt = p.block_tables ? p.block_tables + (size_t)u.b * p.max_blocks : nullptr;
+      const int n_pages = bt ? (si.kv_len + p.block_size - 1) / p.block_size : 0;
       bool ok = true;
       int issued[2] = {0, 0};  // tiles whose K (0) / V (1) load was issued
-      for (int j = 0; j < n && ok; ++j) {
-        const int s = j % STAGES;
-        const uint32_t par = ((j / STAGES) - 1) & 1;
+      for (int j = 0; j < nmax && ok; ++j) {
+        const int s = j & 1;
+        const uint32_t par = ((j >> 1) - 1) & 1;
         for (int kv = 0; kv < 2; ++kv) {
-          uint64_t* empty = kv ? v_empty + s : k_empty + s;
-          uint64_t* full = kv ? v_full + s : k_full + s;
-          const CUtensorMap* map = kv ? &tmV : &tmK;
-          uint8_t* dst = (kv ? sV : sK) + s * C::KV_BYTES;
-          if (j >= STAGES && !mbar_wait(empty, par, status, kv ? kDevTimeoutVEmpty : kDevTimeoutKEmpty)) {
+          if (j >= 2 && !mbar_wait((kv ? v_empty : k_empty) + s, par, status,
+                                   kv ? kDevTimeoutVEmpty : kDevTimeoutKEmpty)) {
             ok = false;
             break;
           }
+          uint64_t* full = (kv ? v_full : k_full) + s;
           mbar_expect_tx(full, C::KV_BYTES);
-          const int j0 = j * 128;
-          for (int r0 = 0; r0 < 128; r0 += box_rows) {
-            int row;
-            if (!paged) {
-              row = si.cu_kv + j0 + r0;
-            } else {
-              const int pos = j0 + r0;
-              const int pg = pos / bs;
-              row = pg < n_pages ? bt[pg] * bs + (pos % bs) : p.oob_row;
-            }
-            for (int cb = 0; cb < D / C::AW; ++cb)
-              tma_load_3d(dst + cb * C::BLK + r0 * 128, map, full, cb * C::AW, kvh, row);
-          }
+          load_kv_tile<T, D>(kv ? &tmV : &tmK, (kv ? sV : sK) + s * C::KV_BYTES, full, j, si, p, bt, n_pages, kvh);
           issued[kv] = j + 1;
         }
       }
       // never leave the CTA while loads it issued are still landing in shared memory
       for (int kv = 0; kv < 2; ++kv)
-        for (int j = issued[kv] - STAGES < 0 ? 0 : issued[kv] - STAGES; j < issued[kv]; ++j)
-          mbar_wait((kv ? v_full : k_full) + j % STAGES, (j / STAGES) & 1, status,
-                    kv ? kDevTimeoutVFull : kDevTimeoutKFull);
+        for (int j = issued[kv] - 2 < 0 ? 0 : issued[kv] - 2; j < issued[kv]; ++j)
+          mbar_wait((kv ? v_full : k_full) + (j & 1), (j >> 1) & 1, status, kv ? kDevTimeoutVFull : kDevTimeoutKFull);
       mbar_wait(q_full, 0, status, kDevTimeoutQ);
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t q_base = smem_addr(sQ);
-      const uint32_t p_base = smem_addr(sP);
-      bool ok = mbar_wait(q_full, 0, status, kDevTimeoutQ);
-      for (int j = 0; j <= n && ok; ++j) {
-        if (j < n) {
-          const int s = j % STAGES;
-          const int sb = j & 1;
-          if (!mbar_wait(k_full + s, (j / STAGES) & 1, status, kDevTimeoutKFull)) break;
-          if (j >= 2 && !mbar_wait(s_free + sb, ((j - 2) >> 1) & 1, status, kDevTimeoutSFree)) break;
-          tc_fence_after();
-          const uint32_t k_base = smem_addr(sK + s * C::KV_BYTES);
+      auto issue_qk = [&](int b, int s) {
+        const uint32_t qb = q_base + b * C::Q_BYTES;
+        const uint32_t kb = smem_addr(sK + s * C::KV_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < D / C::UK; ++kk) {
-            const int ke = kk * C::UK;
-            const uint32_t off = (ke / C::AW) * C::BLK + (ke % C::AW) * C::ES;
-            mma_ss(tmem + sb * 128, smem_desc_sw128(q_base + off, 16, 1024), smem_desc_sw128(k_base + off, 16, 1024),
-                   C::IDESC_QK, kk > 0, C::ES == 4);
-          }
-          mma_commit(k_empty + s);
-          mma_commit(s_full + sb);
+        for (int kk = 0; kk < D / C::UK; ++kk) {
+          const int ke = kk * C::UK;
+          const uint32_t off = (ke / C::AW) * C::BLK + (ke % C::AW) * C::ES;
+          mma_ss(tmem + b * 128, smem_desc_sw128(qb + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024),
+                 C::IDESC_QK, kk > 0, C::ES == 4);
         }
-        if (j >= 1) {
-          const int jj = j - 1;
-          const int s = jj % STAGES;
-          if (!mbar_wait(v_full + s, (jj / STAGES) & 1, status, kDevTimeoutVFull)) break;
-          if (!mbar_wait(p_full, jj & 1, status, kDevTimeoutPFull)) break;
-          tc_fence_after();
-          const uint32_t v_base = smem_addr(sV + s * C::KV_BYTES);
+      };
+      auto issue_pv = [&](int b, int s, bool acc) {
+        const uint32_t vb = smem_addr(sV + s * C::KV_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < 128 / C::UK; ++kk) {
-            const int ke = kk * C::UK;
-            const uint32_t poff = (ke / C::AW) * C::BLK + (ke % C::AW) * C::ES;
-            // V is the MN-major operand: 16-bit types use the 16-byte-chunk swizzle (8-row atoms),
-            // tf32 the 32-byte-chunk swizzle (4-row atoms), matching how the V tensor map loads it
-            const uint64_t vdesc = C::ES == 4 ? smem_desc(v_base + ke * 128, C::BLK, 512, 1)
-                                              : smem_desc(v_base + ke * 128, C::BLK, 1024, 2);
-            mma_ss(tmem + C::O_COL, smem_desc_sw128(p_base + poff, 16, 1024), vdesc, C::IDESC_PV,
-                   (jj > 0 || kk > 0) ? 1u : 0u, C::ES == 4);
+        for (int kk = 0; kk < 128 / C::UK; ++kk) {
+          const int ke = kk * C::UK;
+          // V is the MN-major operand: 16-bit types use the 16-byte-chunk swizzle (8-row atoms),
+          // tf32 the 32-byte-chunk swizzle (4-row atoms), matching how the V tensor map loads it
+          const uint64_t vdesc = C::ES == 4 ? smem_desc(vb + ke * 128, C::BLK, 512, 1)
+                                            : smem_desc(vb + ke * 128, C::BLK, 1024, 2);
+          // P_b in TMEM over S_b: 8 columns per K step (two 16-bit values per column, or 8 tf32)
+          mma_ts(tmem + 256 + b * D, tmem + b * 128 + kk * 8, vdesc, C::IDESC_PV, (acc || kk > 0) ? 1u : 0u,
+                 C::ES == 4);
+        }
+      };
+      bool ok = mbar_wait(q_full, 0, status, kDevTimeoutQ) && mbar_wait(k_full, 0, status, kDevTimeoutKFull);
+      if (ok) {
+        tc_fence_after();
+        for (int b = 0; b < nb; ++b) {
+          issue_qk(b, 0);
+          mma_commit(s_full + b);
+        }
+        mma_commit(k_empty);
+      }
+      for (int j = 0; j < nmax && ok; ++j) {
+        const int s = j & 1;
+        bool v_ready = false;
+        for (int b = 0; b < nb && ok; ++b) {
+          const int nbt = b == 0 ? n0 : n1;
+          if (j >= nbt) continue;
+          if (!mbar_wait(p_full + b, j & 1, status, kDevTimeoutPFull)) {
+            ok = false;
+            break;
           }
-          mma_commit(v_empty + s);
-          mma_commit(o_done);
+          if (!v_ready && !mbar_wait(v_full + s, (j >> 1) & 1, status, kDevTimeoutVFull)) {
+            ok = false;
+            break;
+          }
+          v_ready = true;
+          tc_fence_after();
+          issue_pv(b, s, j > 0);
+          mma_commit(pv_done + b);
+          const bool last_pv = (b == nb - 1) || (j >= n1);
+          if (last_pv) mma_commit(v_empty + s);
+          if (j == nbt - 1) {
+            mma_commit(o_done + b);
+            continue;
+          }
+          // next key tile for this block; S_b / P_b are reused once P_b(j) * V has completed
+          const int j1 = j + 1;
+          const int s1 = j1 & 1;
+          const bool first_qk = (b == 0) || (j1 >= n0);
+          if (first_qk && !mbar_wait(k_full + s1, (j1 >> 1) & 1, status, kDevTimeoutKFull)) {
+            ok = false;
+            break;
+          }
+          if (!mbar_wait(pv_done + b, j & 1, status, kDevTimeoutODone)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_qk(b, s1);
+          mma_commit(s_full + b);
+          const bool last_qk = (b == nb - 1) || (j1 >= n1);
+          if (last_qk) mma_commit(k_empty + s1);
         }
       }
       // all tensor-core work this thread issued has finished before TMEM is released
@@ -250,53 +295,67 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(fin, 0, status, kDevTimeoutFinal);
     }
     __syncwarp();
-  } else {
-    // ------------------------------------------------------------ softmax / epilogue
-    const int r = threadIdx.x;  // query row in the tile == TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const int qi = u.q0 + r;
+  }
+  } else if ((warp >> 2) < nb) {
+    // ------------------------------------------------------------ softmax / epilogue of block b
+    regs_increase<216>();
+    const int b = warp >> 2;
+    const int r = threadIdx.x & 127;  // query row in the block == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_col = tmem + lane_base + b * 128;
+    const uint32_t o_col = tmem + lane_base + 256 + b * D;
+    const int n = b == 0 ? n0 : n1;
+    const int head = u.head[b];
+    const int qi = u.q0[b] + r;
     const bool row_valid = qi < si.seq_len;
-    const int iabs = qi + (si.kv_len - si.seq_len);
+    const int off = si.kv_len - si.seq_len;
+    const int iabs = qi + off;
     const int mt = p.mask_type;
     const bool alibi = (mt == 3 || mt == 4 || mt == 5);
-    const float slope = alibi ? p.slopes[u.head] : 0.f;
+    const float slope = alibi ? p.slopes[head] : 0.f;
     const float slope_log2 = slope * kLog2e;
-    // last allowed key of this row (inclusive)
+    const float scale = p.scale_log2;
+    const bool raw_max = !alibi && scale > 0.f;  // max of the raw scores, scale folded into the exponent
     const int last_key = (mt == 0) ? si.kv_len - 1 : min(iabs, si.kv_len - 1);
-    float m_run = -INFINITY;
+    float* tbl = sTbl + warp * 2 * C::TBL_FLOATS;
+    const int iabs_w = u.q0[b] + (warp & 3) * 32 + off;  // iabs of the warp's first row
+    float m_run = -INFINITY;  // running max in log2 units (the one P is computed against)
     float l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
-      const int sb = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full + sb, (j >> 1) & 1, status, kDevTimeoutSFull));
+      const int j0 = j * 128;
+      float* t = tbl + (j & 1) * C::TBL_FLOATS;
+      if (mt == 4) {
+        // -slope*log2(e)*sqrt(distance) for distance = iabs_w + k - 127 - j0, k = lane - column + 127
+        for (int k = lane; k < C::TBL_FLOATS; k += 32) {
+          const float dist = static_cast<float>(iabs_w - j0 + k - 127);
+          t[k] = -slope_log2 * sqrtf(fmaxf(dist, 0.f));
+        }
+        __syncwarp();
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full + b, j & 1, status, kDevTimeoutSFull));
       if (!ok) break;
       tc_fence_after();
       float x[128];
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
         uint32_t regs[32];
-        tmem_ld32(tmem + lane_base + sb * 128 + c4 * 32, regs);
+        tmem_ld32(s_col + c4 * 32, regs);
         tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < 32; ++c) x[c4 * 32 + c] = __uint_as_float(regs[c]);
       }
-      tc_fence_before();
-      mbar_arrive(s_free + sb);
-
-      const int j0 = j * 128;
       const int lim = last_key - j0;  // columns c <= lim are allowed
-      const float scale = p.scale_log2;
       if (mt == 3 || mt == 5) {
         // right- and left-aligned bias differ by a per-row constant; both use (j - iabs)
         const float b0 = slope_log2 * static_cast<float>(j0 - iabs);
 #pragma unroll
         for (int c = 0; c < 128; ++c) x[c] = fmaf(x[c], scale, fmaf(slope_log2, static_cast<float>(c), b0));
       } else if (mt == 4) {
-        const float d0 = static_cast<float>(iabs - j0);
+        const float* tl = t + lane + 127;
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          x[c] = fmaf(x[c], scale, -slope_log2 * sqrtf(fmaxf(d0 - static_cast<float>(c), 0.f)));
-      } else {
+        for (int c = 0; c < 128; ++c) x[c] = fmaf(x[c], scale, tl[-c]);
+      } else if (!raw_max) {
 #pragma unroll
         for (int c = 0; c < 128; ++c) x[c] *= scale;
       }
@@ -312,7 +371,8 @@ __global__ void __launch_bounds__(192, 1)
         mx2 = fmaxf(mx2, x[c + 2]);
         mx3 = fmaxf(mx3, x[c + 3]);
       }
-      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+      float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+      if (raw_max) mx *= scale;
       const float m_new = fmaxf(m_run, mx);
       float alpha = 1.f;
       if (m_new - m_run > kRescaleThreshold) {  // false while both are -inf
@@ -320,68 +380,72 @@ __global__ void __launch_bounds__(192, 1)
         m_run = m_new;
       }
       const float m_base = (m_run == -INFINITY) ? 0.f : m_run;
-      float sum0 = 0.f, sum1 = 0.f;
+      // O_b is quiescent here: P_b(j-1) * V completed before S_b(j) was written
+      if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        x[c] = fast_exp2(x[c] - m_base);
-        x[c + 1] = fast_exp2(x[c + 1] - m_base);
-        sum0 += x[c];
-        sum1 += x[c + 1];
-      }
-      l_run = l_run * alpha + (sum0 + sum1);
-
-      // O and the P buffer are owned by the previous P*V until it completes
-      if (j >= 1) {
-        ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, status, kDevTimeoutODone));
-        if (!ok) break;
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        for (int c32 = 0; c32 < D / 32; ++c32) {
+          uint32_t regs[32];
+          tmem_ld32(o_col + c32 * 32, regs);
+          tmem_ld_wait();
 #pragma unroll
-          for (int c32 = 0; c32 < D / 32; ++c32) {
-            uint32_t regs[32];
-            const uint32_t addr = tmem + lane_base + C::O_COL + c32 * 32;
-            tmem_ld32(addr, regs);
-            tmem_ld_wait();
-#pragma unroll
-            for (int c = 0; c < 32; ++c) regs[c] = __float_as_uint(__uint_as_float(regs[c]) * alpha);
-            tmem_st32(addr, regs);
-          }
-          tmem_st_wait();
+          for (int c = 0; c < 32; ++c) regs[c] = __float_as_uint(__uint_as_float(regs[c]) * alpha);
+          tmem_st32(o_col + c32 * 32, regs);
         }
       }
-      // P -> shared memory, K-major 128B-swizzled operand layout
+      float sum0 = 0.f, sum1 = 0.f;
       if constexpr (C::ES == 2) {
 #pragma unroll
-        for (int ch = 0; ch < 16; ++ch) {  // 16 chunks of 8 elements
-          uint4 v;
-          v.x = pack2(x[ch * 8 + 0], x[ch * 8 + 1], (T*)nullptr);
-          v.y = pack2(x[ch * 8 + 2], x[ch * 8 + 3], (T*)nullptr);
-          v.z = pack2(x[ch * 8 + 4], x[ch * 8 + 5], (T*)nullptr);
-          v.w = pack2(x[ch * 8 + 6], x[ch * 8 + 7], (T*)nullptr);
-          st_swizzled16(sP + (ch >> 3) * C::BLK, r, ch & 7, v);
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int c0 = h * 64 + 2 * c;
+            float e0, e1;
+            if (raw_max) {
+              e0 = fast_exp2(fmaf(x[c0], scale, -m_base));
+              e1 = fast_exp2(fmaf(x[c0 + 1], scale, -m_base));
+            } else {
+              e0 = fast_exp2(x[c0] - m_base);
+              e1 = fast_exp2(x[c0 + 1] - m_base);
+            }
+            sum0 += e0;
+            sum1 += e1;
+            pk[c] = pack2(e0, e1, (T*)nullptr);
+          }
+          tmem_st32(s_col + h * 32, pk);
         }
       } else {
 #pragma unroll
-        for (int ch = 0; ch < 32; ++ch) {  // 32 chunks of 4 fp32 (read as tf32)
-          uint4 v = make_uint4(__float_as_uint(x[ch * 4 + 0]), __float_as_uint(x[ch * 4 + 1]),
-                               __float_as_uint(x[ch * 4 + 2]), __float_as_uint(x[ch * 4 + 3]));
-          st_swizzled16(sP + (ch >> 3) * C::BLK, r, ch & 7, v);
+        for (int h = 0; h < 4; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float e =
+                raw_max ? fast_exp2(fmaf(x[h * 32 + c], scale, -m_base)) : fast_exp2(x[h * 32 + c] - m_base);
+            if (c & 1)
+              sum1 += e;
+            else
+              sum0 += e;
+            pk[c] = __float_as_uint(e);
+          }
+          tmem_st32(s_col + h * 32, pk);
         }
       }
-      fence_proxy_async_smem();
+      l_run = l_run * alpha + (sum0 + sum1);
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(p_full + b);
     }
 
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, (n - 1) & 1, status, kDevTimeoutODone));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done + b, 0, status, kDevTimeoutODone));
     if (ok) {
       tc_fence_after();
       const float inv_l = 1.f / l_run;
-      T* orow = reinterpret_cast<T*>(p.out) + ((size_t)(si.cu_q + qi) * p.heads + u.head) * D;
+      T* orow = reinterpret_cast<T*>(p.out) + ((size_t)(si.cu_q + qi) * p.heads + head) * D;
 #pragma unroll
       for (int c32 = 0; c32 < D / 32; ++c32) {
         uint32_t regs[32];
-        tmem_ld32(tmem + lane_base + C::O_COL + c32 * 32, regs);
+        tmem_ld32(o_col + c32 * 32, regs);
         tmem_ld_wait();
         if (row_valid) {
           if constexpr (C::ES == 2) {
@@ -411,30 +475,30 @@ __global__ void __launch_bounds__(192, 1)
       if (row_valid && p.lse) {
         float lse = (m_run == -INFINITY ? 0.f : m_run) * kLn2 + logf(l_run);
         if (mt == 5) lse += slope * static_cast<float>(iabs);  // left-aligned bias = right-aligned + slope*iabs
-        p.lse[(size_t)(si.cu_q + qi) * p.heads + u.head] = lse;
+        p.lse[(size_t)(si.cu_q + qi) * p.heads + head] = lse;
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
-template <typename T, int D, int STAGES>
+template <typename T, int D>
 cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const PrefillParams& p,
                    cudaStream_t stream) {
-  using C = Cfg<T, D, STAGES>;
+  using C = Cfg<T, D>;
   // at least 120 KB so a second CTA never shares the SM (each CTA allocates all 512 TMEM columns)
   constexpr int kSmem = C::SMEM > 120 * 1024 ? C::SMEM : 120 * 1024;
-  auto kern = prefill_kernel<T, D, STAGES>;
+  auto kern = prefill_kernel<T, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   if (p.n_units == 0) return cudaSuccess;
-  kern<<<p.n_units, 192, kSmem, stream>>>(tmQ, tmK, tmV, p);
+  kern<<<p.n_units, 384, kSmem, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }
 
@@ -442,10 +506,10 @@ cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtenso
 
 int prefill_smem_bytes(int32_t dtype, int32_t d) {
   if (dtype == kBF16 || dtype == kF16) {
-    if (d == 128) return Cfg<__half, 128, 2>::SMEM;
-    if (d == 64) return Cfg<__half, 64, 2>::SMEM;
+    if (d == 128) return Cfg<__half, 128>::SMEM;
+    if (d == 64) return Cfg<__half, 64>::SMEM;
   } else if (dtype == kF32) {
-    if (d == 64) return Cfg<float, 64, 1>::SMEM;
+    if (d == 64) return Cfg<float, 64>::SMEM;
   }
   return 0;
 }
@@ -453,13 +517,13 @@ int prefill_smem_bytes(int32_t dtype, int32_t d) {
 cudaError_t launch_prefill(int32_t dtype, int32_t d, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                            const CUtensorMap& tmV, const PrefillParams& p, cudaStream_t stream) {
   if (dtype == kBF16) {
-    if (d == 128) return launch<__nv_bfloat16, 128, 2>(tmQ, tmK, tmV, p, stream);
-    if (d == 64) return launch<__nv_bfloat16, 64, 2>(tmQ, tmK, tmV, p, stream);
+    if (d == 128) return launch<__nv_bfloat16, 128>(tmQ, tmK, tmV, p, stream);
+    if (d == 64) return launch<__nv_bfloat16, 64>(tmQ, tmK, tmV, p, stream);
   } else if (dtype == kF16) {
-    if (d == 128) return launch<__half, 128, 2>(tmQ, tmK, tmV, p, stream);
-    if (d == 64) return launch<__half, 64, 2>(tmQ, tmK, tmV, p, stream);
+    if (d == 128) return launch<__half, 128>(tmQ, tmK, tmV, p, stream);
+    if (d == 64) return launch<__half, 64>(tmQ, tmK, tmV, p, stream);
   } else if (dtype == kF32) {
-    if (d == 64) return launch<float, 64, 1>(tmQ, tmK, tmV, p, stream);
+    if (d == 64) return launch<float, 64>(tmQ, tmK, tmV, p, stream);
   }
   return cudaErrorInvalidValue;
 }
