@@ -175,7 +175,8 @@ ALA_API int varlen_attention(void* workspace, uint64_t workspaceSize, ala_op* op
  *
  * qNope       [tokens, headNum, 512] bf16/f16, device.
  * qRope       [tokens, headNum, 64], same dtype, device.
- * ctKV        [numBlocks, blockSize, kvHeadNum, 512], device (ND layout).
+ * ctKV        [numBlocks, blockSize, kvHeadNum, 512], device (ND layout);
+ *             blockSize a multiple of 16 dividing 64, or a multiple of 64.
  * kRope       [numBlocks, blockSize, kvHeadNum, 64], device.
  * blockTables [batch, maxBlocks] int32, device (entries read must be valid).
  * contextLens [batch] int32, HOST: keys per batch, including the new tokens.
@@ -190,6 +191,8 @@ ALA_API int varlen_attention(void* workspace, uint64_t workspaceSize, ala_op* op
  * cacheMode   KROPE_CTKV (1) only; others return UNSUPPORTED.
  * attenOut    [tokens, headNum, 512], dtype of qNope, device.
  * lse         NULL or [tokens, headNum, 1] fp32, device (natural log).
+ * workspace   256-byte aligned; holds the schedule and, for key ranges split
+ *             across CTAs, fp32 partial outputs merged by lse at the end.
  * ------------------------------------------------------------------------- */
 ALA_API int atb_like_mla_get_workspace_size(
     const ala_tensor* qNope, const ala_tensor* qRope, const ala_tensor* ctKV, const ala_tensor* kRope,

@@ -19,12 +19,17 @@ struct MlaPlan {
   float* lse = nullptr;
   const int32_t* block_tables = nullptr;
   std::vector<int32_t> ctx, qs;
-  // schedule and workspace
-  int32_t n_work = 0, n_splits_total = 0;
-  uint64_t ws_size = 0, off_work = 0, off_rows = 0, off_part_o = 0, off_part_lse = 0;
-  std::vector<uint8_t> image;
+  // schedule and workspace: [status | units | combine list | partial lse | partial O]
+  int32_t n_work = 0, n_splits_total = 0, n_combine = 0;
+  uint64_t ws_size = 0, off_work = 0, off_rows = 0, off_part_o = 0, off_part_lse = 0, image_size = 0;
+  std::vector<uint8_t> image;  // host copy of [status | units | combine list]
+  void* pinned = nullptr;      // page-locked copy of `image`, made on first run
   bool maps_ready = false;
   CUtensorMap tmQn, tmQr, tmKV, tmKR;
+  MlaPlan() = default;
+  MlaPlan(const MlaPlan&) = delete;
+  MlaPlan& operator=(const MlaPlan&) = delete;
+  ~MlaPlan();
 };
 
 int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, const ala_tensor* ctKV,
