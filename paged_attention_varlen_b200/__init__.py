@@ -72,6 +72,9 @@ def lib() -> ctypes.CDLL:
         L.atb_like_mla_get_workspace_size.argtypes = [T, T, T, T, T, T, T, T, T, T, ctypes.c_int32, ctypes.c_float,
                                                       ctypes.c_int32, ctypes.c_int, ctypes.c_int, ctypes.c_uint8, T, T,
                                                       U64P, OPP]
+        L.varlen_attention_noalloc.argtypes = [T, T, T, T, T, T, ctypes.c_int, ctypes.c_int32, ctypes.c_int32,
+                                               ctypes.c_float, T, T, P]
+        L.varlen_attention_noalloc.restype = ctypes.c_int
         for f in ("atb_like_prefix_encoder", "varlen_attention", "atb_like_mla"):
             getattr(L, f).argtypes = [P, ctypes.c_uint64, P, P]
         for f in ("ala_workspace_status", "atb_like_prefix_encoder_get_workspace_size",
@@ -170,6 +173,25 @@ def varlen_attention(q, k, v, seq_len, kv_seq_len, mask_type, heads, kv_heads, q
                                     lse=lse)
     op()
     return (out, lse) if return_lse else out
+
+
+def varlen_attention_noalloc(q, k, v, seq_len, kv_seq_len, mask_type, heads, kv_heads, qk_scale, slopes=None,
+                             out=None, lse=None, stream=None):
+    """varlen_attention through the entry point that allocates nothing on the device.
+
+    For callers that cannot allocate device memory: no workspace is passed; the
+    library's fixed device scratch holds the schedule.  ``out`` (and ``lse``)
+    must be supplied by the caller or are created here with torch.
+    """
+    L = lib()
+    out = torch.empty_like(q) if out is None else out
+    sl, kl = _host_i32(seq_len), _host_i32(kv_seq_len)
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    ts = [tensor(q), tensor(k), tensor(v), tensor(sl), tensor(kl), tensor(slopes)]
+    to, tl = tensor(out), tensor(lse)
+    _check(L.varlen_attention_noalloc(*[_ref(t) for t in ts], int(mask_type), int(heads), int(kv_heads),
+                                      float(qk_scale), _ref(to), _ref(tl), ctypes.c_void_p(s.cuda_stream)))
+    return out
 
 
 def plan_prefix_encoder(q, k, v, block_tables, seq_len, kv_seq_len, mask_type, heads, kv_heads, qk_scale,

@@ -149,6 +149,11 @@ struct ala_op {
 
 extern "C" const char* ala_last_error(void) { return g_last_error.c_str(); }
 
+namespace ala {
+// Lets other translation units of the library report through ala_last_error.
+void set_last_error(const char* msg) { g_last_error = msg; }
+}  // namespace ala
+
 extern "C" void ala_op_destroy(ala_op* op) { delete op; }
 
 extern "C" int ala_workspace_status(const ala_op* op, const void* workspace, ala_stream_t stream, int32_t* code) {
