@@ -46,7 +46,18 @@ if ROOT not in sys.path:
 import synth  # noqa: E402
 
 PROFILE = os.path.join(ROOT, "profiles", "prefill_varlen_causal_bf16.md")
+MLA_PROFILE = os.path.join(ROOT, "profiles", "mla_decode_qs1_bf16.md")
 KERNEL_SOURCES = ["paged_attention_varlen_b200/csrc/prefill.cu", "paged_attention_varlen_b200/csrc/ptx.cuh"]
+MLA_KERNEL_SOURCES = ["paged_attention_varlen_b200/csrc/mla.cu", "paged_attention_varlen_b200/csrc/ptx.cuh"]
+DEFAULT_WORKLOAD = "varlen_causal_bf16"
+WORKLOADS = {
+    "varlen_causal_bf16": lambda: synth.varlen_causal_bf16(),
+    "prefix_paged_alibi_fp16": lambda: synth.prefix_paged_alibi_fp16(),
+    "long_alibi_sqrt_bf16": lambda: synth.long_alibi_bf16(synth.MASK_ALIBI_SQRT),
+    "long_alibi_left_bf16": lambda: synth.long_alibi_bf16(synth.MASK_ALIBI_LEFT),
+    "mla_decode_qs1_bf16": lambda: synth.mla_decode_bf16(1),
+    "mla_spec_qs4_bf16": lambda: synth.mla_decode_bf16(4),
+}
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -250,11 +261,27 @@ def cpu_baseline(case, budget_s=12.0):
                       f"fp64 on the host (valid FLOPs of the sampled rows / time)"}
 
 
+def case_dtype(case):
+    return case.q_nope.dtype if isinstance(case, synth.MlaCase) else case.dtype
+
+
+def op_has_combine(op):
+    # the MLA workspace holds fp32 partials only when some key range was split (then a combine launch follows)
+    return op.workspace_size > 1 << 20
+
+
 def base_config(case):
+    l2 = "flushed before every step (256 MiB write, outside the step events)"
+    if isinstance(case, synth.MlaCase):
+        return {"workload": case.name, "global_batch": len(case.context_lens), "tokens": case.n_tokens,
+                "context_lens": "U[1024,16384] per batch", "heads": case.heads, "kv_lora": 512, "rope": 64,
+                "qseqlen": int(case.q_seq_len[0]), "block_size": case.block_size,
+                "parallelism": "replicas (independent batches)", "l2": l2}
+    mask = {0: "none", 3: "alibi right", 4: "alibi sqrt", 5: "alibi left", 9: "causal"}[case.mask_type]
     return {"workload": case.name, "global_batch": len(case.seq_len), "tokens": case.n_tokens,
-            "seq_len": "U[64,2048] per sequence", "heads": case.heads, "kv_heads": case.kv_heads,
-            "head_size": case.head_size, "mask": "causal", "parallelism": "replicas (independent sequences)",
-            "l2": "flushed before every step (256 MiB write, outside the step events)"}
+            "seq_len": "U[64,2048] per sequence" if case.name.startswith("varlen") else "see workload",
+            "heads": case.heads, "kv_heads": case.kv_heads, "head_size": case.head_size, "mask": mask,
+            "paged": case.paged, "parallelism": "replicas (independent sequences)", "l2": l2}
 
 
 def run_reference(args, rank, world):
@@ -286,6 +313,8 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS),
+                    help="workload of the timed steps (the default is the metric's prefill configuration)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -307,7 +336,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
     barrier = (lambda: dist.barrier()) if dist else (lambda: None)
 
-    case = synth.varlen_causal_bf16()
+    case = WORKLOADS[args.workload]()
+    is_mla = isinstance(case, synth.MlaCase)
     op, tens = plan_case(ala, case, device)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
@@ -319,24 +349,46 @@ def main():
         t = torch.tensor([ms], device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
-    flops = prefill_flops(case)
-    value = world * flops / (ms * 1e-3) / 1e12
+    flops = mla_flops(case) if is_mla else prefill_flops(case)
+    nbytes = mla_bytes(case) if is_mla else prefill_bytes(case)
+    if is_mla:
+        value = world * nbytes / (ms * 1e-3) / 1e9
+        metric, unit = "attention HBM GB/s (MLA decode)", "GB/s"
+    else:
+        value = world * flops / (ms * 1e-3) / 1e12
+        metric, unit = "attention TFLOPS on valid tokens (prefill)", "TFLOPS"
 
     if rank == 0:
         peaks = measured_peaks()
-        src = kernel_source_hash()
-        achieved = flops / (statistics.mean(times) * 1e-3) / 1e12
-        roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": achieved / peaks["bf16_tflops"], "traffic": profiled_traffic(PROFILE, src),
-                    "algorithmic_bytes": prefill_bytes(case), "peak_source": peaks["source"] + " (burst bf16)",
-                    "kernel": "prefill_kernel<bf16,128>", "kernel_source_sha256": src}
-        line = {"metric": "attention TFLOPS on valid tokens (prefill)", "value": value, "unit": "TFLOPS",
+        mean_ms = statistics.mean(times)
+        if is_mla:
+            src = kernel_source_hash(MLA_KERNEL_SOURCES)
+            achieved = nbytes / (mean_ms * 1e-3) / 1e9
+            roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": achieved / peaks["hbm_gbs"], "traffic": profiled_traffic(MLA_PROFILE, src),
+                        "algorithmic_bytes": nbytes, "peak_source": peaks["source"] + " (copy bandwidth)",
+                        "tflops": flops / (mean_ms * 1e-3) / 1e12, "kernel": "mla_kernel<bf16> + mla_combine_kernel",
+                        "kernel_source_sha256": src}
+            launches = args.steps * (2 if op_has_combine(op) else 1)
+        else:
+            src = kernel_source_hash()
+            achieved = flops / (mean_ms * 1e-3) / 1e12
+            roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                        "frac": achieved / peaks["bf16_tflops"], "traffic": profiled_traffic(PROFILE, src),
+                        "algorithmic_bytes": nbytes, "peak_source": peaks["source"] + " (burst bf16)",
+                        "kernel": "prefill_kernel", "kernel_source_sha256": src}
+            launches = args.steps
+        line = {"metric": metric, "value": value, "unit": unit,
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "fp16" if case_dtype(case) == torch.float16 else "bf16",
                 "data": "synthetic", "config": base_config(case), "roofline": roofline,
-                "clocks": clk.summary(), "gpu_launches": args.steps,
-                "valid_flops_per_step": flops, "padding_positions": int(len(case.seq_len) * case.seq_len.max()
-                                                                         - case.seq_len.sum())}
+                "clocks": clk.summary(), "gpu_launches": launches, "valid_flops_per_step": flops}
+        if not is_mla:
+            line["padding_positions"] = int(len(case.seq_len) * case.seq_len.max() - case.seq_len.sum())
+        args.no_e2e = args.no_e2e or is_mla
+        args.no_cpu = args.no_cpu or is_mla
+        args.no_extra = args.no_extra or args.workload != DEFAULT_WORKLOAD
         if not args.no_e2e:
             line["e2e"] = e2e_prefill(ala, case, tens, op, min(args.steps, 10), stream)
         if not args.no_extra:

@@ -41,6 +41,9 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
+#ifndef ALA_POLY_PAIRS_OF_4
+#define ALA_POLY_PAIRS_OF_4 0  // of every 4 column pairs, how many take the FMA-pipe exp2 polynomial
+#endif
 
 template <typename T>
 struct ElemFmt;
@@ -85,6 +88,54 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, __nv_bfloat16*) {
 __device__ __forceinline__ uint32_t pack2(float a, float b, __half*) {
   __half2 v = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// P = 2^(u) for one row's 128 scores, u = x*scale - m taken a pair of columns at a
+// time with packed f32x2 arithmetic; writes P over S in TMEM (16-bit pairs, or
+// fp32 for tf32) and returns the row sum.  MASKED zeroes the columns past `lim`
+// (boundary tiles only, so unmasked tiles carry no compare).  Of every four
+// column pairs, ALA_POLY_PAIRS_OF_4 take the FMA-pipe polynomial instead of MUFU.
+template <typename T, bool MASKED>
+__device__ __forceinline__ float exp_rows(const float (&x)[128], uint64_t scale2, uint64_t negm2, int lim,
+                                          uint32_t s_col) {
+  constexpr bool kHalf = sizeof(T) == 2;
+  constexpr int CHUNK = kHalf ? 64 : 32;  // columns per 32-register TMEM store
+  uint64_t acc[4] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f), f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
+#pragma unroll
+  for (int h = 0; h < 128 / CHUNK; ++h) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int cc = 0; cc < CHUNK / 2; ++cc) {
+      const int c0 = h * CHUNK + 2 * cc;
+      const uint64_t u = fma_x2(f2pack(x[c0], x[c0 + 1]), scale2, negm2);
+      float e0, e1;
+      if ((cc & 3) < ALA_POLY_PAIRS_OF_4) {
+        float u0, u1;
+        f2unpack(u, u0, u1);
+        f2unpack(exp2_poly_x2(f2pack(fmaxf(u0, -125.f), fmaxf(u1, -125.f))), e0, e1);
+      } else {
+        f2unpack(u, e0, e1);
+        e0 = fast_exp2(e0);
+        e1 = fast_exp2(e1);
+      }
+      if constexpr (MASKED) {  // exact zeros for masked keys (the polynomial does not reach 0)
+        e0 = (c0 > lim) ? 0.f : e0;
+        e1 = (c0 + 1 > lim) ? 0.f : e1;
+      }
+      acc[cc & 3] = add_x2(acc[cc & 3], f2pack(e0, e1));
+      if constexpr (kHalf) {
+        pk[cc] = pack2(e0, e1, (T*)nullptr);
+      } else {
+        pk[2 * cc] = __float_as_uint(e0);
+        pk[2 * cc + 1] = __float_as_uint(e1);
+      }
+    }
+    tmem_st32(s_col + h * 32, pk);
+  }
+  const uint64_t a = add_x2(add_x2(acc[0], acc[1]), add_x2(acc[2], acc[3]));
+  float s0, s1;
+  f2unpack(a, s0, s1);
+  return s0 + s1;
 }
 
 template <typename T, int D>
@@ -168,10 +219,10 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // register split: the softmax warpgroups take 216 per thread, warps 8..11 keep 56
-  // (256*216 + 128*56 = 62464 <= 384*168, the registers the block is launched with)
+  // register split: the softmax warpgroups take 216 per thread, warps 8..11 keep 64
+  // (256*216 + 128*64 = 63488 <= 384*168, the registers the block is launched with)
   if (warp >= 8) {
-    regs_decrease<56>();
+    regs_decrease<64>();
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -337,13 +388,13 @@ __global__ void __launch_bounds__(384, 1)
       if (!ok) break;
       tc_fence_after();
       float x[128];
+      {
+        uint32_t sr[4][32];
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        uint32_t regs[32];
-        tmem_ld32(s_col + c4 * 32, regs);
-        tmem_ld_wait();
+        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(s_col + c4 * 32, sr[c4]);
+        tmem_ld_wait();  // one wait for all four loads
 #pragma unroll
-        for (int c = 0; c < 32; ++c) x[c4 * 32 + c] = __uint_as_float(regs[c]);
+        for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c >> 5][c & 31]);
       }
       const int lim = last_key - j0;  // columns c <= lim are allowed
       if (mt == 3 || mt == 5) {
@@ -365,11 +416,11 @@ __global__ void __launch_bounds__(384, 1)
       }
       float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
 #pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, x[c]);
-        mx1 = fmaxf(mx1, x[c + 1]);
-        mx2 = fmaxf(mx2, x[c + 2]);
-        mx3 = fmaxf(mx3, x[c + 3]);
+      for (int c = 4; c < 128; c += 8) {
+        mx0 = max3(mx0, x[c], x[c + 1]);
+        mx1 = max3(mx1, x[c + 2], x[c + 3]);
+        mx2 = max3(mx2, x[c + 4], x[c + 5]);
+        mx3 = max3(mx3, x[c + 6], x[c + 7]);
       }
       float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
       if (raw_max) mx *= scale;
@@ -392,45 +443,13 @@ __global__ void __launch_bounds__(384, 1)
           tmem_st32(o_col + c32 * 32, regs);
         }
       }
-      float sum0 = 0.f, sum1 = 0.f;
-      if constexpr (C::ES == 2) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int c0 = h * 64 + 2 * c;
-            float e0, e1;
-            if (raw_max) {
-              e0 = fast_exp2(fmaf(x[c0], scale, -m_base));
-              e1 = fast_exp2(fmaf(x[c0 + 1], scale, -m_base));
-            } else {
-              e0 = fast_exp2(x[c0] - m_base);
-              e1 = fast_exp2(x[c0 + 1] - m_base);
-            }
-            sum0 += e0;
-            sum1 += e1;
-            pk[c] = pack2(e0, e1, (T*)nullptr);
-          }
-          tmem_st32(s_col + h * 32, pk);
-        }
-      } else {
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float e =
-                raw_max ? fast_exp2(fmaf(x[h * 32 + c], scale, -m_base)) : fast_exp2(x[h * 32 + c] - m_base);
-            if (c & 1)
-              sum1 += e;
-            else
-              sum0 += e;
-            pk[c] = __float_as_uint(e);
-          }
-          tmem_st32(s_col + h * 32, pk);
-        }
-      }
+      // P = 2^(x*scale - m) (raw scores) or 2^(x - m) (biased scores), written over S in TMEM
+      const uint64_t scale2 = f2pack(raw_max ? scale : 1.f, raw_max ? scale : 1.f);
+      const uint64_t negm2 = f2pack(-m_base, -m_base);
+      // warp-uniform choice: exp_rows issues tcgen05.st, which all 32 lanes must execute together
+      const float row_sum = __any_sync(0xffffffffu, lim < 127) ? exp_rows<T, true>(x, scale2, negm2, lim, s_col)
+                                                               : exp_rows<T, false>(x, scale2, negm2, lim, s_col);
+      const float sum0 = row_sum, sum1 = 0.f;
       l_run = l_run * alpha + (sum0 + sum1);
       tmem_st_wait();
       tc_fence_before();
@@ -442,11 +461,13 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       const float inv_l = 1.f / l_run;
       T* orow = reinterpret_cast<T*>(p.out) + ((size_t)(si.cu_q + qi) * p.heads + head) * D;
+      uint32_t orr[D / 32][32];
+#pragma unroll
+      for (int c32 = 0; c32 < D / 32; ++c32) tmem_ld32(o_col + c32 * 32, orr[c32]);
+      tmem_ld_wait();  // one wait for all loads of the row
 #pragma unroll
       for (int c32 = 0; c32 < D / 32; ++c32) {
-        uint32_t regs[32];
-        tmem_ld32(o_col + c32 * 32, regs);
-        tmem_ld_wait();
+        const uint32_t (&regs)[32] = orr[c32];
         if (row_valid) {
           if constexpr (C::ES == 2) {
 #pragma unroll

@@ -56,20 +56,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Same, but the thread is suspended by the hardware for up to `hint_ns` while
+// the phase is incomplete, so a waiting warp takes no issue slots from the
+// warps that share its scheduler.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed.  Returns false
 // (and records `code` in *status) if the limit passes first or another role
-// already reported an error.
+// already reported an error.  Each attempt sleeps up to 1 ms, so an error
+// another role reports is noticed within about a millisecond.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* status, int code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*status != 0) return false;
-      if (global_timer_ns() - t0 > ALA_WAIT_LIMIT_NS) {
-        atomicCAS((int*)status, 0, code);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+    if (*status != 0) return false;
+    if (global_timer_ns() - t0 > ALA_WAIT_LIMIT_NS) {
+      atomicCAS((int*)status, 0, code);
+      return false;
     }
   }
 }
@@ -252,6 +266,53 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// two fp32 values in one 64-bit register pair, for the packed f32x2 arithmetic of sm_100
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t fma_x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add_x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for two values on the FMA pipe instead of the MUFU unit.  x = n + f with
+// n = round(x) taken with the 1.5*2^23 shifter, f in [-1/2, 1/2]; 2^f from a
+// degree-3 minimax polynomial (relative error 7.5e-5 in float32, coefficients
+// from csrc/exp2_poly_fit.py); 2^n added into the exponent field.  Inputs must
+// be >= -125 (the caller clamps), so the result stays a normal float.
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
+  const uint64_t shifter = f2pack(12582912.f, 12582912.f);
+  const uint64_t neg_shifter = f2pack(-12582912.f, -12582912.f);
+  const uint64_t t = add_x2(x, shifter);
+  const uint64_t n = add_x2(t, neg_shifter);
+  const uint64_t f = fma_x2(n, f2pack(-1.f, -1.f), x);
+  uint64_t p = fma_x2(f2pack(5.517166853e-02f, 5.517166853e-02f), f, f2pack(2.426111251e-01f, 2.426111251e-01f));
+  p = fma_x2(p, f, f2pack(6.932609677e-01f, 6.932609677e-01f));
+  p = fma_x2(p, f, f2pack(9.999280572e-01f, 9.999280572e-01f));
+  float t0, t1, p0, p1;
+  f2unpack(t, t0, t1);
+  f2unpack(p, p0, p1);
+  p0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  p1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+  return f2pack(p0, p1);
 }
 
 }  // namespace ala
