@@ -12,7 +12,9 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <queue>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "../../include/ala.h"
@@ -41,6 +43,9 @@ int ok() {
 }
 
 constexpr uint64_t kAlign = 256;
+// SMs of the B200 the persistent prefill grid is planned for (one CTA per SM).  On a
+// part with another SM count the grid still runs correctly, with CTAs queued or SMs idle.
+constexpr size_t kPlannedSms = 148;
 uint64_t align_up(uint64_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 int elem_size(int32_t dtype) { return dtype == ALA_F32 || dtype == ALA_I32 ? 4 : 2; }
@@ -137,8 +142,8 @@ struct ala_op {
   const int32_t* block_tables = nullptr;
   const float* slopes = nullptr;
   float* lse = nullptr;
-  uint64_t off_seqs = 0, off_units = 0, ws_size = 0;
-  int32_t n_units = 0;
+  uint64_t off_seqs = 0, off_units = 0, off_ctas = 0, ws_size = 0;
+  int32_t n_units = 0, n_ctas = 0;
   std::vector<uint8_t> image;  // host copy of the workspace header (status, seqs, units)
   PinnedImage pinned;
   bool maps_ready = false;
@@ -355,17 +360,41 @@ int build_prefill(ala_op* op, const ala_tensor* query, const ala_tensor* key, co
     cq += sl[b];
     ckv += kl[b];
   }
-  // longest first, so the tail of the grid is made of short units
-  auto cost = [](const PrefillUnit& u) { return u.n_tiles[0] + u.n_tiles[1]; };
+  // Persistent grid: one CTA per SM, each running a list of units.  Units are
+  // assigned longest first to the least loaded CTA (greedy LPT); a unit costs
+  // its key tiles plus about one tile of fixed work (Q load, epilogue).
+  auto cost = [](const PrefillUnit& u) { return (int64_t)u.n_tiles[0] + u.n_tiles[1] + 1; };
   std::stable_sort(units.begin(), units.end(),
                    [&](const PrefillUnit& a, const PrefillUnit& b) { return cost(a) > cost(b); });
+  const int32_t n_ctas = (int32_t)std::min<size_t>(units.size(), kPlannedSms);
+  std::vector<std::vector<int32_t>> lists(std::max(n_ctas, 1));
+  {
+    std::priority_queue<std::pair<int64_t, int32_t>, std::vector<std::pair<int64_t, int32_t>>, std::greater<>> load;
+    for (int32_t c = 0; c < n_ctas; ++c) load.push({0, c});
+    for (size_t i = 0; i < units.size(); ++i) {
+      auto [l, c] = load.top();
+      load.pop();
+      lists[c].push_back((int32_t)i);
+      load.push({l + cost(units[i]), c});
+    }
+  }
+  std::vector<PrefillUnit> ordered;
+  std::vector<int32_t> offsets(n_ctas + 1, 0);
+  ordered.reserve(units.size());
+  for (int32_t c = 0; c < n_ctas; ++c) {
+    for (int32_t i : lists[c]) ordered.push_back(units[i]);
+    offsets[c + 1] = (int32_t)ordered.size();
+  }
   op->n_units = (int32_t)units.size();
+  op->n_ctas = n_ctas;
   op->off_seqs = kAlign;
   op->off_units = align_up(op->off_seqs + sizeof(SeqInfo) * std::max(batch, 1));
-  op->ws_size = align_up(op->off_units + sizeof(PrefillUnit) * std::max<size_t>(units.size(), 1));
+  op->off_ctas = align_up(op->off_units + sizeof(PrefillUnit) * std::max<size_t>(units.size(), 1));
+  op->ws_size = align_up(op->off_ctas + sizeof(int32_t) * (n_ctas + 1));
   op->image.assign(op->ws_size, 0);
   std::memcpy(op->image.data() + op->off_seqs, seqs.data(), sizeof(SeqInfo) * batch);
-  std::memcpy(op->image.data() + op->off_units, units.data(), sizeof(PrefillUnit) * units.size());
+  std::memcpy(op->image.data() + op->off_units, ordered.data(), sizeof(PrefillUnit) * ordered.size());
+  std::memcpy(op->image.data() + op->off_ctas, offsets.data(), sizeof(int32_t) * (n_ctas + 1));
   return ALA_OK;
 }
 
@@ -399,6 +428,8 @@ int run_prefill(void* workspace, uint64_t workspaceSize, ala_op* op, ala_stream_
   p.lse = op->lse;
   p.status = reinterpret_cast<int*>(ws);
   p.n_units = op->n_units;
+  p.cta_offsets = reinterpret_cast<const int32_t*>(ws + op->off_ctas);
+  p.n_ctas = op->n_ctas;
   p.max_blocks = op->max_blocks;
   p.block_size = op->block_size;
   p.oob_row = (int32_t)op->kv_rows;

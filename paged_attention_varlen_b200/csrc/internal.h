@@ -44,6 +44,7 @@ struct PrefillUnit {
 
 struct PrefillParams {
   const PrefillUnit* units;
+  const int32_t* cta_offsets;   // [n_ctas + 1]: CTA c runs units [off[c], off[c+1]); null: CTA c runs unit c
   const SeqInfo* seqs;
   const int32_t* block_tables;  // device [batch, max_blocks] or null (contiguous)
   const float* slopes;          // device [heads] or null
@@ -51,6 +52,7 @@ struct PrefillParams {
   float* lse;                   // [nTokens, heads] or null
   int* status;                  // device status word
   int32_t n_units;
+  int32_t n_ctas;               // grid size
   int32_t max_blocks;
   int32_t block_size;
   int32_t oob_row;              // a key row index past the cache (TMA fills zeros there)

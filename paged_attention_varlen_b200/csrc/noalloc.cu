@@ -260,7 +260,9 @@ extern "C" ALA_API int varlen_attention_noalloc(const ala_tensor* query, const a
   p.out = attnOut->data;
   p.lse = lse && lse->data ? static_cast<float*>(lse->data) : nullptr;
   p.status = reinterpret_cast<int*>(scratch);
+  p.cta_offsets = nullptr;  // one CTA per work unit
   p.n_units = (int32_t)nu;
+  p.n_ctas = (int32_t)nu;
   p.max_blocks = 0;
   p.block_size = 0;
   p.oob_row = (int32_t)key->dims[0];

@@ -71,7 +71,7 @@ struct Cfg {
   static constexpr int KV_BYTES = 128 * D * ES;
   static constexpr int TBL_FLOATS = 160;  // per-warp sqrt-bias table: lane - column + 127 in [0, 159)
   static constexpr int TBL_BYTES = 8 * 2 * TBL_FLOATS * 4;
-  static constexpr int N_BARS = 18;
+  static constexpr int N_BARS = 19;
   static constexpr int SMEM = 1024 + 2 * Q_BYTES + 2 * STAGES * KV_BYTES + TBL_BYTES + N_BARS * 8 + 16;
   static constexpr uint32_t IDESC_QK = instr_desc(ElemFmt<T>::fmt, false, false, 128, 128);
   static constexpr uint32_t IDESC_PV = instr_desc(ElemFmt<T>::fmt, false, true, 128, D);
@@ -183,20 +183,19 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* pv_done = bars + 13;  // [2] per block
   uint64_t* o_done = bars + 15;   // [2] per block
   uint64_t* fin = bars + 17;
+  uint64_t* q_empty = bars + 18;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::N_BARS);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const PrefillUnit u = p.units[blockIdx.x];
-  const SeqInfo si = p.seqs[u.b];
-  const int nb = u.n_blocks;
-  const int n0 = u.n_tiles[0];
-  const int n1 = nb > 1 ? u.n_tiles[1] : 0;
-  const int nmax = n0 > n1 ? n0 : n1;
+  // this CTA's work units: a host-balanced list (persistent grid), or unit blockIdx.x alone
+  const int u_begin = p.cta_offsets ? p.cta_offsets[blockIdx.x] : blockIdx.x;
+  const int u_end = p.cta_offsets ? p.cta_offsets[blockIdx.x + 1] : blockIdx.x + 1;
   int* status = p.status;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(k_full + s, 1);
       mbar_init(v_full + s, 1);
@@ -219,50 +218,69 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // register split: the softmax warpgroups take 216 per thread, warps 8..11 keep 64
-  // (256*216 + 128*64 = 63488 <= 384*168, the registers the block is launched with)
+  // Barrier phases run on across units: the K/V ring by a global tile counter, the
+  // per-block S/P/PV barriers by each block's tile counter, q_full / q_empty and
+  // o_done by unit counters.
+  //
+  // register split: the softmax warpgroups take 224 per thread, warps 8..11 keep 56
+  // (256*224 + 128*56 = 64512 = 384*168, all the registers the block is launched with)
   if (warp >= 8) {
-    regs_decrease<64>();
-  if (warp == 8) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    regs_decrease<56>();
+    if (warp == 8 && lane == 0) {
+      // ------------------------------------------------------------ producer
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      const int kvh = u.head[0] / p.group;
-      mbar_expect_tx(q_full, nb * C::Q_BYTES);
-      for (int b = 0; b < nb; ++b)
-        for (int cb = 0; cb < D / C::AW; ++cb)
-          tma_load_3d(sQ + b * C::Q_BYTES + cb * C::BLK, &tmQ, q_full, cb * C::AW, u.head[b], si.cu_q + u.q0[b]);
-      const int32_t* bt = p.block_tables ? p.block_tables + (size_t)u.b * p.max_blocks : nullptr;
-      const int n_pages = bt ? (si.kv_len + p.block_size - 1) / p.block_size : 0;
       bool ok = true;
-      int issued[2] = {0, 0};  // tiles whose K (0) / V (1) load was issued
-      for (int j = 0; j < nmax && ok; ++j) {
-        const int s = j & 1;
-        const uint32_t par = ((j >> 1) - 1) & 1;
-        for (int kv = 0; kv < 2; ++kv) {
-          if (j >= 2 && !mbar_wait((kv ? v_empty : k_empty) + s, par, status,
-                                   kv ? kDevTimeoutVEmpty : kDevTimeoutKEmpty)) {
-            ok = false;
-            break;
+      uint32_t kv_iter = 0;               // K/V tiles loaded so far (all units)
+      uint32_t issued[2] = {0, 0};        // K (0) / V (1) loads issued
+      int q_loads = 0;
+      for (int ui = u_begin; ui < u_end && ok; ++ui) {
+        const PrefillUnit u = p.units[ui];
+        const SeqInfo si = p.seqs[u.b];
+        const int nb = u.n_blocks;
+        const int nmax = (nb > 1 && u.n_tiles[1] > u.n_tiles[0]) ? u.n_tiles[1] : u.n_tiles[0];
+        const int kvh = u.head[0] / p.group;
+        const int32_t* bt = p.block_tables ? p.block_tables + (size_t)u.b * p.max_blocks : nullptr;
+        const int n_pages = bt ? (si.kv_len + p.block_size - 1) / p.block_size : 0;
+        for (int j = 0; j < nmax && ok; ++j) {
+          const uint32_t g = kv_iter + j;
+          const int s = g & 1;
+          for (int kv = 0; kv < 2; ++kv) {
+            if (g >= 2 && !mbar_wait((kv ? v_empty : k_empty) + s, ((g >> 1) - 1) & 1, status,
+                                     kv ? kDevTimeoutVEmpty : kDevTimeoutKEmpty)) {
+              ok = false;
+              break;
+            }
+            uint64_t* full = (kv ? v_full : k_full) + s;
+            mbar_expect_tx(full, C::KV_BYTES);
+            load_kv_tile<T, D>(kv ? &tmV : &tmK, (kv ? sV : sK) + s * C::KV_BYTES, full, j, si, p, bt, n_pages, kvh);
+            issued[kv] = g + 1;
           }
-          uint64_t* full = (kv ? v_full : k_full) + s;
-          mbar_expect_tx(full, C::KV_BYTES);
-          load_kv_tile<T, D>(kv ? &tmV : &tmK, (kv ? sV : sK) + s * C::KV_BYTES, full, j, si, p, bt, n_pages, kvh);
-          issued[kv] = j + 1;
+          if (j == 0 && ok) {
+            // Q after the first K/V tile, so both latencies overlap; the Q buffers are free
+            // once the previous unit's last QK has finished
+            if (q_loads > 0 && !mbar_wait(q_empty, (q_loads - 1) & 1, status, kDevTimeoutQ)) {
+              ok = false;
+              break;
+            }
+            mbar_expect_tx(q_full, nb * C::Q_BYTES);
+            for (int b = 0; b < nb; ++b)
+              for (int cb = 0; cb < D / C::AW; ++cb)
+                tma_load_3d(sQ + b * C::Q_BYTES + cb * C::BLK, &tmQ, q_full, cb * C::AW, u.head[b],
+                            si.cu_q + u.q0[b]);
+            ++q_loads;
+          }
         }
+        kv_iter += nmax;
       }
       // never leave the CTA while loads it issued are still landing in shared memory
       for (int kv = 0; kv < 2; ++kv)
-        for (int j = issued[kv] - 2 < 0 ? 0 : issued[kv] - 2; j < issued[kv]; ++j)
-          mbar_wait((kv ? v_full : k_full) + (j & 1), (j >> 1) & 1, status, kv ? kDevTimeoutVFull : kDevTimeoutKFull);
-      mbar_wait(q_full, 0, status, kDevTimeoutQ);
-    }
-    __syncwarp();
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+        for (uint32_t g = issued[kv] >= 2 ? issued[kv] - 2 : 0; g < issued[kv]; ++g)
+          mbar_wait((kv ? v_full : k_full) + (g & 1), (g >> 1) & 1, status, kv ? kDevTimeoutVFull : kDevTimeoutKFull);
+      if (q_loads > 0) mbar_wait(q_full, (q_loads - 1) & 1, status, kDevTimeoutQ);
+    } else if (warp == 9 && lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
       const uint32_t q_base = smem_addr(sQ);
       auto issue_qk = [&](int b, int s) {
         const uint32_t qb = q_base + b * C::Q_BYTES;
@@ -289,185 +307,219 @@ __global__ void __launch_bounds__(384, 1)
                  C::ES == 4);
         }
       };
-      bool ok = mbar_wait(q_full, 0, status, kDevTimeoutQ) && mbar_wait(k_full, 0, status, kDevTimeoutKFull);
-      if (ok) {
-        tc_fence_after();
+      bool ok = true;
+      uint32_t kv_iter = 0;
+      uint32_t sp[2] = {0, 0};  // tiles block 0 / 1 processed in earlier units
+      for (int ui = u_begin; ui < u_end && ok; ++ui) {
+        const int it = ui - u_begin;
+        const PrefillUnit u = p.units[ui];
+        const int nb = u.n_blocks;
+        const int n0 = u.n_tiles[0];
+        const int n1 = nb > 1 ? u.n_tiles[1] : 0;
+        const int nmax = n0 > n1 ? n0 : n1;
+        if (!mbar_wait(q_full, it & 1, status, kDevTimeoutQ) ||
+            !mbar_wait(k_full + (kv_iter & 1), (kv_iter >> 1) & 1, status, kDevTimeoutKFull)) {
+          ok = false;
+          break;
+        }
         for (int b = 0; b < nb; ++b) {
-          issue_qk(b, 0);
-          mma_commit(s_full + b);
-        }
-        mma_commit(k_empty);
-      }
-      for (int j = 0; j < nmax && ok; ++j) {
-        const int s = j & 1;
-        bool v_ready = false;
-        for (int b = 0; b < nb && ok; ++b) {
-          const int nbt = b == 0 ? n0 : n1;
-          if (j >= nbt) continue;
-          if (!mbar_wait(p_full + b, j & 1, status, kDevTimeoutPFull)) {
-            ok = false;
-            break;
-          }
-          if (!v_ready && !mbar_wait(v_full + s, (j >> 1) & 1, status, kDevTimeoutVFull)) {
-            ok = false;
-            break;
-          }
-          v_ready = true;
-          tc_fence_after();
-          issue_pv(b, s, j > 0);
-          mma_commit(pv_done + b);
-          const bool last_pv = (b == nb - 1) || (j >= n1);
-          if (last_pv) mma_commit(v_empty + s);
-          if (j == nbt - 1) {
-            mma_commit(o_done + b);
-            continue;
-          }
-          // next key tile for this block; S_b / P_b are reused once P_b(j) * V has completed
-          const int j1 = j + 1;
-          const int s1 = j1 & 1;
-          const bool first_qk = (b == 0) || (j1 >= n0);
-          if (first_qk && !mbar_wait(k_full + s1, (j1 >> 1) & 1, status, kDevTimeoutKFull)) {
-            ok = false;
-            break;
-          }
-          if (!mbar_wait(pv_done + b, j & 1, status, kDevTimeoutODone)) {
+          // S_b / P_b are free once the previous unit's last P_b * V has completed
+          if (sp[b] > 0 && !mbar_wait(pv_done + b, (sp[b] - 1) & 1, status, kDevTimeoutODone)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          issue_qk(b, s1);
+          issue_qk(b, kv_iter & 1);
           mma_commit(s_full + b);
-          const bool last_qk = (b == nb - 1) || (j1 >= n1);
-          if (last_qk) mma_commit(k_empty + s1);
         }
+        if (!ok) break;
+        mma_commit(k_empty + (kv_iter & 1));
+        if (nmax == 1) mma_commit(q_empty);
+        for (int j = 0; j < nmax && ok; ++j) {
+          const uint32_t g = kv_iter + j;
+          const int s = g & 1;
+          bool v_ready = false;
+          for (int b = 0; b < nb && ok; ++b) {
+            const int nbt = b == 0 ? n0 : n1;
+            if (j >= nbt) continue;
+            const uint32_t ph = sp[b] + j;  // this block's barrier phase for tile j
+            if (!mbar_wait(p_full + b, ph & 1, status, kDevTimeoutPFull)) {
+              ok = false;
+              break;
+            }
+            if (!v_ready && !mbar_wait(v_full + s, (g >> 1) & 1, status, kDevTimeoutVFull)) {
+              ok = false;
+              break;
+            }
+            v_ready = true;
+            tc_fence_after();
+            issue_pv(b, s, j > 0);
+            mma_commit(pv_done + b);
+            const bool last_pv = (b == nb - 1) || (j >= n1);
+            if (last_pv) mma_commit(v_empty + s);
+            if (j == nbt - 1) {
+              mma_commit(o_done + b);
+              continue;
+            }
+            // next key tile for this block; S_b / P_b are reused once P_b(j) * V has completed
+            const uint32_t g1 = g + 1;
+            const int s1 = g1 & 1;
+            const bool first_qk = (b == 0) || (j + 1 >= n0);
+            if (first_qk && !mbar_wait(k_full + s1, (g1 >> 1) & 1, status, kDevTimeoutKFull)) {
+              ok = false;
+              break;
+            }
+            if (!mbar_wait(pv_done + b, ph & 1, status, kDevTimeoutODone)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_qk(b, s1);
+            mma_commit(s_full + b);
+            const bool last_qk = (b == nb - 1) || (j + 1 >= n1);
+            if (last_qk) {
+              mma_commit(k_empty + s1);
+              if (j + 1 == nmax - 1) mma_commit(q_empty);  // the unit's last QK: Q buffers free
+            }
+          }
+        }
+        sp[0] += n0;
+        sp[1] += n1;
+        kv_iter += nmax;
       }
       // all tensor-core work this thread issued has finished before TMEM is released
       mma_commit(fin);
       mbar_wait(fin, 0, status, kDevTimeoutFinal);
     }
     __syncwarp();
-  }
-  } else if ((warp >> 2) < nb) {
+  } else {
     // ------------------------------------------------------------ softmax / epilogue of block b
-    regs_increase<216>();
+    regs_increase<224>();
     const int b = warp >> 2;
     const int r = threadIdx.x & 127;  // query row in the block == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t s_col = tmem + lane_base + b * 128;
     const uint32_t o_col = tmem + lane_base + 256 + b * D;
-    const int n = b == 0 ? n0 : n1;
-    const int head = u.head[b];
-    const int qi = u.q0[b] + r;
-    const bool row_valid = qi < si.seq_len;
-    const int off = si.kv_len - si.seq_len;
-    const int iabs = qi + off;
     const int mt = p.mask_type;
     const bool alibi = (mt == 3 || mt == 4 || mt == 5);
-    const float slope = alibi ? p.slopes[head] : 0.f;
-    const float slope_log2 = slope * kLog2e;
     const float scale = p.scale_log2;
     const bool raw_max = !alibi && scale > 0.f;  // max of the raw scores, scale folded into the exponent
-    const int last_key = (mt == 0) ? si.kv_len - 1 : min(iabs, si.kv_len - 1);
     float* tbl = sTbl + warp * 2 * C::TBL_FLOATS;
-    const int iabs_w = u.q0[b] + (warp & 3) * 32 + off;  // iabs of the warp's first row
-    float m_run = -INFINITY;  // running max in log2 units (the one P is computed against)
-    float l_run = 0.f;
+    uint32_t sp = 0;  // tiles this block processed in earlier units (barrier phases)
+    uint32_t up = 0;  // units this block took part in (o_done phases)
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      const int j0 = j * 128;
-      float* t = tbl + (j & 1) * C::TBL_FLOATS;
-      if (mt == 4) {
-        // -slope*log2(e)*sqrt(distance) for distance = iabs_w + k - 127 - j0, k = lane - column + 127
-        for (int k = lane; k < C::TBL_FLOATS; k += 32) {
-          const float dist = static_cast<float>(iabs_w - j0 + k - 127);
-          t[k] = -slope_log2 * sqrtf(fmaxf(dist, 0.f));
+    for (int ui = u_begin; ui < u_end && ok; ++ui) {
+      const PrefillUnit u = p.units[ui];
+      if (b >= u.n_blocks) continue;
+      const SeqInfo si = p.seqs[u.b];
+      const int n = u.n_tiles[b];
+      const int head = u.head[b];
+      const int qi = u.q0[b] + r;
+      const bool row_valid = qi < si.seq_len;
+      const int off = si.kv_len - si.seq_len;
+      const int iabs = qi + off;
+      const float slope = alibi ? p.slopes[head] : 0.f;
+      const float slope_log2 = slope * kLog2e;
+      const int last_key = (mt == 0) ? si.kv_len - 1 : min(iabs, si.kv_len - 1);
+      const int iabs_w = u.q0[b] + (warp & 3) * 32 + off;  // iabs of the warp's first row
+      float m_run = -INFINITY;  // running max in log2 units (the one P is computed against)
+      float l_run = 0.f;
+      for (int j = 0; j < n; ++j) {
+        const uint32_t ph = sp + j;
+        const int j0 = j * 128;
+        float* t = tbl + (ph & 1) * C::TBL_FLOATS;
+        if (mt == 4) {
+          // -slope*log2(e)*sqrt(distance) for distance = iabs_w + k - 127 - j0, k = lane - column + 127
+          for (int k = lane; k < C::TBL_FLOATS; k += 32) {
+            const float dist = static_cast<float>(iabs_w - j0 + k - 127);
+            t[k] = -slope_log2 * sqrtf(fmaxf(dist, 0.f));
+          }
+          __syncwarp();
         }
-        __syncwarp();
+        ok = __all_sync(0xffffffffu, mbar_wait(s_full + b, ph & 1, status, kDevTimeoutSFull));
+        if (!ok) break;
+        tc_fence_after();
+        float x[128];
+        {
+          uint32_t sr[4][32];
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(s_col + c4 * 32, sr[c4]);
+          tmem_ld_wait();  // one wait for all four loads
+#pragma unroll
+          for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c >> 5][c & 31]);
+        }
+        const int lim = last_key - j0;  // columns c <= lim are allowed
+        if (mt == 3 || mt == 5) {
+          // right- and left-aligned bias differ by a per-row constant; both use (j - iabs)
+          const float b0 = slope_log2 * static_cast<float>(j0 - iabs);
+#pragma unroll
+          for (int c = 0; c < 128; ++c) x[c] = fmaf(x[c], scale, fmaf(slope_log2, static_cast<float>(c), b0));
+        } else if (mt == 4) {
+          const float* tl = t + lane + 127;
+#pragma unroll
+          for (int c = 0; c < 128; ++c) x[c] = fmaf(x[c], scale, tl[-c]);
+        } else if (!raw_max) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) x[c] *= scale;
+        }
+        if (lim < 127) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) x[c] = (c > lim) ? -INFINITY : x[c];
+        }
+        float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
+#pragma unroll
+        for (int c = 4; c < 128; c += 8) {
+          mx0 = max3(mx0, x[c], x[c + 1]);
+          mx1 = max3(mx1, x[c + 2], x[c + 3]);
+          mx2 = max3(mx2, x[c + 4], x[c + 5]);
+          mx3 = max3(mx3, x[c + 6], x[c + 7]);
+        }
+        float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        if (raw_max) mx *= scale;
+        const float m_new = fmaxf(m_run, mx);
+        float alpha = 1.f;
+        if (m_new - m_run > kRescaleThreshold) {  // false while both are -inf
+          alpha = fast_exp2(m_run - m_new);
+          m_run = m_new;
+        }
+        const float m_base = (m_run == -INFINITY) ? 0.f : m_run;
+        // O_b is quiescent here: P_b(j-1) * V completed before S_b(j) was written
+        if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int c32 = 0; c32 < D / 32; ++c32) {
+            uint32_t regs[32];
+            tmem_ld32(o_col + c32 * 32, regs);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) regs[c] = __float_as_uint(__uint_as_float(regs[c]) * alpha);
+            tmem_st32(o_col + c32 * 32, regs);
+          }
+        }
+        // P = 2^(x*scale - m) (raw scores) or 2^(x - m) (biased scores), written over S in TMEM
+        const uint64_t scale2 = f2pack(raw_max ? scale : 1.f, raw_max ? scale : 1.f);
+        const uint64_t negm2 = f2pack(-m_base, -m_base);
+        // warp-uniform choice: exp_rows issues tcgen05.st, which all 32 lanes must execute together
+        const float row_sum = __any_sync(0xffffffffu, lim < 127) ? exp_rows<T, true>(x, scale2, negm2, lim, s_col)
+                                                                 : exp_rows<T, false>(x, scale2, negm2, lim, s_col);
+        l_run = l_run * alpha + row_sum;
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(p_full + b);
       }
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full + b, j & 1, status, kDevTimeoutSFull));
+      sp += n;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done + b, up & 1, status, kDevTimeoutODone));
+      ++up;
       if (!ok) break;
-      tc_fence_after();
-      float x[128];
-      {
-        uint32_t sr[4][32];
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(s_col + c4 * 32, sr[c4]);
-        tmem_ld_wait();  // one wait for all four loads
-#pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c >> 5][c & 31]);
-      }
-      const int lim = last_key - j0;  // columns c <= lim are allowed
-      if (mt == 3 || mt == 5) {
-        // right- and left-aligned bias differ by a per-row constant; both use (j - iabs)
-        const float b0 = slope_log2 * static_cast<float>(j0 - iabs);
-#pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] = fmaf(x[c], scale, fmaf(slope_log2, static_cast<float>(c), b0));
-      } else if (mt == 4) {
-        const float* tl = t + lane + 127;
-#pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] = fmaf(x[c], scale, tl[-c]);
-      } else if (!raw_max) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] *= scale;
-      }
-      if (lim < 127) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] = (c > lim) ? -INFINITY : x[c];
-      }
-      float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
-#pragma unroll
-      for (int c = 4; c < 128; c += 8) {
-        mx0 = max3(mx0, x[c], x[c + 1]);
-        mx1 = max3(mx1, x[c + 2], x[c + 3]);
-        mx2 = max3(mx2, x[c + 4], x[c + 5]);
-        mx3 = max3(mx3, x[c + 6], x[c + 7]);
-      }
-      float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-      if (raw_max) mx *= scale;
-      const float m_new = fmaxf(m_run, mx);
-      float alpha = 1.f;
-      if (m_new - m_run > kRescaleThreshold) {  // false while both are -inf
-        alpha = fast_exp2(m_run - m_new);
-        m_run = m_new;
-      }
-      const float m_base = (m_run == -INFINITY) ? 0.f : m_run;
-      // O_b is quiescent here: P_b(j-1) * V completed before S_b(j) was written
-      if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-        for (int c32 = 0; c32 < D / 32; ++c32) {
-          uint32_t regs[32];
-          tmem_ld32(o_col + c32 * 32, regs);
-          tmem_ld_wait();
-#pragma unroll
-          for (int c = 0; c < 32; ++c) regs[c] = __float_as_uint(__uint_as_float(regs[c]) * alpha);
-          tmem_st32(o_col + c32 * 32, regs);
-        }
-      }
-      // P = 2^(x*scale - m) (raw scores) or 2^(x - m) (biased scores), written over S in TMEM
-      const uint64_t scale2 = f2pack(raw_max ? scale : 1.f, raw_max ? scale : 1.f);
-      const uint64_t negm2 = f2pack(-m_base, -m_base);
-      // warp-uniform choice: exp_rows issues tcgen05.st, which all 32 lanes must execute together
-      const float row_sum = __any_sync(0xffffffffu, lim < 127) ? exp_rows<T, true>(x, scale2, negm2, lim, s_col)
-                                                               : exp_rows<T, false>(x, scale2, negm2, lim, s_col);
-      const float sum0 = row_sum, sum1 = 0.f;
-      l_run = l_run * alpha + (sum0 + sum1);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(p_full + b);
-    }
-
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done + b, 0, status, kDevTimeoutODone));
-    if (ok) {
       tc_fence_after();
       const float inv_l = 1.f / l_run;
       T* orow = reinterpret_cast<T*>(p.out) + ((size_t)(si.cu_q + qi) * p.heads + head) * D;
       uint32_t orr[D / 32][32];
 #pragma unroll
       for (int c32 = 0; c32 < D / 32; ++c32) tmem_ld32(o_col + c32 * 32, orr[c32]);
-      tmem_ld_wait();  // one wait for all loads of the row
+      tmem_ld_wait();  // one wait for all loads of the row; the next unit's P_b * V may then overwrite O_b
 #pragma unroll
       for (int c32 = 0; c32 < D / 32; ++c32) {
-        const uint32_t (&regs)[32] = orr[c32];
+        const uint32_t(&regs)[32] = orr[c32];
         if (row_valid) {
           if constexpr (C::ES == 2) {
 #pragma unroll
@@ -518,8 +570,8 @@ cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtenso
   auto kern = prefill_kernel<T, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
-  if (p.n_units == 0) return cudaSuccess;
-  kern<<<p.n_units, 384, kSmem, stream>>>(tmQ, tmK, tmV, p);
+  if (p.n_ctas == 0) return cudaSuccess;
+  kern<<<p.n_ctas, 384, kSmem, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }
 
