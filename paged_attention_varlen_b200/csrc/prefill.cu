@@ -141,7 +141,7 @@ __device__ __forceinline__ float exp_rows(const float (&x)[128], uint64_t scale2
 template <typename T, int D>
 __device__ __forceinline__ void load_kv_tile(const CUtensorMap* map, uint8_t* dst, uint64_t* full, int j,
                                              const SeqInfo& si, const PrefillParams& p, const int32_t* bt,
-                                             int n_pages, int kvh) {
+                                             int n_pages, int kvh, bool leader) {
   using C = Cfg<T, D>;
   const bool paged = bt != nullptr;
   const int bs = p.block_size;
@@ -156,8 +156,10 @@ __device__ __forceinline__ void load_kv_tile(const CUtensorMap* map, uint8_t* ds
       const int pg = pos / bs;
       row = pg < n_pages ? bt[pg] * bs + (pos % bs) : p.oob_row;  // past the last page: zero fill
     }
+    if (leader) {
 #pragma unroll
-    for (int cb = 0; cb < D / C::AW; ++cb) tma_load_3d(dst + cb * C::BLK + r0 * 128, map, full, cb * C::AW, kvh, row);
+      for (int cb = 0; cb < D / C::AW; ++cb) tma_load_3d(dst + cb * C::BLK + r0 * 128, map, full, cb * C::AW, kvh, row);
+    }
   }
 }
 
@@ -222,18 +224,22 @@ __global__ void __launch_bounds__(384, 1)
   // per-block S/P/PV barriers by each block's tile counter, q_full / q_empty and
   // o_done by unit counters.
   //
-  // register split: the softmax warpgroups take 224 per thread, warps 8..11 keep 56
-  // (256*224 + 128*56 = 64512 = 384*168, all the registers the block is launched with)
+  // register split: the softmax warpgroups take 216 per thread, warps 8..11 keep 72
+  // (256*216 + 128*72 = 64512 = 384*168, all the registers the block is launched with)
   if (warp >= 8) {
-    regs_decrease<56>();
-    if (warp == 8 && lane == 0) {
+    regs_decrease<72>();
+    if (warp == 8) {
       // ------------------------------------------------------------ producer
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
+      // the whole warp walks the schedule (warp-uniform values); one elected lane issues the copies
+      const bool leader = elect_one();
+      if (leader) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+      }
       bool ok = true;
       uint32_t kv_iter = 0;               // K/V tiles loaded so far (all units)
-      uint32_t issued[2] = {0, 0};        // K (0) / V (1) loads issued
+      uint32_t issued_k = 0, issued_v = 0;  // K / V loads issued
       int q_loads = 0;
       for (int ui = u_begin; ui < u_end && ok; ++ui) {
         const PrefillUnit u = p.units[ui];
@@ -247,69 +253,88 @@ __global__ void __launch_bounds__(384, 1)
           const uint32_t g = kv_iter + j;
           const int s = g & 1;
           for (int kv = 0; kv < 2; ++kv) {
-            if (g >= 2 && !mbar_wait((kv ? v_empty : k_empty) + s, ((g >> 1) - 1) & 1, status,
-                                     kv ? kDevTimeoutVEmpty : kDevTimeoutKEmpty)) {
+            if (g >= 2 && !__all_sync(0xffffffffu, mbar_wait((kv ? v_empty : k_empty) + s, ((g >> 1) - 1) & 1, status,
+                                                              kv ? kDevTimeoutVEmpty : kDevTimeoutKEmpty))) {
               ok = false;
               break;
             }
             uint64_t* full = (kv ? v_full : k_full) + s;
-            mbar_expect_tx(full, C::KV_BYTES);
-            load_kv_tile<T, D>(kv ? &tmV : &tmK, (kv ? sV : sK) + s * C::KV_BYTES, full, j, si, p, bt, n_pages, kvh);
-            issued[kv] = g + 1;
+            if (leader) mbar_expect_tx(full, C::KV_BYTES);
+            load_kv_tile<T, D>(kv ? &tmV : &tmK, (kv ? sV : sK) + s * C::KV_BYTES, full, j, si, p, bt, n_pages, kvh,
+                               leader);
+            if (kv) issued_v = g + 1; else issued_k = g + 1;
           }
           if (j == 0 && ok) {
             // Q after the first K/V tile, so both latencies overlap; the Q buffers are free
             // once the previous unit's last QK has finished
-            if (q_loads > 0 && !mbar_wait(q_empty, (q_loads - 1) & 1, status, kDevTimeoutQ)) {
+            if (q_loads > 0 && !__all_sync(0xffffffffu, mbar_wait(q_empty, (q_loads - 1) & 1, status, kDevTimeoutQ))) {
               ok = false;
               break;
             }
-            mbar_expect_tx(q_full, nb * C::Q_BYTES);
-            for (int b = 0; b < nb; ++b)
-              for (int cb = 0; cb < D / C::AW; ++cb)
-                tma_load_3d(sQ + b * C::Q_BYTES + cb * C::BLK, &tmQ, q_full, cb * C::AW, u.head[b],
-                            si.cu_q + u.q0[b]);
+            if (leader) {
+              mbar_expect_tx(q_full, nb * C::Q_BYTES);
+#pragma unroll
+              for (int b = 0; b < 2; ++b) {
+                if (b >= nb) break;
+#pragma unroll
+                for (int cb = 0; cb < D / C::AW; ++cb)
+                  tma_load_3d(sQ + b * C::Q_BYTES + cb * C::BLK, &tmQ, q_full, cb * C::AW, b ? u.head[1] : u.head[0],
+                              si.cu_q + (b ? u.q0[1] : u.q0[0]));
+              }
+            }
             ++q_loads;
           }
         }
         kv_iter += nmax;
       }
       // never leave the CTA while loads it issued are still landing in shared memory
-      for (int kv = 0; kv < 2; ++kv)
-        for (uint32_t g = issued[kv] >= 2 ? issued[kv] - 2 : 0; g < issued[kv]; ++g)
-          mbar_wait((kv ? v_full : k_full) + (g & 1), (g >> 1) & 1, status, kv ? kDevTimeoutVFull : kDevTimeoutKFull);
+      for (uint32_t g = issued_k >= 2 ? issued_k - 2 : 0; g < issued_k; ++g)
+        mbar_wait(k_full + (g & 1), (g >> 1) & 1, status, kDevTimeoutKFull);
+      for (uint32_t g = issued_v >= 2 ? issued_v - 2 : 0; g < issued_v; ++g)
+        mbar_wait(v_full + (g & 1), (g >> 1) & 1, status, kDevTimeoutVFull);
       if (q_loads > 0) mbar_wait(q_full, (q_loads - 1) & 1, status, kDevTimeoutQ);
-    } else if (warp == 9 && lane == 0) {
+    } else if (warp == 9) {
       // ------------------------------------------------------------ MMA issuer
-      const uint32_t q_base = smem_addr(sQ);
+      // the whole warp walks the schedule with warp-uniform descriptors; one elected lane issues
+      const bool leader = elect_one();
+      // base shared-memory descriptors; a K step adds its byte offset >> 4 to the start-address field
+      const uint64_t dq = smem_desc_sw128(smem_addr(sQ), 16, 1024);
+      const uint64_t dk = smem_desc_sw128(smem_addr(sK), 16, 1024);
+      // V is the MN-major operand: 16-bit types use the 16-byte-chunk swizzle (8-row atoms),
+      // tf32 the 32-byte-chunk swizzle (4-row atoms), matching how the V tensor map loads it
+      const uint64_t dv = C::ES == 4 ? smem_desc(smem_addr(sV), C::BLK, 512, 1) : smem_desc(smem_addr(sV), C::BLK, 1024, 2);
+      constexpr uint64_t kQStep = C::Q_BYTES >> 4, kKVStep = C::KV_BYTES >> 4;
       auto issue_qk = [&](int b, int s) {
-        const uint32_t qb = q_base + b * C::Q_BYTES;
-        const uint32_t kb = smem_addr(sK + s * C::KV_BYTES);
+        if (leader) {
+          const uint64_t a0 = dq + b * kQStep, b0 = dk + s * kKVStep;
 #pragma unroll
-        for (int kk = 0; kk < D / C::UK; ++kk) {
-          const int ke = kk * C::UK;
-          const uint32_t off = (ke / C::AW) * C::BLK + (ke % C::AW) * C::ES;
-          mma_ss(tmem + b * 128, smem_desc_sw128(qb + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024),
-                 C::IDESC_QK, kk > 0, C::ES == 4);
+          for (int kk = 0; kk < D / C::UK; ++kk) {
+            const int ke = kk * C::UK;
+            const uint64_t off = ((ke / C::AW) * C::BLK + (ke % C::AW) * C::ES) >> 4;
+            mma_ss(tmem + b * 128, a0 + off, b0 + off, C::IDESC_QK, kk > 0, C::ES == 4);
+          }
         }
       };
       auto issue_pv = [&](int b, int s, bool acc) {
-        const uint32_t vb = smem_addr(sV + s * C::KV_BYTES);
+        if (leader) {
+          const uint64_t v0 = dv + s * kKVStep;
 #pragma unroll
-        for (int kk = 0; kk < 128 / C::UK; ++kk) {
-          const int ke = kk * C::UK;
-          // V is the MN-major operand: 16-bit types use the 16-byte-chunk swizzle (8-row atoms),
-          // tf32 the 32-byte-chunk swizzle (4-row atoms), matching how the V tensor map loads it
-          const uint64_t vdesc = C::ES == 4 ? smem_desc(vb + ke * 128, C::BLK, 512, 1)
-                                            : smem_desc(vb + ke * 128, C::BLK, 1024, 2);
-          // P_b in TMEM over S_b: 8 columns per K step (two 16-bit values per column, or 8 tf32)
-          mma_ts(tmem + 256 + b * D, tmem + b * 128 + kk * 8, vdesc, C::IDESC_PV, (acc || kk > 0) ? 1u : 0u,
-                 C::ES == 4);
+          for (int kk = 0; kk < 128 / C::UK; ++kk) {
+            // P_b in TMEM over S_b: 8 columns per K step (two 16-bit values per column, or 8 tf32)
+            mma_ts(tmem + 256 + b * D, tmem + b * 128 + kk * 8, v0 + ((kk * C::UK * 128) >> 4), C::IDESC_PV,
+                   (acc || kk > 0) ? 1u : 0u, C::ES == 4);
+          }
         }
+      };
+      auto commit = [&](uint64_t* bar) {
+        if (leader) mma_commit(bar);
+      };
+      auto wait_all = [&](uint64_t* bar, uint32_t parity, int code) {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, status, code));
       };
       bool ok = true;
       uint32_t kv_iter = 0;
-      uint32_t sp[2] = {0, 0};  // tiles block 0 / 1 processed in earlier units
+      uint32_t sp0 = 0, sp1 = 0;  // tiles block 0 / 1 processed in earlier units
       for (int ui = u_begin; ui < u_end && ok; ++ui) {
         const int it = ui - u_begin;
         const PrefillUnit u = p.units[ui];
@@ -317,24 +342,25 @@ __global__ void __launch_bounds__(384, 1)
         const int n0 = u.n_tiles[0];
         const int n1 = nb > 1 ? u.n_tiles[1] : 0;
         const int nmax = n0 > n1 ? n0 : n1;
-        if (!mbar_wait(q_full, it & 1, status, kDevTimeoutQ) ||
-            !mbar_wait(k_full + (kv_iter & 1), (kv_iter >> 1) & 1, status, kDevTimeoutKFull)) {
+        if (!wait_all(q_full, it & 1, kDevTimeoutQ) ||
+            !wait_all(k_full + (kv_iter & 1), (kv_iter >> 1) & 1, kDevTimeoutKFull)) {
           ok = false;
           break;
         }
         for (int b = 0; b < nb; ++b) {
           // S_b / P_b are free once the previous unit's last P_b * V has completed
-          if (sp[b] > 0 && !mbar_wait(pv_done + b, (sp[b] - 1) & 1, status, kDevTimeoutODone)) {
+          const uint32_t spb = b ? sp1 : sp0;
+          if (spb > 0 && !wait_all(pv_done + b, (spb - 1) & 1, kDevTimeoutODone)) {
             ok = false;
             break;
           }
           tc_fence_after();
           issue_qk(b, kv_iter & 1);
-          mma_commit(s_full + b);
+          commit(s_full + b);
         }
         if (!ok) break;
-        mma_commit(k_empty + (kv_iter & 1));
-        if (nmax == 1) mma_commit(q_empty);
+        commit(k_empty + (kv_iter & 1));
+        if (nmax == 1) commit(q_empty);
         for (int j = 0; j < nmax && ok; ++j) {
           const uint32_t g = kv_iter + j;
           const int s = g & 1;
@@ -342,59 +368,59 @@ __global__ void __launch_bounds__(384, 1)
           for (int b = 0; b < nb && ok; ++b) {
             const int nbt = b == 0 ? n0 : n1;
             if (j >= nbt) continue;
-            const uint32_t ph = sp[b] + j;  // this block's barrier phase for tile j
-            if (!mbar_wait(p_full + b, ph & 1, status, kDevTimeoutPFull)) {
+            const uint32_t ph = (b ? sp1 : sp0) + j;  // this block's barrier phase for tile j
+            if (!wait_all(p_full + b, ph & 1, kDevTimeoutPFull)) {
               ok = false;
               break;
             }
-            if (!v_ready && !mbar_wait(v_full + s, (g >> 1) & 1, status, kDevTimeoutVFull)) {
+            if (!v_ready && !wait_all(v_full + s, (g >> 1) & 1, kDevTimeoutVFull)) {
               ok = false;
               break;
             }
             v_ready = true;
             tc_fence_after();
             issue_pv(b, s, j > 0);
-            mma_commit(pv_done + b);
+            commit(pv_done + b);
             const bool last_pv = (b == nb - 1) || (j >= n1);
-            if (last_pv) mma_commit(v_empty + s);
+            if (last_pv) commit(v_empty + s);
             if (j == nbt - 1) {
-              mma_commit(o_done + b);
+              commit(o_done + b);
               continue;
             }
             // next key tile for this block; S_b / P_b are reused once P_b(j) * V has completed
             const uint32_t g1 = g + 1;
             const int s1 = g1 & 1;
             const bool first_qk = (b == 0) || (j + 1 >= n0);
-            if (first_qk && !mbar_wait(k_full + s1, (g1 >> 1) & 1, status, kDevTimeoutKFull)) {
+            if (first_qk && !wait_all(k_full + s1, (g1 >> 1) & 1, kDevTimeoutKFull)) {
               ok = false;
               break;
             }
-            if (!mbar_wait(pv_done + b, ph & 1, status, kDevTimeoutODone)) {
+            if (!wait_all(pv_done + b, ph & 1, kDevTimeoutODone)) {
               ok = false;
               break;
             }
             tc_fence_after();
             issue_qk(b, s1);
-            mma_commit(s_full + b);
+            commit(s_full + b);
             const bool last_qk = (b == nb - 1) || (j + 1 >= n1);
             if (last_qk) {
-              mma_commit(k_empty + s1);
-              if (j + 1 == nmax - 1) mma_commit(q_empty);  // the unit's last QK: Q buffers free
+              commit(k_empty + s1);
+              if (j + 1 == nmax - 1) commit(q_empty);  // the unit's last QK: Q buffers free
             }
           }
         }
-        sp[0] += n0;
-        sp[1] += n1;
+        sp0 += n0;
+        sp1 += n1;
         kv_iter += nmax;
       }
       // all tensor-core work this thread issued has finished before TMEM is released
-      mma_commit(fin);
-      mbar_wait(fin, 0, status, kDevTimeoutFinal);
+      commit(fin);
+      wait_all(fin, 0, kDevTimeoutFinal);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax / epilogue of block b
-    regs_increase<224>();
+    regs_increase<216>();
     const int b = warp >> 2;
     const int r = threadIdx.x & 127;  // query row in the block == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -412,16 +438,17 @@ __global__ void __launch_bounds__(384, 1)
       const PrefillUnit u = p.units[ui];
       if (b >= u.n_blocks) continue;
       const SeqInfo si = p.seqs[u.b];
-      const int n = u.n_tiles[b];
-      const int head = u.head[b];
-      const int qi = u.q0[b] + r;
+      const int n = b ? u.n_tiles[1] : u.n_tiles[0];
+      const int head = b ? u.head[1] : u.head[0];
+      const int q0 = b ? u.q0[1] : u.q0[0];
+      const int qi = q0 + r;
       const bool row_valid = qi < si.seq_len;
       const int off = si.kv_len - si.seq_len;
       const int iabs = qi + off;
       const float slope = alibi ? p.slopes[head] : 0.f;
       const float slope_log2 = slope * kLog2e;
       const int last_key = (mt == 0) ? si.kv_len - 1 : min(iabs, si.kv_len - 1);
-      const int iabs_w = u.q0[b] + (warp & 3) * 32 + off;  // iabs of the warp's first row
+      const int iabs_w = q0 + (warp & 3) * 32 + off;  // iabs of the warp's first row
       float m_run = -INFINITY;  // running max in log2 units (the one P is computed against)
       float l_run = 0.f;
       for (int j = 0; j < n; ++j) {
