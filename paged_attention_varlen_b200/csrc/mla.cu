@@ -150,92 +150,104 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // the whole warp walks the tiles (warp-uniform values); one elected lane issues the copies
+    const bool leader = elect_one();
+    const int h0 = u.group * kHeadsPerCta;
+    if (leader) {
       tma_prefetch_desc(&tmQn);
       tma_prefetch_desc(&tmQr);
       tma_prefetch_desc(&tmKV);
       tma_prefetch_desc(&tmKR);
-      const int h0 = u.group * kHeadsPerCta;
       mbar_expect_tx(q_full, kQBytes);
       for (int cb = 0; cb < 8; ++cb) tma_load_3d(sQ + cb * kBlk, &tmQn, q_full, cb * 64, h0, u.token);
       tma_load_3d(sQ + 8 * kBlk, &tmQr, q_full, 0, h0, u.token);
-      const int32_t* bt = p.block_tables + (size_t)u.b * p.max_blocks;
-      const int bs = p.block_size;
-      const int box_rows = bs < kTileKeys ? bs : kTileKeys;
-      const int n_pages = (u.last_key + 1 + bs - 1) / bs;
-      bool ok = true;
-      int issued = 0;
-      for (int j = 0; j < n && ok; ++j) {
-        const int s = j & 1;
-        if (j >= kStages && !mbar_wait(kv_empty + s, ((j >> 1) - 1) & 1, status, kDevTimeoutKEmpty)) {
-          ok = false;
-          break;
-        }
-        uint8_t* dst = sKV + s * kKvBytes;
-        mbar_expect_tx(kv_full + s, kKvBytes);
-        const int j0 = u.kv_begin + j * kTileKeys;
-        for (int r0 = 0; r0 < kTileKeys; r0 += box_rows) {
-          const int pos = j0 + r0;
-          const int pg = pos / bs;
-          const int row = pg < n_pages ? bt[pg] * bs + (pos % bs) : p.oob_row;  // past the last page: zeros
+    }
+    const int32_t* bt = p.block_tables + (size_t)u.b * p.max_blocks;
+    const int bs = p.block_size;
+    const int box_rows = bs < kTileKeys ? bs : kTileKeys;
+    const int n_pages = (u.last_key + 1 + bs - 1) / bs;
+    bool ok = true;
+    int issued = 0;
+    for (int j = 0; j < n && ok; ++j) {
+      const int s = j & 1;
+      if (j >= kStages &&
+          !__all_sync(0xffffffffu, mbar_wait(kv_empty + s, ((j >> 1) - 1) & 1, status, kDevTimeoutKEmpty))) {
+        ok = false;
+        break;
+      }
+      uint8_t* dst = sKV + s * kKvBytes;
+      if (leader) mbar_expect_tx(kv_full + s, kKvBytes);
+      const int j0 = u.kv_begin + j * kTileKeys;
+      for (int r0 = 0; r0 < kTileKeys; r0 += box_rows) {
+        const int pos = j0 + r0;
+        const int pg = pos / bs;
+        const int row = pg < n_pages ? bt[pg] * bs + (pos % bs) : p.oob_row;  // past the last page: zeros
+        if (leader) {
           for (int cb = 0; cb < 8; ++cb) tma_load_2d(dst + cb * kBlk + r0 * 128, &tmKV, kv_full + s, cb * 64, row);
           tma_load_2d(dst + 8 * kBlk + r0 * 128, &tmKR, kv_full + s, 0, row);
         }
-        issued = j + 1;
       }
-      for (int j = issued - kStages < 0 ? 0 : issued - kStages; j < issued; ++j)
-        mbar_wait(kv_full + (j & 1), (j >> 1) & 1, status, kDevTimeoutKFull);
-      mbar_wait(q_full, 0, status, kDevTimeoutQ);
+      issued = j + 1;
     }
-    __syncwarp();
+    for (int j = issued - kStages < 0 ? 0 : issued - kStages; j < issued; ++j)
+      mbar_wait(kv_full + (j & 1), (j >> 1) & 1, status, kDevTimeoutKFull);
+    mbar_wait(q_full, 0, status, kDevTimeoutQ);
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t fmt = std::is_same<T, __half>::value ? 0u : 1u;
-      constexpr uint32_t idesc_qk = instr_desc(fmt, false, false, 64, kTileKeys);
-      constexpr uint32_t idesc_pv = instr_desc(fmt, false, true, 64, 256);
-      const uint32_t q_base = smem_addr(sQ);
-      const uint32_t p_base = smem_addr(sP);
-      auto issue_pv = [&](int jj) {
-        const uint32_t kvb = smem_addr(sKV + (jj & 1) * kKvBytes);
-#pragma unroll
-        for (int kk = 0; kk < kTileKeys / 16; ++kk) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            // V = ctKV columns [256h, 256h+256): four 64-wide column blocks, MN-major
-            const uint64_t vdesc = smem_desc(kvb + 4 * h * kBlk + kk * 16 * 128, kBlk, 1024, 2);
-            mma_ss(tmem + ((uint32_t)(16 * h) << 16), smem_desc_sw128(p_base + kk * 32, 16, 1024), vdesc, idesc_pv,
-                   (jj > 0 || kk > 0) ? 1u : 0u, false);
-          }
-        }
-        mma_commit(kv_empty + (jj & 1));
-        mma_commit(o_done);
-      };
-      bool ok = mbar_wait(q_full, 0, status, kDevTimeoutQ);
-      for (int j = 0; j <= n && ok; ++j) {
-        if (j < n) {
-          if (!mbar_wait(kv_full + (j & 1), (j >> 1) & 1, status, kDevTimeoutKFull)) break;
-          if (j >= 1 && !mbar_wait(s_free, (j - 1) & 1, status, kDevTimeoutSFree)) break;
-          tc_fence_after();
-          const uint32_t kvb = smem_addr(sKV + (j & 1) * kKvBytes);
+    // the whole warp walks the schedule with warp-uniform descriptors; one elected lane issues
+    const bool leader = elect_one();
+    constexpr uint32_t fmt = std::is_same<T, __half>::value ? 0u : 1u;
+    constexpr uint32_t idesc_qk = instr_desc(fmt, false, false, 64, kTileKeys);
+    constexpr uint32_t idesc_pv = instr_desc(fmt, false, true, 64, 256);
+    // base descriptors; a step adds its byte offset >> 4 to the start-address field
+    const uint64_t dq = smem_desc_sw128(smem_addr(sQ), 16, 1024);
+    const uint64_t dkv = smem_desc_sw128(smem_addr(sKV), 16, 1024);
+    const uint64_t dv = smem_desc(smem_addr(sKV), kBlk, 1024, 2);  // ctKV as the MN-major V operand
+    const uint64_t dp = smem_desc_sw128(smem_addr(sP), 16, 1024);
+    auto wait_all = [&](uint64_t* bar, uint32_t parity, int code) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, status, code));
+    };
+    auto commit = [&](uint64_t* bar) {
+      if (leader) mma_commit(bar);
+    };
+    bool ok = wait_all(q_full, 0, kDevTimeoutQ);
+    for (int j = 0; j <= n && ok; ++j) {
+      if (j < n) {
+        if (!wait_all(kv_full + (j & 1), (j >> 1) & 1, kDevTimeoutKFull)) break;
+        if (j >= 1 && !wait_all(s_free, (j - 1) & 1, kDevTimeoutSFree)) break;
+        tc_fence_after();
+        if (leader) {
+          const uint64_t kv0 = dkv + (uint64_t)((j & 1) * kKvBytes >> 4);
 #pragma unroll
           for (int kk = 0; kk < 576 / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kBlk + (kk & 3) * 32;
-            mma_ss(tmem + kSCol, smem_desc_sw128(q_base + off, 16, 1024), smem_desc_sw128(kvb + off, 16, 1024),
-                   idesc_qk, kk > 0, false);
+            const uint64_t off = ((kk >> 2) * kBlk + (kk & 3) * 32) >> 4;
+            mma_ss(tmem + kSCol, dq + off, kv0 + off, idesc_qk, kk > 0, false);
           }
-          mma_commit(s_full);
         }
-        if (j >= 1) {
-          if (!mbar_wait(p_full, (j - 1) & 1, status, kDevTimeoutPFull)) break;
-          tc_fence_after();
-          issue_pv(j - 1);
-        }
+        commit(s_full);
       }
-      mma_commit(fin);
-      mbar_wait(fin, 0, status, kDevTimeoutFinal);
+      if (j >= 1) {
+        const int jj = j - 1;
+        if (!wait_all(p_full, jj & 1, kDevTimeoutPFull)) break;
+        tc_fence_after();
+        if (leader) {
+          const uint64_t v0 = dv + (uint64_t)((jj & 1) * kKvBytes >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kTileKeys / 16; ++kk) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              // V = ctKV columns [256h, 256h+256): four 64-wide column blocks, MN-major
+              mma_ss(tmem + ((uint32_t)(16 * h) << 16), dp + ((kk * 32) >> 4),
+                     v0 + ((4 * h * kBlk + kk * 16 * 128) >> 4), idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u, false);
+            }
+          }
+        }
+        commit(kv_empty + (jj & 1));
+        commit(o_done);
+      }
     }
-    __syncwarp();
+    commit(fin);
+    wait_all(fin, 0, kDevTimeoutFinal);
   } else {
     // ------------------------------------------------------------ softmax / epilogue
     const bool upper = lane >= 16;            // lanes 16..31 hold the upper 256 output columns
