@@ -255,6 +255,7 @@ __global__ void __launch_bounds__(192, 1)
     const int head = u.group * kHeadsPerCta + hl;
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const float scale = p.scale_log2;
+    const bool raw_max = scale > 0.f;  // max of the raw scores, scale folded into the exponent
     float m_run = -INFINITY;
     float l_run = 0.f;
     bool ok = true;
@@ -274,12 +275,24 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       mbar_arrive(s_free);
       const int lim = u.last_key - (u.kv_begin + j * kTileKeys);  // columns c <= lim are allowed
-      float mx = -INFINITY;
+      if (!raw_max) {
 #pragma unroll
-      for (int c = 0; c < kTileKeys; ++c) {
-        x[c] = (c > lim) ? -INFINITY : x[c] * scale;
-        mx = fmaxf(mx, x[c]);
+        for (int c = 0; c < kTileKeys; ++c) x[c] *= scale;
       }
+      if (__any_sync(0xffffffffu, lim < kTileKeys - 1)) {  // only a range's last tile can hold masked keys
+#pragma unroll
+        for (int c = 0; c < kTileKeys; ++c) x[c] = (c > lim) ? -INFINITY : x[c];
+      }
+      float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
+#pragma unroll
+      for (int c = 4; c < kTileKeys; c += 8) {
+        mx0 = max3(mx0, x[c], x[c + 1]);
+        mx1 = max3(mx1, x[c + 2], x[c + 3]);
+        mx2 = max3(mx2, x[c + 4], x[c + 5]);
+        mx3 = max3(mx3, x[c + 6], x[c + 7]);
+      }
+      float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+      if (raw_max) mx *= scale;
       const float m_new = fmaxf(m_run, mx);
       float alpha = 1.f;
       if (m_new - m_run > kRescaleThreshold) {
@@ -287,13 +300,24 @@ __global__ void __launch_bounds__(192, 1)
         m_run = m_new;
       }
       const float m_base = (m_run == -INFINITY) ? 0.f : m_run;
-      float sum = 0.f;
+      // P = 2^(x*scale - m), a pair of columns at a time (-inf masked keys give exactly 0)
+      const uint64_t scale2 = f2pack(raw_max ? scale : 1.f, raw_max ? scale : 1.f);
+      const uint64_t negm2 = f2pack(-m_base, -m_base);
+      uint64_t acc0 = f2pack(0.f, 0.f), acc1 = f2pack(0.f, 0.f);
+      uint32_t pk[kTileKeys / 2];
 #pragma unroll
-      for (int c = 0; c < kTileKeys; ++c) {
-        x[c] = fast_exp2(x[c] - m_base);
-        sum += x[c];
+      for (int c = 0; c < kTileKeys; c += 2) {
+        float e0, e1;
+        f2unpack(fma_x2(f2pack(x[c], x[c + 1]), scale2, negm2), e0, e1);
+        e0 = fast_exp2(e0);
+        e1 = fast_exp2(e1);
+        if ((c >> 1) & 1) acc1 = add_x2(acc1, f2pack(e0, e1));
+        else acc0 = add_x2(acc0, f2pack(e0, e1));
+        pk[c >> 1] = pack2(e0, e1, (T*)nullptr);
       }
-      l_run = l_run * alpha + sum;
+      float s0, s1;
+      f2unpack(add_x2(acc0, acc1), s0, s1);
+      l_run = l_run * alpha + (s0 + s1);
       if (j >= 1) {
         ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, status, kDevTimeoutODone));
         if (!ok) break;
@@ -316,15 +340,10 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (!upper) {
         // P row hl: 64 keys x 16 bit = 128 bytes, K-major 128B-swizzled
+        const uint32_t prow = smem_addr(sP) + hl * 128;
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint4 v;
-          v.x = pack2(x[ch * 8 + 0], x[ch * 8 + 1], (T*)nullptr);
-          v.y = pack2(x[ch * 8 + 2], x[ch * 8 + 3], (T*)nullptr);
-          v.z = pack2(x[ch * 8 + 4], x[ch * 8 + 5], (T*)nullptr);
-          v.w = pack2(x[ch * 8 + 6], x[ch * 8 + 7], (T*)nullptr);
-          *reinterpret_cast<uint4*>(sP + hl * 128 + ((ch ^ (hl & 7)) << 4)) = v;
-        }
+        for (int ch = 0; ch < 8; ++ch)
+          st_shared_v4(prow + ((ch ^ (hl & 7)) << 4), make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]));
       }
       fence_proxy_async_smem();
       tc_fence_before();

@@ -118,9 +118,12 @@ __device__ __forceinline__ float exp_rows(const float (&x)[128], uint64_t scale2
         e0 = fast_exp2(e0);
         e1 = fast_exp2(e1);
       }
-      if constexpr (MASKED) {  // exact zeros for masked keys (the polynomial does not reach 0)
-        e0 = (c0 > lim) ? 0.f : e0;
-        e1 = (c0 + 1 > lim) ? 0.f : e1;
+      if constexpr (MASKED) {
+        // masked keys hold -inf, which ex2 maps to exactly 0; only polynomial lanes need zeroing
+        if ((cc & 3) < ALA_POLY_PAIRS_OF_4) {
+          e0 = (c0 > lim) ? 0.f : e0;
+          e1 = (c0 + 1 > lim) ? 0.f : e1;
+        }
       }
       acc[cc & 3] = add_x2(acc[cc & 3], f2pack(e0, e1));
       if constexpr (kHalf) {

@@ -78,14 +78,21 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* status, int code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (;;) {
+  for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
-    if (*status != 0) return false;
-    if (global_timer_ns() - t0 > ALA_WAIT_LIMIT_NS) {
-      atomicCAS((int*)status, 0, code);
-      return false;
+    if ((it & 15u) == 0) {  // the status word and the clock are checked every 16 attempts
+      if (*status != 0) return false;
+      if (global_timer_ns() - t0 > ALA_WAIT_LIMIT_NS) {
+        atomicCAS((int*)status, 0, code);
+        return false;
+      }
     }
   }
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
 }
 
 // One lane of the (fully converged) warp gets true.

@@ -86,3 +86,13 @@ def test_mla_full_size_sampled(qs):
     check_out(out.reshape(-1, 512)[idx], ref)
     check_lse(lse.reshape(-1)[idx], lref)
     assert torch.isfinite(out.float()).all()
+
+
+def test_mla_negative_qk_scale():
+    ctx = np.array([100, 700], dtype=np.int32)
+    case = synth.make_mla("neg", ctx, 2, 128, 41, block_size=64)
+    case.qk_scale = -0.03
+    out, lse, _ = _run(case)
+    ref, lref = _oracle(case)
+    check_out(out.reshape(-1, 512), ref)
+    check_lse(lse.reshape(-1), lref)

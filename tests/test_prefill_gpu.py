@@ -155,3 +155,12 @@ def test_full_prefix_paged_alibi_fp16():
 @pytest.mark.parametrize("variant", [synth.MASK_ALIBI_SQRT, synth.MASK_ALIBI_LEFT])
 def test_full_long_alibi_bf16(variant):
     _sampled_check(synth.long_alibi_bf16(variant), n=192)
+
+
+@pytest.mark.parametrize("mask_type", [0, 3, 9])
+def test_negative_qk_scale(mask_type):
+    """A negative qkScale reverses the score order; the max must be taken after scaling."""
+    L = [70, 200]
+    case = synth.make_prefill("neg", L, [a + 30 for a in L], 8, 4, 128, torch.bfloat16, mask_type, 29,
+                              qk_scale=-0.06)
+    _full_check(case)
