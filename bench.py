@@ -61,6 +61,20 @@ WORKLOADS = {
 L2_FLUSH_BYTES = 256 << 20
 
 
+def max_over_ranks(value: float, dist=None, device="cpu") -> float:
+    """The largest per-rank value (the slowest rank's step time); identity without a process group."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, work_per_rank: float, ms: float, scale: float) -> float:
+    """Whole-job rate: every rank processes the same work (weak scaling) in at most `ms`."""
+    return world * work_per_rank / (ms * 1e-3) / scale
+
+
 def kernel_source_hash(paths=KERNEL_SOURCES) -> str:
     h = hashlib.sha256()
     for p in paths:
@@ -344,18 +358,14 @@ def main():
 
     with ClockSampler(local) as clk:
         times = time_steps(op, args.steps, args.warmup, flush, stream, barrier)
-    ms = statistics.mean(times)
-    if dist:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(statistics.mean(times), dist, device)
     flops = mla_flops(case) if is_mla else prefill_flops(case)
     nbytes = mla_bytes(case) if is_mla else prefill_bytes(case)
     if is_mla:
-        value = world * nbytes / (ms * 1e-3) / 1e9
+        value = job_throughput(world, nbytes, ms, 1e9)
         metric, unit = "attention HBM GB/s (MLA decode)", "GB/s"
     else:
-        value = world * flops / (ms * 1e-3) / 1e12
+        value = job_throughput(world, flops, ms, 1e12)
         metric, unit = "attention TFLOPS on valid tokens (prefill)", "TFLOPS"
 
     if rank == 0:
