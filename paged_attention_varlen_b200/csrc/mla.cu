@@ -4,25 +4,36 @@
 // the speculative causal rule (token t of a batch with qseqlen tokens allows
 // keys j <= contextLens - qseqlen + t), plus the natural-log lse.
 //
-// Work split.  The 512-wide fp32 output of 128 heads would fill all of tensor
-// memory, so one CTA handles 64 heads (M = 64 MMAs; the output is kept as two
-// 256-column accumulators in the two lane halves of the same TMEM columns) of
-// one query token over one range of keys.  The two head groups of a token read
-// the same cache tiles, which L2 serves once from HBM.  Long key ranges are
-// split so every SM has work; each split leaves an fp32 partial (O, lse) in the
-// workspace and mla_combine_kernel merges them by lse (the same merge the MLA
-// page's ring mode returns the lse for).
+// Rows.  Every MMA has M = 64 rows: tpc consecutive query tokens of one batch
+// times 64/tpc heads (tpc = 4, 2 or 1: the largest that divides every batch's
+// qseqlen), so the speculative tokens of a batch share each cache tile the CTA
+// stages.  The 512-wide fp32 output of 64 rows is kept as two 256-column
+// accumulators in the two lane halves of the same tensor-memory columns.  The
+// heads / (64/tpc) "groups" of a batch read the same cache tiles; L2 serves
+// them once from HBM.
 //
-//   warp 4      TMA producer: the 64x576 query tile once; then 64-token tiles of
-//               ctKV (512) and kRope (64) gathered through the block table into
-//               a 2-deep ring.
-//   warp 5      tcgen05 issuer: S = Q K^T (64 x 64, K = 576), O += P V with V
-//               the ctKV part of the same tile (two N = 256 halves).
-//   warps 0..3  softmax: lane l < 16 of warp w owns head 16w + l; it scales and
-//               masks its S row in registers, keeps the online max / sum, writes
-//               P to shared memory, rescales O when the max grew by more than 2^8,
-//               and at the end normalises O (lanes >= 16 hold the upper 256
-//               columns of the same heads) and stores it.
+// Persistent schedule.  The key tiles of all chunks (a chunk = the tpc tokens
+// one CTA row block covers), laid end to end, are cut into equal contiguous
+// ranges, one per "lane"; the grid is lanes x groups CTAs (at most one per SM),
+// and a CTA walks the pieces of its lane in order.  A chunk cut by a lane
+// boundary leaves an fp32 partial (O, lse) per piece, which mla_combine_kernel
+// merges by lse (the merge the MLA page's ring mode returns the lse for).
+//
+//   warp 4      TMA producer: 64-key tiles of ctKV (512) and kRope (64)
+//               gathered through the block table into a two-deep ring (or
+//               32-key tiles, four deep, with ALA_MLA_TILE_KEYS=32), running
+//               ahead across piece boundaries and asking L2 for the tiles after.
+//   warp 5      tcgen05 issuer: S = Q K^T (64 x 64, K = 576) and O += P V with V
+//               the ctKV part of the same tile (two N = 256 halves); it issues
+//               whichever of the next QK and the next PV is ready first, so a
+//               tile's PV, which frees its ring slot, never waits behind the
+//               next tile's load.
+//   warps 0..3  softmax: lane l < 16 of warp w owns row 16w + l; it scales and
+//               masks its S row, keeps the online max / sum, writes P to shared
+//               memory and rescales O when the max grew by more than 2^8.  At
+//               the end of a piece all 128 threads normalise O into the Q
+//               buffer (free until the next piece's query) and one thread
+//               writes it out with TMA stores, then loads the next query.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -44,47 +55,71 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
 
-constexpr int kHeadsPerCta = 64;
-constexpr int kTileKeys = 64;
+#ifndef ALA_MLA_TILE_KEYS
+#define ALA_MLA_TILE_KEYS 64  // keys per ring slot: 64 (two slots) or 32 (four slots)
+#endif
+
+#ifndef ALA_MLA_PREFETCH_TILES
+#define ALA_MLA_PREFETCH_TILES 2  // the producer asks L2 for the tiles this far ahead of its loads
+#endif
+
+#ifndef ALA_MLA_SPIN
+#define ALA_MLA_SPIN 1  // 1: the MMA warp polls its barriers instead of sleeping on them; 2: softmax too
+#endif
+
+constexpr int kRows = 64;                  // attention rows per CTA: the M of every MMA
+constexpr int kTileKeys = ALA_MLA_TILE_KEYS;
+static_assert(kTileKeys == 32 || kTileKeys == 64, "tile of 32 or 64 keys");
 constexpr int kDNope = 512;
-constexpr int kBlk = 64 * 128;                     // one 64-row x 128-byte swizzle column block
-constexpr int kQBytes = 9 * kBlk;                  // 64 heads x 576 x 2 B
-constexpr int kKvBytes = 9 * kBlk;                 // 64 keys x 576 x 2 B
-constexpr int kPBytes = kBlk;                      // 64 heads x 64 keys x 2 B
-constexpr int kStages = 2;
-constexpr int kNBars = 1 + 4 + 5;                  // q_full, kv_full[2], kv_empty[2], s_full, s_free, p_full, o_done, fin
+constexpr int kQBlk = kRows * 128;         // one 64-column block of the 64 query rows (8 KB)
+constexpr int kKvBlk = kTileKeys * 128;    // one 64-column block of a key tile
+constexpr int kQBytes = 9 * kQBlk;         // 64 rows x 576 x 2 B
+constexpr int kKvBytes = 9 * kKvBlk;       // 32 keys x 576 x 2 B
+constexpr int kPBytes = kRows * 128;       // P rows of 128 B (2 B per key)
+constexpr int kStages = 128 / kTileKeys;   // the ring holds 128 keys
+// q_full, kv_full[4], kv_empty[4], s_full, s_free, p_full, o_done, fin, st_full, st_free
+constexpr int kNBars = 1 + 2 * kStages + 7;
 constexpr int kSmem = 1024 + kQBytes + kStages * kKvBytes + kPBytes + kNBars * 8 + 16;
 static_assert(kSmem <= 232448, "shared memory budget");
-constexpr uint32_t kSCol = 256;                    // S: columns [256, 320), lanes of half 0
+static_assert(8 * kQBlk <= kQBytes, "the output staging (eight 8 KB boxes) must fit in the query buffer");
+constexpr uint32_t kSCol = 256;            // S: columns [256, 256 + kTileKeys), lanes of half 0
 constexpr uint32_t kTmemCols = 512;
+constexpr int kPlannedSms = 148;           // SMs of the part the schedule is cut for
+constexpr int kMinLaneTiles = 8;           // shortest key range worth a lane of its own
+constexpr unsigned kFull = 0xffffffffu;
 
-struct MlaUnit {
+struct MlaPiece {
   int32_t b;         // batch
-  int32_t token;     // packed query token
-  int32_t t;         // token index within its batch
-  int32_t group;     // head group (heads 64*group .. +63)
-  int32_t kv_begin;  // first key of the range (multiple of 64)
-  int32_t n_tiles;   // 64-key tiles in the range
-  int32_t last_key;  // last allowed key of this token (inclusive)
-  int32_t part;      // partial slot, or -1 when this unit writes the final output
+  int32_t token0;    // first packed query token of the chunk
+  int32_t kv_begin;  // first key of the range (a multiple of 32)
+  int32_t n_tiles;   // 32-key tiles in the range
+  int32_t last;      // last allowed key of the chunk's first token; token t of the chunk allows last + t
+  int32_t part;      // partial slot (rows part*tpc .. +tpc-1 of the partials), or -1: final output
+  int32_t pad[2];
 };
 
 struct MlaCombine {
-  int32_t token;
-  int32_t part_begin;
+  int32_t token;       // packed query token
+  int32_t part_begin;  // its chunk's first partial slot
   int32_t n_parts;
-  int32_t pad;
+  int32_t t_local;     // token index within the chunk
 };
 
 struct MlaParams {
-  const MlaUnit* units;
+  const MlaPiece* pieces;
+  const int32_t* lane_off;  // [n_lanes + 1]: lane l walks pieces [lane_off[l], lane_off[l+1])
   const int32_t* block_tables;
-  void* out;          // [tokens, heads, 512]
-  float* lse;         // [tokens, heads] or null
-  float* part_o;      // [parts, heads, 512]
-  float* part_lse;    // [parts, heads]
+  const uint8_t* ct_kv;     // [numBlocks * blockSize, 512] (the L2 prefetch reads raw rows)
+  const uint8_t* k_rope;    // [numBlocks * blockSize, 64]
+  void* out;                // [tokens, heads, 512] (written by TMA stores and by the combine)
+  float* lse;               // [tokens, heads] or null
+  float* part_o;            // [parts * tpc, heads, 512]
+  float* part_lse;          // [parts * tpc, heads]
   int* status;
   int32_t heads;
+  int32_t groups;           // heads / hpc
+  int32_t tpc;              // query tokens per CTA row block
+  int32_t hpc;              // heads per CTA row block (64 / tpc)
   int32_t max_blocks;
   int32_t block_size;
   int32_t oob_row;
@@ -100,30 +135,59 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, __half*) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// The 64 x 576 query rows of one chunk: eight 64-column blocks of qNope, then qRope.
+__device__ __forceinline__ void load_query(uint8_t* sQ, uint64_t* q_full, const CUtensorMap* tmQn,
+                                           const CUtensorMap* tmQr, int h0, int token0) {
+  mbar_expect_tx(q_full, kQBytes);
+  for (int cb = 0; cb < 8; ++cb) tma_load_3d(sQ + cb * kQBlk, tmQn, q_full, cb * 64, h0, token0);
+  tma_load_3d(sQ + 8 * kQBlk, tmQr, q_full, 0, h0, token0);
+}
+
+// Warp-uniform wait on all lanes (each lane observes the phase itself).
+__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, int* status, int code) {
+  return __all_sync(kFull, mbar_wait(bar, parity, status, code));
+}
+// The same for the waits on the QK -> softmax -> PV chain (ALA_MLA_SPIN: 1 = the MMA warp polls,
+// 2 = the softmax warps too).
+__device__ __forceinline__ bool wait_mma(uint64_t* bar, uint32_t parity, int* status, int code) {
+  if (ALA_MLA_SPIN >= 1) return __all_sync(kFull, mbar_wait_spin(bar, parity, status, code));
+  return __all_sync(kFull, mbar_wait(bar, parity, status, code));
+}
+__device__ __forceinline__ bool wait_smx(uint64_t* bar, uint32_t parity, int* status, int code) {
+  if (ALA_MLA_SPIN >= 2) return __all_sync(kFull, mbar_wait_spin(bar, parity, status, code));
+  return __all_sync(kFull, mbar_wait(bar, parity, status, code));
+}
+
 template <typename T>
 __global__ void __launch_bounds__(192, 1)
     mla_kernel(const __grid_constant__ CUtensorMap tmQn, const __grid_constant__ CUtensorMap tmQr,
-               const __grid_constant__ CUtensorMap tmKV, const __grid_constant__ CUtensorMap tmKR, const MlaParams p) {
+               const __grid_constant__ CUtensorMap tmKV, const __grid_constant__ CUtensorMap tmKR,
+               const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmPO,
+               const MlaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
+  uint8_t* sQ = smem;  // the chunk's query rows; between pieces, the output staging area
   uint8_t* sKV = sQ + kQBytes;
   uint8_t* sP = sKV + kStages * kKvBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sP + kPBytes);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;   // [2]
-  uint64_t* kv_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;
-  uint64_t* s_free = bars + 6;
-  uint64_t* p_full = bars + 7;
-  uint64_t* o_done = bars + 8;
-  uint64_t* fin = bars + 9;
+  uint64_t* kv_full = bars + 1;             // [kStages]
+  uint64_t* kv_empty = bars + 1 + kStages;  // [kStages]
+  uint64_t* s_full = bars + 1 + 2 * kStages;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_done = s_full + 3;
+  uint64_t* fin = s_full + 4;
+  uint64_t* st_full = s_full + 5;  // the 128 softmax threads have written a round of output boxes
+  uint64_t* st_free = s_full + 6;  // the stores of a round have read their boxes
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNBars);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const MlaUnit u = p.units[blockIdx.x];
-  const int n = u.n_tiles;
+  const int ln = blockIdx.x / p.groups;
+  const int h0 = (blockIdx.x - ln * p.groups) * p.hpc;  // first head of this CTA's group
+  const int k0 = p.lane_off[ln];
+  const int k1 = p.lane_off[ln + 1];
   int* status = p.status;
 
   if (threadIdx.x == 0) {
@@ -137,6 +201,8 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(p_full, 128);
     mbar_init(o_done, 1);
     mbar_init(fin, 1);
+    mbar_init(st_full, 128);
+    mbar_init(st_free, 1);
     fence_mbar_init();
   }
   if (warp == 5) {
@@ -152,245 +218,363 @@ __global__ void __launch_bounds__(192, 1)
     // ------------------------------------------------------------ producer
     // the whole warp walks the tiles (warp-uniform values); one elected lane issues the copies
     const bool leader = elect_one();
-    const int h0 = u.group * kHeadsPerCta;
     if (leader) {
       tma_prefetch_desc(&tmQn);
       tma_prefetch_desc(&tmQr);
       tma_prefetch_desc(&tmKV);
       tma_prefetch_desc(&tmKR);
-      mbar_expect_tx(q_full, kQBytes);
-      for (int cb = 0; cb < 8; ++cb) tma_load_3d(sQ + cb * kBlk, &tmQn, q_full, cb * 64, h0, u.token);
-      tma_load_3d(sQ + 8 * kBlk, &tmQr, q_full, 0, h0, u.token);
+      if (k0 < k1) load_query(sQ, q_full, &tmQn, &tmQr, h0, p.pieces[k0].token0);
     }
-    const int32_t* bt = p.block_tables + (size_t)u.b * p.max_blocks;
     const int bs = p.block_size;
     const int box_rows = bs < kTileKeys ? bs : kTileKeys;
-    const int n_pages = (u.last_key + 1 + bs - 1) / bs;
     bool ok = true;
-    int issued = 0;
-    for (int j = 0; j < n && ok; ++j) {
-      const int s = j & 1;
-      if (j >= kStages &&
-          !__all_sync(0xffffffffu, mbar_wait(kv_empty + s, ((j >> 1) - 1) & 1, status, kDevTimeoutKEmpty))) {
-        ok = false;
-        break;
-      }
-      uint8_t* dst = sKV + s * kKvBytes;
-      if (leader) mbar_expect_tx(kv_full + s, kKvBytes);
-      const int j0 = u.kv_begin + j * kTileKeys;
-      for (int r0 = 0; r0 < kTileKeys; r0 += box_rows) {
-        const int pos = j0 + r0;
-        const int pg = pos / bs;
-        const int row = pg < n_pages ? bt[pg] * bs + (pos % bs) : p.oob_row;  // past the last page: zeros
-        if (leader) {
-          for (int cb = 0; cb < 8; ++cb) tma_load_2d(dst + cb * kBlk + r0 * 128, &tmKV, kv_full + s, cb * 64, row);
-          tma_load_2d(dst + 8 * kBlk + r0 * 128, &tmKR, kv_full + s, 0, row);
+    int G = 0;  // tiles issued so far by this CTA
+    // L2 prefetch cursor (piece kf, tile jf, CTA tile Gf), kept ALA_MLA_PREFETCH_TILES tiles ahead of the loads
+    int kf = k0, jf = 0, Gf = 0;
+    MlaPiece pf = k0 < k1 ? p.pieces[k0] : MlaPiece{};
+    for (int k = k0; k < k1 && ok; ++k) {
+      const MlaPiece pc = p.pieces[k];
+      const int32_t* bt = p.block_tables + (size_t)pc.b * p.max_blocks;
+      const int n_pages = (pc.last + p.tpc + bs - 1) / bs;  // pages holding keys <= the chunk's last allowed key
+      for (int j = 0; j < pc.n_tiles; ++j) {
+        if (ALA_MLA_PREFETCH_TILES > 0) {
+          for (; kf < k1 && Gf <= G + ALA_MLA_PREFETCH_TILES; ++Gf) {
+            if (leader) {
+              const int32_t* btf = p.block_tables + (size_t)pf.b * p.max_blocks;
+              const int npf = (pf.last + p.tpc + bs - 1) / bs;
+              for (int r0 = 0; r0 < kTileKeys; r0 += box_rows) {
+                const int pos = pf.kv_begin + jf * kTileKeys + r0;
+                const int pg = pos / bs;
+                const size_t row = pg < npf ? (size_t)btf[pg] * bs + (pos - pg * bs) : (size_t)p.oob_row;
+                if (row < (size_t)p.oob_row) {  // a block index outside the cache is never touched
+                  bulk_prefetch_l2(p.ct_kv + row * 1024, box_rows * 1024);
+                  bulk_prefetch_l2(p.k_rope + row * 128, box_rows * 128);
+                }
+              }
+            }
+            if (++jf == pf.n_tiles) {
+              jf = 0;
+              if (++kf < k1) pf = p.pieces[kf];
+            }
+          }
         }
+        const int s = G & (kStages - 1);
+        if (G >= kStages && !wait_all(kv_empty + s, ((G / kStages) - 1) & 1, status, kDevTimeoutKEmpty)) {
+          ok = false;
+          break;
+        }
+        uint8_t* dst = sKV + s * kKvBytes;
+        if (leader) mbar_expect_tx(kv_full + s, kKvBytes);
+        const int j0 = pc.kv_begin + j * kTileKeys;
+        for (int r0 = 0; r0 < kTileKeys; r0 += box_rows) {
+          const int pos = j0 + r0;
+          const int pg = pos / bs;
+          const int row = pg < n_pages ? bt[pg] * bs + (pos - pg * bs) : p.oob_row;  // past the last page: zeros
+          if (leader) {
+            for (int cb = 0; cb < 8; ++cb) tma_load_2d(dst + cb * kKvBlk + r0 * 128, &tmKV, kv_full + s, cb * 64, row);
+            tma_load_2d(dst + 8 * kKvBlk + r0 * 128, &tmKR, kv_full + s, 0, row);
+          }
+        }
+        ++G;
       }
-      issued = j + 1;
     }
-    for (int j = issued - kStages < 0 ? 0 : issued - kStages; j < issued; ++j)
-      mbar_wait(kv_full + (j & 1), (j >> 1) & 1, status, kDevTimeoutKFull);
-    mbar_wait(q_full, 0, status, kDevTimeoutQ);
+    // no copy may be in flight when the CTA exits
+    for (int t = G - kStages < 0 ? 0 : G - kStages; t < G; ++t)
+      mbar_wait(kv_full + (t & (kStages - 1)), (t / kStages) & 1, status, kDevTimeoutKFull);
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
     // the whole warp walks the schedule with warp-uniform descriptors; one elected lane issues
     const bool leader = elect_one();
     constexpr uint32_t fmt = std::is_same<T, __half>::value ? 0u : 1u;
-    constexpr uint32_t idesc_qk = instr_desc(fmt, false, false, 64, kTileKeys);
-    constexpr uint32_t idesc_pv = instr_desc(fmt, false, true, 64, 256);
+    constexpr uint32_t idesc_qk = instr_desc(fmt, false, false, kRows, kTileKeys);
+    constexpr uint32_t idesc_pv = instr_desc(fmt, false, true, kRows, 256);
     // base descriptors; a step adds its byte offset >> 4 to the start-address field
     const uint64_t dq = smem_desc_sw128(smem_addr(sQ), 16, 1024);
-    const uint64_t dkv = smem_desc_sw128(smem_addr(sKV), 16, 1024);
-    const uint64_t dv = smem_desc(smem_addr(sKV), kBlk, 1024, 2);  // ctKV as the MN-major V operand
+    const uint64_t dk = smem_desc_sw128(smem_addr(sKV), 16, 1024);
+    const uint64_t dv = smem_desc(smem_addr(sKV), kKvBlk, 1024, 2);  // ctKV as the MN-major V operand
     const uint64_t dp = smem_desc_sw128(smem_addr(sP), 16, 1024);
-    auto wait_all = [&](uint64_t* bar, uint32_t parity, int code) {
-      return __all_sync(0xffffffffu, mbar_wait(bar, parity, status, code));
-    };
-    auto commit = [&](uint64_t* bar) {
-      if (leader) mma_commit(bar);
-    };
-    bool ok = wait_all(q_full, 0, kDevTimeoutQ);
-    for (int j = 0; j <= n && ok; ++j) {
-      if (j < n) {
-        if (!wait_all(kv_full + (j & 1), (j >> 1) & 1, kDevTimeoutKFull)) break;
-        if (j >= 1 && !wait_all(s_free, (j - 1) & 1, kDevTimeoutSFree)) break;
-        tc_fence_after();
-        if (leader) {
-          const uint64_t kv0 = dkv + (uint64_t)((j & 1) * kKvBytes >> 4);
-#pragma unroll
-          for (int kk = 0; kk < 576 / 16; ++kk) {
-            const uint64_t off = ((kk >> 2) * kBlk + (kk & 3) * 32) >> 4;
-            mma_ss(tmem + kSCol, dq + off, kv0 + off, idesc_qk, kk > 0, false);
+    int total = 0;
+    for (int k = k0; k < k1; ++k) total += p.pieces[k].n_tiles;
+    // QK cursor: piece kq, tile jq of nq, tile Gq of the CTA; PV cursor likewise
+    int kq = k0, jq = 0, nq = k0 < k1 ? p.pieces[k0].n_tiles : 0, Gq = 0;
+    int kp = k0, jp = 0, np = nq, Gp = 0;
+    bool ok = true;
+    while (ok && Gp < total) {
+      // QK(Gq) needs its tile, the S buffer (softmax has read S(Gq-1)) and, first in a piece, the query;
+      // PV(Gp) needs P(Gp).  QK may lead PV by one tile: S and P are single-buffered.
+      const bool can_pv = Gp < Gq;
+      const bool can_qk = Gq < total && Gq - Gp < 2;
+      bool do_pv = can_pv;
+      if (can_pv && can_qk) {
+        const uint64_t t0 = global_timer_ns();
+        for (uint32_t it = 1;; ++it) {
+          if (__all_sync(kFull, mbar_test_wait(p_full, Gp & 1))) {
+            do_pv = true;
+            break;
+          }
+          const bool qk_ready = mbar_test_wait(kv_full + (Gq & (kStages - 1)), (Gq / kStages) & 1) &&
+                                (Gq == 0 || mbar_test_wait(s_free, (Gq - 1) & 1)) &&
+                                (jq > 0 || mbar_test_wait(q_full, (kq - k0) & 1));
+          if (__all_sync(kFull, qk_ready)) {
+            do_pv = false;
+            break;
+          }
+          if (!ALA_MLA_SPIN) __nanosleep(32);
+          if ((it & 255u) == 0) {
+            if (*(volatile int*)status != 0) ok = false;
+            else if (global_timer_ns() - t0 > ALA_WAIT_LIMIT_NS) {
+              atomicCAS(status, 0, kDevTimeoutPFull);
+              ok = false;
+            }
+            if (__any_sync(kFull, !ok)) {
+              ok = false;
+              break;
+            }
           }
         }
-        commit(s_full);
+        if (!ok) break;
       }
-      if (j >= 1) {
-        const int jj = j - 1;
-        if (!wait_all(p_full, jj & 1, kDevTimeoutPFull)) break;
+      if (do_pv) {
+        if (!wait_mma(p_full, Gp & 1, status, kDevTimeoutPFull)) break;
         tc_fence_after();
         if (leader) {
-          const uint64_t v0 = dv + (uint64_t)((jj & 1) * kKvBytes >> 4);
+          const uint64_t v0 = dv + (uint64_t)(((Gp & (kStages - 1)) * kKvBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < kTileKeys / 16; ++kk) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               // V = ctKV columns [256h, 256h+256): four 64-wide column blocks, MN-major
               mma_ss(tmem + ((uint32_t)(16 * h) << 16), dp + ((kk * 32) >> 4),
-                     v0 + ((4 * h * kBlk + kk * 16 * 128) >> 4), idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u, false);
+                     v0 + ((4 * h * kKvBlk + kk * 16 * 128) >> 4), idesc_pv, (jp > 0 || kk > 0) ? 1u : 0u, false);
             }
           }
+          mma_commit(kv_empty + (Gp & (kStages - 1)));
+          mma_commit(o_done);
         }
-        commit(kv_empty + (jj & 1));
-        commit(o_done);
+        __syncwarp();
+        ++Gp;
+        if (++jp == np) {
+          ++kp;
+          jp = 0;
+          np = kp < k1 ? p.pieces[kp].n_tiles : 0;
+        }
+      } else {
+        if (!wait_mma(kv_full + (Gq & (kStages - 1)), (Gq / kStages) & 1, status, kDevTimeoutKFull)) break;
+        if (Gq >= 1 && !wait_mma(s_free, (Gq - 1) & 1, status, kDevTimeoutSFree)) break;
+        if (jq == 0 && !wait_mma(q_full, (kq - k0) & 1, status, kDevTimeoutQ)) break;
+        tc_fence_after();
+        if (leader) {
+          const uint64_t kt = dk + (uint64_t)(((Gq & (kStages - 1)) * kKvBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < 576 / 16; ++kk) {
+            mma_ss(tmem + kSCol, dq + (uint64_t)(((kk >> 2) * kQBlk + (kk & 3) * 32) >> 4),
+                   kt + (uint64_t)(((kk >> 2) * kKvBlk + (kk & 3) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u, false);
+          }
+          mma_commit(s_full);
+        }
+        __syncwarp();
+        ++Gq;
+        if (++jq == nq) {
+          ++kq;
+          jq = 0;
+          nq = kq < k1 ? p.pieces[kq].n_tiles : 0;
+        }
       }
     }
-    commit(fin);
-    wait_all(fin, 0, kDevTimeoutFinal);
+    if (leader) mma_commit(fin);
+    __syncwarp();
+    wait_all(fin, 0, status, kDevTimeoutFinal);
   } else {
     // ------------------------------------------------------------ softmax / epilogue
     const bool upper = lane >= 16;            // lanes 16..31 hold the upper 256 output columns
-    const int hl = (warp * 16) + (lane & 15); // head within the group
-    const int head = u.group * kHeadsPerCta + hl;
+    const int hr = (warp * 16) + (lane & 15); // row within the CTA: token t_local, head h0 + hl
+    const int t_local = hr / p.hpc;
+    const int head = h0 + (hr - t_local * p.hpc);
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t stage_row = smem_addr(sQ) + hr * 128;  // this row in each 8 KB staging box
+    const int sw = hr & 7;                                // 128-byte swizzle of the row's 16-byte chunks
     const float scale = p.scale_log2;
     const bool raw_max = scale > 0.f;  // max of the raw scores, scale folded into the exponent
-    float m_run = -INFINITY;
-    float l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full, j & 1, status, kDevTimeoutSFull));
-      if (!ok) break;
-      tc_fence_after();
-      float x[kTileKeys];
-#pragma unroll
-      for (int c32 = 0; c32 < kTileKeys / 32; ++c32) {
-        uint32_t regs[32];
-        tmem_ld32(tmem + lane_base + kSCol + c32 * 32, regs);
-        tmem_ld_wait();
-#pragma unroll
-        for (int c = 0; c < 32; ++c) x[c32 * 32 + c] = __uint_as_float(regs[c]);
-      }
-      tc_fence_before();
-      mbar_arrive(s_free);
-      const int lim = u.last_key - (u.kv_begin + j * kTileKeys);  // columns c <= lim are allowed
-      if (!raw_max) {
-#pragma unroll
-        for (int c = 0; c < kTileKeys; ++c) x[c] *= scale;
-      }
-      if (__any_sync(0xffffffffu, lim < kTileKeys - 1)) {  // only a range's last tile can hold masked keys
-#pragma unroll
-        for (int c = 0; c < kTileKeys; ++c) x[c] = (c > lim) ? -INFINITY : x[c];
-      }
-      float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
-#pragma unroll
-      for (int c = 4; c < kTileKeys; c += 8) {
-        mx0 = max3(mx0, x[c], x[c + 1]);
-        mx1 = max3(mx1, x[c + 2], x[c + 3]);
-        mx2 = max3(mx2, x[c + 4], x[c + 5]);
-        mx3 = max3(mx3, x[c + 6], x[c + 7]);
-      }
-      float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-      if (raw_max) mx *= scale;
-      const float m_new = fmaxf(m_run, mx);
-      float alpha = 1.f;
-      if (m_new - m_run > kRescaleThreshold) {
-        alpha = fast_exp2(m_run - m_new);
-        m_run = m_new;
-      }
-      const float m_base = (m_run == -INFINITY) ? 0.f : m_run;
-      // P = 2^(x*scale - m), a pair of columns at a time (-inf masked keys give exactly 0)
-      const uint64_t scale2 = f2pack(raw_max ? scale : 1.f, raw_max ? scale : 1.f);
-      const uint64_t negm2 = f2pack(-m_base, -m_base);
-      uint64_t acc0 = f2pack(0.f, 0.f), acc1 = f2pack(0.f, 0.f);
-      uint32_t pk[kTileKeys / 2];
-#pragma unroll
-      for (int c = 0; c < kTileKeys; c += 2) {
-        float e0, e1;
-        f2unpack(fma_x2(f2pack(x[c], x[c + 1]), scale2, negm2), e0, e1);
-        e0 = fast_exp2(e0);
-        e1 = fast_exp2(e1);
-        if ((c >> 1) & 1) acc1 = add_x2(acc1, f2pack(e0, e1));
-        else acc0 = add_x2(acc0, f2pack(e0, e1));
-        pk[c >> 1] = pack2(e0, e1, (T*)nullptr);
-      }
-      float s0, s1;
-      f2unpack(add_x2(acc0, acc1), s0, s1);
-      l_run = l_run * alpha + (s0 + s1);
-      if (j >= 1) {
-        ok = __all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, status, kDevTimeoutODone));
+    int G = 0;  // tiles consumed
+    int R = 0;  // output staging rounds
+    for (int k = k0; k < k1 && ok; ++k) {
+      const MlaPiece pc = p.pieces[k];
+      const int row_last = pc.last + t_local;
+      float m_run = -INFINITY;
+      float l_run = 0.f;
+      for (int j = 0; j < pc.n_tiles; ++j, ++G) {
+        ok = wait_smx(s_full, G & 1, status, kDevTimeoutSFull);
         if (!ok) break;
         tc_fence_after();
-        // lanes 16..31 scale the upper half of the heads owned by lanes 0..15
-        const float a_row = __shfl_sync(0xffffffffu, alpha, lane & 15);
-        if (__any_sync(0xffffffffu, a_row != 1.f)) {
+        float x[kTileKeys];
+        {
+          uint32_t regs[kTileKeys / 32][32];
 #pragma unroll
-          for (int c32 = 0; c32 < 256 / 32; ++c32) {
-            uint32_t regs[32];
-            const uint32_t addr = tmem + lane_base + c32 * 32;
-            tmem_ld32(addr, regs);
-            tmem_ld_wait();
+          for (int c32 = 0; c32 < kTileKeys / 32; ++c32) tmem_ld32(tmem + lane_base + kSCol + c32 * 32, regs[c32]);
+          tmem_ld_wait();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) regs[c] = __float_as_uint(__uint_as_float(regs[c]) * a_row);
-            tmem_st32(addr, regs);
-          }
-          tmem_st_wait();
+          for (int c = 0; c < kTileKeys; ++c) x[c] = __uint_as_float(regs[c >> 5][c & 31]);
         }
-      }
-      if (!upper) {
-        // P row hl: 64 keys x 16 bit = 128 bytes, K-major 128B-swizzled
-        const uint32_t prow = smem_addr(sP) + hl * 128;
+        tc_fence_before();
+        mbar_arrive(s_free);
+        const int lim = row_last - (pc.kv_begin + j * kTileKeys);  // columns c <= lim are allowed
+        if (!raw_max) {
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          st_shared_v4(prow + ((ch ^ (hl & 7)) << 4), make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]));
+          for (int c = 0; c < kTileKeys; ++c) x[c] *= scale;
+        }
+        if (__any_sync(kFull, lim < kTileKeys - 1)) {  // only a range's last tiles can hold masked keys
+#pragma unroll
+          for (int c = 0; c < kTileKeys; ++c) x[c] = (c > lim) ? -INFINITY : x[c];
+        }
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kTileKeys; c += 8) {
+          mx0 = max3(mx0, x[c], x[c + 1]);
+          mx1 = max3(mx1, x[c + 2], x[c + 3]);
+          mx2 = max3(mx2, x[c + 4], x[c + 5]);
+          mx3 = max3(mx3, x[c + 6], x[c + 7]);
+        }
+        float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        if (raw_max) mx *= scale;
+        const float m_new = fmaxf(m_run, mx);
+        float alpha = 1.f;
+        if (m_new - m_run > kRescaleThreshold) {  // false while both are -inf
+          alpha = fast_exp2(m_run - m_new);
+          m_run = m_new;
+        }
+        const float m_base = (m_run == -INFINITY) ? 0.f : m_run;
+        // P = 2^(x*scale - m), a pair of columns at a time (-inf masked keys give exactly 0)
+        const uint64_t scale2 = f2pack(raw_max ? scale : 1.f, raw_max ? scale : 1.f);
+        const uint64_t negm2 = f2pack(-m_base, -m_base);
+        uint64_t acc0 = f2pack(0.f, 0.f), acc1 = f2pack(0.f, 0.f);
+        uint32_t pk[kTileKeys / 2];
+#pragma unroll
+        for (int c = 0; c < kTileKeys; c += 2) {
+          float e0, e1;
+          f2unpack(fma_x2(f2pack(x[c], x[c + 1]), scale2, negm2), e0, e1);
+          e0 = fast_exp2(e0);
+          e1 = fast_exp2(e1);
+          if ((c >> 1) & 1) acc1 = add_x2(acc1, f2pack(e0, e1));
+          else acc0 = add_x2(acc0, f2pack(e0, e1));
+          pk[c >> 1] = pack2(e0, e1, (T*)nullptr);
+        }
+        float s0, s1;
+        f2unpack(add_x2(acc0, acc1), s0, s1);
+        l_run = l_run * alpha + (s0 + s1);
+        if (j >= 1) {
+          ok = wait_smx(o_done, (G - 1) & 1, status, kDevTimeoutODone);
+          if (!ok) break;
+          tc_fence_after();
+          // lanes 16..31 scale the upper half of the rows owned by lanes 0..15
+          const float a_row = __shfl_sync(kFull, alpha, lane & 15);
+          if (__any_sync(kFull, a_row != 1.f)) {
+#pragma unroll
+            for (int c32 = 0; c32 < 256 / 32; ++c32) {
+              uint32_t regs[32];
+              const uint32_t addr = tmem + lane_base + c32 * 32;
+              tmem_ld32(addr, regs);
+              tmem_ld_wait();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) regs[c] = __float_as_uint(__uint_as_float(regs[c]) * a_row);
+              tmem_st32(addr, regs);
+            }
+            tmem_st_wait();
+          }
+        }
+        if (!upper) {
+          // P row hr: kTileKeys keys x 16 bit = the first kTileKeys/8 16-byte chunks of a 128B-swizzled row
+          const uint32_t prow = smem_addr(sP) + hr * 128;
+#pragma unroll
+          for (int ch = 0; ch < kTileKeys / 8; ++ch)
+            st_shared_v4(prow + ((ch ^ sw) << 4), make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]));
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(p_full);
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(p_full);
-    }
-    if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(o_done, (n - 1) & 1, status, kDevTimeoutODone));
-    if (ok) {
+      if (!ok) break;
+      // ---- epilogue of the piece: O / l into the staging boxes, TMA stores, then the next query
+      ok = wait_smx(o_done, (G - 1) & 1, status, kDevTimeoutODone);
+      if (!ok) break;
       tc_fence_after();
-      const float l_row = __shfl_sync(0xffffffffu, l_run, lane & 15);
-      const float m_row = __shfl_sync(0xffffffffu, m_run, lane & 15);
-      const float inv_l = 1.f / l_row;
-      const int col0 = upper ? 256 : 0;
-      if (u.part < 0) {
-        T* orow = reinterpret_cast<T*>(p.out) + ((size_t)u.token * p.heads + head) * kDNope + col0;
+      const float l_row = __shfl_sync(kFull, l_run, lane & 15);
+      const float m_row = __shfl_sync(kFull, m_run, lane & 15);
+      // a row whose allowed keys all lie before this range (possible only in a partial) contributes nothing
+      const bool empty = !(l_row > 0.f);
+      const float inv_l = empty ? 0.f : 1.f / l_row;
+      const float lse_row = empty ? -INFINITY : (m_row == -INFINITY ? 0.f : m_row) * kLn2 + logf(l_row);
+      const uint32_t half_box = upper ? 4u * kQBlk : 0u;
+      const bool final_out = pc.part < 0;
+      const int n_rounds = final_out ? 1 : 2;
+      for (int r = 0; r < n_rounds && ok; ++r, ++R) {
+        // the previous round's boxes must have been read by its stores
+        if (R > 0 && !(ok = wait_all(st_free, (R - 1) & 1, status, kDevTimeoutFinal))) break;
+        if (final_out) {
+          // output in T: box (u, b) holds columns 256u + 64b .. +63 of the 64 rows
 #pragma unroll
-        for (int c32 = 0; c32 < 8; ++c32) {
-          uint32_t regs[32];
-          tmem_ld32(tmem + lane_base + c32 * 32, regs);
-          tmem_ld_wait();
+          for (int b = 0; b < 4; ++b) {
+            uint32_t ra[32], rb[32];
+            tmem_ld32(tmem + lane_base + b * 64, ra);
+            tmem_ld32(tmem + lane_base + b * 64 + 32, rb);
+            tmem_ld_wait();
+            const uint32_t box = stage_row + half_box + b * kQBlk;
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4) {
-            uint4 v;
-            v.x = pack2(__uint_as_float(regs[v4 * 8 + 0]) * inv_l, __uint_as_float(regs[v4 * 8 + 1]) * inv_l, (T*)nullptr);
-            v.y = pack2(__uint_as_float(regs[v4 * 8 + 2]) * inv_l, __uint_as_float(regs[v4 * 8 + 3]) * inv_l, (T*)nullptr);
-            v.z = pack2(__uint_as_float(regs[v4 * 8 + 4]) * inv_l, __uint_as_float(regs[v4 * 8 + 5]) * inv_l, (T*)nullptr);
-            v.w = pack2(__uint_as_float(regs[v4 * 8 + 6]) * inv_l, __uint_as_float(regs[v4 * 8 + 7]) * inv_l, (T*)nullptr);
-            *reinterpret_cast<uint4*>(orow + c32 * 32 + v4 * 8) = v;
+            for (int c = 0; c < 8; ++c) {
+              const uint32_t* q = c < 4 ? ra + 8 * c : rb + 8 * (c - 4);
+              uint4 v;
+              v.x = pack2(__uint_as_float(q[0]) * inv_l, __uint_as_float(q[1]) * inv_l, (T*)nullptr);
+              v.y = pack2(__uint_as_float(q[2]) * inv_l, __uint_as_float(q[3]) * inv_l, (T*)nullptr);
+              v.z = pack2(__uint_as_float(q[4]) * inv_l, __uint_as_float(q[5]) * inv_l, (T*)nullptr);
+              v.w = pack2(__uint_as_float(q[6]) * inv_l, __uint_as_float(q[7]) * inv_l, (T*)nullptr);
+              st_shared_v4(box + ((c ^ sw) << 4), v);
+            }
+          }
+        } else {
+          // fp32 partial, round r: box (u, b) holds columns 256u + 32(4r + b) .. +31
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            uint32_t ra[32];
+            tmem_ld32(tmem + lane_base + (4 * r + b) * 32, ra);
+            tmem_ld_wait();
+            const uint32_t box = stage_row + half_box + b * kQBlk;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              st_shared_v4(box + ((c ^ sw) << 4),
+                           make_uint4(__float_as_uint(__uint_as_float(ra[4 * c + 0]) * inv_l),
+                                      __float_as_uint(__uint_as_float(ra[4 * c + 1]) * inv_l),
+                                      __float_as_uint(__uint_as_float(ra[4 * c + 2]) * inv_l),
+                                      __float_as_uint(__uint_as_float(ra[4 * c + 3]) * inv_l)));
           }
         }
-        if (!upper && p.lse) p.lse[(size_t)u.token * p.heads + head] = (m_row == -INFINITY ? 0.f : m_row) * kLn2 + logf(l_row);
-      } else {
-        float* prow = p.part_o + ((size_t)u.part * p.heads + head) * kDNope + col0;
-#pragma unroll
-        for (int c32 = 0; c32 < 8; ++c32) {
-          uint32_t regs[32];
-          tmem_ld32(tmem + lane_base + c32 * 32, regs);
-          tmem_ld_wait();
-#pragma unroll
-          for (int v4 = 0; v4 < 8; ++v4)
-            *reinterpret_cast<float4*>(prow + c32 * 32 + v4 * 4) =
-                make_float4(__uint_as_float(regs[v4 * 4 + 0]) * inv_l, __uint_as_float(regs[v4 * 4 + 1]) * inv_l,
-                            __uint_as_float(regs[v4 * 4 + 2]) * inv_l, __uint_as_float(regs[v4 * 4 + 3]) * inv_l);
+        fence_proxy_async_smem();
+        mbar_arrive(st_full);
+        if (threadIdx.x == 0) {
+          if (mbar_wait(st_full, R & 1, status, kDevTimeoutFinal)) {
+            for (int b = 0; b < 8; ++b) {
+              if (final_out)
+                tma_store_3d(&tmO, sQ + b * kQBlk, (b >> 2) * 256 + (b & 3) * 64, h0, pc.token0);
+              else
+                tma_store_3d(&tmPO, sQ + b * kQBlk, (b >> 2) * 256 + (4 * r + (b & 3)) * 32, h0, pc.part * p.tpc);
+            }
+            bulk_commit_group();
+            bulk_wait_read_all();
+          }
+          mbar_arrive(st_free);
         }
-        if (!upper)
-          p.part_lse[(size_t)u.part * p.heads + head] = (m_row == -INFINITY ? 0.f : m_row) * kLn2 + logf(l_row);
       }
+      if (!ok) break;
+      if (!upper) {
+        if (final_out) {
+          if (p.lse) p.lse[(size_t)(pc.token0 + t_local) * p.heads + head] = lse_row;
+        } else {
+          p.part_lse[((size_t)pc.part * p.tpc + t_local) * p.heads + head] = lse_row;
+        }
+      }
+      // the staging boxes have been read: the buffer takes the next piece's query
+      if (threadIdx.x == 0 && k + 1 < k1) load_query(sQ, q_full, &tmQn, &tmQr, h0, p.pieces[k + 1].token0);
     }
+    if (threadIdx.x == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -401,7 +585,7 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-// Merge of the partial results of one token's key splits by their lse:
+// Merge of the partial results of one token's key ranges by their lse:
 // lse = log sum_s exp(lse_s), O = sum_s exp(lse_s - lse) O_s.
 // One CTA per (token, 8 heads); one warp per head, 16 output columns per lane.
 template <typename T>
@@ -410,17 +594,18 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaCombine* work
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int head = blockIdx.y * 8 + warp;
   if (head >= p.heads) return;
+  auto row = [&](int s) { return ((size_t)(w.part_begin + s) * p.tpc + w.t_local) * p.heads + head; };
   float m = -INFINITY;
-  for (int s = 0; s < w.n_parts; ++s) m = fmaxf(m, p.part_lse[(size_t)(w.part_begin + s) * p.heads + head]);
+  for (int s = 0; s < w.n_parts; ++s) m = fmaxf(m, p.part_lse[row(s)]);
   float l = 0.f;
-  for (int s = 0; s < w.n_parts; ++s) l += __expf(p.part_lse[(size_t)(w.part_begin + s) * p.heads + head] - m);
+  for (int s = 0; s < w.n_parts; ++s) l += __expf(p.part_lse[row(s)] - m);
   const float lse = m + __logf(l);
   float acc[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
   for (int s = 0; s < w.n_parts; ++s) {
-    const size_t pr = (size_t)(w.part_begin + s) * p.heads + head;
-    const float wgt = __expf(p.part_lse[pr] - lse);
+    const size_t pr = row(s);
+    const float wgt = __expf(p.part_lse[pr] - lse);  // 0 for a part whose rows saw no allowed key
     const float4* src = reinterpret_cast<const float4*>(p.part_o + pr * kDNope);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -464,14 +649,16 @@ EncodeTiledFn encoder() {
   return fn;
 }
 
-// rank-2 or rank-3 map with a 64-element (128-byte) inner box and 128B swizzle
+// rank-2 or rank-3 map with a 128-byte inner box and 128B swizzle
 bool encode(CUtensorMap* map, void* base, int32_t dtype, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
             const cuuint32_t* box) {
   EncodeTiledFn enc = encoder();
   if (!enc) return false;
   cuuint32_t estr[3] = {1, 1, 1};
-  return enc(map, dtype == ALA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base,
-             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  const CUtensorMapDataType t = dtype == ALA_F16   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                : dtype == ALA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                                   : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return enc(map, t, rank, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -522,7 +709,7 @@ int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, co
       kRope->dims[3] != 64)
     return mfail(err, n, ALA_INVALID_SHAPE, "kRope must be [numBlocks, blockSize, 1, 64]");
   const int64_t bs = ctKV->dims[1];
-  if (!(bs > 0 && bs % 16 == 0 && (kTileKeys % bs == 0 || bs % kTileKeys == 0)))
+  if (!(bs > 0 && bs % 16 == 0 && (64 % bs == 0 || bs % 64 == 0)))  // also tiles both 32- and 64-key rings
     return mfail(err, n, ALA_UNSUPPORTED, "blockSize must be a multiple of 16 dividing 64, or a multiple of 64");
   if (attenOut->ndim != 3 || attenOut->dims[0] != tokens || attenOut->dims[1] != headNum || attenOut->dims[2] != 512)
     return mfail(err, n, ALA_INVALID_SHAPE, "attenOut must be [tokens, headNum, 512]");
@@ -582,55 +769,92 @@ int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, co
   plan->qs.assign(batch, 1);
   if (qs) plan->qs.assign(qs, qs + batch);
 
-  // ---- schedule: per token, its allowed keys split into ranges of chunk_tiles 64-key tiles
-  const int groups = headNum / kHeadsPerCta;
+  // ---- row blocks: tpc tokens x hpc heads, tpc the largest of 4, 2, 1 dividing every qseqlen
+  int32_t tpc = 4;
+  for (; tpc > 1; tpc >>= 1) {
+    bool divides = true;
+    for (int32_t b = 0; b < batch; ++b) divides = divides && plan->qs[b] % tpc == 0;
+    if (divides) break;
+  }
+  const int32_t hpc = kRows / tpc;
+  const int32_t groups = headNum / hpc;
+  plan->tpc = tpc;
+  plan->hpc = hpc;
+  plan->groups = groups;
+
+  // ---- chunks and their 32-key tiles, end to end
+  struct Chunk {
+    int32_t b, token0, last, tiles;
+  };
+  std::vector<Chunk> chunks;
   int64_t total_tiles = 0;
-  for (int32_t b = 0; b < batch; ++b)
-    for (int32_t t = 0; t < plan->qs[b]; ++t) total_tiles += (cl[b] - plan->qs[b] + t + 1 + kTileKeys - 1) / kTileKeys;
-  total_tiles *= groups;
-  // about three units per SM of a 148-SM part, each at least 8 tiles
-  const int64_t target_units = 148 * 3;
-  const int32_t chunk_tiles = (int32_t)std::max<int64_t>(8, (total_tiles + target_units - 1) / target_units);
-  std::vector<MlaUnit> units;
-  std::vector<MlaCombine> comb;
-  int32_t token = 0, parts = 0;
-  for (int32_t b = 0; b < batch; ++b) {
-    for (int32_t t = 0; t < plan->qs[b]; ++t, ++token) {
-      const int32_t last = cl[b] - plan->qs[b] + t;
-      const int32_t tiles = (last + 1 + kTileKeys - 1) / kTileKeys;
-      const int32_t splits = (tiles + chunk_tiles - 1) / chunk_tiles;
-      const int32_t part0 = splits > 1 ? parts : -1;
-      if (splits > 1) {
-        comb.push_back(MlaCombine{token, parts, splits, 0});
-        parts += splits;
-      }
-      for (int32_t s = 0; s < splits; ++s) {
-        const int32_t t0 = s * chunk_tiles;
-        const int32_t nt = std::min(chunk_tiles, tiles - t0);
-        for (int32_t g = 0; g < groups; ++g)
-          units.push_back(MlaUnit{b, token, t, g, t0 * kTileKeys, nt, last, splits > 1 ? part0 + s : -1});
-      }
+  for (int32_t b = 0, token = 0; b < batch; token += plan->qs[b], ++b) {
+    for (int32_t t0 = 0; t0 < plan->qs[b]; t0 += tpc) {
+      const int32_t last = cl[b] - plan->qs[b] + t0;           // the chunk's first token's last allowed key
+      const int32_t tiles = (last + tpc + kTileKeys - 1) / kTileKeys;  // keys 0 .. last + tpc - 1
+      chunks.push_back(Chunk{b, token + t0, last, tiles});
+      total_tiles += tiles;
     }
   }
-  std::stable_sort(units.begin(), units.end(), [](const MlaUnit& a, const MlaUnit& c) { return a.n_tiles > c.n_tiles; });
-  plan->n_work = (int32_t)units.size();
+  // ---- lanes: equal contiguous ranges of that sequence, one CTA per lane and group
+  const int64_t lanes_max = std::max<int64_t>(1, kPlannedSms / groups);
+  const int64_t per_lane = std::max<int64_t>(kMinLaneTiles, (total_tiles + lanes_max - 1) / lanes_max);
+  std::vector<MlaPiece> pieces;
+  std::vector<int32_t> piece_lane;
+  std::vector<MlaCombine> comb;
+  int32_t parts = 0, lane_id = 0;
+  int64_t pos = 0, lane_end = per_lane;
+  for (const Chunk& ch : chunks) {
+    const size_t first = pieces.size();
+    for (int32_t t = 0; t < ch.tiles;) {
+      const int32_t take = (int32_t)std::min<int64_t>(lane_end - pos, ch.tiles - t);
+      pieces.push_back(MlaPiece{ch.b, ch.token0, t * kTileKeys, take, ch.last, -1, {0, 0}});
+      piece_lane.push_back(lane_id);
+      pos += take;
+      t += take;
+      if (pos == lane_end) {
+        ++lane_id;
+        lane_end += per_lane;
+      }
+    }
+    const int32_t np = (int32_t)(pieces.size() - first);
+    if (np > 1) {
+      for (int32_t i = 0; i < np; ++i) pieces[first + i].part = parts + i;
+      for (int32_t t = 0; t < tpc; ++t) comb.push_back(MlaCombine{ch.token0 + t, parts, np, t});
+      parts += np;
+    }
+  }
+  const int32_t n_lanes = pieces.empty() ? 0 : piece_lane.back() + 1;
+  std::vector<int32_t> lane_off(n_lanes + 1, 0);
+  for (int32_t l = 0, i = 0; l <= n_lanes; ++l) {
+    while (i < (int32_t)pieces.size() && piece_lane[i] < l) ++i;
+    lane_off[l] = i;
+  }
+  plan->n_lanes = n_lanes;
+  plan->n_work = n_lanes * groups;
   plan->n_splits_total = parts;
   plan->n_combine = (int32_t)comb.size();
   auto align = [](uint64_t x) { return (x + 255) / 256 * 256; };
   plan->off_work = 256;
-  plan->off_rows = align(plan->off_work + sizeof(MlaUnit) * std::max<size_t>(units.size(), 1));
+  plan->off_lanes = align(plan->off_work + sizeof(MlaPiece) * std::max<size_t>(pieces.size(), 1));
+  plan->off_rows = align(plan->off_lanes + sizeof(int32_t) * lane_off.size());
   plan->off_part_lse = align(plan->off_rows + sizeof(MlaCombine) * std::max<size_t>(comb.size(), 1));
-  plan->off_part_o = align(plan->off_part_lse + sizeof(float) * (uint64_t)parts * headNum);
-  plan->ws_size = align(plan->off_part_o + sizeof(float) * (uint64_t)parts * headNum * kDNope);
+  const uint64_t part_rows = (uint64_t)parts * tpc * headNum;
+  plan->off_part_o = align(plan->off_part_lse + sizeof(float) * part_rows);
+  plan->ws_size = align(plan->off_part_o + sizeof(float) * part_rows * kDNope);
   plan->image_size = plan->off_part_lse;  // only the schedule is uploaded; partials are written by the kernel
   plan->image.assign(plan->image_size, 0);
-  std::memcpy(plan->image.data() + plan->off_work, units.data(), sizeof(MlaUnit) * units.size());
+  std::memcpy(plan->image.data() + plan->off_work, pieces.data(), sizeof(MlaPiece) * pieces.size());
+  std::memcpy(plan->image.data() + plan->off_lanes, lane_off.data(), sizeof(int32_t) * lane_off.size());
   std::memcpy(plan->image.data() + plan->off_rows, comb.data(), sizeof(MlaCombine) * comb.size());
   return ALA_OK;
 }
 
 int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size_t n) {
   if (reinterpret_cast<uintptr_t>(workspace) % 256) return mfail(err, n, ALA_INVALID_PARAM, "workspace must be 256-byte aligned");
+  if (plan->n_work == 0) return ALA_OK;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const cuuint32_t tpc = (cuuint32_t)plan->tpc, hpc = (cuuint32_t)plan->hpc;
   if (!plan->maps_ready) {
     const int es = 2;
     const cuuint64_t rows = (cuuint64_t)plan->num_blocks * plan->block_size;
@@ -639,7 +863,7 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
     cuuint64_t qn_str[2] = {512 * es, (cuuint64_t)plan->heads * 512 * es};
     cuuint64_t qr_dims[3] = {64, (cuuint64_t)plan->heads, (cuuint64_t)plan->tokens};
     cuuint64_t qr_str[2] = {64 * es, (cuuint64_t)plan->heads * 64 * es};
-    cuuint32_t q_box[3] = {64, kHeadsPerCta, 1};
+    cuuint32_t q_box[3] = {64, hpc, tpc};
     cuuint64_t kv_dims[2] = {512, rows};
     cuuint64_t kv_str[1] = {512 * es};
     cuuint64_t kr_dims[2] = {64, rows};
@@ -648,9 +872,20 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
     if (!encode(&plan->tmQn, plan->q_nope, plan->dtype, 3, qn_dims, qn_str, q_box) ||
         !encode(&plan->tmQr, plan->q_rope, plan->dtype, 3, qr_dims, qr_str, q_box) ||
         !encode(&plan->tmKV, plan->ct_kv, plan->dtype, 2, kv_dims, kv_str, kv_box) ||
-        !encode(&plan->tmKR, plan->k_rope, plan->dtype, 2, kr_dims, kr_str, kv_box))
+        !encode(&plan->tmKR, plan->k_rope, plan->dtype, 2, kr_dims, kr_str, kv_box) ||
+        !encode(&plan->tmO, plan->out, plan->dtype, 3, qn_dims, qn_str, q_box))
       return mfail(err, n, ALA_CUDA_ERROR, "cuTensorMapEncodeTiled failed (pointers must be 16-byte aligned)");
     plan->maps_ready = true;
+  }
+  if (plan->n_splits_total == 0) {
+    plan->tmPO = plan->tmO;  // never used: every piece writes the final output
+  } else if (plan->tmPO_base != ws + plan->off_part_o) {
+    cuuint64_t po_dims[3] = {512, (cuuint64_t)plan->heads, (cuuint64_t)plan->n_splits_total * tpc};
+    cuuint64_t po_str[2] = {512 * 4, (cuuint64_t)plan->heads * 512 * 4};
+    cuuint32_t po_box[3] = {32, hpc, tpc};
+    if (!encode(&plan->tmPO, ws + plan->off_part_o, ALA_F32, 3, po_dims, po_str, po_box))
+      return mfail(err, n, ALA_CUDA_ERROR, "cuTensorMapEncodeTiled failed for the partial-output map");
+    plan->tmPO_base = ws + plan->off_part_o;
   }
   if (!plan->pinned) {
     if (cudaHostAlloc(&plan->pinned, plan->image_size, cudaHostAllocDefault) == cudaSuccess)
@@ -663,24 +898,29 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
   if (cudaMemcpyAsync(workspace, plan->pinned ? plan->pinned : plan->image.data(), plan->image_size,
                       cudaMemcpyHostToDevice, stream) != cudaSuccess)
     return mfail(err, n, ALA_CUDA_ERROR, "schedule upload failed");
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
   MlaParams p{};
-  p.units = reinterpret_cast<const MlaUnit*>(ws + plan->off_work);
+  p.pieces = reinterpret_cast<const MlaPiece*>(ws + plan->off_work);
+  p.lane_off = reinterpret_cast<const int32_t*>(ws + plan->off_lanes);
   p.block_tables = plan->block_tables;
+  p.ct_kv = static_cast<const uint8_t*>(plan->ct_kv);
+  p.k_rope = static_cast<const uint8_t*>(plan->k_rope);
   p.out = plan->out;
   p.lse = plan->lse;
   p.part_o = reinterpret_cast<float*>(ws + plan->off_part_o);
   p.part_lse = reinterpret_cast<float*>(ws + plan->off_part_lse);
   p.status = reinterpret_cast<int*>(ws);
   p.heads = plan->heads;
+  p.groups = plan->groups;
+  p.tpc = plan->tpc;
+  p.hpc = plan->hpc;
   p.max_blocks = plan->max_blocks;
   p.block_size = plan->block_size;
   p.oob_row = (int32_t)(plan->num_blocks * plan->block_size);
   p.scale_log2 = plan->qk_scale * kLog2e;
   auto kern = plan->dtype == ALA_F16 ? mla_kernel<__half> : mla_kernel<__nv_bfloat16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-  if (e == cudaSuccess && plan->n_work > 0) {
-    kern<<<plan->n_work, 192, kSmem, stream>>>(plan->tmQn, plan->tmQr, plan->tmKV, plan->tmKR, p);
+  if (e == cudaSuccess) {
+    kern<<<plan->n_work, 192, kSmem, stream>>>(plan->tmQn, plan->tmQr, plan->tmKV, plan->tmKR, plan->tmO, plan->tmPO, p);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess && plan->n_combine > 0) {

@@ -19,13 +19,18 @@ struct MlaPlan {
   float* lse = nullptr;
   const int32_t* block_tables = nullptr;
   std::vector<int32_t> ctx, qs;
-  // schedule and workspace: [status | units | combine list | partial lse | partial O]
-  int32_t n_work = 0, n_splits_total = 0, n_combine = 0;
-  uint64_t ws_size = 0, off_work = 0, off_rows = 0, off_part_o = 0, off_part_lse = 0, image_size = 0;
-  std::vector<uint8_t> image;  // host copy of [status | units | combine list]
+  // row blocks of tpc tokens x hpc heads; groups = heads / hpc
+  int32_t tpc = 1, hpc = 64, groups = 1;
+  // schedule and workspace: [status | pieces | lane offsets | combine list | partial lse | partial O]
+  int32_t n_lanes = 0, n_work = 0, n_splits_total = 0, n_combine = 0;
+  uint64_t ws_size = 0, off_work = 0, off_lanes = 0, off_rows = 0, off_part_o = 0, off_part_lse = 0,
+           image_size = 0;
+  std::vector<uint8_t> image;  // host copy of [status | pieces | lane offsets | combine list]
   void* pinned = nullptr;      // page-locked copy of `image`, made on first run
   bool maps_ready = false;
-  CUtensorMap tmQn, tmQr, tmKV, tmKR;
+  CUtensorMap tmQn, tmQr, tmKV, tmKR, tmO;
+  CUtensorMap tmPO;                // partial-output map, bound to the workspace it was encoded for
+  const void* tmPO_base = nullptr;
   MlaPlan() = default;
   MlaPlan(const MlaPlan&) = delete;
   MlaPlan& operator=(const MlaPlan&) = delete;

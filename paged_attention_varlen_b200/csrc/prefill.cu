@@ -496,9 +496,9 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int c = 0; c < 128; ++c) x[c] = (c > lim) ? -INFINITY : x[c];
         }
-        float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-        for (int c = 4; c < 128; c += 8) {
+        for (int c = 0; c < 128; c += 8) {
           mx0 = max3(mx0, x[c], x[c + 1]);
           mx1 = max3(mx1, x[c + 2], x[c + 3]);
           mx2 = max3(mx2, x[c + 4], x[c + 5]);

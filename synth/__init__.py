@@ -229,8 +229,9 @@ def make_mla(name, context_lens, qs, heads, seed, rng=None, block_size=128, d_no
     rng = rng if rng is not None else np.random.Generator(np.random.PCG64(seed))
     context_lens = np.asarray(context_lens, dtype=np.int32)
     batch = len(context_lens)
-    q_seq_len = np.full(batch, qs, dtype=np.int32)
-    tokens = batch * qs
+    q_seq_len = np.broadcast_to(np.asarray(qs, dtype=np.int32), (batch,)).copy()  # one count or one per batch
+    tokens = int(q_seq_len.sum())
+    spec = bool((q_seq_len > 1).any())
     q_nope = _normal(rng, (tokens, heads, d_nope), sigma, dtype)
     q_rope = _normal(rng, (tokens, heads, d_rope), sigma, dtype)
     n_kv = int(context_lens.sum())
@@ -240,8 +241,8 @@ def make_mla(name, context_lens, qs, heads, seed, rng=None, block_size=128, d_no
     return MlaCase(name=name, dtype=dtype, q_nope=q_nope, q_rope=q_rope, ct_kv=ct_kv, k_rope=k_rope,
                    block_tables=bt, context_lens=context_lens, q_seq_len=q_seq_len, heads=heads,
                    qk_scale=1.0 / math.sqrt(d_nope + d_rope),
-                   calc_type=MLA_CALC_SPEC if qs > 1 else MLA_CALC_UNDEFINED,
-                   mask_type=MLA_MASK_SPEC if qs > 1 else MLA_MASK_UNDEFINED, block_size=block_size)
+                   calc_type=MLA_CALC_SPEC if spec else MLA_CALC_UNDEFINED,
+                   mask_type=MLA_MASK_SPEC if spec else MLA_MASK_UNDEFINED, block_size=block_size)
 
 
 def mla_decode_bf16(qs: int, seed=1004, batch=64, lo=1024, hi=16384, heads=128) -> MlaCase:

@@ -43,7 +43,7 @@ def _oracle(case, rows=None):
 
 
 @pytest.mark.parametrize("qs", [1, 4])
-@pytest.mark.parametrize("block_size", [16, 64, 128])
+@pytest.mark.parametrize("block_size", [16, 32, 64, 128])
 def test_mla_small_ragged(qs, block_size):
     ctx = np.array([qs, 63, 64, 65, 700, 1100], dtype=np.int32)
     case = synth.make_mla("small", ctx, qs, 128, 5 + qs, block_size=block_size)
@@ -56,6 +56,29 @@ def test_mla_small_ragged(qs, block_size):
 def test_mla_fp16_and_64_heads():
     ctx = np.array([300, 5, 900], dtype=np.int32)
     case = synth.make_mla("f16", ctx, 2, 64, 31, block_size=64, dtype=torch.float16)
+    out, lse, _ = _run(case)
+    ref, lref = _oracle(case)
+    check_out(out.reshape(-1, 512), ref)
+    check_lse(lse.reshape(-1), lref)
+
+
+def test_mla_mixed_qseqlen():
+    # qseqlen 1, 3, 4, 2: one query token per CTA row block, 64 heads of it
+    ctx = np.array([50, 700, 1300, 20], dtype=np.int32)
+    qs = np.array([1, 3, 4, 2], dtype=np.int32)
+    case = synth.make_mla("mixed", ctx, qs, 128, 43, block_size=32)
+    out, lse, _ = _run(case)
+    ref, lref = _oracle(case)
+    check_out(out.reshape(-1, 512), ref)
+    check_lse(lse.reshape(-1), lref)
+
+
+def test_mla_spec_range_past_some_rows():
+    # four speculative tokens share each CTA; the second batch's key range is cut just before its
+    # last 32-key tile (keys 128..), which only its last token may see, so three of the four tokens
+    # have no allowed key in that range and their partial carries lse = -inf
+    ctx = np.array([100, 129, 300], dtype=np.int32)
+    case = synth.make_mla("spec_cut", ctx, 4, 128, 44, block_size=32)
     out, lse, _ = _run(case)
     ref, lref = _oracle(case)
     check_out(out.reshape(-1, 512), ref)
