@@ -7,10 +7,8 @@
 // Rows.  Every MMA has M = 64 rows: tpc consecutive query tokens of one batch
 // times 64/tpc heads (tpc = 4, 2 or 1: the largest that divides every batch's
 // qseqlen), so the speculative tokens of a batch share each cache tile the CTA
-// stages.  The 512-wide fp32 output of 64 rows is kept as two 256-column
-// accumulators in the two lane halves of the same tensor-memory columns.  The
-// heads / (64/tpc) "groups" of a batch read the same cache tiles; L2 serves
-// them once from HBM.
+// stages.  The heads / (64/tpc) "groups" of a batch read the same cache tiles;
+// L2 serves them once from HBM.
 //
 // Persistent schedule.  The key tiles of all chunks (a chunk = the tpc tokens
 // one CTA row block covers), laid end to end, are cut into equal contiguous
@@ -19,21 +17,27 @@
 // boundary leaves an fp32 partial (O, lse) per piece, which mla_combine_kernel
 // merges by lse (the merge the MLA page's ring mode returns the lse for).
 //
-//   warp 4      TMA producer: 64-key tiles of ctKV (512) and kRope (64)
-//               gathered through the block table into a two-deep ring (or
-//               32-key tiles, four deep, with ALA_MLA_TILE_KEYS=32), running
-//               ahead across piece boundaries and asking L2 for the tiles after.
-//   warp 5      tcgen05 issuer: S = Q K^T (64 x 64, K = 576) and O += P V with V
-//               the ctKV part of the same tile (two N = 256 halves); it issues
-//               whichever of the next QK and the next PV is ready first, so a
-//               tile's PV, which frees its ring slot, never waits behind the
-//               next tile's load.
-//   warps 0..3  softmax: lane l < 16 of warp w owns row 16w + l; it scales and
-//               masks its S row, keeps the online max / sum, writes P to shared
-//               memory and rescales O when the max grew by more than 2^8.  At
-//               the end of a piece all 128 threads normalise O into the Q
-//               buffer (free until the next piece's query) and one thread
-//               writes it out with TMA stores, then loads the next query.
+// Memory.  qNope (64 rows x 512) sits in tensor memory as the A operand of the
+// QK MMAs, so shared memory holds only qRope and a three-deep ring of 64-key
+// tiles (ctKV 64 KB + kRope 8 KB each).  Once S(j) is computed, the softmax
+// writes P(j) over tile j's kRope block; the PV of the tile reads P and V from
+// the same slot.  Tensor memory: lanes 0..15 of each 32-lane quarter hold qNope
+// (columns 0..255) and S (256..319); lanes 16..31 hold O (columns 0..511).
+//
+//   warp 4      TMA producer (one thread): ctKV + kRope tiles gathered through
+//               the block table (one 3-D box per tile when a tile lies in one
+//               page), running ahead across piece boundaries and asking L2 for
+//               the tiles after.
+//   warp 5      tcgen05 issuer (one thread): S = qNope K^T (TS, A in tensor
+//               memory) + qRope kRope^T (SS), and O += P V with V the ctKV part
+//               of the tile (two N = 256 halves); it issues whichever of the
+//               next QK and the next PV is ready.
+//   warps 0..3  softmax: lane l < 16 of warp w owns S row 16w + l (scale, mask,
+//               online max / sum, P); lane 16 + l owns the O row and rescales
+//               it when the max grew by more than 2^8.  At the end of a piece
+//               the O rows are normalised into the last tile's slot and one
+//               thread writes them out with TMA stores; then the 128 threads
+//               load the next chunk's query into tensor memory.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -55,37 +59,32 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
 
-#ifndef ALA_MLA_TILE_KEYS
-#define ALA_MLA_TILE_KEYS 64  // keys per ring slot: 64 (two slots) or 32 (four slots)
-#endif
-
 #ifndef ALA_MLA_PREFETCH_TILES
 #define ALA_MLA_PREFETCH_TILES 2  // the producer asks L2 for the tiles this far ahead of its loads
 #endif
 
-#ifndef ALA_MLA_SPIN
-#define ALA_MLA_SPIN 1  // 1: the MMA warp polls its barriers instead of sleeping on them; 2: softmax too
-#endif
-
 constexpr int kRows = 64;                  // attention rows per CTA: the M of every MMA
-constexpr int kTileKeys = ALA_MLA_TILE_KEYS;
-static_assert(kTileKeys == 32 || kTileKeys == 64, "tile of 32 or 64 keys");
+constexpr int kTileKeys = 64;
 constexpr int kDNope = 512;
-constexpr int kQBlk = kRows * 128;         // one 64-column block of the 64 query rows (8 KB)
-constexpr int kKvBlk = kTileKeys * 128;    // one 64-column block of a key tile
-constexpr int kQBytes = 9 * kQBlk;         // 64 rows x 576 x 2 B
-constexpr int kKvBytes = 9 * kKvBlk;       // 32 keys x 576 x 2 B
-constexpr int kPBytes = kRows * 128;       // P rows of 128 B (2 B per key)
-constexpr int kStages = 128 / kTileKeys;   // the ring holds 128 keys
-// q_full, kv_full[4], kv_empty[4], s_full, s_free, p_full, o_done, fin, st_full, st_free
-constexpr int kNBars = 1 + 2 * kStages + 7;
-constexpr int kSmem = 1024 + kQBytes + kStages * kKvBytes + kPBytes + kNBars * 8 + 16;
+constexpr int kBlk = kRows * 128;          // one 64-column block of 64 rows (query rows or keys): 8 KB
+constexpr int kQrBytes = kBlk;             // the 64 x 64 qRope rows (qNope lives in tensor memory)
+constexpr int kKvBytes = 9 * kBlk;         // 64 keys x 576 x 2 B: ctKV blocks 0..7, kRope block 8
+constexpr int kPOff = 8 * kBlk;            // P(j) overwrites tile j's kRope block once S(j) is computed
+constexpr int kStages = 3;
+// q_full, kv_full[3], kv_empty[3], p_full[3], pv_last, s_full, s_free, fin, st_full, st_free
+constexpr int kNBars = 1 + 3 * kStages + 6;
+constexpr int kSmem = 1024 + kQrBytes + kStages * kKvBytes + kNBars * 8 + 16;
 static_assert(kSmem <= 232448, "shared memory budget");
-static_assert(8 * kQBlk <= kQBytes, "the output staging (eight 8 KB boxes) must fit in the query buffer");
-constexpr uint32_t kSCol = 256;            // S: columns [256, 256 + kTileKeys), lanes of half 0
+static_assert(8 * kBlk <= kKvBytes, "the output staging (eight 8 KB boxes) must fit in a ring slot");
+// tensor memory: lanes 0..15 of each 32-lane quarter hold qNope (columns 0..255, the A operand of the
+// QK MMAs, which must accumulate at lane offset 0) and S (columns 256..319); lanes 16..31 hold O
+// (columns 0..511: output columns 0..255 and 256..511 as two N = 256 accumulators)
+constexpr uint32_t kQnCol = 0;
+constexpr uint32_t kSCol = 256;
+constexpr uint32_t kOLane = 16;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPlannedSms = 148;           // SMs of the part the schedule is cut for
-constexpr int kMinLaneTiles = 8;           // shortest key range worth a lane of its own
+constexpr int kMinLaneTiles = 4;           // shortest key range worth a lane of its own
 constexpr unsigned kFull = 0xffffffffu;
 
 struct MlaPiece {
@@ -109,6 +108,7 @@ struct MlaParams {
   const MlaPiece* pieces;
   const int32_t* lane_off;  // [n_lanes + 1]: lane l walks pieces [lane_off[l], lane_off[l+1])
   const int32_t* block_tables;
+  const uint8_t* q_nope;    // [tokens, heads, 512] (rows go to tensor memory through registers)
   const uint8_t* ct_kv;     // [numBlocks * blockSize, 512] (the L2 prefetch reads raw rows)
   const uint8_t* k_rope;    // [numBlocks * blockSize, 64]
   void* out;                // [tokens, heads, 512] (written by TMA stores and by the combine)
@@ -135,51 +135,62 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, __half*) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// The 64 x 576 query rows of one chunk: eight 64-column blocks of qNope, then qRope.
-__device__ __forceinline__ void load_query(uint8_t* sQ, uint64_t* q_full, const CUtensorMap* tmQn,
-                                           const CUtensorMap* tmQr, int h0, int token0) {
-  mbar_expect_tx(q_full, kQBytes);
-  for (int cb = 0; cb < 8; ++cb) tma_load_3d(sQ + cb * kQBlk, tmQn, q_full, cb * 64, h0, token0);
-  tma_load_3d(sQ + 8 * kQBlk, tmQr, q_full, 0, h0, token0);
-}
-
 // Warp-uniform wait on all lanes (each lane observes the phase itself).
 __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, int* status, int code) {
   return __all_sync(kFull, mbar_wait(bar, parity, status, code));
 }
-// The same for the waits on the QK -> softmax -> PV chain (ALA_MLA_SPIN: 1 = the MMA warp polls,
-// 2 = the softmax warps too).
-__device__ __forceinline__ bool wait_mma(uint64_t* bar, uint32_t parity, int* status, int code) {
-  if (ALA_MLA_SPIN >= 1) return __all_sync(kFull, mbar_wait_spin(bar, parity, status, code));
-  return __all_sync(kFull, mbar_wait(bar, parity, status, code));
-}
-__device__ __forceinline__ bool wait_smx(uint64_t* bar, uint32_t parity, int* status, int code) {
-  if (ALA_MLA_SPIN >= 2) return __all_sync(kFull, mbar_wait_spin(bar, parity, status, code));
-  return __all_sync(kFull, mbar_wait(bar, parity, status, code));
+
+// Loads one chunk's query into place: qNope rows into tensor memory (lanes 0..15 of the warp's
+// quarter, by the 128 softmax threads: row 16w + l is token t, head h of the chunk) and the qRope
+// rows into shared memory by TMA (thread 0).  Every thread arrives on q_full once.
+// Tensor-memory stores are warp-wide: lanes 16..31 write zeros into their columns 0..255, which
+// hold O, so this runs only while O is free (before the piece's first PV, after the last epilogue).
+__device__ __forceinline__ void load_query(const MlaParams& p, const CUtensorMap* tmQr, uint8_t* sQr,
+                                           uint64_t* q_full, uint32_t tmem_warp, int h0, int token0, int t_local,
+                                           int head, bool upper) {
+  if (threadIdx.x == 0) {
+    mbar_expect_tx_only(q_full, kQrBytes);  // thread 0 arrives below, with the others
+    tma_load_3d(sQr, tmQr, q_full, 0, h0, token0);
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(p.q_nope + (((size_t)(token0 + t_local) * p.heads + head) * kDNope) * 2);
+#pragma unroll
+  for (int c32 = 0; c32 < 8; ++c32) {  // 32 columns = 64 elements = 128 B of the row per store
+    uint32_t r[32];
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const uint4 w = upper ? make_uint4(0u, 0u, 0u, 0u) : __ldg(src + c32 * 8 + v);
+      r[4 * v + 0] = w.x;
+      r[4 * v + 1] = w.y;
+      r[4 * v + 2] = w.z;
+      r[4 * v + 3] = w.w;
+    }
+    tmem_st32(tmem_warp + kQnCol + c32 * 32, r);
+  }
+  tmem_st_wait();
+  tc_fence_before();
+  mbar_arrive(q_full);
 }
 
 template <typename T>
 __global__ void __launch_bounds__(192, 1)
-    mla_kernel(const __grid_constant__ CUtensorMap tmQn, const __grid_constant__ CUtensorMap tmQr,
-               const __grid_constant__ CUtensorMap tmKV, const __grid_constant__ CUtensorMap tmKR,
-               const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmPO,
-               const MlaParams p) {
+    mla_kernel(const __grid_constant__ CUtensorMap tmQr, const __grid_constant__ CUtensorMap tmKV,
+               const __grid_constant__ CUtensorMap tmKV3, const __grid_constant__ CUtensorMap tmKR,
+               const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmPO, const MlaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;  // the chunk's query rows; between pieces, the output staging area
-  uint8_t* sKV = sQ + kQBytes;
-  uint8_t* sP = sKV + kStages * kKvBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + kPBytes);
+  uint8_t* sQr = smem;  // the chunk's qRope rows
+  uint8_t* sKV = sQr + kQrBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + kStages * kKvBytes);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;             // [kStages]
-  uint64_t* kv_empty = bars + 1 + kStages;  // [kStages]
-  uint64_t* s_full = bars + 1 + 2 * kStages;
-  uint64_t* s_free = s_full + 1;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_done = s_full + 3;
-  uint64_t* fin = s_full + 4;
-  uint64_t* st_full = s_full + 5;  // the 128 softmax threads have written a round of output boxes
-  uint64_t* st_free = s_full + 6;  // the stores of a round have read their boxes
+  uint64_t* kv_full = bars + 1;               // [kStages] tile loaded
+  uint64_t* kv_empty = bars + 1 + kStages;    // [kStages] slot free again
+  uint64_t* p_full = bars + 1 + 2 * kStages;  // [kStages] P of the slot's tile written
+  uint64_t* pv_last = bars + 1 + 3 * kStages; // the last PV of a piece is complete
+  uint64_t* s_full = pv_last + 1;
+  uint64_t* s_free = pv_last + 2;
+  uint64_t* fin = pv_last + 3;
+  uint64_t* st_full = pv_last + 4;  // the 128 softmax threads have written a round of output boxes
+  uint64_t* st_free = pv_last + 5;  // the stores of a round have read their boxes
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNBars);
 
   const int warp = threadIdx.x >> 5;
@@ -191,15 +202,15 @@ __global__ void __launch_bounds__(192, 1)
   int* status = p.status;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    mbar_init(q_full, 128);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(kv_full + s, 1);
       mbar_init(kv_empty + s, 1);
+      mbar_init(p_full + s, 128);
     }
+    mbar_init(pv_last, 1);
     mbar_init(s_full, 1);
     mbar_init(s_free, 128);
-    mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
     mbar_init(fin, 1);
     mbar_init(st_full, 128);
     mbar_init(st_free, 1);
@@ -215,41 +226,40 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 4) {
-    // ------------------------------------------------------------ producer
-    // the whole warp walks the tiles (warp-uniform values); one elected lane issues the copies
-    const bool leader = elect_one();
-    if (leader) {
-      tma_prefetch_desc(&tmQn);
+    // ------------------------------------------------------------ producer (one elected thread)
+    if (elect_one()) {
       tma_prefetch_desc(&tmQr);
       tma_prefetch_desc(&tmKV);
+      tma_prefetch_desc(&tmKV3);
       tma_prefetch_desc(&tmKR);
-      if (k0 < k1) load_query(sQ, q_full, &tmQn, &tmQr, h0, p.pieces[k0].token0);
-    }
-    const int bs = p.block_size;
-    const int box_rows = bs < kTileKeys ? bs : kTileKeys;
-    bool ok = true;
-    int G = 0;  // tiles issued so far by this CTA
-    // L2 prefetch cursor (piece kf, tile jf, CTA tile Gf), kept ALA_MLA_PREFETCH_TILES tiles ahead of the loads
-    int kf = k0, jf = 0, Gf = 0;
-    MlaPiece pf = k0 < k1 ? p.pieces[k0] : MlaPiece{};
-    for (int k = k0; k < k1 && ok; ++k) {
-      const MlaPiece pc = p.pieces[k];
-      const int32_t* bt = p.block_tables + (size_t)pc.b * p.max_blocks;
-      const int n_pages = (pc.last + p.tpc + bs - 1) / bs;  // pages holding keys <= the chunk's last allowed key
-      for (int j = 0; j < pc.n_tiles; ++j) {
-        if (ALA_MLA_PREFETCH_TILES > 0) {
-          for (; kf < k1 && Gf <= G + ALA_MLA_PREFETCH_TILES; ++Gf) {
-            if (leader) {
-              const int32_t* btf = p.block_tables + (size_t)pf.b * p.max_blocks;
-              const int npf = (pf.last + p.tpc + bs - 1) / bs;
-              for (int r0 = 0; r0 < kTileKeys; r0 += box_rows) {
-                const int pos = pf.kv_begin + jf * kTileKeys + r0;
-                const int pg = pos / bs;
-                const size_t row = pg < npf ? (size_t)btf[pg] * bs + (pos - pg * bs) : (size_t)p.oob_row;
-                if (row < (size_t)p.oob_row) {  // a block index outside the cache is never touched
-                  bulk_prefetch_l2(p.ct_kv + row * 1024, box_rows * 1024);
-                  bulk_prefetch_l2(p.k_rope + row * 128, box_rows * 128);
-                }
+      const int bs = p.block_size;
+      const bool whole = bs % kTileKeys == 0;  // a tile lies in one page: one 3-D box holds its ctKV part
+      const int box_rows = bs < kTileKeys ? bs : kTileKeys;
+      int G = 0;  // tiles issued so far by this CTA
+      // L2 prefetch cursor (piece kf, tile jf, CTA tile Gf), kept ALA_MLA_PREFETCH_TILES tiles ahead of the loads
+      int kf = k0, jf = 0, Gf = 0;
+      MlaPiece pf = k0 < k1 ? p.pieces[k0] : MlaPiece{};
+      bool ok = true;
+      for (int k = k0; k < k1 && ok; ++k) {
+        const MlaPiece pc = p.pieces[k];
+        const int32_t* bt = p.block_tables + (size_t)pc.b * p.max_blocks;
+        const int n_pages = (pc.last + p.tpc + bs - 1) / bs;  // pages holding keys <= the chunk's last allowed key
+        if (k + 1 < k1) {  // the next chunk's qNope rows, for the softmax threads' loads at the piece boundary
+          const MlaPiece pn = p.pieces[k + 1];
+          for (int t = 0; t < p.tpc; ++t)
+            bulk_prefetch_l2(p.q_nope + (((size_t)(pn.token0 + t) * p.heads + h0) * kDNope) * 2, p.hpc * kDNope * 2);
+        }
+        for (int j = 0; j < pc.n_tiles; ++j) {
+          for (; ALA_MLA_PREFETCH_TILES > 0 && kf < k1 && Gf <= G + ALA_MLA_PREFETCH_TILES; ++Gf) {
+            const int32_t* btf = p.block_tables + (size_t)pf.b * p.max_blocks;
+            const int npf = (pf.last + p.tpc + bs - 1) / bs;
+            for (int r0 = 0; r0 < kTileKeys; r0 += box_rows) {
+              const int pos = pf.kv_begin + jf * kTileKeys + r0;
+              const int pg = pos / bs;
+              const size_t row = pg < npf ? (size_t)btf[pg] * bs + (pos - pg * bs) : (size_t)p.oob_row;
+              if (row < (size_t)p.oob_row) {  // a block index outside the cache is never touched
+                bulk_prefetch_l2(p.ct_kv + row * 1024, box_rows * 1024);
+                bulk_prefetch_l2(p.k_rope + row * 128, box_rows * 128);
               }
             }
             if (++jf == pf.n_tiles) {
@@ -257,167 +267,140 @@ __global__ void __launch_bounds__(192, 1)
               if (++kf < k1) pf = p.pieces[kf];
             }
           }
-        }
-        const int s = G & (kStages - 1);
-        if (G >= kStages && !wait_all(kv_empty + s, ((G / kStages) - 1) & 1, status, kDevTimeoutKEmpty)) {
-          ok = false;
-          break;
-        }
-        uint8_t* dst = sKV + s * kKvBytes;
-        if (leader) mbar_expect_tx(kv_full + s, kKvBytes);
-        const int j0 = pc.kv_begin + j * kTileKeys;
-        for (int r0 = 0; r0 < kTileKeys; r0 += box_rows) {
-          const int pos = j0 + r0;
-          const int pg = pos / bs;
-          const int row = pg < n_pages ? bt[pg] * bs + (pos - pg * bs) : p.oob_row;  // past the last page: zeros
-          if (leader) {
-            for (int cb = 0; cb < 8; ++cb) tma_load_2d(dst + cb * kKvBlk + r0 * 128, &tmKV, kv_full + s, cb * 64, row);
-            tma_load_2d(dst + 8 * kKvBlk + r0 * 128, &tmKR, kv_full + s, 0, row);
+          const int s = G % kStages;
+          if (G >= kStages && !mbar_wait(kv_empty + s, ((G / kStages) - 1) & 1, status, kDevTimeoutKEmpty)) {
+            ok = false;
+            break;
           }
+          uint8_t* dst = sKV + s * kKvBytes;
+          mbar_expect_tx(kv_full + s, kKvBytes);
+          const int j0 = pc.kv_begin + j * kTileKeys;
+          for (int r0 = 0; r0 < kTileKeys; r0 += box_rows) {
+            const int pos = j0 + r0;
+            const int pg = pos / bs;
+            const int row = pg < n_pages ? bt[pg] * bs + (pos - pg * bs) : p.oob_row;  // past the last page: zeros
+            if (whole) {
+              tma_load_3d(dst, &tmKV3, kv_full + s, 0, row, 0);  // [column block][key][64 elements]
+            } else {
+              for (int cb = 0; cb < 8; ++cb) tma_load_2d(dst + cb * kBlk + r0 * 128, &tmKV, kv_full + s, cb * 64, row);
+            }
+            tma_load_2d(dst + 8 * kBlk + r0 * 128, &tmKR, kv_full + s, 0, row);
+          }
+          ++G;
         }
-        ++G;
       }
+      // no copy may be in flight when the CTA exits
+      for (int t = G - kStages < 0 ? 0 : G - kStages; t < G; ++t)
+        mbar_wait(kv_full + (t % kStages), (t / kStages) & 1, status, kDevTimeoutKFull);
     }
-    // no copy may be in flight when the CTA exits
-    for (int t = G - kStages < 0 ? 0 : G - kStages; t < G; ++t)
-      mbar_wait(kv_full + (t & (kStages - 1)), (t / kStages) & 1, status, kDevTimeoutKFull);
   } else if (warp == 5) {
-    // ------------------------------------------------------------ MMA issuer
-    // the whole warp walks the schedule with warp-uniform descriptors; one elected lane issues
-    const bool leader = elect_one();
-    constexpr uint32_t fmt = std::is_same<T, __half>::value ? 0u : 1u;
-    constexpr uint32_t idesc_qk = instr_desc(fmt, false, false, kRows, kTileKeys);
-    constexpr uint32_t idesc_pv = instr_desc(fmt, false, true, kRows, 256);
-    // base descriptors; a step adds its byte offset >> 4 to the start-address field
-    const uint64_t dq = smem_desc_sw128(smem_addr(sQ), 16, 1024);
-    const uint64_t dk = smem_desc_sw128(smem_addr(sKV), 16, 1024);
-    const uint64_t dv = smem_desc(smem_addr(sKV), kKvBlk, 1024, 2);  // ctKV as the MN-major V operand
-    const uint64_t dp = smem_desc_sw128(smem_addr(sP), 16, 1024);
-    int total = 0;
-    for (int k = k0; k < k1; ++k) total += p.pieces[k].n_tiles;
-    // QK cursor: piece kq, tile jq of nq, tile Gq of the CTA; PV cursor likewise
-    int kq = k0, jq = 0, nq = k0 < k1 ? p.pieces[k0].n_tiles : 0, Gq = 0;
-    int kp = k0, jp = 0, np = nq, Gp = 0;
-    bool ok = true;
-    while (ok && Gp < total) {
-      // QK(Gq) needs its tile, the S buffer (softmax has read S(Gq-1)) and, first in a piece, the query;
-      // PV(Gp) needs P(Gp).  QK may lead PV by one tile: S and P are single-buffered.
-      const bool can_pv = Gp < Gq;
-      const bool can_qk = Gq < total && Gq - Gp < 2;
-      bool do_pv = can_pv;
-      if (can_pv && can_qk) {
-        const uint64_t t0 = global_timer_ns();
-        for (uint32_t it = 1;; ++it) {
-          if (__all_sync(kFull, mbar_test_wait(p_full, Gp & 1))) {
-            do_pv = true;
-            break;
+    // ------------------------------------------------------------ MMA issuer (one elected thread)
+    if (elect_one()) {
+      constexpr uint32_t fmt = std::is_same<T, __half>::value ? 0u : 1u;
+      constexpr uint32_t idesc_qk = instr_desc(fmt, false, false, kRows, kTileKeys);
+      constexpr uint32_t idesc_pv = instr_desc(fmt, false, true, kRows, 256);
+      // base descriptors; a step adds its byte offset >> 4 to the start-address field
+      const uint64_t dqr = smem_desc_sw128(smem_addr(sQr), 16, 1024);
+      const uint64_t dk = smem_desc_sw128(smem_addr(sKV), 16, 1024);
+      const uint64_t dv = smem_desc(smem_addr(sKV), kBlk, 1024, 2);          // ctKV as the MN-major V operand
+      const uint64_t dp = smem_desc_sw128(smem_addr(sKV + kPOff), 16, 1024);  // P in the slot's kRope block
+      int total = 0;
+      for (int k = k0; k < k1; ++k) total += p.pieces[k].n_tiles;
+      // QK cursor: piece kq, tile jq of nq, tile Gq of the CTA; PV cursor likewise
+      int kq = k0, jq = 0, nq = k0 < k1 ? p.pieces[k0].n_tiles : 0, Gq = 0;
+      int kp = k0, jp = 0, np = nq, Gp = 0;
+      bool ok = true;
+      uint64_t t_prog = global_timer_ns();  // last time something was issued
+      uint32_t it = 0;
+      while (ok && Gp < total) {
+        // QK(Gq) needs its tile, the S buffer (softmax is done with S(Gq-1)) and, first in a piece, the
+        // query; it may lead PV by one tile (S is single-buffered).  PV(Gp) needs P(Gp).
+        const int sq = Gq % kStages;
+        if (Gq < total && Gq - Gp < 2 && mbar_test_wait(kv_full + sq, (Gq / kStages) & 1) &&
+            (Gq == 0 || mbar_test_wait(s_free, (Gq - 1) & 1)) && (jq > 0 || mbar_test_wait(q_full, (kq - k0) & 1))) {
+          tc_fence_after();
+          const uint64_t so = (uint64_t)((sq * kKvBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kDNope / 16; ++kk)  // qNope from tensor memory (8 columns per 16 elements)
+            mma_ts(tmem + kSCol, tmem + kQnCol + kk * 8, dk + so + (uint64_t)(((kk >> 2) * kBlk + (kk & 3) * 32) >> 4),
+                   idesc_qk, kk > 0 ? 1u : 0u, false);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // qRope x kRope from shared memory
+            mma_ss(tmem + kSCol, dqr + (uint64_t)((kk * 32) >> 4), dk + so + (uint64_t)((8 * kBlk + kk * 32) >> 4),
+                   idesc_qk, 1u, false);
+          mma_commit(s_full);
+          ++Gq;
+          if (++jq == nq) {
+            ++kq;
+            jq = 0;
+            nq = kq < k1 ? p.pieces[kq].n_tiles : 0;
           }
-          const bool qk_ready = mbar_test_wait(kv_full + (Gq & (kStages - 1)), (Gq / kStages) & 1) &&
-                                (Gq == 0 || mbar_test_wait(s_free, (Gq - 1) & 1)) &&
-                                (jq > 0 || mbar_test_wait(q_full, (kq - k0) & 1));
-          if (__all_sync(kFull, qk_ready)) {
-            do_pv = false;
-            break;
-          }
-          if (!ALA_MLA_SPIN) __nanosleep(32);
-          if ((it & 255u) == 0) {
-            if (*(volatile int*)status != 0) ok = false;
-            else if (global_timer_ns() - t0 > ALA_WAIT_LIMIT_NS) {
-              atomicCAS(status, 0, kDevTimeoutPFull);
-              ok = false;
-            }
-            if (__any_sync(kFull, !ok)) {
-              ok = false;
-              break;
-            }
-          }
-        }
-        if (!ok) break;
-      }
-      if (do_pv) {
-        if (!wait_mma(p_full, Gp & 1, status, kDevTimeoutPFull)) break;
-        tc_fence_after();
-        if (leader) {
-          const uint64_t v0 = dv + (uint64_t)(((Gp & (kStages - 1)) * kKvBytes) >> 4);
+          t_prog = global_timer_ns();
+        } else if (Gp < Gq && mbar_test_wait(p_full + (Gp % kStages), (Gp / kStages) & 1)) {
+          tc_fence_after();
+          const uint64_t so = (uint64_t)(((Gp % kStages) * kKvBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < kTileKeys / 16; ++kk) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              // V = ctKV columns [256h, 256h+256): four 64-wide column blocks, MN-major
-              mma_ss(tmem + ((uint32_t)(16 * h) << 16), dp + ((kk * 32) >> 4),
-                     v0 + ((4 * h * kKvBlk + kk * 16 * 128) >> 4), idesc_pv, (jp > 0 || kk > 0) ? 1u : 0u, false);
+              // V = ctKV columns [256h, 256h+256): four 64-wide column blocks, MN-major; O at lane 16
+              mma_ss(tmem + (kOLane << 16) + 256 * h, dp + so + ((kk * 32) >> 4),
+                     dv + so + ((4 * h * kBlk + kk * 16 * 128) >> 4), idesc_pv, (jp > 0 || kk > 0) ? 1u : 0u, false);
             }
           }
-          mma_commit(kv_empty + (Gp & (kStages - 1)));
-          mma_commit(o_done);
-        }
-        __syncwarp();
-        ++Gp;
-        if (++jp == np) {
-          ++kp;
-          jp = 0;
-          np = kp < k1 ? p.pieces[kp].n_tiles : 0;
-        }
-      } else {
-        if (!wait_mma(kv_full + (Gq & (kStages - 1)), (Gq / kStages) & 1, status, kDevTimeoutKFull)) break;
-        if (Gq >= 1 && !wait_mma(s_free, (Gq - 1) & 1, status, kDevTimeoutSFree)) break;
-        if (jq == 0 && !wait_mma(q_full, (kq - k0) & 1, status, kDevTimeoutQ)) break;
-        tc_fence_after();
-        if (leader) {
-          const uint64_t kt = dk + (uint64_t)(((Gq & (kStages - 1)) * kKvBytes) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < 576 / 16; ++kk) {
-            mma_ss(tmem + kSCol, dq + (uint64_t)(((kk >> 2) * kQBlk + (kk & 3) * 32) >> 4),
-                   kt + (uint64_t)(((kk >> 2) * kKvBlk + (kk & 3) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u, false);
+          // the last tile of a piece: its slot is the epilogue's staging area and is freed by the epilogue
+          mma_commit(jp + 1 == np ? pv_last : kv_empty + (Gp % kStages));
+          ++Gp;
+          if (++jp == np) {
+            ++kp;
+            jp = 0;
+            np = kp < k1 ? p.pieces[kp].n_tiles : 0;
           }
-          mma_commit(s_full);
-        }
-        __syncwarp();
-        ++Gq;
-        if (++jq == nq) {
-          ++kq;
-          jq = 0;
-          nq = kq < k1 ? p.pieces[kq].n_tiles : 0;
+          t_prog = global_timer_ns();
+        } else if ((++it & 1023u) == 0) {
+          if (*(volatile int*)status != 0) ok = false;
+          else if (global_timer_ns() - t_prog > ALA_WAIT_LIMIT_NS) {
+            atomicCAS(status, 0, Gq - Gp < 2 && Gq < total ? kDevTimeoutKFull : kDevTimeoutPFull);
+            ok = false;
+          }
         }
       }
+      mma_commit(fin);
+      mbar_wait(fin, 0, status, kDevTimeoutFinal);
     }
-    if (leader) mma_commit(fin);
-    __syncwarp();
-    wait_all(fin, 0, status, kDevTimeoutFinal);
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    const bool upper = lane >= 16;            // lanes 16..31 hold the upper 256 output columns
+    // lanes 0..15 of warp w own S row 16w + l; lanes 16..31 own O row 16w + (l - 16)
+    const bool upper = lane >= 16;
     const int hr = (warp * 16) + (lane & 15); // row within the CTA: token t_local, head h0 + hl
     const int t_local = hr / p.hpc;
     const int head = h0 + (hr - t_local * p.hpc);
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t stage_row = smem_addr(sQ) + hr * 128;  // this row in each 8 KB staging box
-    const int sw = hr & 7;                                // 128-byte swizzle of the row's 16-byte chunks
+    const uint32_t tmem_warp = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int sw = hr & 7;  // 128-byte swizzle of the row's 16-byte chunks
     const float scale = p.scale_log2;
     const bool raw_max = scale > 0.f;  // max of the raw scores, scale folded into the exponent
     bool ok = true;
     int G = 0;  // tiles consumed
     int R = 0;  // output staging rounds
+    if (k0 < k1) load_query(p, &tmQr, sQr, q_full, tmem_warp, h0, p.pieces[k0].token0, t_local, head, upper);
     for (int k = k0; k < k1 && ok; ++k) {
       const MlaPiece pc = p.pieces[k];
       const int row_last = pc.last + t_local;
       float m_run = -INFINITY;
       float l_run = 0.f;
       for (int j = 0; j < pc.n_tiles; ++j, ++G) {
-        ok = wait_smx(s_full, G & 1, status, kDevTimeoutSFull);
+        ok = wait_all(s_full, G & 1, status, kDevTimeoutSFull);
         if (!ok) break;
         tc_fence_after();
         float x[kTileKeys];
         {
-          uint32_t regs[kTileKeys / 32][32];
-#pragma unroll
-          for (int c32 = 0; c32 < kTileKeys / 32; ++c32) tmem_ld32(tmem + lane_base + kSCol + c32 * 32, regs[c32]);
+          uint32_t regs[2][32];
+          tmem_ld32(tmem_warp + kSCol, regs[0]);
+          tmem_ld32(tmem_warp + kSCol + 32, regs[1]);
           tmem_ld_wait();
 #pragma unroll
           for (int c = 0; c < kTileKeys; ++c) x[c] = __uint_as_float(regs[c >> 5][c & 31]);
         }
-        tc_fence_before();
-        mbar_arrive(s_free);
         const int lim = row_last - (pc.kv_begin + j * kTileKeys);  // columns c <= lim are allowed
         if (!raw_max) {
 #pragma unroll
@@ -443,6 +426,29 @@ __global__ void __launch_bounds__(192, 1)
           alpha = fast_exp2(m_run - m_new);
           m_run = m_new;
         }
+        // lanes 16..31 scale the O rows whose S rows lanes 0..15 own
+        const float a_row = __shfl_sync(kFull, alpha, lane & 15);
+        if (j >= 1 && __any_sync(kFull, a_row != 1.f)) {
+          // O must hold P(j-1) V(j-1) before it is scaled, and no MMA may run while the warp-wide
+          // tensor-memory stores rewrite this quarter (lanes 0..15 store back qNope and S unchanged):
+          // S(j+1) is not computed before s_free below, and PV(j) waits for P(j)
+          ok = wait_all(kv_empty + ((G - 1) % kStages), ((G - 1) / kStages) & 1, status, kDevTimeoutODone);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll 2
+          for (int c32 = 0; c32 < 512 / 32; ++c32) {
+            uint32_t regs[32];
+            const uint32_t addr = tmem_warp + c32 * 32;
+            tmem_ld32(addr, regs);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) regs[c] = upper ? __float_as_uint(__uint_as_float(regs[c]) * a_row) : regs[c];
+            tmem_st32(addr, regs);
+          }
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        mbar_arrive(s_free);
         const float m_base = (m_run == -INFINITY) ? 0.f : m_run;
         // P = 2^(x*scale - m), a pair of columns at a time (-inf masked keys give exactly 0)
         const uint64_t scale2 = f2pack(raw_max ? scale : 1.f, raw_max ? scale : 1.f);
@@ -462,40 +468,21 @@ __global__ void __launch_bounds__(192, 1)
         float s0, s1;
         f2unpack(add_x2(acc0, acc1), s0, s1);
         l_run = l_run * alpha + (s0 + s1);
-        if (j >= 1) {
-          ok = wait_smx(o_done, (G - 1) & 1, status, kDevTimeoutODone);
-          if (!ok) break;
-          tc_fence_after();
-          // lanes 16..31 scale the upper half of the rows owned by lanes 0..15
-          const float a_row = __shfl_sync(kFull, alpha, lane & 15);
-          if (__any_sync(kFull, a_row != 1.f)) {
-#pragma unroll
-            for (int c32 = 0; c32 < 256 / 32; ++c32) {
-              uint32_t regs[32];
-              const uint32_t addr = tmem + lane_base + c32 * 32;
-              tmem_ld32(addr, regs);
-              tmem_ld_wait();
-#pragma unroll
-              for (int c = 0; c < 32; ++c) regs[c] = __float_as_uint(__uint_as_float(regs[c]) * a_row);
-              tmem_st32(addr, regs);
-            }
-            tmem_st_wait();
-          }
-        }
         if (!upper) {
-          // P row hr: kTileKeys keys x 16 bit = the first kTileKeys/8 16-byte chunks of a 128B-swizzled row
-          const uint32_t prow = smem_addr(sP) + hr * 128;
+          // P row hr into this tile's kRope block (S(j) is computed, so the block is dead): 64 keys x 16 bit
+          const uint32_t prow = smem_addr(sKV + (G % kStages) * kKvBytes + kPOff) + hr * 128;
 #pragma unroll
           for (int ch = 0; ch < kTileKeys / 8; ++ch)
             st_shared_v4(prow + ((ch ^ sw) << 4), make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]));
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(p_full);
+        mbar_arrive(p_full + (G % kStages));
       }
       if (!ok) break;
-      // ---- epilogue of the piece: O / l into the staging boxes, TMA stores, then the next query
-      ok = wait_smx(o_done, (G - 1) & 1, status, kDevTimeoutODone);
+      // ---- epilogue of the piece: O / l staged in the last tile's slot, TMA stores, then the next query
+      const int s_last = (G - 1) % kStages;
+      ok = wait_all(pv_last, (k - k0) & 1, status, kDevTimeoutODone);
       if (!ok) break;
       tc_fence_after();
       const float l_row = __shfl_sync(kFull, l_run, lane & 15);
@@ -504,47 +491,52 @@ __global__ void __launch_bounds__(192, 1)
       const bool empty = !(l_row > 0.f);
       const float inv_l = empty ? 0.f : 1.f / l_row;
       const float lse_row = empty ? -INFINITY : (m_row == -INFINITY ? 0.f : m_row) * kLn2 + logf(l_row);
-      const uint32_t half_box = upper ? 4u * kQBlk : 0u;
+      uint8_t* stage = sKV + s_last * kKvBytes;
+      const uint32_t stage_row = smem_addr(stage) + hr * 128;  // this row in each 8 KB staging box
       const bool final_out = pc.part < 0;
       const int n_rounds = final_out ? 1 : 2;
       for (int r = 0; r < n_rounds && ok; ++r, ++R) {
         // the previous round's boxes must have been read by its stores
         if (R > 0 && !(ok = wait_all(st_free, (R - 1) & 1, status, kDevTimeoutFinal))) break;
         if (final_out) {
-          // output in T: box (u, b) holds columns 256u + 64b .. +63 of the 64 rows
-#pragma unroll
-          for (int b = 0; b < 4; ++b) {
+          // output in T: box b holds columns 64b .. 64b+63 of the 64 rows (lanes 16..31 hold all of O)
+#pragma unroll 1
+          for (int b = 0; b < 8; ++b) {
             uint32_t ra[32], rb[32];
-            tmem_ld32(tmem + lane_base + b * 64, ra);
-            tmem_ld32(tmem + lane_base + b * 64 + 32, rb);
+            tmem_ld32(tmem_warp + b * 64, ra);
+            tmem_ld32(tmem_warp + b * 64 + 32, rb);
             tmem_ld_wait();
-            const uint32_t box = stage_row + half_box + b * kQBlk;
+            if (upper) {
+              const uint32_t box = stage_row + b * kBlk;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const uint32_t* q = c < 4 ? ra + 8 * c : rb + 8 * (c - 4);
-              uint4 v;
-              v.x = pack2(__uint_as_float(q[0]) * inv_l, __uint_as_float(q[1]) * inv_l, (T*)nullptr);
-              v.y = pack2(__uint_as_float(q[2]) * inv_l, __uint_as_float(q[3]) * inv_l, (T*)nullptr);
-              v.z = pack2(__uint_as_float(q[4]) * inv_l, __uint_as_float(q[5]) * inv_l, (T*)nullptr);
-              v.w = pack2(__uint_as_float(q[6]) * inv_l, __uint_as_float(q[7]) * inv_l, (T*)nullptr);
-              st_shared_v4(box + ((c ^ sw) << 4), v);
+              for (int c = 0; c < 8; ++c) {
+                const uint32_t* q = c < 4 ? ra + 8 * c : rb + 8 * (c - 4);
+                uint4 v;
+                v.x = pack2(__uint_as_float(q[0]) * inv_l, __uint_as_float(q[1]) * inv_l, (T*)nullptr);
+                v.y = pack2(__uint_as_float(q[2]) * inv_l, __uint_as_float(q[3]) * inv_l, (T*)nullptr);
+                v.z = pack2(__uint_as_float(q[4]) * inv_l, __uint_as_float(q[5]) * inv_l, (T*)nullptr);
+                v.w = pack2(__uint_as_float(q[6]) * inv_l, __uint_as_float(q[7]) * inv_l, (T*)nullptr);
+                st_shared_v4(box + ((c ^ sw) << 4), v);
+              }
             }
           }
         } else {
-          // fp32 partial, round r: box (u, b) holds columns 256u + 32(4r + b) .. +31
-#pragma unroll
-          for (int b = 0; b < 4; ++b) {
+          // fp32 partial, round r: box b holds columns 256r + 32b .. +31
+#pragma unroll 1
+          for (int b = 0; b < 8; ++b) {
             uint32_t ra[32];
-            tmem_ld32(tmem + lane_base + (4 * r + b) * 32, ra);
+            tmem_ld32(tmem_warp + 256 * r + 32 * b, ra);
             tmem_ld_wait();
-            const uint32_t box = stage_row + half_box + b * kQBlk;
+            if (upper) {
+              const uint32_t box = stage_row + b * kBlk;
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-              st_shared_v4(box + ((c ^ sw) << 4),
-                           make_uint4(__float_as_uint(__uint_as_float(ra[4 * c + 0]) * inv_l),
-                                      __float_as_uint(__uint_as_float(ra[4 * c + 1]) * inv_l),
-                                      __float_as_uint(__uint_as_float(ra[4 * c + 2]) * inv_l),
-                                      __float_as_uint(__uint_as_float(ra[4 * c + 3]) * inv_l)));
+              for (int c = 0; c < 8; ++c)
+                st_shared_v4(box + ((c ^ sw) << 4),
+                             make_uint4(__float_as_uint(__uint_as_float(ra[4 * c + 0]) * inv_l),
+                                        __float_as_uint(__uint_as_float(ra[4 * c + 1]) * inv_l),
+                                        __float_as_uint(__uint_as_float(ra[4 * c + 2]) * inv_l),
+                                        __float_as_uint(__uint_as_float(ra[4 * c + 3]) * inv_l)));
+            }
           }
         }
         fence_proxy_async_smem();
@@ -553,9 +545,9 @@ __global__ void __launch_bounds__(192, 1)
           if (mbar_wait(st_full, R & 1, status, kDevTimeoutFinal)) {
             for (int b = 0; b < 8; ++b) {
               if (final_out)
-                tma_store_3d(&tmO, sQ + b * kQBlk, (b >> 2) * 256 + (b & 3) * 64, h0, pc.token0);
+                tma_store_3d(&tmO, stage + b * kBlk, 64 * b, h0, pc.token0);
               else
-                tma_store_3d(&tmPO, sQ + b * kQBlk, (b >> 2) * 256 + (4 * r + (b & 3)) * 32, h0, pc.part * p.tpc);
+                tma_store_3d(&tmPO, stage + b * kBlk, 256 * r + 32 * b, h0, pc.part * p.tpc);
             }
             bulk_commit_group();
             bulk_wait_read_all();
@@ -571,8 +563,18 @@ __global__ void __launch_bounds__(192, 1)
           p.part_lse[((size_t)pc.part * p.tpc + t_local) * p.heads + head] = lse_row;
         }
       }
-      // the staging boxes have been read: the buffer takes the next piece's query
-      if (threadIdx.x == 0 && k + 1 < k1) load_query(sQ, q_full, &tmQn, &tmQr, h0, p.pieces[k + 1].token0);
+      // O has been read: the next chunk's query may go in (its qNope stores clobber O)
+      tc_fence_before();
+      if (k + 1 < k1) {
+        const MlaPiece pn = p.pieces[k + 1];
+        load_query(p, &tmQr, sQr, q_full, tmem_warp, h0, pn.token0, t_local, head, upper);
+      }
+      // the staging slot goes back to the producer once the stores have read it
+      if (threadIdx.x == 0) {
+        ok = mbar_wait(st_free, (R - 1) & 1, status, kDevTimeoutFinal);
+        mbar_arrive(kv_empty + s_last);
+      }
+      ok = __all_sync(kFull, ok);
     }
     if (threadIdx.x == 0) bulk_wait_all();
   }
@@ -869,7 +871,13 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
     cuuint64_t kr_dims[2] = {64, rows};
     cuuint64_t kr_str[1] = {64 * es};
     cuuint32_t kv_box[2] = {64, kv_box_rows};
-    if (!encode(&plan->tmQn, plan->q_nope, plan->dtype, 3, qn_dims, qn_str, q_box) ||
+    // ctKV seen as (64 elements, rows, 8 column blocks): one box is a whole 64-key tile, laid out
+    // [column block][key][64 elements] as the 128B-swizzled K-major operand wants it
+    cuuint64_t kv3_dims[3] = {64, rows, 8};
+    cuuint64_t kv3_str[2] = {512 * es, 64 * es};
+    cuuint32_t kv3_box[3] = {64, (cuuint32_t)kTileKeys, 8};
+    if (!encode(&plan->tmKV3, plan->ct_kv, plan->dtype, 3, kv3_dims, kv3_str, kv3_box) ||
+        !encode(&plan->tmQn, plan->q_nope, plan->dtype, 3, qn_dims, qn_str, q_box) ||
         !encode(&plan->tmQr, plan->q_rope, plan->dtype, 3, qr_dims, qr_str, q_box) ||
         !encode(&plan->tmKV, plan->ct_kv, plan->dtype, 2, kv_dims, kv_str, kv_box) ||
         !encode(&plan->tmKR, plan->k_rope, plan->dtype, 2, kr_dims, kr_str, kv_box) ||
@@ -902,6 +910,7 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
   p.pieces = reinterpret_cast<const MlaPiece*>(ws + plan->off_work);
   p.lane_off = reinterpret_cast<const int32_t*>(ws + plan->off_lanes);
   p.block_tables = plan->block_tables;
+  p.q_nope = static_cast<const uint8_t*>(plan->q_nope);
   p.ct_kv = static_cast<const uint8_t*>(plan->ct_kv);
   p.k_rope = static_cast<const uint8_t*>(plan->k_rope);
   p.out = plan->out;
@@ -920,7 +929,7 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
   auto kern = plan->dtype == ALA_F16 ? mla_kernel<__half> : mla_kernel<__nv_bfloat16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e == cudaSuccess) {
-    kern<<<plan->n_work, 192, kSmem, stream>>>(plan->tmQn, plan->tmQr, plan->tmKV, plan->tmKR, plan->tmO, plan->tmPO, p);
+    kern<<<plan->n_work, 192, kSmem, stream>>>(plan->tmQr, plan->tmKV, plan->tmKV3, plan->tmKR, plan->tmO, plan->tmPO, p);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess && plan->n_combine > 0) {
