@@ -310,8 +310,9 @@ __global__ void __launch_bounds__(192, 1)
       int kq = k0, jq = 0, nq = k0 < k1 ? p.pieces[k0].n_tiles : 0, Gq = 0;
       int kp = k0, jp = 0, np = nq, Gp = 0;
       bool ok = true;
-      uint64_t t_prog = global_timer_ns();  // last time something was issued
+      uint64_t t_prog = global_timer_ns();  // when the idle loop last saw progress
       uint32_t it = 0;
+      bool progressed = false;
       while (ok && Gp < total) {
         // QK(Gq) needs its tile, the S buffer (softmax is done with S(Gq-1)) and, first in a piece, the
         // query; it may lead PV by one tile (S is single-buffered).  PV(Gp) needs P(Gp).
@@ -335,7 +336,7 @@ __global__ void __launch_bounds__(192, 1)
             jq = 0;
             nq = kq < k1 ? p.pieces[kq].n_tiles : 0;
           }
-          t_prog = global_timer_ns();
+          progressed = true;
         } else if (Gp < Gq && mbar_test_wait(p_full + (Gp % kStages), (Gp / kStages) & 1)) {
           tc_fence_after();
           const uint64_t so = (uint64_t)(((Gp % kStages) * kKvBytes) >> 4);
@@ -356,10 +357,15 @@ __global__ void __launch_bounds__(192, 1)
             jp = 0;
             np = kp < k1 ? p.pieces[kp].n_tiles : 0;
           }
-          t_prog = global_timer_ns();
+          progressed = true;
         } else if ((++it & 1023u) == 0) {
+          const uint64_t now = global_timer_ns();
+          if (progressed) {
+            t_prog = now;
+            progressed = false;
+          }
           if (*(volatile int*)status != 0) ok = false;
-          else if (global_timer_ns() - t_prog > ALA_WAIT_LIMIT_NS) {
+          else if (now - t_prog > ALA_WAIT_LIMIT_NS) {
             atomicCAS(status, 0, Gq - Gp < 2 && Gq < total ? kDevTimeoutKFull : kDevTimeoutPFull);
             ok = false;
           }

@@ -16,7 +16,9 @@
 //                  O_b += P_b V_j         (TS MMA: P_b read from TMEM)
 //                in the order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so the
 //                tensor core works on one block while the other block's
-//                softmax runs.
+//                softmax runs.  P_b V_j goes in two halves of 64 keys: the
+//                first starts as soon as the softmax has written P for keys
+//                0..63, while it still computes the rest.
 //   warps 0..3,  softmax of block 0 / block 1: thread r owns row r (TMEM lane
 //   4..7         r).  It reads its S row, applies qkScale, the ALiBi bias and
 //                the causal / prefix-offset rule in registers (the mask is
@@ -43,6 +45,9 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 #ifndef ALA_POLY_PAIRS_OF_4
 #define ALA_POLY_PAIRS_OF_4 0  // of every 4 column pairs, how many take the FMA-pipe exp2 polynomial
+#endif
+#ifndef ALA_PREFILL_SPIN
+#define ALA_PREFILL_SPIN 0  // 1: the MMA warp polls its barriers instead of sleeping on them
 #endif
 
 template <typename T>
@@ -71,7 +76,7 @@ struct Cfg {
   static constexpr int KV_BYTES = 128 * D * ES;
   static constexpr int TBL_FLOATS = 160;  // per-warp sqrt-bias table: lane - column + 127 in [0, 159)
   static constexpr int TBL_BYTES = 8 * 2 * TBL_FLOATS * 4;
-  static constexpr int N_BARS = 19;
+  static constexpr int N_BARS = 21;
   static constexpr int SMEM = 1024 + 2 * Q_BYTES + 2 * STAGES * KV_BYTES + TBL_BYTES + N_BARS * 8 + 16;
   static constexpr uint32_t IDESC_QK = instr_desc(ElemFmt<T>::fmt, false, false, 128, 128);
   static constexpr uint32_t IDESC_PV = instr_desc(ElemFmt<T>::fmt, false, true, 128, D);
@@ -97,7 +102,7 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, __half*) {
 // column pairs, ALA_POLY_PAIRS_OF_4 take the FMA-pipe polynomial instead of MUFU.
 template <typename T, bool MASKED>
 __device__ __forceinline__ float exp_rows(const float (&x)[128], uint64_t scale2, uint64_t negm2, int lim,
-                                          uint32_t s_col) {
+                                          uint32_t s_col, uint64_t* p_lo) {
   constexpr bool kHalf = sizeof(T) == 2;
   constexpr int CHUNK = kHalf ? 64 : 32;  // columns per 32-register TMEM store
   uint64_t acc[4] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f), f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
@@ -134,6 +139,12 @@ __device__ __forceinline__ float exp_rows(const float (&x)[128], uint64_t scale2
       }
     }
     tmem_st32(s_col + h * 32, pk);
+    if (h == 128 / CHUNK / 2 - 1) {
+      // P of keys 0..63 is in place: the first half of P*V may start while the rest is computed
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_lo);
+    }
   }
   const uint64_t a = add_x2(add_x2(acc[0], acc[1]), add_x2(acc[2], acc[3]));
   float s0, s1;
@@ -184,11 +195,12 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* k_empty = bars + 5;   // [2]
   uint64_t* v_empty = bars + 7;   // [2]
   uint64_t* s_full = bars + 9;    // [2] per block
-  uint64_t* p_full = bars + 11;   // [2] per block
+  uint64_t* p_full = bars + 11;   // [2] per block: P of keys 64..127 written (all of P)
   uint64_t* pv_done = bars + 13;  // [2] per block
   uint64_t* o_done = bars + 15;   // [2] per block
   uint64_t* fin = bars + 17;
   uint64_t* q_empty = bars + 18;
+  uint64_t* p_lo = bars + 19;     // [2] per block: P of keys 0..63 written
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::N_BARS);
 
   const int warp = threadIdx.x >> 5;
@@ -208,6 +220,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(v_empty + s, 1);
       mbar_init(s_full + s, 1);
       mbar_init(p_full + s, 128);
+      mbar_init(p_lo + s, 128);
       mbar_init(pv_done + s, 1);
       mbar_init(o_done + s, 1);
     }
@@ -318,11 +331,11 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       };
-      auto issue_pv = [&](int b, int s, bool acc) {
+      auto issue_pv = [&](int b, int s, bool acc, int half) {
         if (leader) {
           const uint64_t v0 = dv + s * kKVStep;
 #pragma unroll
-          for (int kk = 0; kk < 128 / C::UK; ++kk) {
+          for (int kk = half * 64 / C::UK; kk < (half + 1) * 64 / C::UK; ++kk) {
             // P_b in TMEM over S_b: 8 columns per K step (two 16-bit values per column, or 8 tf32)
             mma_ts(tmem + 256 + b * D, tmem + b * 128 + kk * 8, v0 + ((kk * C::UK * 128) >> 4), C::IDESC_PV,
                    (acc || kk > 0) ? 1u : 0u, C::ES == 4);
@@ -333,6 +346,7 @@ __global__ void __launch_bounds__(384, 1)
         if (leader) mma_commit(bar);
       };
       auto wait_all = [&](uint64_t* bar, uint32_t parity, int code) {
+        if (ALA_PREFILL_SPIN) return __all_sync(0xffffffffu, mbar_wait_spin(bar, parity, status, code));
         return __all_sync(0xffffffffu, mbar_wait(bar, parity, status, code));
       };
       bool ok = true;
@@ -372,7 +386,7 @@ __global__ void __launch_bounds__(384, 1)
             const int nbt = b == 0 ? n0 : n1;
             if (j >= nbt) continue;
             const uint32_t ph = (b ? sp1 : sp0) + j;  // this block's barrier phase for tile j
-            if (!wait_all(p_full + b, ph & 1, kDevTimeoutPFull)) {
+            if (!wait_all(p_lo + b, ph & 1, kDevTimeoutPFull)) {
               ok = false;
               break;
             }
@@ -382,7 +396,13 @@ __global__ void __launch_bounds__(384, 1)
             }
             v_ready = true;
             tc_fence_after();
-            issue_pv(b, s, j > 0);
+            issue_pv(b, s, j > 0, 0);  // keys 0..63
+            if (!wait_all(p_full + b, ph & 1, kDevTimeoutPFull)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_pv(b, s, true, 1);   // keys 64..127
             commit(pv_done + b);
             const bool last_pv = (b == nb - 1) || (j >= n1);
             if (last_pv) commit(v_empty + s);
@@ -529,8 +549,9 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t scale2 = f2pack(raw_max ? scale : 1.f, raw_max ? scale : 1.f);
         const uint64_t negm2 = f2pack(-m_base, -m_base);
         // warp-uniform choice: exp_rows issues tcgen05.st, which all 32 lanes must execute together
-        const float row_sum = __any_sync(0xffffffffu, lim < 127) ? exp_rows<T, true>(x, scale2, negm2, lim, s_col)
-                                                                 : exp_rows<T, false>(x, scale2, negm2, lim, s_col);
+        const float row_sum = __any_sync(0xffffffffu, lim < 127)
+                                  ? exp_rows<T, true>(x, scale2, negm2, lim, s_col, p_lo + b)
+                                  : exp_rows<T, false>(x, scale2, negm2, lim, s_col, p_lo + b);
         l_run = l_run * alpha + row_sum;
         tmem_st_wait();
         tc_fence_before();
