@@ -210,10 +210,14 @@ ALA_API int varlen_attention_noalloc(const ala_tensor* query, const ala_tensor* 
  * qkDescale, pvDescale  must be NULL (int8 cache not built).
  * headNum     128 (multiple of 64 accepted); kvHeadNum must be 1.
  * maskType    UNDEFINED (0) with one token per batch, or SPEC (1).
- * calcType    UNDEFINED (0) or SPEC (1); RING and PREFILL return UNSUPPORTED.
+ * calcType    UNDEFINED (0), SPEC (1) or RING (2); PREFILL returns UNSUPPORTED.
+ *             RING (ring attention) computes the same attention over the keys
+ *             this call is given and requires lse, so that results over
+ *             disjoint key ranges can be merged with ala_lse_merge.
  * cacheMode   KROPE_CTKV (1) only; others return UNSUPPORTED.
  * attenOut    [tokens, headNum, 512], dtype of qNope, device.
- * lse         NULL or [tokens, headNum, 1] fp32, device (natural log).
+ * lse         NULL or [tokens, headNum, 1] fp32, device (natural log);
+ *             required with calcType RING (NULL_REQUIRED otherwise).
  * workspace   256-byte aligned; holds the schedule and, for key ranges split
  *             across CTAs, fp32 partial outputs merged by lse at the end.
  * ------------------------------------------------------------------------- */
@@ -225,6 +229,26 @@ ALA_API int atb_like_mla_get_workspace_size(
     ala_tensor* lse, uint64_t* workspaceSize, ala_op** op);
 
 ALA_API int atb_like_mla(void* workspace, uint64_t workspaceSize, ala_op* op, ala_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Merge of two partial attention results over disjoint key ranges by their
+ * log-sum-exp (ATB "MLA" page, parameter table, rows calcType (ring mode) and
+ * lse).  Per output row r:
+ *   lse[r] = log(exp(lseA[r]) + exp(lseB[r])),
+ *   out[r] = exp(lseA[r] - lse[r]) outA[r] + exp(lseB[r] - lse[r]) outB[r];
+ * a row whose lseA and lseB are both -inf gets lse = -inf and out = 0.
+ *
+ * outA, outB, out  same shape [..., d] (1 to 4 dims, 1 <= d <= 1024), same
+ *                  dtype (bf16, f16 or f32), device; rows = product of the
+ *                  leading dims.  Each is normalised over its own keys.
+ * lseA, lseB, lse  fp32 with one value per row (any shape of `rows`
+ *                  elements, e.g. [tokens, headNum, 1]), device, natural log.
+ * out / lse may be the same memory as outA / lseA or outB / lseB (in-place
+ * accumulation over a ring).  Runs asynchronously on `stream`; allocates
+ * nothing.  Returns a status code before any GPU work on invalid arguments.
+ * ------------------------------------------------------------------------- */
+ALA_API int ala_lse_merge(const ala_tensor* outA, const ala_tensor* lseA, const ala_tensor* outB,
+                          const ala_tensor* lseB, ala_tensor* out, ala_tensor* lse, ala_stream_t stream);
 
 #ifdef __cplusplus
 }

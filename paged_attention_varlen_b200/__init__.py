@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
         L.varlen_attention_noalloc.argtypes = [T, T, T, T, T, T, ctypes.c_int, ctypes.c_int32, ctypes.c_int32,
                                                ctypes.c_float, T, T, P]
         L.varlen_attention_noalloc.restype = ctypes.c_int
+        L.ala_lse_merge.argtypes = [T, T, T, T, T, T, P]
+        L.ala_lse_merge.restype = ctypes.c_int
         for f in ("atb_like_prefix_encoder", "varlen_attention", "atb_like_mla"):
             getattr(L, f).argtypes = [P, ctypes.c_uint64, P, P]
         for f in ("ala_workspace_status", "atb_like_prefix_encoder_get_workspace_size",
@@ -242,9 +244,25 @@ def plan_mla(q_nope, q_rope, ct_kv, k_rope, block_tables, context_lens, q_seq_le
 
 def atb_like_mla(q_nope, q_rope, ct_kv, k_rope, block_tables, context_lens, q_seq_len, heads, qk_scale,
                  mask_type=MLA_MASK_UNDEFINED, calc_type=MLA_CALC_UNDEFINED, return_lse=False):
+    return_lse = return_lse or calc_type == MLA_CALC_RING  # ring mode always returns the lse
     lse = (torch.empty((q_nope.shape[0], heads, 1), dtype=torch.float32, device=q_nope.device)
            if return_lse else None)
     op, out = plan_mla(q_nope, q_rope, ct_kv, k_rope, block_tables, context_lens, q_seq_len, heads, qk_scale,
                        mask_type, calc_type, lse=lse)
     op()
     return (out, lse) if return_lse else out
+
+
+def lse_merge(out_a, lse_a, out_b, lse_b, out=None, lse=None, stream=None):
+    """Merge two partial results over disjoint key ranges by their lse (ala_lse_merge).
+
+    ``out`` / ``lse`` default to new tensors; passing ``out_a`` / ``lse_a`` merges in place.
+    Returns (out, lse).
+    """
+    L = lib()
+    out = torch.empty_like(out_a) if out is None else out
+    lse = torch.empty_like(lse_a) if lse is None else lse
+    s = stream if stream is not None else torch.cuda.current_stream(out_a.device)
+    ts = [tensor(out_a), tensor(lse_a), tensor(out_b), tensor(lse_b), tensor(out), tensor(lse)]
+    _check(L.ala_lse_merge(*[_ref(t) for t in ts], ctypes.c_void_p(s.cuda_stream)))
+    return out, lse

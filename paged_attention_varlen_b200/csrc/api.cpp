@@ -516,6 +516,12 @@ extern "C" int atb_like_mla_get_workspace_size(const ala_tensor* qNope, const al
   const char* fn = "atb_like_mla_get_workspace_size";
   if (!workspaceSize || !op) return fail(ALA_NULL_REQUIRED, "%s: workspaceSize and op are required", fn);
   *op = nullptr;
+  if (calcType == ALA_MLA_CALC_RING) {
+    // ring attention: the same attention over the keys this call is given, with the lse it needs to merge
+    // the result with the other ranges' (ala_lse_merge); one token per batch, or qseqlen tokens with SPEC
+    if (!lse || !lse->data) return fail(ALA_NULL_REQUIRED, "%s: lse is required with calcType RING", fn);
+    calcType = (qSeqLen && qSeqLen->data) ? ALA_MLA_CALC_SPEC : ALA_MLA_CALC_UNDEFINED;
+  }
   ala_op* o = new ala_op();
   o->kind = ala_op::kMla;
   char err[512] = {0};
@@ -542,5 +548,43 @@ extern "C" int atb_like_mla(void* workspace, uint64_t workspaceSize, ala_op* op,
   char err[512] = {0};
   int st = mla_run(&op->mla, workspace, reinterpret_cast<cudaStream_t>(stream), err, sizeof err);
   if (st != ALA_OK) return fail(st, "%s: %s", fn, err);
+  return ok();
+}
+
+extern "C" int ala_lse_merge(const ala_tensor* outA, const ala_tensor* lseA, const ala_tensor* outB,
+                             const ala_tensor* lseB, ala_tensor* out, ala_tensor* lse, ala_stream_t stream) {
+  const char* fn = "ala_lse_merge";
+  const ala_tensor* ts[6] = {outA, lseA, outB, lseB, out, lse};
+  for (const ala_tensor* t : ts)
+    if (!t || !t->data) return fail(ALA_NULL_REQUIRED, "%s: all six tensors are required", fn);
+  const int32_t dt = outA->dtype;
+  if (dt != ALA_BF16 && dt != ALA_F16 && dt != ALA_F32)
+    return fail(ALA_INVALID_DTYPE, "%s: outputs must be bf16, f16 or f32", fn);
+  if (outB->dtype != dt || out->dtype != dt) return fail(ALA_INVALID_DTYPE, "%s: outA, outB and out differ in dtype", fn);
+  if (lseA->dtype != ALA_F32 || lseB->dtype != ALA_F32 || lse->dtype != ALA_F32)
+    return fail(ALA_INVALID_DTYPE, "%s: lse tensors must be fp32", fn);
+  if (outA->ndim < 1 || outA->ndim > 4) return fail(ALA_INVALID_SHAPE, "%s: outA must have 1 to 4 dims", fn);
+  const ala_tensor* same[2] = {outB, out};
+  for (const ala_tensor* t : same) {
+    if (t->ndim != outA->ndim) return fail(ALA_INVALID_SHAPE, "%s: outA, outB and out differ in shape", fn);
+    for (int i = 0; i < outA->ndim; ++i)
+      if (t->dims[i] != outA->dims[i]) return fail(ALA_INVALID_SHAPE, "%s: outA, outB and out differ in shape", fn);
+  }
+  const int64_t d = outA->dims[outA->ndim - 1];
+  if (d <= 0 || d > 1024) return fail(ALA_INVALID_SHAPE, "%s: the last dim must be in 1..1024", fn);
+  int64_t rows = 1;
+  for (int i = 0; i + 1 < outA->ndim; ++i) rows *= outA->dims[i];
+  const ala_tensor* lses[3] = {lseA, lseB, lse};
+  for (const ala_tensor* t : lses) {
+    int64_t ne = 1;
+    for (int i = 0; i < t->ndim; ++i) ne *= t->dims[i];
+    if (t->ndim < 1 || t->ndim > 4 || ne != rows)
+      return fail(ALA_INVALID_SHAPE, "%s: every lse must hold one value per output row", fn);
+  }
+  const cudaError_t e = ala::launch_lse_merge(dt, outA->data, static_cast<const float*>(lseA->data), outB->data,
+                                              static_cast<const float*>(lseB->data), out->data,
+                                              static_cast<float*>(lse->data), rows, (int)d,
+                                              reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(ALA_CUDA_ERROR, "%s: %s", fn, cudaGetErrorString(e));
   return ok();
 }

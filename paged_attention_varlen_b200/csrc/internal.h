@@ -71,4 +71,9 @@ cudaError_t launch_prefill(int32_t dtype, int32_t d, const CUtensorMap& tmQ, con
 // Dynamic shared memory the prefill kernel needs (0 if the combination is unsupported).
 int prefill_smem_bytes(int32_t dtype, int32_t d);
 
+// Merges two partial results (rows x d, each normalised over its own keys) by their lse; out / lse may
+// alias the inputs.  d <= 1024.
+cudaError_t launch_lse_merge(int32_t dtype, const void* a, const float* lse_a, const void* b, const float* lse_b,
+                             void* out, float* lse, int64_t rows, int d, cudaStream_t stream);
+
 }  // namespace ala

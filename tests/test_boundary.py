@@ -127,7 +127,7 @@ def _plan_mla(**over):
     a.update(over)
     return ala.plan_mla(a["q_nope"], a["q_rope"], a["ct_kv"], a["k_rope"], a["block_tables"], a["context_lens"],
                         a["q_seq_len"], a["heads"], a["qk_scale"], a["mask_type"], a["calc_type"], a["cache_mode"],
-                        kv_heads=a["kv_heads"])
+                        kv_heads=a["kv_heads"], lse=a.get("lse"))
 
 
 def test_mla_plan_ok():
@@ -136,9 +136,50 @@ def test_mla_plan_ok():
               q_seq_len=[2, 2, 2], mask_type=1, calc_type=1)
 
 
+def test_mla_ring_plans_with_lse():
+    # ring mode computes the same attention and requires the lse it is merged with
+    lse = torch.zeros(3, 128, 1, dtype=torch.float32)
+    _plan_mla(calc_type=2, lse=lse)
+    _plan_mla(q_nope=torch.zeros(6, 128, 512, dtype=torch.bfloat16), q_rope=torch.zeros(6, 128, 64, dtype=torch.bfloat16),
+              q_seq_len=[2, 2, 2], mask_type=1, calc_type=2, lse=torch.zeros(6, 128, 1, dtype=torch.float32))
+
+
+def _merge_args(n=4, d=512, dtype=torch.bfloat16):
+    return dict(out_a=torch.zeros(n, 2, d, dtype=dtype), lse_a=torch.zeros(n, 2, 1), out_b=torch.zeros(n, 2, d, dtype=dtype),
+                lse_b=torch.zeros(n, 2, 1), out=torch.zeros(n, 2, d, dtype=dtype), lse=torch.zeros(n, 2, 1))
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(out_b=torch.zeros(4, 2, 256, dtype=torch.bfloat16)), 2),   # shapes differ
+    (dict(out=torch.zeros(4, 2, 512, dtype=torch.float16)), 3),      # dtypes differ
+    (dict(lse_b=torch.zeros(4, 2, 1, dtype=torch.float16)), 3),      # lse must be fp32
+    (dict(lse=torch.zeros(4, 3, 1)), 2),                             # one lse per row
+    (dict(out_a=torch.zeros(4, 2, 2048, dtype=torch.bfloat16), out_b=torch.zeros(4, 2, 2048, dtype=torch.bfloat16),
+          out=torch.zeros(4, 2, 2048, dtype=torch.bfloat16)), 2),    # d <= 1024
+    (dict(out_a=torch.zeros(4, 2, 512, dtype=torch.int32), out_b=torch.zeros(4, 2, 512, dtype=torch.int32),
+          out=torch.zeros(4, 2, 512, dtype=torch.int32)), 3),        # outputs are floating point
+])
+def test_lse_merge_rejects(over, status):
+    # all checks run before any GPU work, so host tensors are enough here
+    a = _merge_args()
+    a.update(over)
+    L = ala.lib()
+    ts = [ala.tensor(a[k]) for k in ("out_a", "lse_a", "out_b", "lse_b", "out", "lse")]
+    st = L.ala_lse_merge(*[ala._ref(t) for t in ts], None)
+    assert st == status, ala.lib().ala_last_error().decode()
+
+
+def test_lse_merge_null_tensor():
+    a = _merge_args()
+    L = ala.lib()
+    ts = [ala.tensor(a[k]) for k in ("out_a", "lse_a", "out_b", "lse_b", "out")]
+    assert L.ala_lse_merge(*[ala._ref(t) for t in ts], None, None) == 1
+
+
 @pytest.mark.parametrize("over,status", [
     (dict(cache_mode=0), 5), (dict(cache_mode=2), 5), (dict(cache_mode=3), 5),
-    (dict(calc_type=2), 5), (dict(calc_type=3), 5),
+    (dict(calc_type=2), 1),                        # RING needs lse
+    (dict(calc_type=3), 5),
     (dict(mask_type=3), 4),                        # ALiBi only on the encoder paths
     (dict(kv_heads=2), 5),
     (dict(context_lens=[5, 100, 129]), 4),         # needs 3 blocks > 2

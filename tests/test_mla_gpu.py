@@ -119,3 +119,70 @@ def test_mla_negative_qk_scale():
     ref, lref = _oracle(case)
     check_out(out.reshape(-1, 512), ref)
     check_lse(lse.reshape(-1), lref)
+
+
+def _ring_ranges(case, bs):
+    """Each batch's keys cut at a page boundary into [0, cut) and [cut, ctx): two block tables over the same cache."""
+    ctx = case.context_lens
+    cut = np.maximum(ctx // (2 * bs), 1) * bs
+    assert (cut < ctx).all()
+    bt = case.block_tables
+    bt_a = np.full_like(bt, -1)
+    bt_b = np.full_like(bt, -1)
+    for b in range(len(ctx)):
+        pa = cut[b] // bs
+        nb = (ctx[b] - cut[b] + bs - 1) // bs
+        bt_a[b, :pa] = bt[b, :pa]
+        bt_b[b, :nb] = bt[b, pa:pa + nb]
+    return (cut.astype(np.int32), bt_a), ((ctx - cut).astype(np.int32), bt_b)
+
+
+def test_mla_ring_ranges_merged_equal_the_whole_context():
+    # calcType RING over two disjoint key ranges, merged by lse (ala_lse_merge), against the oracle over all keys
+    bs = 64
+    ctx = np.array([700, 1100, 300, 129], dtype=np.int32)
+    case = synth.make_mla("ring", ctx, 1, 128, 45, block_size=bs)
+    d = "cuda"
+    qn, qr = case.q_nope.to(d), case.q_rope.to(d)
+    ck, kr = case.ct_kv.to(d), case.k_rope.to(d)
+    parts = []
+    for cl, bt in _ring_ranges(case, bs):
+        out, lse = ala.atb_like_mla(qn, qr, ck, kr, torch.from_numpy(bt).to(d), cl, None, case.heads, case.qk_scale,
+                                    synth.MLA_MASK_UNDEFINED, ala.MLA_CALC_RING)
+        parts.append((out, lse))
+    (oa, la), (ob, lb) = parts
+    out, lse = ala.lse_merge(oa, la, ob, lb)
+    torch.cuda.synchronize()
+    ref, lref = _oracle(case)
+    check_out(out.reshape(-1, 512), ref)
+    check_lse(lse.reshape(-1), lref)
+    # in place over the first range's buffers gives the same result
+    ala.lse_merge(oa, la, ob, lb, out=oa, lse=la)
+    torch.cuda.synchronize()
+    assert torch.equal(oa, out) and torch.equal(la, lse)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_lse_merge_matches_the_oracle(dtype):
+    rng = np.random.Generator(np.random.PCG64(46))
+    n, heads, dv = 96, 3, 512
+    oa = torch.from_numpy(rng.standard_normal((n, heads, dv)).astype(np.float32)).to(dtype)
+    ob = torch.from_numpy(rng.standard_normal((n, heads, dv)).astype(np.float32)).to(dtype)
+    la = (rng.standard_normal((n, heads, 1)) * 4).astype(np.float32)
+    lb = (rng.standard_normal((n, heads, 1)) * 4).astype(np.float32)
+    la[5, 0, 0] = -np.inf                           # one side saw no allowed key
+    lb[7, 1, 0] = -np.inf
+    la[9, 2, 0] = lb[9, 2, 0] = -np.inf             # neither side: lse -inf, output 0
+    ref, lref = oracle.lse_merge(np.stack([oa.double().numpy().reshape(-1, dv), ob.double().numpy().reshape(-1, dv)]),
+                                 np.stack([la.reshape(-1), lb.reshape(-1)]).astype(np.float64))
+    out, lse = ala.lse_merge(oa.cuda(), torch.from_numpy(la).cuda(), ob.cuda(), torch.from_numpy(lb).cuda())
+    torch.cuda.synchronize()
+    got = out.reshape(-1, dv).double().cpu().numpy()
+    gl = lse.reshape(-1).double().cpu().numpy()
+    both = 9 * heads + 2
+    assert gl[both] == -np.inf and lref[both] == -np.inf
+    assert (got[both] == 0).all() and (ref[both] == 0).all()
+    keep = np.arange(n * heads) != both
+    tol = 2e-2 if dtype == torch.bfloat16 else 1e-5
+    assert np.abs(got[keep] - ref[keep]).max() <= tol
+    assert (np.abs(gl[keep] - lref[keep]) / np.maximum(1, np.abs(lref[keep]))).max() <= 1e-5
