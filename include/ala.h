@@ -148,6 +148,18 @@ ALA_API int atb_like_prefix_encoder_get_workspace_size(
 
 ALA_API int atb_like_prefix_encoder(void* workspace, uint64_t workspaceSize, ala_op* op, ala_stream_t stream);
 
+/* The same operation with the natural-log lse of every (token, head) row also
+ * written, so that attention over a prefix split into chunks can be merged
+ * with ala_lse_merge (the MLA page's lse output, applied to this encoder).
+ * lse: [nTokens, headNum] (or [nTokens, headNum, 1]) fp32, device, required;
+ * for left-aligned ALiBi (maskType 5) it is the lse of the left-aligned
+ * scores.  Execute with atb_like_prefix_encoder. */
+ALA_API int atb_like_prefix_encoder_lse_get_workspace_size(
+    const ala_tensor* query, const ala_tensor* key, const ala_tensor* value, const ala_tensor* blockTables,
+    const ala_tensor* mask, const ala_tensor* seqLen, const ala_tensor* kvSeqLen, const ala_tensor* slopes,
+    int maskType, int32_t headNum, int32_t kvHeadNum, float qkScale, ala_tensor* attnOut, ala_tensor* lse,
+    uint64_t* workspaceSize, ala_op** op);
+
 /* ---------------------------------------------------------------------------
  * varlen_attention: the same operation with K/V packed contiguously instead of
  * paged (the contiguous full-prefill reading of the pages' PA_ENCODER mode).

@@ -75,6 +75,10 @@ def lib() -> ctypes.CDLL:
         L.varlen_attention_noalloc.argtypes = [T, T, T, T, T, T, ctypes.c_int, ctypes.c_int32, ctypes.c_int32,
                                                ctypes.c_float, T, T, P]
         L.varlen_attention_noalloc.restype = ctypes.c_int
+        L.atb_like_prefix_encoder_lse_get_workspace_size.argtypes = [T, T, T, T, T, T, T, T, ctypes.c_int,
+                                                                     ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
+                                                                     T, T, U64P, OPP]
+        L.atb_like_prefix_encoder_lse_get_workspace_size.restype = ctypes.c_int
         L.ala_lse_merge.argtypes = [T, T, T, T, T, T, P]
         L.ala_lse_merge.restype = ctypes.c_int
         for f in ("atb_like_prefix_encoder", "varlen_attention", "atb_like_mla"):
@@ -197,8 +201,9 @@ def varlen_attention_noalloc(q, k, v, seq_len, kv_seq_len, mask_type, heads, kv_
 
 
 def plan_prefix_encoder(q, k, v, block_tables, seq_len, kv_seq_len, mask_type, heads, kv_heads, qk_scale,
-                        slopes=None, mask=None, out=None) -> tuple[Op, torch.Tensor]:
-    """Plan the paged PrefixEncoder call; returns (op, out)."""
+                        slopes=None, mask=None, out=None, lse=None) -> tuple[Op, torch.Tensor]:
+    """Plan the paged PrefixEncoder call; returns (op, out).  With ``lse`` ([nTokens, heads] fp32) the
+    lse-returning entry point is used."""
     L = lib()
     out = torch.empty_like(q) if out is None else out
     sl, kl = _host_i32(seq_len), _host_i32(kv_seq_len)
@@ -207,11 +212,16 @@ def plan_prefix_encoder(q, k, v, block_tables, seq_len, kv_seq_len, mask_type, h
     to = tensor(out)
     ws = ctypes.c_uint64(0)
     h = ctypes.c_void_p(0)
-    _check(L.atb_like_prefix_encoder_get_workspace_size(*[_ref(t) for t in ts], int(mask_type), int(heads),
-                                                        int(kv_heads), float(qk_scale), _ref(to), ctypes.byref(ws),
-                                                        ctypes.byref(h)))
+    if lse is None:
+        _check(L.atb_like_prefix_encoder_get_workspace_size(*[_ref(t) for t in ts], int(mask_type), int(heads),
+                                                            int(kv_heads), float(qk_scale), _ref(to),
+                                                            ctypes.byref(ws), ctypes.byref(h)))
+    else:
+        _check(L.atb_like_prefix_encoder_lse_get_workspace_size(*[_ref(t) for t in ts], int(mask_type), int(heads),
+                                                                int(kv_heads), float(qk_scale), _ref(to),
+                                                                _ref(tensor(lse)), ctypes.byref(ws), ctypes.byref(h)))
     return Op(h, ws.value, L.atb_like_prefix_encoder, q.device,
-              (q, k, v, block_tables, mask, sl, kl, slopes, out)), out
+              (q, k, v, block_tables, mask, sl, kl, slopes, out, lse)), out
 
 
 def atb_like_prefix_encoder(q, k, v, block_tables, seq_len, kv_seq_len, mask_type, heads, kv_heads, qk_scale,

@@ -444,12 +444,12 @@ int run_prefill(void* workspace, uint64_t workspaceSize, ala_op* op, ala_stream_
 
 }  // namespace
 
-extern "C" int atb_like_prefix_encoder_get_workspace_size(
-    const ala_tensor* query, const ala_tensor* key, const ala_tensor* value, const ala_tensor* blockTables,
-    const ala_tensor* mask, const ala_tensor* seqLen, const ala_tensor* kvSeqLen, const ala_tensor* slopes,
-    int maskType, int32_t headNum, int32_t kvHeadNum, float qkScale, ala_tensor* attnOut, uint64_t* workspaceSize,
-    ala_op** op) {
-  const char* fn = "atb_like_prefix_encoder_get_workspace_size";
+namespace {
+int plan_prefix_encoder(const ala_tensor* query, const ala_tensor* key, const ala_tensor* value,
+                        const ala_tensor* blockTables, const ala_tensor* mask, const ala_tensor* seqLen,
+                        const ala_tensor* kvSeqLen, const ala_tensor* slopes, int maskType, int32_t headNum,
+                        int32_t kvHeadNum, float qkScale, ala_tensor* attnOut, ala_tensor* lse,
+                        uint64_t* workspaceSize, ala_op** op, const char* fn) {
   if (!workspaceSize || !op) return fail(ALA_NULL_REQUIRED, "%s: workspaceSize and op are required", fn);
   *op = nullptr;
   if (!blockTables) return fail(ALA_NULL_REQUIRED, "%s: blockTables is required", fn);
@@ -465,7 +465,7 @@ extern "C" int atb_like_prefix_encoder_get_workspace_size(
   }
   ala_op* o = new ala_op();
   int st = build_prefill(o, query, key, value, blockTables, seqLen, kvSeqLen, slopes, maskType, headNum, kvHeadNum,
-                         qkScale, attnOut, nullptr, fn);
+                         qkScale, attnOut, lse, fn);
   if (st != ALA_OK) {
     delete o;
     return st;
@@ -473,6 +473,28 @@ extern "C" int atb_like_prefix_encoder_get_workspace_size(
   *workspaceSize = o->ws_size;
   *op = o;
   return ok();
+}
+}  // namespace
+
+extern "C" int atb_like_prefix_encoder_get_workspace_size(
+    const ala_tensor* query, const ala_tensor* key, const ala_tensor* value, const ala_tensor* blockTables,
+    const ala_tensor* mask, const ala_tensor* seqLen, const ala_tensor* kvSeqLen, const ala_tensor* slopes,
+    int maskType, int32_t headNum, int32_t kvHeadNum, float qkScale, ala_tensor* attnOut, uint64_t* workspaceSize,
+    ala_op** op) {
+  return plan_prefix_encoder(query, key, value, blockTables, mask, seqLen, kvSeqLen, slopes, maskType, headNum,
+                             kvHeadNum, qkScale, attnOut, nullptr, workspaceSize, op,
+                             "atb_like_prefix_encoder_get_workspace_size");
+}
+
+extern "C" int atb_like_prefix_encoder_lse_get_workspace_size(
+    const ala_tensor* query, const ala_tensor* key, const ala_tensor* value, const ala_tensor* blockTables,
+    const ala_tensor* mask, const ala_tensor* seqLen, const ala_tensor* kvSeqLen, const ala_tensor* slopes,
+    int maskType, int32_t headNum, int32_t kvHeadNum, float qkScale, ala_tensor* attnOut, ala_tensor* lse,
+    uint64_t* workspaceSize, ala_op** op) {
+  const char* fn = "atb_like_prefix_encoder_lse_get_workspace_size";
+  if (!lse || !lse->data) return fail(ALA_NULL_REQUIRED, "%s: lse is required", fn);
+  return plan_prefix_encoder(query, key, value, blockTables, mask, seqLen, kvSeqLen, slopes, maskType, headNum,
+                             kvHeadNum, qkScale, attnOut, lse, workspaceSize, op, fn);
 }
 
 extern "C" int atb_like_prefix_encoder(void* workspace, uint64_t workspaceSize, ala_op* op, ala_stream_t stream) {

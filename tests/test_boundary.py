@@ -144,6 +144,30 @@ def test_mla_ring_plans_with_lse():
               q_seq_len=[2, 2, 2], mask_type=1, calc_type=2, lse=torch.zeros(6, 128, 1, dtype=torch.float32))
 
 
+def test_prefix_encoder_lse_entry_requires_lse():
+    L = ala.lib()
+    q = torch.zeros(4, 2, 128, dtype=torch.float16)
+    kv = torch.zeros(2, 64, 2, 128, dtype=torch.float16)
+    bt = torch.zeros(1, 2, dtype=torch.int32)
+    sl = np.array([4], dtype=np.int32)
+    kl = np.array([70], dtype=np.int32)
+    ts = [ala.tensor(x) for x in (q, kv, kv, bt)] + [None] + [ala.tensor(sl), ala.tensor(kl), None]
+    ws = ctypes.c_uint64(0)
+    h = ctypes.c_void_p(0)
+    args = [ala._ref(t) for t in ts] + [9, 2, 2, ctypes.c_float(0.1), ala._ref(ala.tensor(q))]
+    st = L.atb_like_prefix_encoder_lse_get_workspace_size(*args, None, ctypes.byref(ws), ctypes.byref(h))
+    assert st == 1
+    lse = torch.zeros(4, 2, dtype=torch.float32)
+    st = L.atb_like_prefix_encoder_lse_get_workspace_size(*args, ala._ref(ala.tensor(lse)), ctypes.byref(ws),
+                                                          ctypes.byref(h))
+    assert st == 0, L.ala_last_error().decode()
+    L.ala_op_destroy(h)
+    bad = torch.zeros(4, 3, dtype=torch.float32)  # one value per (token, head)
+    st = L.atb_like_prefix_encoder_lse_get_workspace_size(*args, ala._ref(ala.tensor(bad)), ctypes.byref(ws),
+                                                          ctypes.byref(h))
+    assert st == 2
+
+
 def _merge_args(n=4, d=512, dtype=torch.bfloat16):
     return dict(out_a=torch.zeros(n, 2, d, dtype=dtype), lse_a=torch.zeros(n, 2, 1), out_b=torch.zeros(n, 2, d, dtype=dtype),
                 lse_b=torch.zeros(n, 2, 1), out=torch.zeros(n, 2, d, dtype=dtype), lse=torch.zeros(n, 2, 1))

@@ -186,3 +186,15 @@ def test_lse_merge_matches_the_oracle(dtype):
     tol = 2e-2 if dtype == torch.bfloat16 else 1e-5
     assert np.abs(got[keep] - ref[keep]).max() <= tol
     assert (np.abs(gl[keep] - lref[keep]) / np.maximum(1, np.abs(lref[keep]))).max() <= 1e-5
+
+
+@pytest.mark.parametrize("heads,qs,block_size", [(256, 1, 128), (128, 2, 64), (64, 4, 128)])
+def test_mla_row_block_shapes(heads, qs, block_size):
+    # rows per CTA = tokens per chunk x heads per group: 1 x 64 (four groups of a 256-head token),
+    # 2 x 32 and 4 x 16 (64 heads: four groups of 16)
+    ctx = np.array([90, 640, 1500, qs + 3], dtype=np.int32)
+    case = synth.make_mla(f"rows_{heads}_{qs}", ctx, qs, heads, 47 + qs, block_size=block_size)
+    out, lse, _ = _run(case)
+    ref, lref = _oracle(case)
+    check_out(out.reshape(-1, 512), ref)
+    check_lse(lse.reshape(-1), lref)

@@ -36,8 +36,11 @@ def _run(case, want_lse=True):
     q, k, v, slopes, bt = _dev(case)
     lse = None
     if case.paged:
+        # the lse-returning PrefixEncoder entry point (the plain one shares everything else)
+        if want_lse:
+            lse = torch.empty((q.shape[0], case.heads), dtype=torch.float32, device="cuda")
         op, out = ala.plan_prefix_encoder(q, k, v, bt, case.seq_len, case.kv_seq_len, case.mask_type, case.heads,
-                                          case.kv_heads, case.qk_scale, slopes)
+                                          case.kv_heads, case.qk_scale, slopes, lse=lse)
     else:
         if want_lse:
             lse = torch.empty((q.shape[0], case.heads), dtype=torch.float32, device="cuda")
