@@ -222,10 +222,14 @@ ALA_API int varlen_attention_noalloc(const ala_tensor* query, const ala_tensor* 
  * qkDescale, pvDescale  must be NULL (int8 cache not built).
  * headNum     128 (multiple of 64 accepted); kvHeadNum must be 1.
  * maskType    UNDEFINED (0) with one token per batch, or SPEC (1).
- * calcType    UNDEFINED (0), SPEC (1) or RING (2); PREFILL returns UNSUPPORTED.
+ * calcType    UNDEFINED (0), SPEC (1), RING (2) or PREFILL (3).
  *             RING (ring attention) computes the same attention over the keys
  *             this call is given and requires lse, so that results over
  *             disjoint key ranges can be merged with ala_lse_merge.
+ *             PREFILL (full prefill) requires qSeqLen (the new tokens of each
+ *             batch, at the end of its context) and applies the causal rule
+ *             token t -> keys j <= contextLens - qSeqLen + t whatever maskType
+ *             (UNDEFINED or SPEC) says.
  * cacheMode   KROPE_CTKV (1) only; others return UNSUPPORTED.
  * attenOut    [tokens, headNum, 512], dtype of qNope, device.
  * lse         NULL or [tokens, headNum, 1] fp32, device (natural log);

@@ -538,6 +538,15 @@ extern "C" int atb_like_mla_get_workspace_size(const ala_tensor* qNope, const al
   const char* fn = "atb_like_mla_get_workspace_size";
   if (!workspaceSize || !op) return fail(ALA_NULL_REQUIRED, "%s: workspaceSize and op are required", fn);
   *op = nullptr;
+  if (calcType == ALA_MLA_CALC_PREFILL) {
+    // full prefill: every query token of a batch attends causally to the keys up to its own position, i.e.
+    // token t of the qseqlen new tokens allows keys j <= contextLens - qseqlen + t (the speculative rule)
+    if (!qSeqLen || !qSeqLen->data) return fail(ALA_NULL_REQUIRED, "%s: qseqlen is required with calcType PREFILL", fn);
+    if (maskType != ALA_MLA_MASK_UNDEFINED && maskType != ALA_MLA_MASK_SPEC)
+      return fail(ALA_INVALID_PARAM, "%s: calcType PREFILL takes maskType UNDEFINED or SPEC (causal either way)", fn);
+    calcType = ALA_MLA_CALC_SPEC;
+    maskType = ALA_MLA_MASK_SPEC;
+  }
   if (calcType == ALA_MLA_CALC_RING) {
     // ring attention: the same attention over the keys this call is given, with the lse it needs to merge
     // the result with the other ranges' (ala_lse_merge); one token per batch, or qseqlen tokens with SPEC

@@ -136,6 +136,13 @@ def test_mla_plan_ok():
               q_seq_len=[2, 2, 2], mask_type=1, calc_type=1)
 
 
+def test_mla_prefill_plans_with_qseqlen():
+    _plan_mla(q_nope=torch.zeros(9, 128, 512, dtype=torch.bfloat16), q_rope=torch.zeros(9, 128, 64, dtype=torch.bfloat16),
+              q_seq_len=[1, 5, 3], calc_type=3)
+    _plan_mla(q_nope=torch.zeros(9, 128, 512, dtype=torch.bfloat16), q_rope=torch.zeros(9, 128, 64, dtype=torch.bfloat16),
+              q_seq_len=[1, 5, 3], calc_type=3, mask_type=1)
+
+
 def test_mla_ring_plans_with_lse():
     # ring mode computes the same attention and requires the lse it is merged with
     lse = torch.zeros(3, 128, 1, dtype=torch.float32)
@@ -203,7 +210,8 @@ def test_lse_merge_null_tensor():
 @pytest.mark.parametrize("over,status", [
     (dict(cache_mode=0), 5), (dict(cache_mode=2), 5), (dict(cache_mode=3), 5),
     (dict(calc_type=2), 1),                        # RING needs lse
-    (dict(calc_type=3), 5),
+    (dict(calc_type=3), 1),                        # PREFILL needs qseqlen
+    (dict(calc_type=3, q_seq_len=[1, 1, 1], mask_type=2), 4),  # PREFILL is causal: UNDEFINED or SPEC only
     (dict(mask_type=3), 4),                        # ALiBi only on the encoder paths
     (dict(kv_heads=2), 5),
     (dict(context_lens=[5, 100, 129]), 4),         # needs 3 blocks > 2

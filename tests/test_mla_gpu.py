@@ -28,7 +28,7 @@ def _run(case):
     ck, kr = case.ct_kv.to(d), case.k_rope.to(d)
     bt = torch.from_numpy(case.block_tables).to(d)
     lse = torch.empty((case.n_tokens, case.heads, 1), dtype=torch.float32, device=d)
-    qs = case.q_seq_len if case.calc_type == synth.MLA_CALC_SPEC else None
+    qs = case.q_seq_len if case.calc_type in (synth.MLA_CALC_SPEC, ala.MLA_CALC_PREFILL) else None
     op, out = ala.plan_mla(qn, qr, ck, kr, bt, case.context_lens, qs, case.heads, case.qk_scale, case.mask_type,
                            case.calc_type, lse=lse)
     op()
@@ -194,6 +194,19 @@ def test_mla_row_block_shapes(heads, qs, block_size):
     # 2 x 32 and 4 x 16 (64 heads: four groups of 16)
     ctx = np.array([90, 640, 1500, qs + 3], dtype=np.int32)
     case = synth.make_mla(f"rows_{heads}_{qs}", ctx, qs, heads, 47 + qs, block_size=block_size)
+    out, lse, _ = _run(case)
+    ref, lref = _oracle(case)
+    check_out(out.reshape(-1, 512), ref)
+    check_lse(lse.reshape(-1), lref)
+
+
+def test_mla_prefill_is_causal_within_each_batch():
+    # calcType PREFILL: all new tokens of a batch (one batch without a prefix) attend causally
+    ctx = np.array([100, 300, 520], dtype=np.int32)
+    qs = np.array([37, 300, 64], dtype=np.int32)
+    case = synth.make_mla("prefill", ctx, qs, 64, 49, block_size=64)
+    case.calc_type = ala.MLA_CALC_PREFILL
+    case.mask_type = synth.MLA_MASK_UNDEFINED
     out, lse, _ = _run(case)
     ref, lref = _oracle(case)
     check_out(out.reshape(-1, 512), ref)
