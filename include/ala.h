@@ -138,7 +138,7 @@ ALA_API int ala_workspace_status(const ala_op* op, const void* workspace, ala_st
  * qkScale     multiplies Q K^T before the bias is added.
  * headSize    64 or 128 (ALiBi masks: <= 128, per the compressed-mask page's
  *             constraints).
- * attnOut     same shape and dtype as query, device.
+ * attnOut     same shape and dtype as query, device, 32-byte aligned.
  * ------------------------------------------------------------------------- */
 ALA_API int atb_like_prefix_encoder_get_workspace_size(
     const ala_tensor* query, const ala_tensor* key, const ala_tensor* value, const ala_tensor* blockTables,
@@ -170,7 +170,7 @@ ALA_API int atb_like_prefix_encoder_lse_get_workspace_size(
  * seqLen, kvSeqLen, slopes, headNum, kvHeadNum, qkScale as above; maskType
  *             0, 3, 4, 5 or 9.  f32 inputs run on tf32 tensor cores
  *             (headSize 64 only).
- * attnOut     like query.
+ * attnOut     like query, 32-byte aligned.
  * lse         NULL or [nTokens, headNum] fp32, device: natural-log
  *             log-sum-exp of each row's scaled, biased, masked scores.
  * ------------------------------------------------------------------------- */

@@ -198,6 +198,8 @@ int build_prefill(ala_op* op, const ala_tensor* query, const ala_tensor* key, co
     return fail(ALA_INVALID_DTYPE, "%s: query dtype must be f16, bf16 or f32", fn);
   if (key->dtype != dt || value->dtype != dt || attnOut->dtype != dt)
     return fail(ALA_INVALID_DTYPE, "%s: key, value and attnOut must have the query's dtype", fn);
+  if (reinterpret_cast<uintptr_t>(attnOut->data) % 32)
+    return fail(ALA_INVALID_PARAM, "%s: attnOut must be 32-byte aligned (the kernel writes rows in 32-byte pieces)", fn);
   if (seqLen->dtype != ALA_I32 || kvSeqLen->dtype != ALA_I32)
     return fail(ALA_INVALID_DTYPE, "%s: seqLen and kvSeqLen must be int32 (host)", fn);
 

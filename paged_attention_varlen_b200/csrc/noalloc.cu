@@ -135,6 +135,8 @@ extern "C" ALA_API int varlen_attention_noalloc(const ala_tensor* query, const a
     return nfail(ALA_INVALID_DTYPE, "%s: query dtype must be f16, bf16 or f32", fn);
   if (key->dtype != dt || value->dtype != dt || attnOut->dtype != dt)
     return nfail(ALA_INVALID_DTYPE, "%s: key, value and attnOut must have the query's dtype", fn);
+  if (reinterpret_cast<uintptr_t>(attnOut->data) % 32)
+    return nfail(ALA_INVALID_PARAM, "%s: attnOut must be 32-byte aligned (the kernel writes rows in 32-byte pieces)", fn);
   if (seqLen->dtype != ALA_I32 || kvSeqLen->dtype != ALA_I32)
     return nfail(ALA_INVALID_DTYPE, "%s: seqLen and kvSeqLen must be int32 (host)", fn);
   if (query->ndim != 3 || query->dims[1] != headNum)

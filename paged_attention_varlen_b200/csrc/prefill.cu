@@ -86,6 +86,14 @@ struct Cfg {
   static_assert(256 + 2 * D <= 512, "tensor memory budget");
 };
 
+// One 32-byte store (address 32-byte aligned): whole sectors, half the instructions of 16-byte stores.
+__device__ __forceinline__ void st_global_v8(void* p, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t a4,
+                                             uint32_t a5, uint32_t a6, uint32_t a7) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a0), "r"(a1), "r"(a2), "r"(a3),
+               "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+               : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack2(float a, float b, __nv_bfloat16*) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -572,26 +580,25 @@ __global__ void __launch_bounds__(384, 1)
       for (int c32 = 0; c32 < D / 32; ++c32) {
         const uint32_t(&regs)[32] = orr[c32];
         if (row_valid) {
+          // rows start on 128-byte boundaries (D * element size), so every 32-byte store is aligned
           if constexpr (C::ES == 2) {
 #pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4) {
-              uint4 v;
-              v.x = pack2(__uint_as_float(regs[v4 * 8 + 0]) * inv_l, __uint_as_float(regs[v4 * 8 + 1]) * inv_l,
-                          (T*)nullptr);
-              v.y = pack2(__uint_as_float(regs[v4 * 8 + 2]) * inv_l, __uint_as_float(regs[v4 * 8 + 3]) * inv_l,
-                          (T*)nullptr);
-              v.z = pack2(__uint_as_float(regs[v4 * 8 + 4]) * inv_l, __uint_as_float(regs[v4 * 8 + 5]) * inv_l,
-                          (T*)nullptr);
-              v.w = pack2(__uint_as_float(regs[v4 * 8 + 6]) * inv_l, __uint_as_float(regs[v4 * 8 + 7]) * inv_l,
-                          (T*)nullptr);
-              *reinterpret_cast<uint4*>(orow + c32 * 32 + v4 * 8) = v;
+            for (int v8 = 0; v8 < 2; ++v8) {
+              uint32_t w[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                w[i] = pack2(__uint_as_float(regs[v8 * 16 + 2 * i]) * inv_l,
+                             __uint_as_float(regs[v8 * 16 + 2 * i + 1]) * inv_l, (T*)nullptr);
+              st_global_v8(orow + c32 * 32 + v8 * 16, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
             }
           } else {
 #pragma unroll
-            for (int v4 = 0; v4 < 8; ++v4) {
-              float4 v = make_float4(__uint_as_float(regs[v4 * 4 + 0]) * inv_l, __uint_as_float(regs[v4 * 4 + 1]) * inv_l,
-                                     __uint_as_float(regs[v4 * 4 + 2]) * inv_l, __uint_as_float(regs[v4 * 4 + 3]) * inv_l);
-              *reinterpret_cast<float4*>(reinterpret_cast<float*>(orow) + c32 * 32 + v4 * 4) = v;
+            for (int v8 = 0; v8 < 4; ++v8) {
+              uint32_t w[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) w[i] = __float_as_uint(__uint_as_float(regs[v8 * 8 + i]) * inv_l);
+              st_global_v8(reinterpret_cast<float*>(orow) + c32 * 32 + v8 * 8, w[0], w[1], w[2], w[3], w[4], w[5],
+                           w[6], w[7]);
             }
           }
         }

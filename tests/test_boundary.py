@@ -52,6 +52,19 @@ def test_valid_plan_needs_no_gpu():
     assert op.workspace_size > 0 and out.shape == (10, 4, 128)
 
 
+def test_output_must_be_32_byte_aligned():
+    # the kernel writes output rows in 32-byte pieces: a 16-byte-aligned output is refused on the host
+    a = _varlen_args()
+    q = a["q"]
+    buf = torch.zeros(q.numel() + 8, dtype=q.dtype)
+    out = buf[8:].view(q.shape)  # 16 bytes past a 256-byte boundary
+    assert out.data_ptr() % 32 == 16
+    with pytest.raises(ala.AlaError) as e:
+        ala.plan_varlen_attention(q, a["k"], a["v"], a["seq_len"], a["kv_seq_len"], a["mask_type"], a["heads"],
+                                  a["kv_heads"], a["qk_scale"], a["slopes"], out=out)
+    assert e.value.status == 4 and "32-byte" in str(e.value)
+
+
 @pytest.mark.parametrize("over,status", [
     (dict(heads=0), 4),                                          # headNum must be > 0
     (dict(kv_heads=3), 4),                                       # kvHeadNum must divide headNum
