@@ -22,7 +22,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 
 MASK_NONE, MASK_ALIBI, MASK_ALIBI_SQRT, MASK_ALIBI_LEFT, MASK_CAUSAL = 0, 3, 4, 5, 9
 
-_DTYPE_CODE = {torch.float16: 0, torch.bfloat16: 1, torch.float32: 2}
+_DTYPE_CODE = {torch.float16: 0, torch.bfloat16: 1, torch.float32: 2, torch.int8: 3}
 
 
 def build(force: bool = False) -> str:
@@ -50,9 +50,11 @@ def _load():
         _lib.oracle_expand_causal_compressed.argtypes = [P, I64, I64, P]
         _lib.oracle_mla.argtypes = [P, P, P, P, ctypes.c_int, P, I64, I32, P, P, I32, I32, I32, I32, D, P, I64,
                                     P, P]
+        _lib.oracle_mla_dequant.argtypes = [P, ctypes.c_int, P, ctypes.c_int, P, ctypes.c_int, P, P, P, P, I64,
+                                            I32, P, P, I32, I32, I32, I32, D, P, I64, P, P]
         _lib.oracle_lse_merge.argtypes = [I32, I64, I32, P, P, P, P]
         for f in ("oracle_attention", "oracle_build_mask", "oracle_attention_explicit",
-                  "oracle_expand_causal_compressed", "oracle_mla", "oracle_lse_merge"):
+                  "oracle_expand_causal_compressed", "oracle_mla", "oracle_mla_dequant", "oracle_lse_merge"):
             getattr(_lib, f).restype = ctypes.c_int
     return _lib
 
@@ -165,6 +167,37 @@ def mla(q_nope, q_rope, ct_kv, k_rope, block_tables, block_size, context_lens, q
                         0 if rw is None else len(rw), _ptr(out), _ptr(lse))
     if rc != 0:
         raise ValueError("oracle_mla: inconsistent arguments")
+    return out, lse
+
+
+def mla_dequant(q_nope, q_rope, ct_kv, k_rope, qk_descale, pv_descale, block_tables, block_size, context_lens,
+                q_seq_len, heads, qk_scale, rows=None):
+    """MLA over an int8 latent cache in fp64 (the MLA page's qkDescale / pvDescale rows):
+    s = qkScale * (qkDescale[h] * qNope.ctKV + qRope.kRope), O = pvDescale[h] * softmax(s) ctKV,
+    qNope and ctKV taken as stored (int8 or float); a None descale means 1."""
+    lib = _load()
+    qn, cq = _raw(q_nope)
+    qr, cr = _raw(q_rope)
+    ck, ckv = _raw(ct_kv)
+    kr, cr2 = _raw(k_rope)
+    assert cr == cr2
+    qd = None if qk_descale is None else np.ascontiguousarray(np.asarray(qk_descale, dtype=np.float32))
+    pd = None if pv_descale is None else np.ascontiguousarray(np.asarray(pv_descale, dtype=np.float32))
+    for d in (qd, pd):
+        assert d is None or d.shape == (heads,)
+    bt = _i32(block_tables)
+    cl = _i32(context_lens)
+    qs = _i32(q_seq_len) if q_seq_len is not None else np.ones_like(cl)
+    d_nope, d_rope = q_nope.shape[-1], q_rope.shape[-1]
+    rw = None if rows is None else np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    n = len(rw) if rw is not None else int(qs.sum()) * heads
+    out = np.zeros((n, d_nope), dtype=np.float64)
+    lse = np.zeros((n,), dtype=np.float64)
+    rc = lib.oracle_mla_dequant(_ptr(qn), cq, _ptr(qr), cr, _ptr(ck), ckv, _ptr(kr), _ptr(qd), _ptr(pd), _ptr(bt),
+                                bt.shape[1], block_size, _ptr(cl), _ptr(qs), len(cl), heads, d_nope, d_rope,
+                                float(qk_scale), _ptr(rw), 0 if rw is None else len(rw), _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_mla_dequant: inconsistent arguments")
     return out, lse
 
 

@@ -40,6 +40,11 @@
  *  - blockTables row index is the batch index;
  *  - MLA: key = [ctKV ; kRope], value = ctKV, query t of batch b allows
  *    j <= contextLens_b - qseqlen_b + t.
+ *  - MLA with an int8 latent cache (the MLA page's qkDescale / pvDescale
+ *    rows, both [num_heads] float): qkDescale[h] turns the qNope . ctKV dot
+ *    product of the stored numbers into a score (the qRope . kRope part is
+ *    not rescaled), and pvDescale[h] turns the probability-weighted sum of
+ *    the stored ctKV rows into the output.
  */
 #include <math.h>
 #include <stdint.h>
@@ -50,6 +55,7 @@
 #define ORC_F16 0
 #define ORC_BF16 1
 #define ORC_F32 2
+#define ORC_I8 3 /* two's-complement signed 8-bit integer */
 
 /* mask types, numbered as on the ATB PrefixEncoder page (maskType row) plus
  * 0 = no mask (all keys of the sequence allowed). */
@@ -88,6 +94,7 @@ static double orc_load(const void* base, int dtype, int64_t idx) {
   switch (dtype) {
     case ORC_F16: return orc_half_to_double(((const uint16_t*)base)[idx]);
     case ORC_BF16: return orc_bf16_to_double(((const uint16_t*)base)[idx]);
+    case ORC_I8: return (double)((const int8_t*)base)[idx];
     default: return (double)((const float*)base)[idx];
   }
 }
@@ -304,13 +311,22 @@ int oracle_expand_causal_compressed(const double* tri, int64_t seq_len,
  * ctKV  [numBlocks, blockSize, kv_heads(=1), d_nope], kRope [.., d_rope]
  * key_j = [ctKV_j ; kRope_j], value_j = ctKV_j.
  * Query t (0 <= t < qs_b) of batch b allows j <= contextLens_b - qs_b + t
- * (qs_b = 1 gives all j < contextLens_b).  Rows as in oracle_attention.   */
-int oracle_mla(const void* q_nope, const void* q_rope, const void* ct_kv,
-               const void* k_rope, int dtype, const int32_t* block_tables,
-               int64_t max_blocks, int32_t block_size, const int32_t* context_lens,
-               const int32_t* q_seq_len, int32_t batch, int32_t heads,
-               int32_t d_nope, int32_t d_rope, double qk_scale,
-               const int64_t* rows, int64_t n_rows, double* out, double* lse) {
+ * (qs_b = 1 gives all j < contextLens_b).  Rows as in oracle_attention.
+ *
+ * Dequantised form (qk_descale / pv_descale non-NULL, one float per head):
+ *   s_j = qkScale * (qkDescale[h] * qNope . ctKV_j + qRope . kRope_j)
+ *   O   = pvDescale[h] * sum_j softmax(s)_j ctKV_j
+ * with qNope and ctKV read as stored (int8 integers, or floats).  NULL
+ * descales mean 1, which is the plain MLA definition above.              */
+int oracle_mla_dequant(const void* q_nope, int qn_dtype, const void* q_rope,
+                       int rope_dtype, const void* ct_kv, int kv_dtype,
+                       const void* k_rope, const float* qk_descale,
+                       const float* pv_descale, const int32_t* block_tables,
+                       int64_t max_blocks, int32_t block_size,
+                       const int32_t* context_lens, const int32_t* q_seq_len,
+                       int32_t batch, int32_t heads, int32_t d_nope,
+                       int32_t d_rope, double qk_scale, const int64_t* rows,
+                       int64_t n_rows, double* out, double* lse) {
   if (batch < 0 || heads <= 0) return -1;
   int64_t* cu_q = (int64_t*)malloc(sizeof(int64_t) * (batch + 1));
   cu_q[0] = 0;
@@ -336,18 +352,20 @@ int oracle_mla(const void* q_nope, const void* q_rope, const void* ct_kv,
       const int64_t ti = t - cu_q[b];
       const int64_t ctx = context_lens[b];
       const int64_t last = ctx - qs + ti; /* last allowed key */
+      const double qk_d = qk_descale ? (double)qk_descale[h] : 1.0;
+      const double pv_d = pv_descale ? (double)pv_descale[h] : 1.0;
       double m = -INFINITY;
       for (int64_t j = 0; j <= last; ++j) {
         const int64_t blk = block_tables[(int64_t)b * max_blocks + j / block_size];
         const int64_t slot = blk * block_size + j % block_size;
-        double dot = 0.0;
+        double dot_nope = 0.0, dot_rope = 0.0;
         for (int32_t c = 0; c < d_nope; ++c)
-          dot += orc_load(q_nope, dtype, (t * heads + h) * (int64_t)d_nope + c) *
-                 orc_load(ct_kv, dtype, slot * d_nope + c);
+          dot_nope += orc_load(q_nope, qn_dtype, (t * heads + h) * (int64_t)d_nope + c) *
+                      orc_load(ct_kv, kv_dtype, slot * d_nope + c);
         for (int32_t c = 0; c < d_rope; ++c)
-          dot += orc_load(q_rope, dtype, (t * heads + h) * (int64_t)d_rope + c) *
-                 orc_load(k_rope, dtype, slot * d_rope + c);
-        s[j] = qk_scale * dot;
+          dot_rope += orc_load(q_rope, rope_dtype, (t * heads + h) * (int64_t)d_rope + c) *
+                      orc_load(k_rope, rope_dtype, slot * d_rope + c);
+        s[j] = qk_scale * (qk_d * dot_nope + dot_rope);
         if (s[j] > m) m = s[j];
       }
       double l = 0.0;
@@ -359,14 +377,27 @@ int oracle_mla(const void* q_nope, const void* q_rope, const void* ct_kv,
         const int64_t blk = block_tables[(int64_t)b * max_blocks + j / block_size];
         const int64_t slot = blk * block_size + j % block_size;
         for (int32_t c = 0; c < d_nope; ++c)
-          o[c] += p * orc_load(ct_kv, dtype, slot * d_nope + c);
+          o[c] += p * orc_load(ct_kv, kv_dtype, slot * d_nope + c);
       }
+      for (int32_t c = 0; c < d_nope; ++c) o[c] *= pv_d;
       if (lse) lse[r] = m + log(l);
     }
     free(s);
   }
   free(cu_q);
   return 0;
+}
+
+/* The MLA definition with every tensor in one floating dtype. */
+int oracle_mla(const void* q_nope, const void* q_rope, const void* ct_kv,
+               const void* k_rope, int dtype, const int32_t* block_tables,
+               int64_t max_blocks, int32_t block_size, const int32_t* context_lens,
+               const int32_t* q_seq_len, int32_t batch, int32_t heads,
+               int32_t d_nope, int32_t d_rope, double qk_scale,
+               const int64_t* rows, int64_t n_rows, double* out, double* lse) {
+  return oracle_mla_dequant(q_nope, dtype, q_rope, dtype, ct_kv, dtype, k_rope, NULL, NULL,
+                            block_tables, max_blocks, block_size, context_lens, q_seq_len,
+                            batch, heads, d_nope, d_rope, qk_scale, rows, n_rows, out, lse);
 }
 
 /* ---- merge of partial results over disjoint key ranges --------------------

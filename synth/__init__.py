@@ -27,7 +27,7 @@ MASK_NONE, MASK_ALIBI, MASK_ALIBI_SQRT, MASK_ALIBI_LEFT, MASK_CAUSAL = 0, 3, 4, 
 MLA_CALC_UNDEFINED, MLA_CALC_SPEC = 0, 1
 MLA_MASK_UNDEFINED, MLA_MASK_SPEC = 0, 1
 
-_POISON = {torch.float16: 6.0e4, torch.bfloat16: 1.0e30, torch.float32: 1.0e30}
+_POISON = {torch.float16: 6.0e4, torch.bfloat16: 1.0e30, torch.float32: 1.0e30, torch.int8: 127}
 
 
 def alibi_slopes(heads: int) -> np.ndarray:
@@ -212,6 +212,8 @@ class MlaCase:
     calc_type: int
     mask_type: int
     block_size: int
+    qk_descale: np.ndarray | None = None  # [heads] float32, int8 latent cache only
+    pv_descale: np.ndarray | None = None  # [heads] float32, int8 latent cache only
 
     @property
     def n_tokens(self) -> int:
@@ -250,3 +252,61 @@ def mla_decode_bf16(qs: int, seed=1004, batch=64, lo=1024, hi=16384, heads=128) 
     rng = np.random.Generator(np.random.PCG64(seed))
     ctx = rng.integers(lo, hi + 1, size=batch).astype(np.int32)
     return make_mla(f"mla_qs{qs}_bf16_b{batch}_h{heads}", ctx, qs, heads, seed, rng=rng)
+
+
+def _quantize(x: np.ndarray, scale) -> torch.Tensor:
+    """Symmetric int8 codes of float samples: round(x / scale) clipped to [-127, 127]."""
+    return torch.from_numpy(np.clip(np.rint(x / scale), -127, 127).astype(np.int8))
+
+
+def make_mla_int8(name, context_lens, qs, heads, seed, rng=None, block_size=128, d_nope=512, d_rope=64, sigma=0.5,
+                  dtype=torch.bfloat16, qnope_int8=True) -> MlaCase:
+    """An MLA case over an int8 latent cache: ctKV holds int8 codes of N(0, sigma) samples at one scale
+    (4 sigma / 127); qNope is int8 codes at a per-head scale (or plain `dtype` samples); qRope and kRope
+    stay `dtype`.  qk_descale[h] = qNope scale x cache scale (cache scale alone, with a per-head factor in
+    [0.75, 1.25), for a float qNope) and pv_descale[h] = cache scale x a per-head factor in [0.75, 1.25)."""
+    rng = rng if rng is not None else np.random.Generator(np.random.PCG64(seed))
+    context_lens = np.asarray(context_lens, dtype=np.int32)
+    batch = len(context_lens)
+    q_seq_len = np.broadcast_to(np.asarray(qs, dtype=np.int32), (batch,)).copy()
+    tokens = int(q_seq_len.sum())
+    spec = bool((q_seq_len > 1).any())
+    kv_scale = 4.0 * sigma / 127.0
+    head_f = (0.75 + 0.5 * rng.random(heads)).astype(np.float32)
+    qn = rng.standard_normal(size=(tokens, heads, d_nope), dtype=np.float32) * np.float32(sigma)
+    if qnope_int8:
+        q_scale = (kv_scale * head_f).astype(np.float32)
+        q_nope = _quantize(qn, q_scale[None, :, None])
+        qk_descale = (q_scale * np.float32(kv_scale)).astype(np.float32)
+    else:
+        q_nope = torch.from_numpy(qn).to(dtype)
+        qk_descale = (np.float32(kv_scale) * head_f).astype(np.float32)
+    pv_descale = (np.float32(kv_scale) * (0.75 + 0.5 * rng.random(heads))).astype(np.float32)
+    q_rope = _normal(rng, (tokens, heads, d_rope), sigma, dtype)
+    n_kv = int(context_lens.sum())
+    ckv = _quantize(rng.standard_normal(size=(n_kv, 1, d_nope), dtype=np.float32) * np.float32(sigma), kv_scale)
+    kr = _normal(rng, (n_kv, 1, d_rope), sigma, dtype)
+    ct_kv, _, bt = _page(rng, context_lens, block_size, ckv, ckv[:, :, :1], torch.int8)
+    # kRope goes through the same block table: page it again with the table just drawn
+    k_rope = (torch.where(torch.arange(d_rope) % 2 == 0, 1.0, -1.0) * _POISON[dtype]).to(dtype).repeat(
+        ct_kv.shape[0], block_size, 1, 1)
+    pos = 0
+    for b, L in enumerate(context_lens.tolist()):
+        for p_ in range((L + block_size - 1) // block_size):
+            lo, n = p_ * block_size, min(block_size, L - p_ * block_size)
+            k_rope[int(bt[b, p_]), :n] = kr[pos + lo: pos + lo + n]
+        pos += L
+    return MlaCase(name=name, dtype=dtype, q_nope=q_nope, q_rope=q_rope, ct_kv=ct_kv, k_rope=k_rope,
+                   block_tables=bt, context_lens=context_lens, q_seq_len=q_seq_len, heads=heads,
+                   qk_scale=1.0 / math.sqrt(d_nope + d_rope),
+                   calc_type=MLA_CALC_SPEC if spec else MLA_CALC_UNDEFINED,
+                   mask_type=MLA_MASK_SPEC if spec else MLA_MASK_UNDEFINED, block_size=block_size,
+                   qk_descale=qk_descale, pv_descale=pv_descale)
+
+
+def mla_decode_int8(seed=1005, batch=64, lo=1024, hi=16384, heads=128, qs=1) -> MlaCase:
+    """The MLA decode workload over an int8 latent cache: batch 64, contextLens ~ U{1024..16384}, 128 heads,
+    512 + 64, paged bs = 128, int8 qNope and ctKV, bf16 qRope / kRope."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    ctx = rng.integers(lo, hi + 1, size=batch).astype(np.int32)
+    return make_mla_int8(f"mla_qs{qs}_int8_b{batch}_h{heads}", ctx, qs, heads, seed, rng=rng)

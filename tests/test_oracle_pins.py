@@ -345,3 +345,91 @@ def test_row_subset_equals_full_run():
                                slopes=case.slopes, rows=rows)
     np.testing.assert_array_equal(sub, full[rows])
     np.testing.assert_array_equal(ls, lf[rows])
+
+
+# --------------------------------------------------------------------------
+# MLA over an int8 latent cache (MLA page, qkDescale / pvDescale rows)
+# --------------------------------------------------------------------------
+
+def _int8_two_key_case():
+    """Two heads, two cached keys, d_nope 16, d_rope 4, one page (physical block 1 of 2).
+
+    Stored numbers: qNope head 0 = -3, head 1 = 5 (every element); ctKV key 0 = 2, key 1 = -1;
+    qRope head 0 = 0.5, head 1 = -0.25; kRope key 0 = 1, key 1 = 2.  qkDescale = (1/64, 1/32),
+    pvDescale = (0.5, 3), qkScale = 0.5.  By hand:
+      head 0: nope dots 16*(-3*2) = -96 and 16*(-3*-1) = 48; rope dots 4*0.5*1 = 2 and 4*0.5*2 = 4
+              s = 0.5*(-96/64 + 2) = 0.25 and 0.5*(48/64 + 4) = 2.375
+      head 1: nope dots 16*(5*2) = 160 and 16*(5*-1) = -80; rope dots -1 and -2
+              s = 0.5*(160/32 - 1) = 2 and 0.5*(-80/32 - 2) = -2.25
+    The output is pvDescale * (p0 * 2 + p1 * (-1)) in every column, p1 = 1/(1 + exp(s0 - s1)),
+    and lse = s0 + log(1 + exp(s1 - s0))."""
+    qn = torch.tensor([-3, 5], dtype=torch.int8).view(1, 2, 1).expand(1, 2, 16).contiguous()
+    qr = torch.tensor([0.5, -0.25], dtype=torch.bfloat16).view(1, 2, 1).expand(1, 2, 4).contiguous()
+    ck = torch.full((2, 16, 1, 16), 99, dtype=torch.int8)  # block 0 is not referenced
+    ck[1, 0] = 2
+    ck[1, 1] = -1
+    kr = torch.full((2, 16, 1, 4), 7.0, dtype=torch.bfloat16)
+    kr[1, 0] = 1.0
+    kr[1, 1] = 2.0
+    return qn, qr, ck, kr, np.array([[1]], dtype=np.int32)
+
+
+def test_mla_int8_two_key_worked_example():
+    qn, qr, ck, kr, bt = _int8_two_key_case()
+    out, lse = oracle.mla_dequant(qn, qr, ck, kr, [1 / 64, 1 / 32], [0.5, 3.0], bt, 16, [2], [1], 2, 0.5)
+    for h, (s0, s1, pv) in enumerate([(0.25, 2.375, 0.5), (2.0, -2.25, 3.0)]):
+        p1 = 1.0 / (1.0 + math.exp(s0 - s1))
+        expect = pv * ((1.0 - p1) * 2.0 + p1 * -1.0)
+        np.testing.assert_allclose(out[h], np.full(16, expect), rtol=0, atol=1e-13)
+        assert abs(lse[h] - (s0 + math.log1p(math.exp(s1 - s0)))) < 1e-13
+
+
+@pytest.mark.parametrize("qn_int8", [True, False])
+@pytest.mark.parametrize("qs", [1, 3])
+def test_mla_int8_equals_sdpa_with_prescaled_operands(qn_int8, qs):
+    """The dequantised scores are qkScale * [qkDescale*qNope ; qRope] . [ctKV ; kRope]: torch's float64
+    scaled_dot_product_attention on those concatenated operands, with the speculative causal mask,
+    times pvDescale, must give the same rows."""
+    rng = np.random.Generator(np.random.PCG64(71))
+    heads, d_nope, d_rope, bs = 3, 24, 8, 16
+    ctx = np.array([5, 40, 33], dtype=np.int32)
+    case = synth.make_mla_int8("q8", ctx, qs, heads, 71, rng=rng, block_size=bs, d_nope=d_nope, d_rope=d_rope,
+                               qnope_int8=qn_int8)
+    out, lse = oracle.mla_dequant(case.q_nope, case.q_rope, case.ct_kv, case.k_rope, case.qk_descale,
+                                  case.pv_descale, case.block_tables, bs, case.context_lens, case.q_seq_len, heads,
+                                  case.qk_scale)
+    qkd = torch.from_numpy(case.qk_descale.astype(np.float64))
+    pvd = torch.from_numpy(case.pv_descale.astype(np.float64))
+    t0 = 0
+    for b, L in enumerate(ctx.tolist()):
+        keys = []
+        for j in range(L):
+            blk = int(case.block_tables[b, j // bs])
+            keys.append((case.ct_kv[blk, j % bs, 0].double(), case.k_rope[blk, j % bs, 0].double()))
+        kn = torch.stack([k[0] for k in keys])                      # [L, d_nope]
+        kcat = torch.cat([kn, torch.stack([k[1] for k in keys])], dim=-1)
+        for t in range(qs):
+            allow = torch.arange(L) <= L - qs + t
+            for h in range(heads):
+                q = torch.cat([case.q_nope[t0 + t, h].double() * qkd[h], case.q_rope[t0 + t, h].double()])
+                o = F.scaled_dot_product_attention(q.view(1, 1, 1, -1), kcat.view(1, 1, L, -1), kn.view(1, 1, L, -1),
+                                                   attn_mask=allow.view(1, 1, 1, L), scale=case.qk_scale)
+                row = (t0 + t) * heads + h
+                np.testing.assert_allclose(out[row], (o.view(-1) * pvd[h]).numpy(), rtol=1e-12, atol=1e-12)
+                s = case.qk_scale * (kcat[allow] @ q)
+                assert abs(lse[row] - torch.logsumexp(s, 0).item()) < 1e-12
+        t0 += qs
+
+
+def test_mla_int8_output_is_linear_in_pv_descale_and_lse_ignores_it():
+    rng = np.random.Generator(np.random.PCG64(73))
+    case = synth.make_mla_int8("q8", np.array([70], dtype=np.int32), 1, 2, 73, rng=rng, block_size=32, d_nope=16,
+                               d_rope=8, qnope_int8=True)
+    args = (case.block_tables, 32, case.context_lens, case.q_seq_len, 2, case.qk_scale)
+    o1, l1 = oracle.mla_dequant(case.q_nope, case.q_rope, case.ct_kv, case.k_rope, case.qk_descale,
+                                np.ones(2, np.float32), *args)
+    o2, l2 = oracle.mla_dequant(case.q_nope, case.q_rope, case.ct_kv, case.k_rope, case.qk_descale,
+                                np.array([0.25, 4.0], np.float32), *args)
+    np.testing.assert_array_equal(l1, l2)
+    np.testing.assert_array_equal(o2[0], o1[0] * 0.25)
+    np.testing.assert_array_equal(o2[1], o1[1] * 4.0)
