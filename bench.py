@@ -47,6 +47,7 @@ import synth  # noqa: E402
 
 PROFILE = os.path.join(ROOT, "profiles", "prefill_varlen_causal_bf16.md")
 MLA_PROFILE = os.path.join(ROOT, "profiles", "mla_decode_qs1_bf16.md")
+MLA_INT8_PROFILE = os.path.join(ROOT, "profiles", "mla_decode_qs1_int8.md")
 KERNEL_SOURCES = ["paged_attention_varlen_b200/csrc/prefill.cu", "paged_attention_varlen_b200/csrc/ptx.cuh"]
 MLA_KERNEL_SOURCES = ["paged_attention_varlen_b200/csrc/mla.cu", "paged_attention_varlen_b200/csrc/ptx.cuh"]
 DEFAULT_WORKLOAD = "varlen_causal_bf16"
@@ -57,6 +58,7 @@ WORKLOADS = {
     "long_alibi_left_bf16": lambda: synth.long_alibi_bf16(synth.MASK_ALIBI_LEFT),
     "mla_decode_qs1_bf16": lambda: synth.mla_decode_bf16(1),
     "mla_spec_qs4_bf16": lambda: synth.mla_decode_bf16(4),
+    "mla_decode_qs1_int8": lambda: synth.mla_decode_int8(),
 }
 L2_FLUSH_BYTES = 256 << 20
 
@@ -173,9 +175,10 @@ def mla_flops(case) -> float:
 
 
 def mla_bytes(case) -> float:
-    es = case.q_nope.element_size()
-    kv = int(case.context_lens.sum()) * 576 * es
-    q = case.n_tokens * case.heads * 576 * es
+    """Each cached ctKV + kRope row once, the query, the output and the fp32 lse (per-head descales: 1 KB)."""
+    es = case.q_rope.element_size()
+    kv = int(case.context_lens.sum()) * (512 * case.ct_kv.element_size() + 64 * es)
+    q = case.n_tokens * case.heads * (512 * case.q_nope.element_size() + 64 * es)
     o = case.n_tokens * case.heads * 512 * es + case.n_tokens * case.heads * 4
     return kv + q + o
 
@@ -186,9 +189,13 @@ def plan_case(ala, case, device):
         t = {"q_nope": case.q_nope.to(device), "q_rope": case.q_rope.to(device), "ct_kv": case.ct_kv.to(device),
              "k_rope": case.k_rope.to(device), "bt": torch.from_numpy(case.block_tables).to(device)}
         t["lse"] = torch.empty((case.n_tokens, case.heads, 1), dtype=torch.float32, device=device)
+        if case.qk_descale is not None:  # int8 latent cache
+            t["qk_descale"] = torch.from_numpy(case.qk_descale).to(device)
+            t["pv_descale"] = torch.from_numpy(case.pv_descale).to(device)
         op, out = ala.plan_mla(t["q_nope"], t["q_rope"], t["ct_kv"], t["k_rope"], t["bt"], case.context_lens,
                                case.q_seq_len if case.calc_type == synth.MLA_CALC_SPEC else None, case.heads,
-                               case.qk_scale, case.mask_type, case.calc_type, lse=t["lse"])
+                               case.qk_scale, case.mask_type, case.calc_type, lse=t["lse"],
+                               qk_descale=t.get("qk_descale"), pv_descale=t.get("pv_descale"))
         t["out"] = out
         return op, t
     t = {"q": case.q.to(device), "k": case.k.to(device), "v": case.v.to(device)}
@@ -276,7 +283,7 @@ def cpu_baseline(case, budget_s=12.0):
 
 
 def case_dtype(case):
-    return case.q_nope.dtype if isinstance(case, synth.MlaCase) else case.dtype
+    return case.q_rope.dtype if isinstance(case, synth.MlaCase) else case.dtype
 
 
 def op_has_combine(op):
@@ -290,6 +297,8 @@ def base_config(case):
         return {"workload": case.name, "global_batch": len(case.context_lens), "tokens": case.n_tokens,
                 "context_lens": "U[1024,16384] per batch", "heads": case.heads, "kv_lora": 512, "rope": 64,
                 "qseqlen": int(case.q_seq_len[0]), "block_size": case.block_size,
+                "cache": ("int8 ctKV and qNope codes, per-head qkDescale / pvDescale" if case.qk_descale is not None
+                          else str(case.q_rope.dtype).replace("torch.", "")),
                 "parallelism": "replicas (independent batches)", "l2": l2}
     mask = {0: "none", 3: "alibi right", 4: "alibi sqrt", 5: "alibi left", 9: "causal"}[case.mask_type]
     return {"workload": case.name, "global_batch": len(case.seq_len), "tokens": case.n_tokens,
@@ -374,10 +383,13 @@ def main():
         if is_mla:
             src = kernel_source_hash(MLA_KERNEL_SOURCES)
             achieved = nbytes / (mean_ms * 1e-3) / 1e9
+            int8 = case.qk_descale is not None
             roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                        "frac": achieved / peaks["hbm_gbs"], "traffic": profiled_traffic(MLA_PROFILE, src),
+                        "frac": achieved / peaks["hbm_gbs"],
+                        "traffic": profiled_traffic(MLA_INT8_PROFILE if int8 else MLA_PROFILE, src),
                         "algorithmic_bytes": nbytes, "peak_source": peaks["source"] + " (copy bandwidth)",
-                        "tflops": flops / (mean_ms * 1e-3) / 1e12, "kernel": "mla_kernel<bf16> + mla_combine_kernel",
+                        "tflops": flops / (mean_ms * 1e-3) / 1e12,
+                        "kernel": ("mla_kernel<bf16, int8 cache>" if int8 else "mla_kernel<bf16>") + " + mla_combine_kernel",
                         "kernel_source_sha256": src}
             launches = args.steps * (2 if op_has_combine(op) else 1)
         else:
@@ -430,8 +442,7 @@ def extra_workloads(ala, device, flush, stream, peaks, main_case, args):
         tf = prefill_flops(case) / (ms * 1e-3) / 1e12
         out[case.name] = {"ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / peaks["bf16_tflops"]}
         del op
-    for qs in (1, 4):
-        case = synth.mla_decode_bf16(qs)
+    for case in (synth.mla_decode_bf16(1), synth.mla_decode_bf16(4), synth.mla_decode_int8()):
         try:
             op, _ = plan_case(ala, case, device)
             ms = statistics.mean(time_steps(op, steps, 3, flush, stream))

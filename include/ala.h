@@ -59,7 +59,7 @@ extern "C" {
 typedef struct CUstream_st* ala_stream_t; /* same type as cudaStream_t */
 
 /* dtype codes */
-enum { ALA_F16 = 0, ALA_BF16 = 1, ALA_F32 = 2, ALA_I32 = 3 };
+enum { ALA_F16 = 0, ALA_BF16 = 1, ALA_F32 = 2, ALA_I32 = 3, ALA_I8 = 4 };
 
 typedef struct ala_tensor {
   void* data;
@@ -208,9 +208,11 @@ ALA_API int varlen_attention_noalloc(const ala_tensor* query, const ala_tensor* 
  * MLA decode / speculative decode (ATB "MLA" page, definition and parameter
  * table).  key_j = [ctKV_j ; kRope_j] (576 dims), value_j = ctKV_j (512).
  *
- * qNope       [tokens, headNum, 512] bf16/f16, device.
- * qRope       [tokens, headNum, 64], same dtype, device.
- * ctKV        [numBlocks, blockSize, kvHeadNum, 512], device (ND layout);
+ * qNope       [tokens, headNum, 512] bf16/f16 (qRope's dtype), device; with
+ *             cacheMode 2 also int8 codes (16-byte aligned).
+ * qRope       [tokens, headNum, 64] bf16/f16, device: the compute and output type.
+ * ctKV        [numBlocks, blockSize, kvHeadNum, 512], device (ND layout), qRope's
+ *             dtype, or int8 codes with cacheMode 2 (16-byte aligned);
  *             blockSize a multiple of 16 dividing 64, or a multiple of 64.
  * kRope       [numBlocks, blockSize, kvHeadNum, 64], device.
  * blockTables [batch, maxBlocks] int32, device (entries read must be valid).
@@ -219,7 +221,11 @@ ALA_API int varlen_attention_noalloc(const ala_tensor* query, const ala_tensor* 
  * qSeqLen     [batch] int32, HOST: query tokens per batch; required when
  *             calcType = SPEC, else NULL (one token each).  Token t of batch
  *             b allows keys j <= contextLens_b - qSeqLen_b + t.
- * qkDescale, pvDescale  must be NULL (int8 cache not built).
+ * qkDescale, pvDescale  [headNum] fp32, device, required with cacheMode 2
+ *             and NULL otherwise.  Reading of the page's two rows: the score
+ *             is qkScale * (qkDescale[h] * qNope.ctKV + qRope.kRope) with qNope
+ *             and ctKV taken as stored (int8 codes, or floats), and the output
+ *             is pvDescale[h] * sum_j p_j ctKV_j.
  * headNum     128 (multiple of 64 accepted); kvHeadNum must be 1.
  * maskType    UNDEFINED (0) with one token per batch, or SPEC (1).
  * calcType    UNDEFINED (0), SPEC (1), RING (2) or PREFILL (3).
@@ -230,8 +236,10 @@ ALA_API int varlen_attention_noalloc(const ala_tensor* query, const ala_tensor* 
  *             batch, at the end of its context) and applies the causal rule
  *             token t -> keys j <= contextLens - qSeqLen + t whatever maskType
  *             (UNDEFINED or SPEC) says.
- * cacheMode   KROPE_CTKV (1) only; others return UNSUPPORTED.
- * attenOut    [tokens, headNum, 512], dtype of qNope, device.
+ * cacheMode   KROPE_CTKV (1), or INT8_NZCACHE (2): the int8 latent cache,
+ *             kept here in the same ND layout as mode 1 (the page's NZ fractal
+ *             layout is Ascend's); 0 and 3 return UNSUPPORTED.
+ * attenOut    [tokens, headNum, 512], dtype of qRope, device.
  * lse         NULL or [tokens, headNum, 1] fp32, device (natural log);
  *             required with calcType RING (NULL_REQUIRED otherwise).
  * workspace   256-byte aligned; holds the schedule and, for key ranges split

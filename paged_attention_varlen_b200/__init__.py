@@ -23,7 +23,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libala.so")
 
-F16, BF16, F32, I32 = 0, 1, 2, 3
+F16, BF16, F32, I32, I8 = 0, 1, 2, 3, 4
 MASK_NONE, MASK_ALIBI, MASK_ALIBI_SQRT, MASK_ALIBI_LEFT, MASK_CAUSAL = 0, 3, 4, 5, 9
 MLA_MASK_UNDEFINED, MLA_MASK_SPEC, MLA_MASK_FREE = 0, 1, 2
 MLA_CALC_UNDEFINED, MLA_CALC_SPEC, MLA_CALC_RING, MLA_CALC_PREFILL = 0, 1, 2, 3
@@ -32,7 +32,7 @@ MLA_CACHE_KVCACHE, MLA_CACHE_KROPE_CTKV, MLA_CACHE_INT8_NZ, MLA_CACHE_NZ = 0, 1,
 STATUS = {0: "OK", 1: "NULL_REQUIRED", 2: "INVALID_SHAPE", 3: "INVALID_DTYPE", 4: "INVALID_PARAM",
           5: "UNSUPPORTED", 6: "WORKSPACE_TOO_SMALL", 7: "CUDA_ERROR", 8: "DEVICE_TIMEOUT"}
 
-_TORCH_DTYPE = {torch.float16: F16, torch.bfloat16: BF16, torch.float32: F32, torch.int32: I32}
+_TORCH_DTYPE = {torch.float16: F16, torch.bfloat16: BF16, torch.float32: F32, torch.int32: I32, torch.int8: I8}
 _NP_DTYPE = {np.dtype(np.int32): I32, np.dtype(np.float32): F32}
 
 
@@ -233,15 +233,22 @@ def atb_like_prefix_encoder(q, k, v, block_tables, seq_len, kv_seq_len, mask_typ
 
 
 def plan_mla(q_nope, q_rope, ct_kv, k_rope, block_tables, context_lens, q_seq_len, heads, qk_scale,
-             mask_type=MLA_MASK_UNDEFINED, calc_type=MLA_CALC_UNDEFINED, cache_mode=MLA_CACHE_KROPE_CTKV,
-             lse=None, out=None, kv_heads=1) -> tuple[Op, torch.Tensor]:
-    """Plan the MLA decode/spec call; returns (op, attenOut)."""
+             mask_type=MLA_MASK_UNDEFINED, calc_type=MLA_CALC_UNDEFINED, cache_mode=None,
+             lse=None, out=None, kv_heads=1, qk_descale=None, pv_descale=None) -> tuple[Op, torch.Tensor]:
+    """Plan the MLA decode/spec call; returns (op, attenOut).
+
+    An int8 ``ct_kv`` selects the int8 latent cache (cacheMode INT8_NZCACHE, ND layout) and needs
+    ``qk_descale`` / ``pv_descale`` ([heads] fp32 on the device); ``q_nope`` may then be int8 too.
+    """
     L = lib()
-    out = torch.empty_like(q_nope) if out is None else out
+    if cache_mode is None:
+        cache_mode = MLA_CACHE_INT8_NZ if ct_kv.dtype == torch.int8 else MLA_CACHE_KROPE_CTKV
+    out = (torch.empty(q_rope.shape[:-1] + (q_nope.shape[-1],), dtype=q_rope.dtype, device=q_rope.device)
+           if out is None else out)
     cl = _host_i32(context_lens)
     qs = None if q_seq_len is None else _host_i32(q_seq_len)
     ts = [tensor(q_nope), tensor(q_rope), tensor(ct_kv), tensor(k_rope), tensor(block_tables), tensor(cl), None,
-          tensor(qs), None, None]
+          tensor(qs), tensor(qk_descale), tensor(pv_descale)]
     to, tl = tensor(out), tensor(lse)
     ws = ctypes.c_uint64(0)
     h = ctypes.c_void_p(0)
@@ -249,16 +256,17 @@ def plan_mla(q_nope, q_rope, ct_kv, k_rope, block_tables, context_lens, q_seq_le
                                              int(mask_type), int(calc_type), int(cache_mode), _ref(to), _ref(tl),
                                              ctypes.byref(ws), ctypes.byref(h)))
     return Op(h, ws.value, L.atb_like_mla, q_nope.device,
-              (q_nope, q_rope, ct_kv, k_rope, block_tables, cl, qs, out, lse)), out
+              (q_nope, q_rope, ct_kv, k_rope, block_tables, cl, qs, out, lse, qk_descale, pv_descale)), out
 
 
 def atb_like_mla(q_nope, q_rope, ct_kv, k_rope, block_tables, context_lens, q_seq_len, heads, qk_scale,
-                 mask_type=MLA_MASK_UNDEFINED, calc_type=MLA_CALC_UNDEFINED, return_lse=False):
+                 mask_type=MLA_MASK_UNDEFINED, calc_type=MLA_CALC_UNDEFINED, return_lse=False, qk_descale=None,
+                 pv_descale=None):
     return_lse = return_lse or calc_type == MLA_CALC_RING  # ring mode always returns the lse
     lse = (torch.empty((q_nope.shape[0], heads, 1), dtype=torch.float32, device=q_nope.device)
            if return_lse else None)
     op, out = plan_mla(q_nope, q_rope, ct_kv, k_rope, block_tables, context_lens, q_seq_len, heads, qk_scale,
-                       mask_type, calc_type, lse=lse)
+                       mask_type, calc_type, lse=lse, qk_descale=qk_descale, pv_descale=pv_descale)
     op()
     return (out, lse) if return_lse else out
 

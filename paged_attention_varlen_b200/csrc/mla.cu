@@ -38,6 +38,17 @@
 //               the O rows are normalised into the last tile's slot and one
 //               thread writes them out with TMA stores; then the 128 threads
 //               load the next chunk's query into tensor memory.
+//
+// int8 latent cache (the MLA page's INT8 cache mode with its qkDescale and
+// pvDescale rows, kept in the ND layout here).  The producer stages each tile's
+// int8 ctKV codes (32 KB) in the upper half of the slot's ctKV area, three
+// tiles ahead as above; four more warps (6..9) read them, wait until all 128
+// have (their T output overwrites that half), and write the tile as T (every
+// int8 code is a T value) in the swizzled layout the MMAs read, so the QK and
+// PV MMAs are the same T MMAs as above on half the cache bytes.  The
+// qRope kRope part goes to its own accumulator (columns 320..383) so that the
+// softmax forms qkDescale[h] * qNope.ctKV + qRope.kRope; pvDescale[h] joins the
+// 1 / l of the epilogue.  An int8 qNope is converted on its way into tensor memory.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -71,8 +82,9 @@ constexpr int kQrBytes = kBlk;             // the 64 x 64 qRope rows (qNope live
 constexpr int kKvBytes = 9 * kBlk;         // 64 keys x 576 x 2 B: ctKV blocks 0..7, kRope block 8
 constexpr int kPOff = 8 * kBlk;            // P(j) overwrites tile j's kRope block once S(j) is computed
 constexpr int kStages = 3;
-// q_full, kv_full[3], kv_empty[3], p_full[3], pv_last, s_full, s_free, fin, st_full, st_free
-constexpr int kNBars = 1 + 3 * kStages + 6;
+// q_full, kv_full[3], kv_empty[3], p_full[3], pv_last, s_full, s_free, fin, st_full, st_free, cv_full[3], cv_read
+constexpr int kNBars = 1 + 3 * kStages + 6 + kStages + 1;
+constexpr int kI8Off = 4 * kBlk;           // int8 cache: the tile's codes ([4][64 keys][128 B], 128B swizzle)
 constexpr int kSmem = 1024 + kQrBytes + kStages * kKvBytes + kNBars * 8 + 16;
 static_assert(kSmem <= 232448, "shared memory budget");
 static_assert(8 * kBlk <= kKvBytes, "the output staging (eight 8 KB boxes) must fit in a ring slot");
@@ -81,6 +93,8 @@ static_assert(8 * kBlk <= kKvBytes, "the output staging (eight 8 KB boxes) must 
 // (columns 0..511: output columns 0..255 and 256..511 as two N = 256 accumulators)
 constexpr uint32_t kQnCol = 0;
 constexpr uint32_t kSCol = 256;
+constexpr uint32_t kSRCol = 320;           // int8 cache: the qRope kRope part of S, lanes 0..15
+constexpr int kConvWarp0 = 6;              // int8 cache: warps 6..9 convert ctKV tiles
 constexpr uint32_t kOLane = 16;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPlannedSms = 148;           // SMs of the part the schedule is cut for
@@ -124,6 +138,9 @@ struct MlaParams {
   int32_t block_size;
   int32_t oob_row;
   float scale_log2;
+  const float* qk_descale;  // [heads], int8 cache only
+  const float* pv_descale;  // [heads], int8 cache only
+  int32_t qn_int8;          // qNope holds int8 codes (int8 cache only)
 };
 
 __device__ __forceinline__ uint32_t pack2(float a, float b, __nv_bfloat16*) {
@@ -133,6 +150,38 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, __nv_bfloat16*) {
 __device__ __forceinline__ uint32_t pack2(float a, float b, __half*) {
   __half2 v = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Four int8 codes (one 32-bit word, the first code in the low byte) to four T values, exactly,
+// as two words of packed pairs.  The code v is biased to v + 128 in [0, 255] and placed in the low
+// mantissa bits of a float whose unit in the last place is 1 (2^23 in binary32, 2^10 in binary16);
+// subtracting that base plus 128 leaves v.  A binary32 integer of magnitude <= 128 has zeros in its
+// low 16 bits, so its upper half is the exact bf16.
+__device__ __forceinline__ void i8x4_to_pairs(uint32_t w, uint32_t& lo, uint32_t& hi, __nv_bfloat16*) {
+  const uint32_t u = w ^ 0x80808080u;
+  const uint64_t bias = f2pack(-8388736.f, -8388736.f);  // -(2^23 + 128)
+  const uint64_t a = add_x2(f2pack(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540)),
+                                   __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7541))), bias);
+  const uint64_t b = add_x2(f2pack(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7542)),
+                                   __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7543))), bias);
+  lo = __byte_perm(static_cast<uint32_t>(a), static_cast<uint32_t>(a >> 32), 0x7632);
+  hi = __byte_perm(static_cast<uint32_t>(b), static_cast<uint32_t>(b >> 32), 0x7632);
+}
+__device__ __forceinline__ void i8x4_to_pairs(uint32_t w, uint32_t& lo, uint32_t& hi, __half*) {
+  const uint32_t u = w ^ 0x80808080u;
+  uint32_t a = __byte_perm(u, 0x64646464u, 0x4140);  // binary16 1024 + (v + 128) for codes 0 and 1
+  uint32_t b = __byte_perm(u, 0x64646464u, 0x4342);  // ... and for codes 2 and 3
+  const __half2 bias = __half2half2(__ushort_as_half(static_cast<unsigned short>(0x6480u)));  // 1152
+  const __half2 ha = __hsub2(*reinterpret_cast<const __half2*>(&a), bias);
+  const __half2 hb = __hsub2(*reinterpret_cast<const __half2*>(&b), bias);
+  lo = *reinterpret_cast<const uint32_t*>(&ha);
+  hi = *reinterpret_cast<const uint32_t*>(&hb);
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
+  return v;
 }
 
 // Warp-uniform wait on all lanes (each lane observes the phase itself).
@@ -145,6 +194,8 @@ __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, int* st
 // rows into shared memory by TMA (thread 0).  Every thread arrives on q_full once.
 // Tensor-memory stores are warp-wide: lanes 16..31 write zeros into their columns 0..255, which
 // hold O, so this runs only while O is free (before the piece's first PV, after the last epilogue).
+// An int8 qNope (int8 cache only) is converted to T exactly on the way.
+template <typename T>
 __device__ __forceinline__ void load_query(const MlaParams& p, const CUtensorMap* tmQr, uint8_t* sQr,
                                            uint64_t* q_full, uint32_t tmem_warp, int h0, int token0, int t_local,
                                            int head, bool upper) {
@@ -152,27 +203,46 @@ __device__ __forceinline__ void load_query(const MlaParams& p, const CUtensorMap
     mbar_expect_tx_only(q_full, kQrBytes);  // thread 0 arrives below, with the others
     tma_load_3d(sQr, tmQr, q_full, 0, h0, token0);
   }
-  const uint4* src = reinterpret_cast<const uint4*>(p.q_nope + (((size_t)(token0 + t_local) * p.heads + head) * kDNope) * 2);
+  const size_t row = (size_t)(token0 + t_local) * p.heads + head;
+  if (p.qn_int8) {
+    const uint4* src = reinterpret_cast<const uint4*>(p.q_nope + row * kDNope);
 #pragma unroll
-  for (int c32 = 0; c32 < 8; ++c32) {  // 32 columns = 64 elements = 128 B of the row per store
-    uint32_t r[32];
+    for (int c32 = 0; c32 < 8; ++c32) {  // 32 columns = 64 elements = 64 B of int8 codes per store
+      uint32_t r[32];
 #pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      const uint4 w = upper ? make_uint4(0u, 0u, 0u, 0u) : __ldg(src + c32 * 8 + v);
-      r[4 * v + 0] = w.x;
-      r[4 * v + 1] = w.y;
-      r[4 * v + 2] = w.z;
-      r[4 * v + 3] = w.w;
+      for (int v = 0; v < 4; ++v) {
+        const uint4 w = upper ? make_uint4(0u, 0u, 0u, 0u) : __ldg(src + c32 * 4 + v);
+        i8x4_to_pairs(w.x, r[8 * v + 0], r[8 * v + 1], (T*)nullptr);
+        i8x4_to_pairs(w.y, r[8 * v + 2], r[8 * v + 3], (T*)nullptr);
+        i8x4_to_pairs(w.z, r[8 * v + 4], r[8 * v + 5], (T*)nullptr);
+        i8x4_to_pairs(w.w, r[8 * v + 6], r[8 * v + 7], (T*)nullptr);
+      }
+      tmem_st32(tmem_warp + kQnCol + c32 * 32, r);
     }
-    tmem_st32(tmem_warp + kQnCol + c32 * 32, r);
+  } else {
+    const uint4* src = reinterpret_cast<const uint4*>(p.q_nope + row * kDNope * 2);
+#pragma unroll
+    for (int c32 = 0; c32 < 8; ++c32) {  // 32 columns = 64 elements = 128 B of the row per store
+      uint32_t r[32];
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        const uint4 w = upper ? make_uint4(0u, 0u, 0u, 0u) : __ldg(src + c32 * 8 + v);
+        r[4 * v + 0] = w.x;
+        r[4 * v + 1] = w.y;
+        r[4 * v + 2] = w.z;
+        r[4 * v + 3] = w.w;
+      }
+      tmem_st32(tmem_warp + kQnCol + c32 * 32, r);
+    }
   }
   tmem_st_wait();
   tc_fence_before();
   mbar_arrive(q_full);
 }
 
-template <typename T>
-__global__ void __launch_bounds__(192, 1)
+// KV8: int8 latent cache (warps 6..9 convert the ctKV tiles)
+template <typename T, bool KV8>
+__global__ void __launch_bounds__(KV8 ? 320 : 192, 1)
     mla_kernel(const __grid_constant__ CUtensorMap tmQr, const __grid_constant__ CUtensorMap tmKV,
                const __grid_constant__ CUtensorMap tmKV3, const __grid_constant__ CUtensorMap tmKR,
                const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmPO, const MlaParams p) {
@@ -191,6 +261,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* fin = pv_last + 3;
   uint64_t* st_full = pv_last + 4;  // the 128 softmax threads have written a round of output boxes
   uint64_t* st_free = pv_last + 5;  // the stores of a round have read their boxes
+  uint64_t* cv_full = pv_last + 6;  // [kStages] int8 cache: the converters have written the slot's ctKV
+  uint64_t* cv_read = pv_last + 6 + kStages;  // int8 cache: the 128 converters have read a tile's codes
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNBars);
 
   const int warp = threadIdx.x >> 5;
@@ -214,6 +286,10 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(fin, 1);
     mbar_init(st_full, 128);
     mbar_init(st_free, 1);
+    if (KV8) {
+      for (int s = 0; s < kStages; ++s) mbar_init(cv_full + s, 128);
+      mbar_init(cv_read, 128);
+    }
     fence_mbar_init();
   }
   if (warp == 5) {
@@ -246,8 +322,9 @@ __global__ void __launch_bounds__(192, 1)
         const int n_pages = (pc.last + p.tpc + bs - 1) / bs;  // pages holding keys <= the chunk's last allowed key
         if (k + 1 < k1) {  // the next chunk's qNope rows, for the softmax threads' loads at the piece boundary
           const MlaPiece pn = p.pieces[k + 1];
+          const int qes = p.qn_int8 ? 1 : 2;
           for (int t = 0; t < p.tpc; ++t)
-            bulk_prefetch_l2(p.q_nope + (((size_t)(pn.token0 + t) * p.heads + h0) * kDNope) * 2, p.hpc * kDNope * 2);
+            bulk_prefetch_l2(p.q_nope + (((size_t)(pn.token0 + t) * p.heads + h0) * kDNope) * qes, p.hpc * kDNope * qes);
         }
         for (int j = 0; j < pc.n_tiles; ++j) {
           for (; ALA_MLA_PREFETCH_TILES > 0 && kf < k1 && Gf <= G + ALA_MLA_PREFETCH_TILES; ++Gf) {
@@ -258,7 +335,8 @@ __global__ void __launch_bounds__(192, 1)
               const int pg = pos / bs;
               const size_t row = pg < npf ? (size_t)btf[pg] * bs + (pos - pg * bs) : (size_t)p.oob_row;
               if (row < (size_t)p.oob_row) {  // a block index outside the cache is never touched
-                bulk_prefetch_l2(p.ct_kv + row * 1024, box_rows * 1024);
+                constexpr int kRowBytes = KV8 ? kDNope : 2 * kDNope;
+                bulk_prefetch_l2(p.ct_kv + row * kRowBytes, box_rows * kRowBytes);
                 bulk_prefetch_l2(p.k_rope + row * 128, box_rows * 128);
               }
             }
@@ -273,13 +351,20 @@ __global__ void __launch_bounds__(192, 1)
             break;
           }
           uint8_t* dst = sKV + s * kKvBytes;
-          mbar_expect_tx(kv_full + s, kKvBytes);
+          mbar_expect_tx(kv_full + s, KV8 ? 5 * kBlk : kKvBytes);  // int8 cache: 32 KB of codes + kRope
           const int j0 = pc.kv_begin + j * kTileKeys;
           for (int r0 = 0; r0 < kTileKeys; r0 += box_rows) {
             const int pos = j0 + r0;
             const int pg = pos / bs;
             const int row = pg < n_pages ? bt[pg] * bs + (pos - pg * bs) : p.oob_row;  // past the last page: zeros
-            if (whole) {
+            if (KV8) {  // the codes, [4 blocks of 128 columns][key][128 B], into the upper half of the ctKV area
+              if (whole) {
+                tma_load_3d(dst + kI8Off, &tmKV3, kv_full + s, 0, row, 0);
+              } else {
+                for (int cb = 0; cb < 4; ++cb)
+                  tma_load_2d(dst + kI8Off + cb * kBlk + r0 * 128, &tmKV, kv_full + s, cb * 128, row);
+              }
+            } else if (whole) {
               tma_load_3d(dst, &tmKV3, kv_full + s, 0, row, 0);  // [column block][key][64 elements]
             } else {
               for (int cb = 0; cb < 8; ++cb) tma_load_2d(dst + cb * kBlk + r0 * 128, &tmKV, kv_full + s, cb * 64, row);
@@ -318,6 +403,7 @@ __global__ void __launch_bounds__(192, 1)
         // query; it may lead PV by one tile (S is single-buffered).  PV(Gp) needs P(Gp).
         const int sq = Gq % kStages;
         if (Gq < total && Gq - Gp < 2 && mbar_test_wait(kv_full + sq, (Gq / kStages) & 1) &&
+            (!KV8 || mbar_test_wait(cv_full + sq, (Gq / kStages) & 1)) &&
             (Gq == 0 || mbar_test_wait(s_free, (Gq - 1) & 1)) && (jq > 0 || mbar_test_wait(q_full, (kq - k0) & 1))) {
           tc_fence_after();
           const uint64_t so = (uint64_t)((sq * kKvBytes) >> 4);
@@ -326,9 +412,9 @@ __global__ void __launch_bounds__(192, 1)
             mma_ts(tmem + kSCol, tmem + kQnCol + kk * 8, dk + so + (uint64_t)(((kk >> 2) * kBlk + (kk & 3) * 32) >> 4),
                    idesc_qk, kk > 0 ? 1u : 0u, false);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)  // qRope x kRope from shared memory
-            mma_ss(tmem + kSCol, dqr + (uint64_t)((kk * 32) >> 4), dk + so + (uint64_t)((8 * kBlk + kk * 32) >> 4),
-                   idesc_qk, 1u, false);
+          for (int kk = 0; kk < 4; ++kk)  // qRope x kRope from shared memory (own accumulator with an int8 cache)
+            mma_ss(tmem + (KV8 ? kSRCol : kSCol), dqr + (uint64_t)((kk * 32) >> 4),
+                   dk + so + (uint64_t)((8 * kBlk + kk * 32) >> 4), idesc_qk, (!KV8 || kk > 0) ? 1u : 0u, false);
           mma_commit(s_full);
           ++Gq;
           if (++jq == nq) {
@@ -374,6 +460,62 @@ __global__ void __launch_bounds__(192, 1)
       mma_commit(fin);
       mbar_wait(fin, 0, status, kDevTimeoutFinal);
     }
+  } else if (KV8 && warp >= kConvWarp0) {
+    // ------------------------------------------------------------ int8 ctKV -> T (warps 6..9)
+    // Thread ct handles keys kk0 + 8m (m = 0..7) of every tile and, of each, the 16-byte chunks of
+    // codes c0 and c0 + 16 (columns 16c .. 16c+15).  Both its shared-memory reads (the codes, 128B
+    // swizzle) and its writes hit each 16-byte bank group four times per warp (no conflicts).
+    const int ct = threadIdx.x - kConvWarp0 * 32;
+    const int kk0 = ct & 7;
+    const int c0 = ct >> 3;
+    int G = 0;
+    bool ok = true;
+    for (int k = k0; k < k1 && ok; ++k) {
+      const int n_tiles = p.pieces[k].n_tiles;
+      for (int j = 0; j < n_tiles; ++j, ++G) {
+        const int s = G % kStages;
+        if (!wait_all(kv_full + s, (G / kStages) & 1, status, kDevTimeoutKFull)) {
+          ok = false;
+          break;
+        }
+        const uint32_t slot = smem_addr(sKV + s * kKvBytes);
+        uint4 v[8][2];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int c = c0 + 16 * h;  // 128-column block c >> 3, its 16-byte chunk c & 7
+            v[m][h] = ld_shared_v4(slot + kI8Off + (c >> 3) * kBlk + (kk0 + 8 * m) * 128 + (((c & 7) ^ kk0) << 4));
+          }
+        }
+        // the T tile overwrites the codes: every converter must have read its share first
+        mbar_arrive(cv_read);
+        if (!wait_all(cv_read, G & 1, status, kDevTimeoutKFull)) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const uint32_t key_row = slot + (kk0 + 8 * m) * 128;  // 128B swizzle of key row r: chunk q at q ^ (r & 7)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int c = c0 + 16 * h;
+            const uint4 w = v[m][h];
+            uint32_t o[8];
+            i8x4_to_pairs(w.x, o[0], o[1], (T*)nullptr);
+            i8x4_to_pairs(w.y, o[2], o[3], (T*)nullptr);
+            i8x4_to_pairs(w.z, o[4], o[5], (T*)nullptr);
+            i8x4_to_pairs(w.w, o[6], o[7], (T*)nullptr);
+            const uint32_t blk = key_row + (c >> 2) * kBlk;  // 64-column block of columns 16c .. 16c+15
+            const int q = 2 * (c & 3);                        // their two 16-byte chunks in the block's row
+            st_shared_v4(blk + ((q ^ kk0) << 4), make_uint4(o[0], o[1], o[2], o[3]));
+            st_shared_v4(blk + (((q + 1) ^ kk0) << 4), make_uint4(o[4], o[5], o[6], o[7]));
+          }
+        }
+        fence_proxy_async_smem();  // visible to the tensor cores
+        mbar_arrive(cv_full + s);
+      }
+    }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
     // lanes 0..15 of warp w own S row 16w + l; lanes 16..31 own O row 16w + (l - 16)
@@ -385,10 +527,12 @@ __global__ void __launch_bounds__(192, 1)
     const int sw = hr & 7;  // 128-byte swizzle of the row's 16-byte chunks
     const float scale = p.scale_log2;
     const bool raw_max = scale > 0.f;  // max of the raw scores, scale folded into the exponent
+    const float qk_d = KV8 ? p.qk_descale[head] : 1.f;
+    const float pv_d = KV8 ? p.pv_descale[head] : 1.f;
     bool ok = true;
     int G = 0;  // tiles consumed
     int R = 0;  // output staging rounds
-    if (k0 < k1) load_query(p, &tmQr, sQr, q_full, tmem_warp, h0, p.pieces[k0].token0, t_local, head, upper);
+    if (k0 < k1) load_query<T>(p, &tmQr, sQr, q_full, tmem_warp, h0, p.pieces[k0].token0, t_local, head, upper);
     for (int k = k0; k < k1 && ok; ++k) {
       const MlaPiece pc = p.pieces[k];
       const int row_last = pc.last + t_local;
@@ -403,9 +547,20 @@ __global__ void __launch_bounds__(192, 1)
           uint32_t regs[2][32];
           tmem_ld32(tmem_warp + kSCol, regs[0]);
           tmem_ld32(tmem_warp + kSCol + 32, regs[1]);
-          tmem_ld_wait();
+          if constexpr (KV8) {
+            // score = qkDescale * (qNope . ctKV) + qRope . kRope
+            uint32_t rr[2][32];
+            tmem_ld32(tmem_warp + kSRCol, rr[0]);
+            tmem_ld32(tmem_warp + kSRCol + 32, rr[1]);
+            tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < kTileKeys; ++c) x[c] = __uint_as_float(regs[c >> 5][c & 31]);
+            for (int c = 0; c < kTileKeys; ++c)
+              x[c] = fmaf(qk_d, __uint_as_float(regs[c >> 5][c & 31]), __uint_as_float(rr[c >> 5][c & 31]));
+          } else {
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < kTileKeys; ++c) x[c] = __uint_as_float(regs[c >> 5][c & 31]);
+          }
         }
         const int lim = row_last - (pc.kv_begin + j * kTileKeys);  // columns c <= lim are allowed
         if (!raw_max) {
@@ -495,7 +650,7 @@ __global__ void __launch_bounds__(192, 1)
       const float m_row = __shfl_sync(kFull, m_run, lane & 15);
       // a row whose allowed keys all lie before this range (possible only in a partial) contributes nothing
       const bool empty = !(l_row > 0.f);
-      const float inv_l = empty ? 0.f : 1.f / l_row;
+      const float inv_l = empty ? 0.f : pv_d / l_row;  // pv_d = 1 unless the cache is int8
       const float lse_row = empty ? -INFINITY : (m_row == -INFINITY ? 0.f : m_row) * kLn2 + logf(l_row);
       uint8_t* stage = sKV + s_last * kKvBytes;
       const uint32_t stage_row = smem_addr(stage) + hr * 128;  // this row in each 8 KB staging box
@@ -573,7 +728,7 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       if (k + 1 < k1) {
         const MlaPiece pn = p.pieces[k + 1];
-        load_query(p, &tmQr, sQr, q_full, tmem_warp, h0, pn.token0, t_local, head, upper);
+        load_query<T>(p, &tmQr, sQr, q_full, tmem_warp, h0, pn.token0, t_local, head, upper);
       }
       // the staging slot goes back to the producer once the stores have read it
       if (threadIdx.x == 0) {
@@ -665,6 +820,7 @@ bool encode(CUtensorMap* map, void* base, int32_t dtype, int rank, const cuuint6
   cuuint32_t estr[3] = {1, 1, 1};
   const CUtensorMapDataType t = dtype == ALA_F16   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                 : dtype == ALA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                : dtype == ALA_I8  ? CU_TENSOR_MAP_DATA_TYPE_UINT8  // int8 codes move as bytes
                                                    : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   return enc(map, t, rank, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -682,8 +838,9 @@ int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, co
   if (!qNope->data || !qRope->data || !ctKV->data || !kRope->data || !blockTables->data || !contextLens->data ||
       !attenOut->data)
     return mfail(err, n, ALA_NULL_REQUIRED, "a required tensor has a NULL data pointer");
-  if (cacheMode != ALA_MLA_CACHE_KROPE_CTKV)
-    return mfail(err, n, ALA_UNSUPPORTED, "only cacheMode KROPE_CTKV (1) is built");
+  const bool kv8 = cacheMode == ALA_MLA_CACHE_INT8_NZ;
+  if (cacheMode != ALA_MLA_CACHE_KROPE_CTKV && !kv8)
+    return mfail(err, n, ALA_UNSUPPORTED, "cacheMode must be KROPE_CTKV (1) or INT8_NZCACHE (2, int8 ctKV in the ND layout)");
   if (calcType == ALA_MLA_CALC_RING || calcType == ALA_MLA_CALC_PREFILL)
     return mfail(err, n, ALA_UNSUPPORTED, "calcType RING and PREFILL are not built");
   if (calcType != ALA_MLA_CALC_UNDEFINED && calcType != ALA_MLA_CALC_SPEC)
@@ -694,16 +851,34 @@ int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, co
     return mfail(err, n, maskType == ALA_MLA_MASK_FREE ? ALA_UNSUPPORTED : ALA_INVALID_PARAM,
                  "maskType must be UNDEFINED (0) or SPEC (1)");
   if (mask && mask->data) return mfail(err, n, ALA_INVALID_PARAM, "mask must be NULL: the spec mask is generated");
-  if ((qkDescale && qkDescale->data) || (pvDescale && pvDescale->data))
-    return mfail(err, n, ALA_INVALID_PARAM, "qkDescale/pvDescale must be NULL (int8 cache not built)");
+  if (kv8) {
+    if (!qkDescale || !qkDescale->data || !pvDescale || !pvDescale->data)
+      return mfail(err, n, ALA_NULL_REQUIRED, "qkDescale and pvDescale are required with the int8 cache (cacheMode 2)");
+    if (qkDescale->dtype != ALA_F32 || pvDescale->dtype != ALA_F32)
+      return mfail(err, n, ALA_INVALID_DTYPE, "qkDescale and pvDescale must be fp32");
+    if (qkDescale->ndim != 1 || qkDescale->dims[0] != headNum || pvDescale->ndim != 1 || pvDescale->dims[0] != headNum)
+      return mfail(err, n, ALA_INVALID_SHAPE, "qkDescale and pvDescale must be [headNum]");
+  } else if ((qkDescale && qkDescale->data) || (pvDescale && pvDescale->data)) {
+    return mfail(err, n, ALA_INVALID_PARAM, "qkDescale/pvDescale are passed only with the int8 cache (cacheMode 2)");
+  }
   if (headNum <= 0) return mfail(err, n, ALA_INVALID_PARAM, "headNum must be > 0");
   if (headNum % 64 != 0) return mfail(err, n, ALA_UNSUPPORTED, "headNum must be a multiple of 64");
   if (kvHeadNum != 1) return mfail(err, n, ALA_UNSUPPORTED, "kvHeadNum must be 1");
   if (!std::isfinite(qkScale)) return mfail(err, n, ALA_INVALID_PARAM, "qkScale must be finite");
-  const int32_t dt = qNope->dtype;
-  if (dt != ALA_BF16 && dt != ALA_F16) return mfail(err, n, ALA_INVALID_DTYPE, "qNope must be bf16 or f16");
-  if (qRope->dtype != dt || ctKV->dtype != dt || kRope->dtype != dt || attenOut->dtype != dt)
-    return mfail(err, n, ALA_INVALID_DTYPE, "qRope, ctKV, kRope and attenOut must have qNope's dtype");
+  const int32_t dt = qRope->dtype;  // the MMA and output type
+  if (dt != ALA_BF16 && dt != ALA_F16) return mfail(err, n, ALA_INVALID_DTYPE, "qRope must be bf16 or f16");
+  if (kv8) {
+    if (ctKV->dtype != ALA_I8) return mfail(err, n, ALA_INVALID_DTYPE, "ctKV must be int8 with cacheMode 2");
+    if (qNope->dtype != ALA_I8 && qNope->dtype != dt)
+      return mfail(err, n, ALA_INVALID_DTYPE, "qNope must be int8 or qRope's dtype with cacheMode 2");
+    if (kRope->dtype != dt || attenOut->dtype != dt)
+      return mfail(err, n, ALA_INVALID_DTYPE, "kRope and attenOut must have qRope's dtype");
+    // the converter and query loads read 16-byte pieces
+    if (reinterpret_cast<uintptr_t>(ctKV->data) % 16 || reinterpret_cast<uintptr_t>(qNope->data) % 16)
+      return mfail(err, n, ALA_INVALID_PARAM, "ctKV and qNope must be 16-byte aligned");
+  } else if (qNope->dtype != dt || ctKV->dtype != dt || kRope->dtype != dt || attenOut->dtype != dt) {
+    return mfail(err, n, ALA_INVALID_DTYPE, "qNope, ctKV, kRope and attenOut must have qRope's dtype");
+  }
   if (blockTables->dtype != ALA_I32 || contextLens->dtype != ALA_I32)
     return mfail(err, n, ALA_INVALID_DTYPE, "blockTables and contextLens must be int32");
   if (qNope->ndim != 3 || qNope->dims[1] != headNum || qNope->dims[2] != 512)
@@ -757,6 +932,10 @@ int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, co
   if (ctKV->dims[0] * bs >= ((int64_t)1 << 31)) return mfail(err, n, ALA_UNSUPPORTED, "cache has more than 2^31 rows");
 
   plan->dtype = dt;
+  plan->kv8 = kv8;
+  plan->qn_int8 = kv8 && qNope->dtype == ALA_I8;
+  plan->qk_descale = kv8 ? static_cast<const float*>(qkDescale->data) : nullptr;
+  plan->pv_descale = kv8 ? static_cast<const float*>(pvDescale->data) : nullptr;
   plan->heads = headNum;
   plan->batch = batch;
   plan->block_size = (int32_t)bs;
@@ -882,10 +1061,18 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
     cuuint64_t kv3_dims[3] = {64, rows, 8};
     cuuint64_t kv3_str[2] = {512 * es, 64 * es};
     cuuint32_t kv3_box[3] = {64, (cuuint32_t)kTileKeys, 8};
-    if (!encode(&plan->tmKV3, plan->ct_kv, plan->dtype, 3, kv3_dims, kv3_str, kv3_box) ||
-        !encode(&plan->tmQn, plan->q_nope, plan->dtype, 3, qn_dims, qn_str, q_box) ||
-        !encode(&plan->tmQr, plan->q_rope, plan->dtype, 3, qr_dims, qr_str, q_box) ||
-        !encode(&plan->tmKV, plan->ct_kv, plan->dtype, 2, kv_dims, kv_str, kv_box) ||
+    // int8 codes: 512 bytes a row, seen as 128-byte column blocks (4 per row), same boxes of keys
+    cuuint64_t k8_dims[2] = {512, rows};
+    cuuint64_t k8_str[1] = {512};
+    cuuint32_t k8_box[2] = {128, kv_box_rows};
+    cuuint64_t k83_dims[3] = {128, rows, 4};
+    cuuint64_t k83_str[2] = {512, 128};
+    cuuint32_t k83_box[3] = {128, (cuuint32_t)kTileKeys, 4};
+    const bool kv_ok = plan->kv8 ? (encode(&plan->tmKV3, plan->ct_kv, ALA_I8, 3, k83_dims, k83_str, k83_box) &&
+                                    encode(&plan->tmKV, plan->ct_kv, ALA_I8, 2, k8_dims, k8_str, k8_box))
+                                 : (encode(&plan->tmKV3, plan->ct_kv, plan->dtype, 3, kv3_dims, kv3_str, kv3_box) &&
+                                    encode(&plan->tmKV, plan->ct_kv, plan->dtype, 2, kv_dims, kv_str, kv_box));
+    if (!kv_ok || !encode(&plan->tmQr, plan->q_rope, plan->dtype, 3, qr_dims, qr_str, q_box) ||
         !encode(&plan->tmKR, plan->k_rope, plan->dtype, 2, kr_dims, kr_str, kv_box) ||
         !encode(&plan->tmO, plan->out, plan->dtype, 3, qn_dims, qn_str, q_box))
       return mfail(err, n, ALA_CUDA_ERROR, "cuTensorMapEncodeTiled failed (pointers must be 16-byte aligned)");
@@ -932,10 +1119,17 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
   p.block_size = plan->block_size;
   p.oob_row = (int32_t)(plan->num_blocks * plan->block_size);
   p.scale_log2 = plan->qk_scale * kLog2e;
-  auto kern = plan->dtype == ALA_F16 ? mla_kernel<__half> : mla_kernel<__nv_bfloat16>;
+  p.qk_descale = plan->qk_descale;
+  p.pv_descale = plan->pv_descale;
+  p.qn_int8 = plan->qn_int8 ? 1 : 0;
+  const bool f16 = plan->dtype == ALA_F16;
+  auto kern = plan->kv8 ? (f16 ? mla_kernel<__half, true> : mla_kernel<__nv_bfloat16, true>)
+                        : (f16 ? mla_kernel<__half, false> : mla_kernel<__nv_bfloat16, false>);
+  const int threads = plan->kv8 ? 320 : 192;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e == cudaSuccess) {
-    kern<<<plan->n_work, 192, kSmem, stream>>>(plan->tmQr, plan->tmKV, plan->tmKV3, plan->tmKR, plan->tmO, plan->tmPO, p);
+    kern<<<plan->n_work, threads, kSmem, stream>>>(plan->tmQr, plan->tmKV, plan->tmKV3, plan->tmKR, plan->tmO,
+                                                   plan->tmPO, p);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess && plan->n_combine > 0) {

@@ -13,6 +13,8 @@ namespace ala {
 struct MlaPlan {
   int32_t dtype = 0, heads = 0, batch = 0, block_size = 0, max_blocks = 0;
   int32_t calc_type = 0, mask_type = 0;
+  bool kv8 = false, qn_int8 = false;  // int8 latent cache (cacheMode 2); qNope holds int8 codes
+  const float *qk_descale = nullptr, *pv_descale = nullptr;
   float qk_scale = 1.f;
   int64_t tokens = 0, num_blocks = 0;
   void *q_nope = nullptr, *q_rope = nullptr, *ct_kv = nullptr, *k_rope = nullptr, *out = nullptr;

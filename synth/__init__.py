@@ -304,7 +304,7 @@ def make_mla_int8(name, context_lens, qs, heads, seed, rng=None, block_size=128,
                    qk_descale=qk_descale, pv_descale=pv_descale)
 
 
-def mla_decode_int8(seed=1005, batch=64, lo=1024, hi=16384, heads=128, qs=1) -> MlaCase:
+def mla_decode_int8(seed=1004, batch=64, lo=1024, hi=16384, heads=128, qs=1) -> MlaCase:
     """The MLA decode workload over an int8 latent cache: batch 64, contextLens ~ U{1024..16384}, 128 heads,
     512 + 64, paged bs = 128, int8 qNope and ctKV, bf16 qRope / kRope."""
     rng = np.random.Generator(np.random.PCG64(seed))

@@ -140,7 +140,16 @@ def _plan_mla(**over):
     a.update(over)
     return ala.plan_mla(a["q_nope"], a["q_rope"], a["ct_kv"], a["k_rope"], a["block_tables"], a["context_lens"],
                         a["q_seq_len"], a["heads"], a["qk_scale"], a["mask_type"], a["calc_type"], a["cache_mode"],
-                        kv_heads=a["kv_heads"], lse=a.get("lse"))
+                        kv_heads=a["kv_heads"], lse=a.get("lse"), qk_descale=a.get("qk_descale"),
+                        pv_descale=a.get("pv_descale"))
+
+
+def _int8_cache(**over):
+    # the int8 latent cache (cacheMode 2): int8 ctKV (and qNope) with per-head fp32 descales
+    d = dict(ct_kv=torch.zeros(6, 64, 1, 512, dtype=torch.int8), q_nope=torch.zeros(3, 128, 512, dtype=torch.int8),
+             cache_mode=2, qk_descale=torch.ones(128), pv_descale=torch.ones(128))
+    d.update(over)
+    return d
 
 
 def test_mla_plan_ok():
@@ -154,6 +163,38 @@ def test_mla_prefill_plans_with_qseqlen():
               q_seq_len=[1, 5, 3], calc_type=3)
     _plan_mla(q_nope=torch.zeros(9, 128, 512, dtype=torch.bfloat16), q_rope=torch.zeros(9, 128, 64, dtype=torch.bfloat16),
               q_seq_len=[1, 5, 3], calc_type=3, mask_type=1)
+
+
+def test_mla_int8_cache_plans():
+    _plan_mla(**_int8_cache())
+    _plan_mla(**_int8_cache(q_nope=torch.zeros(3, 128, 512, dtype=torch.bfloat16)))  # float qNope
+    _plan_mla(**_int8_cache(q_nope=torch.zeros(6, 128, 512, dtype=torch.int8),
+                            q_rope=torch.zeros(6, 128, 64, dtype=torch.bfloat16), q_seq_len=[2, 2, 2], mask_type=1,
+                            calc_type=1))
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(qk_descale=None), 1),                                          # both descales are required
+    (dict(pv_descale=None), 1),
+    (dict(qk_descale=torch.ones(64)), 2),                                # one per head
+    (dict(pv_descale=torch.ones(128, dtype=torch.float16)), 3),          # fp32
+    (dict(ct_kv=torch.zeros(6, 64, 1, 512, dtype=torch.bfloat16)), 3),   # cacheMode 2 holds int8 codes
+    (dict(q_nope=torch.zeros(3, 128, 512, dtype=torch.float16)), 3),     # qNope: int8 or qRope's dtype
+    (dict(cache_mode=1), 4),                                             # descales only with cacheMode 2
+])
+def test_mla_int8_cache_rejects(over, status):
+    with pytest.raises(ala.AlaError) as e:
+        _plan_mla(**_int8_cache(**over))
+    assert e.value.status == status, str(e.value)
+
+
+def test_mla_int8_codes_need_cache_mode_2():
+    with pytest.raises(ala.AlaError) as e:
+        _plan_mla(ct_kv=torch.zeros(6, 64, 1, 512, dtype=torch.int8))
+    assert e.value.status == 3
+    with pytest.raises(ala.AlaError) as e:
+        _plan_mla(q_nope=torch.zeros(3, 128, 512, dtype=torch.int8))
+    assert e.value.status == 3
 
 
 def test_mla_ring_plans_with_lse():
@@ -221,7 +262,8 @@ def test_lse_merge_null_tensor():
 
 
 @pytest.mark.parametrize("over,status", [
-    (dict(cache_mode=0), 5), (dict(cache_mode=2), 5), (dict(cache_mode=3), 5),
+    (dict(cache_mode=0), 5), (dict(cache_mode=3), 5),
+    (dict(cache_mode=2), 1),                       # the int8 cache needs its descales
     (dict(calc_type=2), 1),                        # RING needs lse
     (dict(calc_type=3), 1),                        # PREFILL needs qseqlen
     (dict(calc_type=3, q_seq_len=[1, 1, 1], mask_type=2), 4),  # PREFILL is causal: UNDEFINED or SPEC only
