@@ -30,7 +30,7 @@ struct MlaPlan {
   std::vector<uint8_t> image;  // host copy of [status | pieces | lane offsets | combine list]
   void* pinned = nullptr;      // page-locked copy of `image`, made on first run
   bool maps_ready = false;
-  CUtensorMap tmQn, tmQr, tmKV, tmKV3, tmKR, tmO;
+  CUtensorMap tmQr, tmKV, tmKV3, tmKR, tmO;
   CUtensorMap tmPO;                // partial-output map, bound to the workspace it was encoded for
   const void* tmPO_base = nullptr;
   MlaPlan() = default;
