@@ -131,3 +131,36 @@ def test_mla_int8_full_size_sampled():
     check_out(out.reshape(-1, 512)[idx], ref)
     check_lse(lse.reshape(-1)[idx], lref)
     assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("heads,qs,block_size,qn_int8", [(256, 1, 256, True), (128, 2, 32, False), (64, 4, 128, True)])
+def test_mla_int8_row_block_shapes(heads, qs, block_size, qn_int8):
+    # rows per CTA = tokens per chunk x heads per group: 1 x 64 (four groups of a 256-head token, whole
+    # 256-key pages), 2 x 32 (64 heads of two tokens, pages of 32 keys) and 4 x 16
+    ctx = np.array([90, 640, 1500, qs + 3], dtype=np.int32)
+    case = synth.make_mla_int8(f"rows8_{heads}_{qs}", ctx, qs, heads, 53 + qs, block_size=block_size,
+                               qnope_int8=qn_int8)
+    out, lse, _ = _run(case)
+    ref, lref = _oracle(case)
+    check_out(out.reshape(-1, 512), ref)
+    check_lse(lse.reshape(-1), lref)
+
+
+def test_mla_int8_negative_qk_scale():
+    case = synth.make_mla_int8("neg8", np.array([100, 700], dtype=np.int32), 2, 128, 55, block_size=64)
+    case.qk_scale = -0.03
+    out, lse, _ = _run(case)
+    ref, lref = _oracle(case)
+    check_out(out.reshape(-1, 512), ref)
+    check_lse(lse.reshape(-1), lref)
+
+
+def test_mla_int8_prefill_is_causal_within_each_batch():
+    # calcType PREFILL over the int8 cache: all new tokens of a batch attend causally
+    ctx = np.array([100, 300, 520], dtype=np.int32)
+    qs = np.array([37, 300, 64], dtype=np.int32)
+    case = synth.make_mla_int8("prefill8", ctx, qs, 64, 57, block_size=64)
+    out, lse, _ = _run(case, calc_type=ala.MLA_CALC_PREFILL)
+    ref, lref = _oracle(case)
+    check_out(out.reshape(-1, 512), ref)
+    check_lse(lse.reshape(-1), lref)
