@@ -254,7 +254,7 @@ def e2e_prefill(ala, case, tens, op, steps, stream):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
-def cpu_baseline(case, budget_s=12.0):
+def cpu_baseline(case, sample_s=12.0):
     """The fp64 oracle, as it stands, on a bounded random sample of the workload's rows."""
     import oracle
     cu = np.concatenate([[0], np.cumsum(case.seq_len)])
@@ -262,7 +262,7 @@ def cpu_baseline(case, budget_s=12.0):
     rng = np.random.Generator(np.random.PCG64(7))
     n_rows = 256
     total_flops, total_s, rows_done = 0.0, 0.0, 0
-    while total_s < budget_s:
+    while total_s < sample_s:
         rows = rng.choice(case.n_tokens * case.heads, size=n_rows, replace=False)
         t0 = time.perf_counter()
         oracle.attention(case.q, case.k, case.v, case.seq_len, case.kv_seq_len, case.mask_type, case.heads,
@@ -311,10 +311,10 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     case = synth.varlen_causal_bf16()
-    cb = cpu_baseline(case, budget_s=max(3.0, 10.0 / max(1, args.steps + args.warmup)))
+    cb = cpu_baseline(case, sample_s=max(3.0, 10.0 / max(1, args.steps + args.warmup)))
     vals = []
     for _ in range(args.warmup + args.steps):
-        vals.append(cpu_baseline(case, budget_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)))["value"])
+        vals.append(cpu_baseline(case, sample_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)))["value"])
     v = statistics.mean(vals[args.warmup:]) if len(vals) > args.warmup else vals[-1]
     flops = prefill_flops(case)
     line = {"impl": "reference", "metric": "attention TFLOPS on valid tokens (prefill)", "value": v,

@@ -4,7 +4,7 @@ Tolerances (GPU result vs the fp64 oracle on the same stored inputs):
   * attention output (bf16 / fp16 / fp32 stored): max |err| <= 2e-2 and
     mean |err| <= 2e-3;
   * fp32 lse: |err| <= 1e-3 * max(1, |lse_ref|) (relative error, with the
-    reference magnitude floored at 1 so rows whose lse is near 0 are judged
+    reference magnitude floored at 1 so rows whose lse is near 0 are measured
     on the absolute scale).
 """
 import numpy as np
