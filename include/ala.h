@@ -244,6 +244,10 @@ ALA_API int varlen_attention_noalloc(const ala_tensor* query, const ala_tensor* 
  *             required with calcType RING (NULL_REQUIRED otherwise).
  * workspace   256-byte aligned; holds the schedule and, for key ranges split
  *             across CTAs, fp32 partial outputs merged by lse at the end.
+ * Environment: with ALA_MLA_PAIR=1 set when the op is planned, a request with
+ *             one token per batch, a 16-bit cache and headNum a multiple of 128
+ *             runs on the CTA-pair kernel (two CTAs per 128 heads splitting the
+ *             latent dimensions); same results, measured slower, off by default.
  * ------------------------------------------------------------------------- */
 ALA_API int atb_like_mla_get_workspace_size(
     const ala_tensor* qNope, const ala_tensor* qRope, const ala_tensor* ctKV, const ala_tensor* kRope,

@@ -11,6 +11,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <queue>
 #include <string>
@@ -561,6 +562,11 @@ extern "C" int atb_like_mla_get_workspace_size(const ala_tensor* qNope, const al
   int st = mla_plan(&o->mla, qNope, qRope, ctKV, kRope, blockTables, contextLens, mask, qSeqLen, qkDescale,
                     pvDescale, headNum, qkScale, kvHeadNum, maskType, calcType, cacheMode, attenOut, lse, err,
                     sizeof err);
+  if (st == ALA_OK) {
+    // the CTA-pair decode kernel, on request (ALA_MLA_PAIR=1 in the environment when the op is planned)
+    const char* pair = std::getenv("ALA_MLA_PAIR");
+    if (pair && pair[0] == '1' && mla_pair_eligible(&o->mla)) st = mla_pair_plan(&o->mla, err, sizeof err);
+  }
   if (st != ALA_OK) {
     delete o;
     return fail(st, "%s: %s", fn, err);
@@ -579,7 +585,8 @@ extern "C" int atb_like_mla(void* workspace, uint64_t workspaceSize, ala_op* op,
     return fail(ALA_WORKSPACE_TOO_SMALL, "%s: workspace %llu < required %llu", fn, (unsigned long long)workspaceSize,
                 (unsigned long long)op->mla.ws_size);
   char err[512] = {0};
-  int st = mla_run(&op->mla, workspace, reinterpret_cast<cudaStream_t>(stream), err, sizeof err);
+  int st = op->mla.pair ? mla_pair_run(&op->mla, workspace, reinterpret_cast<cudaStream_t>(stream), err, sizeof err)
+                        : mla_run(&op->mla, workspace, reinterpret_cast<cudaStream_t>(stream), err, sizeof err);
   if (st != ALA_OK) return fail(st, "%s: %s", fn, err);
   return ok();
 }
