@@ -183,26 +183,35 @@ ALA_API int varlen_attention(void* workspace, uint64_t workspaceSize, ala_op* op
 
 /* ---------------------------------------------------------------------------
  * varlen_attention_noalloc: varlen_attention in one call that allocates
- * nothing, for callers that cannot call cudaMalloc (code that runs while
- * someone else builds a CUDA graph, runtimes that only hand out pre-sized
- * arenas, hosts whose device allocator belongs to another component).  The
- * pages have no counterpart of this call.
+ * nothing, for callers that cannot call cudaMalloc (runtimes that only hand
+ * out pre-sized arenas, hosts whose device allocator belongs to another
+ * component).  The pages have no counterpart of this call.
  *
- * Arguments as for varlen_attention_get_workspace_size (query 3-D), plus the
- * stream; no workspace and no op.  The schedule lives in a 1 MiB array in
- * device global memory owned by the library (every GPU that loads the library
- * keeps it until exit): at most 4096 sequences and as many 128-row work units
- * as fit; larger calls return ALA_UNSUPPORTED with the limit in the message.
- * Every call rewrites that array (its status word is cleared first), so calls
- * whose GPU work overlaps race on it: order them on one stream or with events.
- * The first call on each device looks up the array's address
- * (cudaGetSymbolAddress, with that device current); make it before any stream
- * capture begins.  A successful call allocates no device or host memory.
+ * Arguments as for varlen_attention_get_workspace_size (query 3-D; lse NULL,
+ * [nTokens, headNum] or [nTokens, headNum, 1]), plus the stream; no workspace
+ * and no op.  The schedule lives in a 1 MiB array in device global memory
+ * owned by the library (every GPU that loads the library keeps it until
+ * exit): at most 4096 sequences and as many 128-row work units as fit; larger
+ * calls return ALA_UNSUPPORTED with the limit in the message.  Every call
+ * rewrites that array (its status word is cleared first), so calls whose GPU
+ * work overlaps race on it: order them on one stream or with events.  The
+ * schedule is uploaded from a library-owned host buffer that the next call
+ * rewrites, so a call on a stream that is being captured returns
+ * ALA_UNSUPPORTED.  The first call on each device looks up the array's
+ * address (cudaGetSymbolAddress, with that device current).  A successful
+ * call allocates no device or host memory.
  * ------------------------------------------------------------------------- */
 ALA_API int varlen_attention_noalloc(const ala_tensor* query, const ala_tensor* key, const ala_tensor* value,
                                      const ala_tensor* seqLen, const ala_tensor* kvSeqLen, const ala_tensor* slopes,
                                      int maskType, int32_t headNum, int32_t kvHeadNum, float qkScale,
                                      ala_tensor* attnOut, ala_tensor* lse, ala_stream_t stream);
+
+/* Status word of the last varlen_attention_noalloc call on the current device:
+ * synchronises `stream`, then reads the word from the library's array (no
+ * allocation).  *code = 0 means every kernel wait completed; nonzero names the
+ * wait that ran out, and the output of that call is incomplete.  The pages
+ * have no counterpart of this call. */
+ALA_API int varlen_attention_noalloc_status(ala_stream_t stream, int32_t* code);
 
 /* ---------------------------------------------------------------------------
  * MLA decode / speculative decode (ATB "MLA" page, definition and parameter

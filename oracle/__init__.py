@@ -51,7 +51,7 @@ def _load():
         _lib.oracle_mla.argtypes = [P, P, P, P, ctypes.c_int, P, I64, I32, P, P, I32, I32, I32, I32, D, P, I64,
                                     P, P]
         _lib.oracle_mla_dequant.argtypes = [P, ctypes.c_int, P, ctypes.c_int, P, ctypes.c_int, P, P, P, P, I64,
-                                            I32, P, P, I32, I32, I32, I32, D, P, I64, P, P]
+                                            I32, P, P, I32, I32, I32, I32, D, P, ctypes.c_int, I64, P, I64, P, P]
         _lib.oracle_lse_merge.argtypes = [I32, I64, I32, P, P, P, P]
         for f in ("oracle_attention", "oracle_build_mask", "oracle_attention_explicit",
                   "oracle_expand_causal_compressed", "oracle_mla", "oracle_mla_dequant", "oracle_lse_merge"):
@@ -146,8 +146,14 @@ def expand_causal_compressed(tri, seq_len, kv_len):
 
 
 def mla(q_nope, q_rope, ct_kv, k_rope, block_tables, block_size, context_lens, q_seq_len, heads, qk_scale,
-        rows=None):
-    """MLA decode/spec attention in fp64: key=[ctKV;kRope], value=ctKV, spec-causal rule."""
+        rows=None, mask=None):
+    """MLA decode/spec attention in fp64: key=[ctKV;kRope], value=ctKV, spec-causal rule.
+
+    With ``mask`` ([tokens, max_seq_len] fp16/bf16 tensor, the MLA page's MASK_TYPE_SPEC mask) every key
+    j < contextLens of a token's batch is considered and mask[token, j] is added to its scaled score."""
+    if mask is not None:
+        return mla_dequant(q_nope, q_rope, ct_kv, k_rope, None, None, block_tables, block_size, context_lens,
+                           q_seq_len, heads, qk_scale, rows=rows, mask=mask)
     lib = _load()
     qn, c1 = _raw(q_nope)
     qr, c2 = _raw(q_rope)
@@ -171,10 +177,10 @@ def mla(q_nope, q_rope, ct_kv, k_rope, block_tables, block_size, context_lens, q
 
 
 def mla_dequant(q_nope, q_rope, ct_kv, k_rope, qk_descale, pv_descale, block_tables, block_size, context_lens,
-                q_seq_len, heads, qk_scale, rows=None):
+                q_seq_len, heads, qk_scale, rows=None, mask=None):
     """MLA over an int8 latent cache in fp64 (the MLA page's qkDescale / pvDescale rows):
     s = qkScale * (qkDescale[h] * qNope.ctKV + qRope.kRope), O = pvDescale[h] * softmax(s) ctKV,
-    qNope and ctKV taken as stored (int8 or float); a None descale means 1."""
+    qNope and ctKV taken as stored (int8 or float); a None descale means 1.  ``mask`` as in ``mla``."""
     lib = _load()
     qn, cq = _raw(q_nope)
     qr, cr = _raw(q_rope)
@@ -193,9 +199,15 @@ def mla_dequant(q_nope, q_rope, ct_kv, k_rope, qk_descale, pv_descale, block_tab
     n = len(rw) if rw is not None else int(qs.sum()) * heads
     out = np.zeros((n, d_nope), dtype=np.float64)
     lse = np.zeros((n,), dtype=np.float64)
+    ma, mc, mcols = None, 0, 0
+    if mask is not None:
+        assert mask.dim() == 2 and mask.shape[0] == int(qs.sum()) and mask.dtype in (torch.float16, torch.bfloat16)
+        ma, mc = _raw(mask)
+        mcols = mask.shape[1]
     rc = lib.oracle_mla_dequant(_ptr(qn), cq, _ptr(qr), cr, _ptr(ck), ckv, _ptr(kr), _ptr(qd), _ptr(pd), _ptr(bt),
                                 bt.shape[1], block_size, _ptr(cl), _ptr(qs), len(cl), heads, d_nope, d_rope,
-                                float(qk_scale), _ptr(rw), 0 if rw is None else len(rw), _ptr(out), _ptr(lse))
+                                float(qk_scale), _ptr(ma), mc, mcols, _ptr(rw), 0 if rw is None else len(rw),
+                                _ptr(out), _ptr(lse))
     if rc != 0:
         raise ValueError("oracle_mla_dequant: inconsistent arguments")
     return out, lse

@@ -317,7 +317,15 @@ int oracle_expand_causal_compressed(const double* tri, int64_t seq_len,
  *   s_j = qkScale * (qkDescale[h] * qNope . ctKV_j + qRope . kRope_j)
  *   O   = pvDescale[h] * sum_j softmax(s)_j ctKV_j
  * with qNope and ctKV read as stored (int8 integers, or floats).  NULL
- * descales mean 1, which is the plain MLA definition above.              */
+ * descales mean 1, which is the plain MLA definition above.
+ *
+ * Explicit mask (MLA page, parameter table, rows mask and maskType: the
+ * MASK_TYPE_SPEC mask is [num_tokens, max_seq_len], fp16/bf16).  With `mask`
+ * non-NULL, packed token t of batch b considers every key j < contextLens_b
+ * and its score becomes s_j + mask[t * mask_cols + j] (the mask is added after
+ * the scale, as in the padding-mask article's formula); the generated
+ * speculative rule is not applied.  A row whose every score is -inf has no
+ * allowed key: O = 0 and lse = -inf.                                      */
 int oracle_mla_dequant(const void* q_nope, int qn_dtype, const void* q_rope,
                        int rope_dtype, const void* ct_kv, int kv_dtype,
                        const void* k_rope, const float* qk_descale,
@@ -325,7 +333,8 @@ int oracle_mla_dequant(const void* q_nope, int qn_dtype, const void* q_rope,
                        int64_t max_blocks, int32_t block_size,
                        const int32_t* context_lens, const int32_t* q_seq_len,
                        int32_t batch, int32_t heads, int32_t d_nope,
-                       int32_t d_rope, double qk_scale, const int64_t* rows,
+                       int32_t d_rope, double qk_scale, const void* mask,
+                       int mask_dtype, int64_t mask_cols, const int64_t* rows,
                        int64_t n_rows, double* out, double* lse) {
   if (batch < 0 || heads <= 0) return -1;
   int64_t* cu_q = (int64_t*)malloc(sizeof(int64_t) * (batch + 1));
@@ -336,6 +345,7 @@ int oracle_mla_dequant(const void* q_nope, int qn_dtype, const void* q_rope,
     if (qs < 1 || context_lens[b] < qs) { free(cu_q); return -1; }
     cu_q[b + 1] = cu_q[b] + qs;
     if (context_lens[b] > max_ctx) max_ctx = context_lens[b];
+    if (mask && context_lens[b] > mask_cols) { free(cu_q); return -1; }
   }
   const int64_t total = rows ? n_rows : cu_q[batch] * heads;
 #pragma omp parallel
@@ -351,7 +361,8 @@ int oracle_mla_dequant(const void* q_nope, int qn_dtype, const void* q_rope,
       const int64_t qs = cu_q[b + 1] - cu_q[b];
       const int64_t ti = t - cu_q[b];
       const int64_t ctx = context_lens[b];
-      const int64_t last = ctx - qs + ti; /* last allowed key */
+      /* last key considered: the speculative rule, or every key with an explicit mask */
+      const int64_t last = mask ? ctx - 1 : ctx - qs + ti;
       const double qk_d = qk_descale ? (double)qk_descale[h] : 1.0;
       const double pv_d = pv_descale ? (double)pv_descale[h] : 1.0;
       double m = -INFINITY;
@@ -366,12 +377,17 @@ int oracle_mla_dequant(const void* q_nope, int qn_dtype, const void* q_rope,
           dot_rope += orc_load(q_rope, rope_dtype, (t * heads + h) * (int64_t)d_rope + c) *
                       orc_load(k_rope, rope_dtype, slot * d_rope + c);
         s[j] = qk_scale * (qk_d * dot_nope + dot_rope);
+        if (mask) s[j] += orc_load(mask, mask_dtype, t * mask_cols + j);
         if (s[j] > m) m = s[j];
+      }
+      double* o = out + r * (int64_t)d_nope;
+      for (int32_t c = 0; c < d_nope; ++c) o[c] = 0.0;
+      if (m == -INFINITY) { /* no allowed key */
+        if (lse) lse[r] = -INFINITY;
+        continue;
       }
       double l = 0.0;
       for (int64_t j = 0; j <= last; ++j) l += exp(s[j] - m);
-      double* o = out + r * (int64_t)d_nope;
-      for (int32_t c = 0; c < d_nope; ++c) o[c] = 0.0;
       for (int64_t j = 0; j <= last; ++j) {
         const double p = exp(s[j] - m) / l;
         const int64_t blk = block_tables[(int64_t)b * max_blocks + j / block_size];
@@ -397,7 +413,8 @@ int oracle_mla(const void* q_nope, const void* q_rope, const void* ct_kv,
                const int64_t* rows, int64_t n_rows, double* out, double* lse) {
   return oracle_mla_dequant(q_nope, dtype, q_rope, dtype, ct_kv, dtype, k_rope, NULL, NULL,
                             block_tables, max_blocks, block_size, context_lens, q_seq_len,
-                            batch, heads, d_nope, d_rope, qk_scale, rows, n_rows, out, lse);
+                            batch, heads, d_nope, d_rope, qk_scale, NULL, 0, 0, rows, n_rows,
+                            out, lse);
 }
 
 /* ---- merge of partial results over disjoint key ranges --------------------

@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
         L.varlen_attention_noalloc.argtypes = [T, T, T, T, T, T, ctypes.c_int, ctypes.c_int32, ctypes.c_int32,
                                                ctypes.c_float, T, T, P]
         L.varlen_attention_noalloc.restype = ctypes.c_int
+        L.varlen_attention_noalloc_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
+        L.varlen_attention_noalloc_status.restype = ctypes.c_int
         L.atb_like_prefix_encoder_lse_get_workspace_size.argtypes = [T, T, T, T, T, T, T, T, ctypes.c_int,
                                                                      ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
                                                                      T, T, U64P, OPP]
@@ -187,7 +189,8 @@ def varlen_attention_noalloc(q, k, v, seq_len, kv_seq_len, mask_type, heads, kv_
 
     For callers that cannot allocate device memory: no workspace is passed; the
     library's fixed device scratch holds the schedule.  ``out`` (and ``lse``)
-    must be supplied by the caller or are created here with torch.
+    must be supplied by the caller or are created here with torch.  A stream
+    that is being captured is refused (AlaError, UNSUPPORTED).
     """
     L = lib()
     out = torch.empty_like(q) if out is None else out
@@ -198,6 +201,14 @@ def varlen_attention_noalloc(q, k, v, seq_len, kv_seq_len, mask_type, heads, kv_
     _check(L.varlen_attention_noalloc(*[_ref(t) for t in ts], int(mask_type), int(heads), int(kv_heads),
                                       float(qk_scale), _ref(to), _ref(tl), ctypes.c_void_p(s.cuda_stream)))
     return out
+
+
+def varlen_attention_noalloc_status(stream=None, device=None) -> int:
+    """Status word of the last varlen_attention_noalloc call (0: every kernel wait completed)."""
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    code = ctypes.c_int32(0)
+    _check(lib().varlen_attention_noalloc_status(ctypes.c_void_p(s.cuda_stream), ctypes.byref(code)))
+    return code.value
 
 
 def plan_prefix_encoder(q, k, v, block_tables, seq_len, kv_seq_len, mask_type, heads, kv_heads, qk_scale,

@@ -87,11 +87,11 @@ CUtensorMapDataType tma_dtype(int32_t dtype) {
                           : dtype == ALA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
 }
 
-// 3-D map over [rows, heads, d] (d innermost), box {128 B of d, 1 head, box_rows rows}, 128B swizzle.
-// `mn_major_operand`: the tile feeds the MMA as an MN-major operand; for 32-bit
-// elements that needs 32-byte swizzle atoms instead of 16-byte ones.
+}  // namespace
+
+namespace ala {
 bool encode_rows_heads_d(CUtensorMap* map, void* base, int32_t dtype, int64_t rows, int64_t heads, int64_t d,
-                         int box_rows, bool mn_major_operand = false) {
+                         int box_rows, bool mn_major_operand) {
   EncodeTiledFn enc = get_encoder();
   if (!enc) return false;
   const int es = elem_size(dtype);
@@ -102,11 +102,9 @@ bool encode_rows_heads_d(CUtensorMap* map, void* base, int32_t dtype, int64_t ro
   const CUtensorMapSwizzle sw =
       (mn_major_operand && es == 4) ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B;
   return enc(map, tma_dtype(dtype), 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-}  // namespace
+}  // namespace ala
 
 // ------------------------------------------------------------------ op
 // Page-locked copy of a host image, made on first use so the per-call upload
@@ -327,46 +325,17 @@ int build_prefill(ala_op* op, const ala_tensor* query, const ala_tensor* key, co
   op->slopes = alibi ? static_cast<const float*>(slopes->data) : nullptr;
   op->lse = lse ? static_cast<float*>(lse->data) : nullptr;
 
-  // schedule: units of up to two 128-row blocks that share a kv head (two query heads
-  // of one group, or two consecutive row tiles of one head when there is no grouping);
-  // each block visits key tiles up to its last allowed key.
+  // schedule: units of up to two 128-row blocks that share a kv head, each visiting key tiles up to
+  // its last allowed key (prefill_units)
   std::vector<SeqInfo> seqs(batch);
+  for (int32_t b = 0, cq = 0, ckv = 0; b < batch; cq += sl[b], ckv += kl[b], ++b) seqs[b] = SeqInfo{cq, sl[b], kl[b], ckv};
   std::vector<PrefillUnit> units;
-  const int32_t group = headNum / kvHeadNum;
-  int32_t cq = 0, ckv = 0;
-  for (int32_t b = 0; b < batch; ++b) {
-    seqs[b] = SeqInfo{cq, sl[b], kl[b], ckv};
-    const int32_t off = kl[b] - sl[b];
-    auto tiles_for = [&](int32_t q0) {
-      const int32_t last_row = std::min(q0 + 127, sl[b] - 1);
-      const int32_t kv_end = maskType == 0 ? kl[b] : std::min(kl[b], last_row + off + 1);
-      return (kv_end + 127) / 128;
-    };
-    if (group >= 2) {
-      for (int32_t q0 = 0; q0 < sl[b]; q0 += 128) {
-        const int32_t nt = tiles_for(q0);
-        for (int32_t g = 0; g < kvHeadNum; ++g)
-          for (int32_t i = 0; i < group; i += 2) {
-            const int32_t h = g * group + i;
-            const bool two = i + 1 < group;
-            units.push_back(PrefillUnit{b, two ? 2 : 1, {q0, q0}, {h, two ? h + 1 : h}, {nt, two ? nt : 0}});
-          }
-      }
-    } else {
-      for (int32_t h = 0; h < headNum; ++h)
-        for (int32_t q0 = 0; q0 < sl[b]; q0 += 256) {
-          const bool two = q0 + 128 < sl[b];
-          units.push_back(PrefillUnit{b, two ? 2 : 1, {q0, q0 + 128}, {h, h},
-                                      {tiles_for(q0), two ? tiles_for(q0 + 128) : 0}});
-        }
-    }
-    cq += sl[b];
-    ckv += kl[b];
-  }
+  units.reserve(prefill_unit_count(batch, sl, headNum, kvHeadNum));
+  prefill_units(batch, sl, kl, maskType, headNum, kvHeadNum, [&](const PrefillUnit& u) { units.push_back(u); });
   // Persistent grid: one CTA per SM, each running a list of units.  Units are
   // assigned longest first to the least loaded CTA (greedy LPT); a unit costs
   // its key tiles plus about one tile of fixed work (Q load, epilogue).
-  auto cost = [](const PrefillUnit& u) { return (int64_t)u.n_tiles[0] + u.n_tiles[1] + 1; };
+  auto cost = prefill_unit_cost;
   std::stable_sort(units.begin(), units.end(),
                    [&](const PrefillUnit& a, const PrefillUnit& b) { return cost(a) > cost(b); });
   const int32_t n_ctas = (int32_t)std::min<size_t>(units.size(), kPlannedSms);
@@ -413,8 +382,8 @@ int run_prefill(void* workspace, uint64_t workspaceSize, ala_op* op, ala_stream_
   if (!op->maps_ready) {
     const int kv_box = op->paged ? std::min(op->block_size, 128) : 128;
     const int64_t q_rows = op->n_tokens;
-    if (!encode_rows_heads_d(&op->tmQ, op->q, op->dtype, q_rows, op->heads, op->head_size, 128) ||
-        !encode_rows_heads_d(&op->tmK, op->k, op->dtype, op->kv_rows, op->kv_heads, op->head_size, kv_box) ||
+    if (!encode_rows_heads_d(&op->tmQ, op->q, op->dtype, q_rows, op->heads, op->head_size, 128, false) ||
+        !encode_rows_heads_d(&op->tmK, op->k, op->dtype, op->kv_rows, op->kv_heads, op->head_size, kv_box, false) ||
         !encode_rows_heads_d(&op->tmV, op->v, op->dtype, op->kv_rows, op->kv_heads, op->head_size, kv_box, true))
       return fail(ALA_CUDA_ERROR, "%s: cuTensorMapEncodeTiled failed (pointers must be 16-byte aligned)", fn);
     op->maps_ready = true;

@@ -62,6 +62,61 @@ struct PrefillParams {
   float scale_log2;             // qkScale * log2(e)
 };
 
+// Work units of one prefill request, in sequence order (every prefill entry point uses this list).
+// Per sequence b, blocks of 128 query rows; two blocks that read the same kv head form a unit: two
+// query heads of a GQA group on the same rows, or, without grouping, two consecutive row tiles of one
+// head.  Each block visits the key tiles up to its last allowed key (the causal rule with the prefix
+// offset kvSeqLen - seqLen; every key for mask type 0).  `emit(const PrefillUnit&)` receives them.
+template <class Emit>
+inline void prefill_units(int32_t batch, const int32_t* seq_len, const int32_t* kv_len, int mask_type,
+                          int32_t heads, int32_t kv_heads, Emit&& emit) {
+  const int32_t group = heads / kv_heads;
+  for (int32_t b = 0; b < batch; ++b) {
+    const int32_t sl = seq_len[b], kl = kv_len[b], off = kl - sl;
+    auto tiles_for = [&](int32_t q0) {
+      const int32_t last_row = (q0 + 127 < sl - 1) ? q0 + 127 : sl - 1;
+      const int32_t causal_end = last_row + off + 1;
+      const int32_t kv_end = (mask_type == 0 || kl < causal_end) ? kl : causal_end;
+      return (kv_end + 127) / 128;
+    };
+    if (group >= 2) {
+      for (int32_t q0 = 0; q0 < sl; q0 += 128) {
+        const int32_t nt = tiles_for(q0);
+        for (int32_t g = 0; g < kv_heads; ++g)
+          for (int32_t i = 0; i < group; i += 2) {
+            const int32_t h = g * group + i;
+            const bool two = i + 1 < group;
+            emit(PrefillUnit{b, two ? 2 : 1, {q0, q0}, {h, two ? h + 1 : h}, {nt, two ? nt : 0}});
+          }
+      }
+    } else {
+      for (int32_t h = 0; h < heads; ++h)
+        for (int32_t q0 = 0; q0 < sl; q0 += 256) {
+          const bool two = q0 + 128 < sl;
+          emit(PrefillUnit{b, two ? 2 : 1, {q0, q0 + 128}, {h, h}, {tiles_for(q0), two ? tiles_for(q0 + 128) : 0}});
+        }
+    }
+  }
+}
+
+// Number of units prefill_units emits (no list is built).
+inline int64_t prefill_unit_count(int32_t batch, const int32_t* seq_len, int32_t heads, int32_t kv_heads) {
+  const int32_t group = heads / kv_heads;
+  int64_t n = 0;
+  for (int32_t b = 0; b < batch; ++b)
+    n += group >= 2 ? (int64_t)((seq_len[b] + 127) / 128) * kv_heads * ((group + 1) / 2)
+                    : (int64_t)heads * ((seq_len[b] + 255) / 256);
+  return n;
+}
+
+// Scheduling cost of a unit: its key tiles plus about one tile of fixed work (Q load, epilogue).
+inline int64_t prefill_unit_cost(const PrefillUnit& u) { return (int64_t)u.n_tiles[0] + u.n_tiles[1] + 1; }
+
+// Tensor map over a [rows, heads, d] tensor (d innermost): box of 128 bytes of d, one head and
+// `box_rows` rows, 128-byte swizzle (32-byte atoms for a 32-bit MN-major operand).  Defined in api.cpp.
+bool encode_rows_heads_d(CUtensorMap* map, void* base, int32_t dtype, int64_t rows, int64_t heads, int64_t d,
+                         int box_rows, bool mn_major_operand);
+
 // dtype codes as in include/ala.h
 enum : int32_t { kF16 = 0, kBF16 = 1, kF32 = 2, kI32 = 3 };
 

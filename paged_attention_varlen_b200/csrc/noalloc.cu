@@ -1,12 +1,12 @@
 // noalloc.cu -- varlen_attention for callers that cannot allocate device memory.
 //
-// Some callers cannot call cudaMalloc at all: code running inside a CUDA graph
-// being built by someone else, runtimes that hand out only pre-sized arenas,
-// or embedded hosts whose allocator is owned by another component.  They can
-// still pass their own inputs and outputs, but not a workspace.  This entry
-// point runs the same prefill kernel as varlen_attention with its scratch (the
-// status word, the per-sequence table and the work units) held in one
-// fixed-size array in device global memory that belongs to this library.
+// Some callers cannot call cudaMalloc at all: runtimes that hand out only
+// pre-sized arenas, or embedded hosts whose device allocator is owned by
+// another component.  They can still pass their own inputs and outputs, but
+// not a workspace.  This entry point runs the same prefill kernel as
+// varlen_attention with its scratch (the status word, the per-sequence table
+// and the work units) held in one fixed-size array in device global memory
+// that belongs to this library.
 //
 // Costs and rules of that choice:
 //   - the array is kNoAllocScratchBytes (1 MiB); every GPU that loads the
@@ -16,9 +16,14 @@
 //   - all calls share the one array, and each call rewrites it (status word
 //     cleared to zero first): two calls whose work overlaps on the GPU race
 //     on it, so callers must order them (one stream, or events);
+//   - the schedule is uploaded from a static host buffer that the next call
+//     rewrites, so a call made while its stream is being captured into a
+//     graph is refused (a replay of that graph would read whatever schedule
+//     the buffer holds by then);
 //   - the first call on each device looks up the array's device address with
-//     cudaGetSymbolAddress (with that device current) and keeps it; make that
-//     first call before any stream capture begins;
+//     cudaGetSymbolAddress (with that device current) and keeps it;
+//   - varlen_attention_noalloc_status reads the array's status word, so a
+//     bounded kernel wait that ran out is visible to the caller;
 //   - nothing here calls cudaMalloc, cudaFree or any other allocating routine:
 //     the schedule is built in a static host buffer and uploaded with one
 //     cudaMemcpyAsync from it.  (A rejected call stores its message in the
@@ -67,40 +72,6 @@ int nfail(int status, const char* fmt, ...) {
   va_end(ap);
   set_last_error(buf);
   return status;
-}
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn tiled_encoder() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// [rows, heads, d] map, 128-byte inner box, 128B swizzle (32-byte atoms for an fp32 MN-major operand)
-bool encode_map(CUtensorMap* map, void* base, int32_t dtype, int64_t rows, int64_t heads, int64_t d, bool mn_fp32) {
-  EncodeTiledFn enc = tiled_encoder();
-  if (!enc) return false;
-  const int es = dtype == ALA_F32 ? 4 : 2;
-  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)std::max<int64_t>(rows, 1)};
-  cuuint64_t strides[2] = {(cuuint64_t)(d * es), (cuuint64_t)(heads * d * es)};
-  cuuint32_t box[3] = {(cuuint32_t)(128 / es), 1, 128};
-  cuuint32_t estr[3] = {1, 1, 1};
-  const CUtensorMapDataType t = dtype == ALA_F16    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
-                                : dtype == ALA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                                    : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-  const CUtensorMapSwizzle sw = (mn_fp32 && es == 4) ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B;
-  return enc(map, t, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool dims_ok(const ala_tensor* t) {
@@ -157,8 +128,14 @@ extern "C" ALA_API int varlen_attention_noalloc(const ala_tensor* query, const a
     return nfail(ALA_UNSUPPORTED, "%s: headSize %lld with this dtype is not built", fn, (long long)d);
   if (seqLen->ndim != 1 || kvSeqLen->ndim != 1 || seqLen->dims[0] != kvSeqLen->dims[0])
     return nfail(ALA_INVALID_SHAPE, "%s: seqLen and kvSeqLen must both be [batch]", fn);
-  if (lse && lse->data && (lse->dtype != ALA_F32 || lse->dims[0] != n_tokens))
-    return nfail(ALA_INVALID_SHAPE, "%s: lse must be fp32 [nTokens, headNum]", fn);
+  if (lse && lse->data) {
+    // [nTokens, headNum] or [nTokens, headNum, 1]: the kernel writes nTokens * headNum floats
+    if (lse->dtype != ALA_F32) return nfail(ALA_INVALID_DTYPE, "%s: lse must be fp32", fn);
+    const bool shape_ok = dims_ok(lse) && lse->dims[0] == n_tokens &&
+                          ((lse->ndim == 2 && lse->dims[1] == headNum) ||
+                           (lse->ndim == 3 && lse->dims[1] == headNum && lse->dims[2] == 1));
+    if (!shape_ok) return nfail(ALA_INVALID_SHAPE, "%s: lse must be [nTokens, headNum] or [nTokens, headNum, 1]", fn);
+  }
   const int32_t batch = (int32_t)seqLen->dims[0];
   if (batch > kMaxBatch)
     return nfail(ALA_UNSUPPORTED, "%s: batch %d exceeds the %d sequences the fixed scratch holds", fn, batch, kMaxBatch);
@@ -177,14 +154,20 @@ extern "C" ALA_API int varlen_attention_noalloc(const ala_tensor* query, const a
 
   // ---- count the work units first, so an oversized call is rejected before anything is written
   const int32_t group = headNum / kvHeadNum;
-  int64_t n_units = 0;
-  for (int32_t b = 0; b < batch; ++b) {
-    const int64_t qt = (sl[b] + 127) / 128;
-    n_units += group >= 2 ? qt * kvHeadNum * ((group + 1) / 2) : (int64_t)headNum * ((sl[b] + 255) / 256);
-  }
+  const int64_t n_units = prefill_unit_count(batch, sl, headNum, kvHeadNum);
   if (n_units > (int64_t)kMaxUnits)
     return nfail(ALA_UNSUPPORTED, "%s: the call needs %lld work units; the fixed %zu-byte scratch holds at most %zu", fn,
                  (long long)n_units, kNoAllocScratchBytes, kMaxUnits);
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &capture) != cudaSuccess)
+    return nfail(ALA_CUDA_ERROR, "%s: cudaStreamIsCapturing failed: %s", fn, cudaGetErrorString(cudaGetLastError()));
+  if (capture != cudaStreamCaptureStatusNone)
+    return nfail(ALA_UNSUPPORTED,
+                 "%s: the stream is being captured; the schedule upload reads a host buffer that later calls "
+                 "rewrite, so a replayed capture would run another call's schedule",
+                 fn);
 
   std::lock_guard<std::mutex> lock(g_mutex);
   int dev = 0;
@@ -204,38 +187,11 @@ extern "C" ALA_API int varlen_attention_noalloc(const ala_tensor* query, const a
   SeqInfo* seqs = reinterpret_cast<SeqInfo*>(g_stage + kStatusBytes);
   PrefillUnit* units = reinterpret_cast<PrefillUnit*>(g_stage + kStatusBytes + kSeqBytes);
   size_t nu = 0;
-  int32_t cq = 0, ckv = 0;
-  for (int32_t b = 0; b < batch; ++b) {
-    seqs[b] = SeqInfo{cq, sl[b], kl[b], ckv};
-    const int32_t off = kl[b] - sl[b];
-    auto tiles_for = [&](int32_t q0) {
-      const int32_t last_row = std::min(q0 + 127, sl[b] - 1);
-      const int32_t kv_end = maskType == 0 ? kl[b] : std::min(kl[b], last_row + off + 1);
-      return (kv_end + 127) / 128;
-    };
-    if (group >= 2) {
-      for (int32_t q0 = 0; q0 < sl[b]; q0 += 128) {
-        const int32_t nt = tiles_for(q0);
-        for (int32_t g = 0; g < kvHeadNum; ++g)
-          for (int32_t i = 0; i < group; i += 2) {
-            const int32_t h = g * group + i;
-            const bool two = i + 1 < group;
-            units[nu++] = PrefillUnit{b, two ? 2 : 1, {q0, q0}, {h, two ? h + 1 : h}, {nt, two ? nt : 0}};
-          }
-      }
-    } else {
-      for (int32_t h = 0; h < headNum; ++h)
-        for (int32_t q0 = 0; q0 < sl[b]; q0 += 256) {
-          const bool two = q0 + 128 < sl[b];
-          units[nu++] = PrefillUnit{b, two ? 2 : 1, {q0, q0 + 128}, {h, h}, {tiles_for(q0), two ? tiles_for(q0 + 128) : 0}};
-        }
-    }
-    cq += sl[b];
-    ckv += kl[b];
-  }
+  for (int32_t b = 0, cq = 0, ckv = 0; b < batch; cq += sl[b], ckv += kl[b], ++b) seqs[b] = SeqInfo{cq, sl[b], kl[b], ckv};
+  prefill_units(batch, sl, kl, maskType, headNum, kvHeadNum, [&](const PrefillUnit& u) { units[nu++] = u; });
   // longest first; ties in a fixed order so every call gets the same schedule
   std::sort(units, units + nu, [](const PrefillUnit& a, const PrefillUnit& c) {
-    const int ca = a.n_tiles[0] + a.n_tiles[1], cc = c.n_tiles[0] + c.n_tiles[1];
+    const int64_t ca = prefill_unit_cost(a), cc = prefill_unit_cost(c);
     if (ca != cc) return ca > cc;
     if (a.b != c.b) return a.b < c.b;
     if (a.q0[0] != c.q0[0]) return a.q0[0] < c.q0[0];
@@ -243,14 +199,14 @@ extern "C" ALA_API int varlen_attention_noalloc(const ala_tensor* query, const a
   });
 
   CUtensorMap tmQ, tmK, tmV;
-  if (!encode_map(&tmQ, query->data, dt, n_tokens, headNum, d, false) ||
-      !encode_map(&tmK, key->data, dt, key->dims[0], kvHeadNum, d, false) ||
-      !encode_map(&tmV, value->data, dt, key->dims[0], kvHeadNum, d, true))
+  if (!encode_rows_heads_d(&tmQ, query->data, dt, n_tokens, headNum, d, 128, false) ||
+      !encode_rows_heads_d(&tmK, key->data, dt, key->dims[0], kvHeadNum, d, 128, false) ||
+      !encode_rows_heads_d(&tmV, value->data, dt, key->dims[0], kvHeadNum, d, 128, true))
     return nfail(ALA_CUDA_ERROR, "%s: cuTensorMapEncodeTiled failed (pointers must be 16-byte aligned)", fn);
 
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const size_t bytes = kStatusBytes + kSeqBytes + nu * sizeof(PrefillUnit);
-  // pageable source: the copy is staged before this call returns, so g_stage may be rewritten by the next call
+  // pageable source on a stream that is not being captured: the copy is staged before this call
+  // returns, so g_stage may be rewritten by the next call
   if (cudaMemcpyAsync(scratch, g_stage, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
     return nfail(ALA_CUDA_ERROR, "%s: schedule upload failed: %s", fn, cudaGetErrorString(cudaGetLastError()));
 
@@ -274,6 +230,20 @@ extern "C" ALA_API int varlen_attention_noalloc(const ala_tensor* query, const a
   p.scale_log2 = qkScale * 1.4426950408889634f;
   const cudaError_t e = launch_prefill(dt, (int32_t)d, tmQ, tmK, tmV, p, st);
   if (e != cudaSuccess) return nfail(ALA_CUDA_ERROR, "%s: kernel launch failed: %s", fn, cudaGetErrorString(e));
+  set_last_error("");
+  return ALA_OK;
+}
+
+extern "C" ALA_API int varlen_attention_noalloc_status(ala_stream_t stream, int32_t* code) {
+  const char* fn = "varlen_attention_noalloc_status";
+  if (!code) return nfail(ALA_NULL_REQUIRED, "%s: code is NULL", fn);
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return nfail(ALA_CUDA_ERROR, "%s: stream sync failed: %s", fn, cudaGetErrorString(cudaGetLastError()));
+  int32_t v = 0;
+  // a copy out of the library's array by symbol: no allocation
+  const cudaError_t e = cudaMemcpyFromSymbol(&v, g_noalloc_scratch, sizeof v, 0, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return nfail(ALA_CUDA_ERROR, "%s: status read failed: %s", fn, cudaGetErrorString(e));
+  *code = v;
   set_last_error("");
   return ALA_OK;
 }

@@ -285,3 +285,40 @@ def test_last_error_is_text():
     with pytest.raises(ala.AlaError) as e:
         _plan_varlen(heads=0)
     assert "headNum" in str(e.value)
+
+
+def _fake(shape, dtype_code, addr=1 << 20):
+    """An ala_tensor over a dummy address: the checks below run before any data is touched."""
+    t = ala.AlaTensor()
+    t.data = addr
+    t.dtype = dtype_code
+    t.ndim = len(shape)
+    for i, s in enumerate(shape):
+        t.dims[i] = s
+    return t
+
+
+def _noalloc_raw(n_tokens, heads, kv_heads, d, seq_len, lse_shape=None):
+    L = ala.lib()
+    sl = np.asarray(seq_len, dtype=np.int32)
+    q = _fake((n_tokens, heads, d), ala.BF16)
+    kv = _fake((n_tokens, kv_heads, d), ala.BF16)
+    out = _fake((n_tokens, heads, d), ala.BF16)
+    lse = None if lse_shape is None else _fake(lse_shape, ala.F32)
+    st = L.varlen_attention_noalloc(ctypes.byref(q), ctypes.byref(kv), ctypes.byref(kv),
+                                    ala._ref(ala.tensor(sl)), ala._ref(ala.tensor(sl)), None, 9, heads, kv_heads,
+                                    ctypes.c_float(0.1), ctypes.byref(out), ala._ref(lse), None)
+    return st, L.ala_last_error().decode()
+
+
+def test_noalloc_refuses_more_work_units_than_its_scratch_holds():
+    # one 2M-token sequence over 8 heads without grouping: 8 x 7813 units of two 128-row blocks, more than
+    # the fixed scratch holds; refused on the host before the device is touched
+    st, msg = _noalloc_raw(2_000_000, 8, 8, 64, [2_000_000])
+    assert st == 5 and "work units" in msg
+
+
+@pytest.mark.parametrize("lse_shape", [(10,), (10, 1), (10, 4, 2), (9, 4)])
+def test_noalloc_refuses_an_lse_of_the_wrong_shape(lse_shape):
+    st, msg = _noalloc_raw(10, 4, 4, 64, [10], lse_shape)
+    assert st == 2 and "lse" in msg

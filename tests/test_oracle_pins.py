@@ -433,3 +433,81 @@ def test_mla_int8_output_is_linear_in_pv_descale_and_lse_ignores_it():
     np.testing.assert_array_equal(l1, l2)
     np.testing.assert_array_equal(o2[0], o1[0] * 0.25)
     np.testing.assert_array_equal(o2[1], o1[1] * 4.0)
+
+
+# --------------------------------------------------------------------------
+# MLA with the explicit MASK_TYPE_SPEC mask tensor (MLA page, rows mask / maskType)
+# --------------------------------------------------------------------------
+
+def _spec_rule_mask(ctx, qs, cols, dtype, masked_value):
+    """[tokens, cols] mask holding 0 where the speculative rule allows key j (j <= ctx - qs + t) and
+    `masked_value` elsewhere."""
+    rows = []
+    for c, q in zip(ctx.tolist(), qs.tolist()):
+        for t in range(q):
+            r = torch.full((cols,), masked_value, dtype=torch.float64)
+            r[:c - q + t + 1] = 0.0
+            rows.append(r)
+    return torch.stack(rows).to(dtype)
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("masked_value", [-math.inf, "lowest"])
+def test_mla_explicit_mask_of_the_spec_rule_equals_the_rule(dtype, masked_value):
+    rng = np.random.Generator(np.random.PCG64(77))
+    ctx = np.array([9, 70, 33], dtype=np.int32)
+    qs = np.array([3, 1, 4], dtype=np.int32)
+    case = synth.make_mla("mm", ctx, qs, 3, 77, rng=rng, block_size=16, d_nope=24, d_rope=8, dtype=dtype)
+    mv = torch.finfo(dtype).min if masked_value == "lowest" else masked_value
+    mask = _spec_rule_mask(ctx, qs, 80, dtype, mv)
+    args = (case.q_nope, case.q_rope, case.ct_kv, case.k_rope, case.block_tables, 16, ctx, qs, 3, case.qk_scale)
+    o_rule, l_rule = oracle.mla(*args)
+    o_mask, l_mask = oracle.mla(*args, mask=mask)
+    np.testing.assert_allclose(o_mask, o_rule, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l_mask, l_rule, rtol=0, atol=1e-12)
+
+
+def test_mla_explicit_mask_equals_sdpa_with_the_additive_mask():
+    """A random, non-causal additive mask (finite values and some -inf) per packed token: torch's float64
+    scaled_dot_product_attention over the concatenated key with the token's mask row as attn_mask."""
+    rng = np.random.Generator(np.random.PCG64(79))
+    heads, d_nope, d_rope, bs, cols = 2, 16, 8, 16, 48
+    ctx = np.array([7, 40, 21], dtype=np.int32)
+    qs = np.array([2, 3, 1], dtype=np.int32)
+    case = synth.make_mla("ms", ctx, qs, heads, 79, rng=rng, block_size=bs, d_nope=d_nope, d_rope=d_rope,
+                          dtype=torch.bfloat16)
+    m = rng.standard_normal((int(qs.sum()), cols)).astype(np.float32) * 2.0
+    m[rng.random(m.shape) < 0.3] = -np.inf
+    m[:, 0] = 0.0  # every row keeps at least key 0
+    mask = torch.from_numpy(m).to(torch.bfloat16)
+    out, lse = oracle.mla(case.q_nope, case.q_rope, case.ct_kv, case.k_rope, case.block_tables, bs, ctx, qs, heads,
+                          case.qk_scale, mask=mask)
+    t0 = 0
+    for b, L in enumerate(ctx.tolist()):
+        keys = [(case.ct_kv[int(case.block_tables[b, j // bs]), j % bs, 0].double(),
+                 case.k_rope[int(case.block_tables[b, j // bs]), j % bs, 0].double()) for j in range(L)]
+        kn = torch.stack([k[0] for k in keys])
+        kcat = torch.cat([kn, torch.stack([k[1] for k in keys])], dim=-1)
+        for t in range(int(qs[b])):
+            bias = mask[t0 + t, :L].double()
+            for h in range(heads):
+                q = torch.cat([case.q_nope[t0 + t, h].double(), case.q_rope[t0 + t, h].double()])
+                o = F.scaled_dot_product_attention(q.view(1, 1, 1, -1), kcat.view(1, 1, L, -1), kn.view(1, 1, L, -1),
+                                                   attn_mask=bias.view(1, 1, 1, L), scale=case.qk_scale)
+                row = (t0 + t) * heads + h
+                np.testing.assert_allclose(out[row], o.view(-1).numpy(), rtol=1e-12, atol=1e-12)
+                s = case.qk_scale * (kcat @ q) + bias
+                assert abs(lse[row] - torch.logsumexp(s, 0).item()) < 1e-12
+        t0 += int(qs[b])
+
+
+def test_mla_explicit_mask_fully_masked_row_gives_zero_and_minus_inf():
+    rng = np.random.Generator(np.random.PCG64(81))
+    ctx = np.array([20], dtype=np.int32)
+    case = synth.make_mla("mz", ctx, 2, 2, 81, rng=rng, block_size=16, d_nope=16, d_rope=8, dtype=torch.float16)
+    mask = torch.zeros((2, 32), dtype=torch.float16)
+    mask[1, :] = -math.inf  # the second token sees no key at all
+    out, lse = oracle.mla(case.q_nope, case.q_rope, case.ct_kv, case.k_rope, case.block_tables, 16, ctx, [2], 2,
+                          case.qk_scale, mask=mask)
+    assert (out[2:] == 0).all() and (lse[2:] == -np.inf).all()
+    assert np.isfinite(out[:2]).all() and np.isfinite(lse[:2]).all()
