@@ -226,7 +226,15 @@ ALA_API int varlen_attention_noalloc_status(ala_stream_t stream, int32_t* code);
  * kRope       [numBlocks, blockSize, kvHeadNum, 64], device.
  * blockTables [batch, maxBlocks] int32, device (entries read must be valid).
  * contextLens [batch] int32, HOST: keys per batch, including the new tokens.
- * mask        must be NULL (the spec mask is generated from the rule).
+ * mask        NULL (the speculative mask is generated from the rule), or with
+ *             maskType SPEC the page's MASK_TYPE_SPEC mask: [tokens,
+ *             maxSeqLen] fp16/bf16, device, maxSeqLen >= every contextLens
+ *             entry.  Token t (packed over the batch) then considers every key
+ *             j < contextLens of its batch, and mask[t][j] is added to the
+ *             scaled score (-inf or a large negative value masks the key); the
+ *             generated rule is not applied.  A token whose keys are all
+ *             masked with -inf gets output 0 and lse -inf.  Must be NULL with
+ *             calcType PREFILL.
  * qSeqLen     [batch] int32, HOST: query tokens per batch; required when
  *             calcType = SPEC, else NULL (one token each).  Token t of batch
  *             b allows keys j <= contextLens_b - qSeqLen_b + t.
@@ -253,10 +261,6 @@ ALA_API int varlen_attention_noalloc_status(ala_stream_t stream, int32_t* code);
  *             required with calcType RING (NULL_REQUIRED otherwise).
  * workspace   256-byte aligned; holds the schedule and, for key ranges split
  *             across CTAs, fp32 partial outputs merged by lse at the end.
- * Environment: with ALA_MLA_PAIR=1 set when the op is planned, a request with
- *             one token per batch, a 16-bit cache and headNum a multiple of 128
- *             runs on the CTA-pair kernel (two CTAs per 128 heads splitting the
- *             latent dimensions); same results, measured slower, off by default.
  * ------------------------------------------------------------------------- */
 ALA_API int atb_like_mla_get_workspace_size(
     const ala_tensor* qNope, const ala_tensor* qRope, const ala_tensor* ctKV, const ala_tensor* kRope,

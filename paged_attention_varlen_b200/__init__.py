@@ -245,11 +245,13 @@ def atb_like_prefix_encoder(q, k, v, block_tables, seq_len, kv_seq_len, mask_typ
 
 def plan_mla(q_nope, q_rope, ct_kv, k_rope, block_tables, context_lens, q_seq_len, heads, qk_scale,
              mask_type=MLA_MASK_UNDEFINED, calc_type=MLA_CALC_UNDEFINED, cache_mode=None,
-             lse=None, out=None, kv_heads=1, qk_descale=None, pv_descale=None) -> tuple[Op, torch.Tensor]:
+             lse=None, out=None, kv_heads=1, qk_descale=None, pv_descale=None, mask=None) -> tuple[Op, torch.Tensor]:
     """Plan the MLA decode/spec call; returns (op, attenOut).
 
     An int8 ``ct_kv`` selects the int8 latent cache (cacheMode INT8_NZCACHE, ND layout) and needs
     ``qk_descale`` / ``pv_descale`` ([heads] fp32 on the device); ``q_nope`` may then be int8 too.
+    ``mask`` ([tokens, maxSeqLen] fp16/bf16 on the device, maskType SPEC) is added to the scaled scores
+    of every key below contextLens in place of the generated speculative rule.
     """
     L = lib()
     if cache_mode is None:
@@ -258,8 +260,8 @@ def plan_mla(q_nope, q_rope, ct_kv, k_rope, block_tables, context_lens, q_seq_le
            if out is None else out)
     cl = _host_i32(context_lens)
     qs = None if q_seq_len is None else _host_i32(q_seq_len)
-    ts = [tensor(q_nope), tensor(q_rope), tensor(ct_kv), tensor(k_rope), tensor(block_tables), tensor(cl), None,
-          tensor(qs), tensor(qk_descale), tensor(pv_descale)]
+    ts = [tensor(q_nope), tensor(q_rope), tensor(ct_kv), tensor(k_rope), tensor(block_tables), tensor(cl),
+          tensor(mask), tensor(qs), tensor(qk_descale), tensor(pv_descale)]
     to, tl = tensor(out), tensor(lse)
     ws = ctypes.c_uint64(0)
     h = ctypes.c_void_p(0)
@@ -267,17 +269,17 @@ def plan_mla(q_nope, q_rope, ct_kv, k_rope, block_tables, context_lens, q_seq_le
                                              int(mask_type), int(calc_type), int(cache_mode), _ref(to), _ref(tl),
                                              ctypes.byref(ws), ctypes.byref(h)))
     return Op(h, ws.value, L.atb_like_mla, q_nope.device,
-              (q_nope, q_rope, ct_kv, k_rope, block_tables, cl, qs, out, lse, qk_descale, pv_descale)), out
+              (q_nope, q_rope, ct_kv, k_rope, block_tables, cl, qs, out, lse, qk_descale, pv_descale, mask)), out
 
 
 def atb_like_mla(q_nope, q_rope, ct_kv, k_rope, block_tables, context_lens, q_seq_len, heads, qk_scale,
                  mask_type=MLA_MASK_UNDEFINED, calc_type=MLA_CALC_UNDEFINED, return_lse=False, qk_descale=None,
-                 pv_descale=None):
+                 pv_descale=None, mask=None):
     return_lse = return_lse or calc_type == MLA_CALC_RING  # ring mode always returns the lse
     lse = (torch.empty((q_nope.shape[0], heads, 1), dtype=torch.float32, device=q_nope.device)
            if return_lse else None)
     op, out = plan_mla(q_nope, q_rope, ct_kv, k_rope, block_tables, context_lens, q_seq_len, heads, qk_scale,
-                       mask_type, calc_type, lse=lse, qk_descale=qk_descale, pv_descale=pv_descale)
+                       mask_type, calc_type, lse=lse, qk_descale=qk_descale, pv_descale=pv_descale, mask=mask)
     op()
     return (out, lse) if return_lse else out
 

@@ -516,6 +516,8 @@ extern "C" int atb_like_mla_get_workspace_size(const ala_tensor* qNope, const al
     if (!qSeqLen || !qSeqLen->data) return fail(ALA_NULL_REQUIRED, "%s: qseqlen is required with calcType PREFILL", fn);
     if (maskType != ALA_MLA_MASK_UNDEFINED && maskType != ALA_MLA_MASK_SPEC)
       return fail(ALA_INVALID_PARAM, "%s: calcType PREFILL takes maskType UNDEFINED or SPEC (causal either way)", fn);
+    if (mask && mask->data)
+      return fail(ALA_INVALID_PARAM, "%s: calcType PREFILL generates its causal mask; mask must be NULL", fn);
     calcType = ALA_MLA_CALC_SPEC;
     maskType = ALA_MLA_MASK_SPEC;
   }
@@ -531,11 +533,6 @@ extern "C" int atb_like_mla_get_workspace_size(const ala_tensor* qNope, const al
   int st = mla_plan(&o->mla, qNope, qRope, ctKV, kRope, blockTables, contextLens, mask, qSeqLen, qkDescale,
                     pvDescale, headNum, qkScale, kvHeadNum, maskType, calcType, cacheMode, attenOut, lse, err,
                     sizeof err);
-  if (st == ALA_OK) {
-    // the CTA-pair decode kernel, on request (ALA_MLA_PAIR=1 in the environment when the op is planned)
-    const char* pair = std::getenv("ALA_MLA_PAIR");
-    if (pair && pair[0] == '1' && mla_pair_eligible(&o->mla)) st = mla_pair_plan(&o->mla, err, sizeof err);
-  }
   if (st != ALA_OK) {
     delete o;
     return fail(st, "%s: %s", fn, err);
@@ -554,8 +551,7 @@ extern "C" int atb_like_mla(void* workspace, uint64_t workspaceSize, ala_op* op,
     return fail(ALA_WORKSPACE_TOO_SMALL, "%s: workspace %llu < required %llu", fn, (unsigned long long)workspaceSize,
                 (unsigned long long)op->mla.ws_size);
   char err[512] = {0};
-  int st = op->mla.pair ? mla_pair_run(&op->mla, workspace, reinterpret_cast<cudaStream_t>(stream), err, sizeof err)
-                        : mla_run(&op->mla, workspace, reinterpret_cast<cudaStream_t>(stream), err, sizeof err);
+  int st = mla_run(&op->mla, workspace, reinterpret_cast<cudaStream_t>(stream), err, sizeof err);
   if (st != ALA_OK) return fail(st, "%s: %s", fn, err);
   return ok();
 }

@@ -106,9 +106,10 @@ struct MlaPiece {
   int32_t token0;    // first packed query token of the chunk
   int32_t kv_begin;  // first key of the range (a multiple of 32)
   int32_t n_tiles;   // 32-key tiles in the range
-  int32_t last;      // last allowed key of the chunk's first token; token t of the chunk allows last + t
+  int32_t last;      // last allowed key of the chunk's first token; token t of the chunk allows last + row_step*t
   int32_t part;      // partial slot (rows part*tpc .. +tpc-1 of the partials), or -1: final output
-  int32_t pad[2];
+  int32_t n_keys;    // keys of the batch the chunk may read (its pages): last + tpc, or contextLens with a mask
+  int32_t row_step;  // 1: the speculative rule; 0: every token reads keys 0..n_keys-1 (explicit mask tensor)
 };
 
 struct MlaCombine {
@@ -141,7 +142,39 @@ struct MlaParams {
   const float* qk_descale;  // [heads], int8 cache only
   const float* pv_descale;  // [heads], int8 cache only
   int32_t qn_int8;          // qNope holds int8 codes (int8 cache only)
+  const uint16_t* mask;     // [tokens, mask_cols] additive mask (fp16 or bf16 bits), or null: the rule
+  int64_t mask_cols;
+  int32_t mask_f16;         // the mask holds fp16 (else bf16)
+  int32_t mask_vec;         // rows start 16-byte aligned: 16-byte loads
 };
+
+// One fp16 or bf16 mask element (its 16 bits) as a float.
+__device__ __forceinline__ float mask_value(uint32_t bits, bool f16) {
+  return f16 ? __half2float(__ushort_as_half(static_cast<unsigned short>(bits))) : __uint_as_float(bits << 16);
+}
+
+// The additive mask of packed token `token` for keys j0 .. j0+63, in log2 units (times log2 e); keys at or
+// past the mask's row length read 0 (they lie past contextLens and are masked by the key limit).
+__device__ __forceinline__ void load_mask_log2(const MlaParams& p, int token, int j0, float (&mk)[64]) {
+  const uint16_t* row = p.mask + (size_t)token * p.mask_cols;
+  const bool f16 = p.mask_f16 != 0;
+  if (p.mask_vec && j0 + 64 <= p.mask_cols) {
+    const uint4* src = reinterpret_cast<const uint4*>(row + j0);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const uint4 w = __ldg(src + v);
+      const uint32_t q[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        mk[8 * v + 2 * i] = mask_value(q[i] & 0xffffu, f16) * kLog2e;
+        mk[8 * v + 2 * i + 1] = mask_value(q[i] >> 16, f16) * kLog2e;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 64; ++c) mk[c] = (j0 + c < p.mask_cols) ? mask_value(__ldg(row + j0 + c), f16) * kLog2e : 0.f;
+  }
+}
 
 __device__ __forceinline__ uint32_t pack2(float a, float b, __nv_bfloat16*) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
@@ -319,7 +352,7 @@ __global__ void __launch_bounds__(KV8 ? 320 : 192, 1)
       for (int k = k0; k < k1 && ok; ++k) {
         const MlaPiece pc = p.pieces[k];
         const int32_t* bt = p.block_tables + (size_t)pc.b * p.max_blocks;
-        const int n_pages = (pc.last + p.tpc + bs - 1) / bs;  // pages holding keys <= the chunk's last allowed key
+        const int n_pages = (pc.n_keys + bs - 1) / bs;  // pages holding the keys the chunk may read
         if (k + 1 < k1) {  // the next chunk's qNope rows, for the softmax threads' loads at the piece boundary
           const MlaPiece pn = p.pieces[k + 1];
           const int qes = p.qn_int8 ? 1 : 2;
@@ -329,7 +362,7 @@ __global__ void __launch_bounds__(KV8 ? 320 : 192, 1)
         for (int j = 0; j < pc.n_tiles; ++j) {
           for (; ALA_MLA_PREFETCH_TILES > 0 && kf < k1 && Gf <= G + ALA_MLA_PREFETCH_TILES; ++Gf) {
             const int32_t* btf = p.block_tables + (size_t)pf.b * p.max_blocks;
-            const int npf = (pf.last + p.tpc + bs - 1) / bs;
+            const int npf = (pf.n_keys + bs - 1) / bs;
             for (int r0 = 0; r0 < kTileKeys; r0 += box_rows) {
               const int pos = pf.kv_begin + jf * kTileKeys + r0;
               const int pg = pos / bs;
@@ -526,7 +559,8 @@ __global__ void __launch_bounds__(KV8 ? 320 : 192, 1)
     const uint32_t tmem_warp = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const int sw = hr & 7;  // 128-byte swizzle of the row's 16-byte chunks
     const float scale = p.scale_log2;
-    const bool raw_max = scale > 0.f;  // max of the raw scores, scale folded into the exponent
+    const bool has_mask = p.mask != nullptr;
+    const bool raw_max = scale > 0.f && !has_mask;  // max of the raw scores, scale folded into the exponent
     const float qk_d = KV8 ? p.qk_descale[head] : 1.f;
     const float pv_d = KV8 ? p.pv_descale[head] : 1.f;
     bool ok = true;
@@ -535,7 +569,7 @@ __global__ void __launch_bounds__(KV8 ? 320 : 192, 1)
     if (k0 < k1) load_query<T>(p, &tmQr, sQr, q_full, tmem_warp, h0, p.pieces[k0].token0, t_local, head, upper);
     for (int k = k0; k < k1 && ok; ++k) {
       const MlaPiece pc = p.pieces[k];
-      const int row_last = pc.last + t_local;
+      const int row_last = min(pc.last + pc.row_step * t_local, pc.n_keys - 1);
       float m_run = -INFINITY;
       float l_run = 0.f;
       for (int j = 0; j < pc.n_tiles; ++j, ++G) {
@@ -563,7 +597,18 @@ __global__ void __launch_bounds__(KV8 ? 320 : 192, 1)
           }
         }
         const int lim = row_last - (pc.kv_begin + j * kTileKeys);  // columns c <= lim are allowed
-        if (!raw_max) {
+        if (has_mask) {
+          // the explicit mask is added after the scale (log2 units); lanes 16..31 hold no score row
+          float mk[kTileKeys];
+          if (!upper) {
+            load_mask_log2(p, pc.token0 + t_local, pc.kv_begin + j * kTileKeys, mk);
+          } else {
+#pragma unroll
+            for (int c = 0; c < kTileKeys; ++c) mk[c] = 0.f;
+          }
+#pragma unroll
+          for (int c = 0; c < kTileKeys; ++c) x[c] = fmaf(x[c], scale, mk[c]);
+        } else if (!raw_max) {
 #pragma unroll
           for (int c = 0; c < kTileKeys; ++c) x[c] *= scale;
         }
@@ -760,13 +805,15 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaCombine* work
   auto row = [&](int s) { return ((size_t)(w.part_begin + s) * p.tpc + w.t_local) * p.heads + head; };
   float m = -INFINITY;
   for (int s = 0; s < w.n_parts; ++s) m = fmaxf(m, p.part_lse[row(s)]);
+  // a row with no allowed key in any part (possible only with an explicit mask) gets O = 0, lse = -inf
+  const bool none = m == -INFINITY;
   float l = 0.f;
-  for (int s = 0; s < w.n_parts; ++s) l += __expf(p.part_lse[row(s)] - m);
-  const float lse = m + __logf(l);
+  for (int s = 0; s < w.n_parts && !none; ++s) l += __expf(p.part_lse[row(s)] - m);
+  const float lse = none ? -INFINITY : m + __logf(l);
   float acc[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  for (int s = 0; s < w.n_parts; ++s) {
+  for (int s = 0; s < w.n_parts && !none; ++s) {
     const size_t pr = row(s);
     const float wgt = __expf(p.part_lse[pr] - lse);  // 0 for a part whose rows saw no allowed key
     const float4* src = reinterpret_cast<const float4*>(p.part_o + pr * kDNope);
@@ -850,7 +897,6 @@ int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, co
   if (maskType != ALA_MLA_MASK_UNDEFINED && maskType != ALA_MLA_MASK_SPEC)
     return mfail(err, n, maskType == ALA_MLA_MASK_FREE ? ALA_UNSUPPORTED : ALA_INVALID_PARAM,
                  "maskType must be UNDEFINED (0) or SPEC (1)");
-  if (mask && mask->data) return mfail(err, n, ALA_INVALID_PARAM, "mask must be NULL: the spec mask is generated");
   if (kv8) {
     if (!qkDescale || !qkDescale->data || !pvDescale || !pvDescale->data)
       return mfail(err, n, ALA_NULL_REQUIRED, "qkDescale and pvDescale are required with the int8 cache (cacheMode 2)");
@@ -907,6 +953,17 @@ int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, co
   } else if (qSeqLen && qSeqLen->data) {
     return mfail(err, n, ALA_INVALID_PARAM, "qseqlen is only passed with calcType SPEC");
   }
+  // the explicit MASK_TYPE_SPEC mask (MLA page, parameter table, rows mask and maskType): [tokens, maxSeqLen]
+  const bool has_mask = mask && mask->data;
+  if (has_mask) {
+    if (maskType != ALA_MLA_MASK_SPEC)
+      return mfail(err, n, ALA_INVALID_PARAM, "a mask tensor is passed only with maskType SPEC (1)");
+    if (mask->dtype != ALA_F16 && mask->dtype != ALA_BF16)
+      return mfail(err, n, ALA_INVALID_DTYPE, "mask must be fp16 or bf16");
+    if (mask->ndim != 2 || mask->dims[0] != tokens || mask->dims[1] < 1)
+      return mfail(err, n, ALA_INVALID_SHAPE, "mask must be [tokens, maxSeqLen]");
+    if (reinterpret_cast<uintptr_t>(mask->data) % 2) return mfail(err, n, ALA_INVALID_PARAM, "mask must be 2-byte aligned");
+  }
   if (lse && lse->data) {
     if (lse->dtype != ALA_F32) return mfail(err, n, ALA_INVALID_DTYPE, "lse must be fp32");
     int64_t ne = 1;
@@ -926,6 +983,8 @@ int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, co
       return mfail(err, n, ALA_INVALID_PARAM, "contextLens needs more blocks than blockTables holds");
     if (q > 1 && maskType != ALA_MLA_MASK_SPEC)
       return mfail(err, n, ALA_INVALID_PARAM, "qseqlen > 1 needs maskType SPEC");
+    if (has_mask && cl[b] > mask->dims[1])
+      return mfail(err, n, ALA_INVALID_SHAPE, "the mask's maxSeqLen is shorter than a contextLens entry");
     sum_q += q;
   }
   if (sum_q != tokens) return mfail(err, n, ALA_INVALID_SHAPE, "sum(qseqlen) != tokens");
@@ -955,6 +1014,9 @@ int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, co
   plan->ctx.assign(cl, cl + batch);
   plan->qs.assign(batch, 1);
   if (qs) plan->qs.assign(qs, qs + batch);
+  plan->mask = has_mask ? static_cast<const uint16_t*>(mask->data) : nullptr;
+  plan->mask_cols = has_mask ? mask->dims[1] : 0;
+  plan->mask_f16 = has_mask && mask->dtype == ALA_F16;
 
   // ---- row blocks: tpc tokens x hpc heads, tpc the largest of 4, 2, 1 dividing every qseqlen
   int32_t tpc = 4;
@@ -971,15 +1033,18 @@ int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, co
 
   // ---- chunks and their 32-key tiles, end to end
   struct Chunk {
-    int32_t b, token0, last, tiles;
+    int32_t b, token0, last, tiles, n_keys, row_step;
   };
   std::vector<Chunk> chunks;
   int64_t total_tiles = 0;
   for (int32_t b = 0, token = 0; b < batch; token += plan->qs[b], ++b) {
     for (int32_t t0 = 0; t0 < plan->qs[b]; t0 += tpc) {
-      const int32_t last = cl[b] - plan->qs[b] + t0;           // the chunk's first token's last allowed key
-      const int32_t tiles = (last + tpc + kTileKeys - 1) / kTileKeys;  // keys 0 .. last + tpc - 1
-      chunks.push_back(Chunk{b, token + t0, last, tiles});
+      // the rule: token t0 + t of the chunk allows keys 0 .. last + t; with an explicit mask every token
+      // reads keys 0 .. contextLens - 1 and the mask decides
+      const int32_t last = has_mask ? cl[b] - 1 : cl[b] - plan->qs[b] + t0;
+      const int32_t n_keys = has_mask ? cl[b] : last + tpc;
+      const int32_t tiles = (n_keys + kTileKeys - 1) / kTileKeys;
+      chunks.push_back(Chunk{b, token + t0, last, tiles, n_keys, has_mask ? 0 : 1});
       total_tiles += tiles;
     }
   }
@@ -995,7 +1060,7 @@ int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, co
     const size_t first = pieces.size();
     for (int32_t t = 0; t < ch.tiles;) {
       const int32_t take = (int32_t)std::min<int64_t>(lane_end - pos, ch.tiles - t);
-      pieces.push_back(MlaPiece{ch.b, ch.token0, t * kTileKeys, take, ch.last, -1, {0, 0}});
+      pieces.push_back(MlaPiece{ch.b, ch.token0, t * kTileKeys, take, ch.last, -1, ch.n_keys, ch.row_step});
       piece_lane.push_back(lane_id);
       pos += take;
       t += take;
@@ -1122,6 +1187,10 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
   p.qk_descale = plan->qk_descale;
   p.pv_descale = plan->pv_descale;
   p.qn_int8 = plan->qn_int8 ? 1 : 0;
+  p.mask = plan->mask;
+  p.mask_cols = plan->mask_cols;
+  p.mask_f16 = plan->mask_f16 ? 1 : 0;
+  p.mask_vec = (reinterpret_cast<uintptr_t>(plan->mask) % 16 == 0 && plan->mask_cols % 8 == 0) ? 1 : 0;
   const bool f16 = plan->dtype == ALA_F16;
   auto kern = plan->kv8 ? (f16 ? mla_kernel<__half, true> : mla_kernel<__nv_bfloat16, true>)
                         : (f16 ? mla_kernel<__half, false> : mla_kernel<__nv_bfloat16, false>);

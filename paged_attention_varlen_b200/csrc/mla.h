@@ -14,13 +14,15 @@ struct MlaPlan {
   int32_t dtype = 0, heads = 0, batch = 0, block_size = 0, max_blocks = 0;
   int32_t calc_type = 0, mask_type = 0;
   bool kv8 = false, qn_int8 = false;  // int8 latent cache (cacheMode 2); qNope holds int8 codes
-  bool pair = false;                   // served by the CTA-pair kernel (mla_pair.cu)
   const float *qk_descale = nullptr, *pv_descale = nullptr;
   float qk_scale = 1.f;
   int64_t tokens = 0, num_blocks = 0;
   void *q_nope = nullptr, *q_rope = nullptr, *ct_kv = nullptr, *k_rope = nullptr, *out = nullptr;
   float* lse = nullptr;
   const int32_t* block_tables = nullptr;
+  const uint16_t* mask = nullptr;      // explicit MASK_TYPE_SPEC mask [tokens, mask_cols], or null
+  int64_t mask_cols = 0;
+  bool mask_f16 = false;
   std::vector<int32_t> ctx, qs;
   // row blocks of tpc tokens x hpc heads; groups = heads / hpc
   int32_t tpc = 1, hpc = 64, groups = 1;
@@ -47,12 +49,5 @@ int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, co
              int calcType, uint8_t cacheMode, ala_tensor* attenOut, ala_tensor* lse, char* err, size_t errlen);
 
 int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size_t errlen);
-
-// The CTA-pair kernel (M = 128 rows per CTA, two CTAs per 128 heads splitting the latent dimensions):
-// decode with one query token per batch, heads a multiple of 128, a 16-bit cache.  mla_pair_plan
-// replaces the schedule mla_plan built (same validated request); mla_pair_run executes it.
-bool mla_pair_eligible(const MlaPlan* plan);
-int mla_pair_plan(MlaPlan* plan, char* err, size_t errlen);
-int mla_pair_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size_t errlen);
 
 }  // namespace ala

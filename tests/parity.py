@@ -46,7 +46,11 @@ def check_out(got: torch.Tensor, ref: np.ndarray, what: str = "out"):
 
 
 def check_lse(got: torch.Tensor, ref: np.ndarray, what: str = "lse"):
+    """lse within the relative bound; a row with no allowed key (reference -inf) must be exactly -inf."""
     g = got.detach().float().cpu().double().numpy().reshape(ref.shape)
+    empty = ref == -np.inf
+    assert (g[empty] == -np.inf).all(), f"{what}: rows without an allowed key must have lse = -inf"
+    g, ref = g[~empty], ref[~empty]
     assert np.isfinite(g).all(), f"{what}: non-finite values in the GPU lse"
     rel = np.abs(g - ref) / np.maximum(1.0, np.abs(ref))
     mx = float(rel.max(initial=0.0))

@@ -141,7 +141,7 @@ def _plan_mla(**over):
     return ala.plan_mla(a["q_nope"], a["q_rope"], a["ct_kv"], a["k_rope"], a["block_tables"], a["context_lens"],
                         a["q_seq_len"], a["heads"], a["qk_scale"], a["mask_type"], a["calc_type"], a["cache_mode"],
                         kv_heads=a["kv_heads"], lse=a.get("lse"), qk_descale=a.get("qk_descale"),
-                        pv_descale=a.get("pv_descale"))
+                        pv_descale=a.get("pv_descale"), mask=a.get("mask"))
 
 
 def _int8_cache(**over):
@@ -322,3 +322,25 @@ def test_noalloc_refuses_more_work_units_than_its_scratch_holds():
 def test_noalloc_refuses_an_lse_of_the_wrong_shape(lse_shape):
     st, msg = _noalloc_raw(10, 4, 4, 64, [10], lse_shape)
     assert st == 2 and "lse" in msg
+
+
+def test_mla_explicit_mask_plans():
+    # the MASK_TYPE_SPEC mask [tokens, maxSeqLen] (fp16 or bf16) with maskType SPEC, one or more tokens per batch
+    _plan_mla(mask_type=1, mask=torch.zeros(3, 128, dtype=torch.bfloat16))
+    _plan_mla(mask_type=1, mask=torch.zeros(3, 200, dtype=torch.float16))
+    _plan_mla(q_nope=torch.zeros(6, 128, 512, dtype=torch.bfloat16), q_rope=torch.zeros(6, 128, 64, dtype=torch.bfloat16),
+              q_seq_len=[2, 2, 2], mask_type=1, calc_type=1, mask=torch.zeros(6, 130, dtype=torch.bfloat16))
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(mask=torch.zeros(3, 128, dtype=torch.bfloat16)), 4),                    # maskType UNDEFINED takes no mask
+    (dict(mask_type=1, mask=torch.zeros(3, 127, dtype=torch.bfloat16)), 2),       # shorter than contextLens 128
+    (dict(mask_type=1, mask=torch.zeros(4, 128, dtype=torch.bfloat16)), 2),       # one row per token
+    (dict(mask_type=1, mask=torch.zeros(3, 128, dtype=torch.float32)), 3),        # fp16 / bf16 only
+    (dict(mask_type=1, mask=torch.zeros(3, 2, 128, dtype=torch.bfloat16)), 2),    # 2-D
+    (dict(q_seq_len=[1, 1, 1], calc_type=3, mask_type=1, mask=torch.zeros(3, 128, dtype=torch.bfloat16)), 4),
+])
+def test_mla_explicit_mask_rejects(over, status):
+    with pytest.raises(ala.AlaError) as e:
+        _plan_mla(**over)
+    assert e.value.status == status, str(e.value)

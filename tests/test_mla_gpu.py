@@ -23,7 +23,7 @@ def built():
     build.build()
 
 
-def _run(case):
+def _run(case, mask=None):
     d = "cuda"
     qn, qr = case.q_nope.to(d), case.q_rope.to(d)
     ck, kr = case.ct_kv.to(d), case.k_rope.to(d)
@@ -32,16 +32,16 @@ def _run(case):
     out = nan_out(qr, (case.n_tokens, case.heads, 512))
     qs = case.q_seq_len if case.calc_type in (synth.MLA_CALC_SPEC, ala.MLA_CALC_PREFILL) else None
     op, out = ala.plan_mla(qn, qr, ck, kr, bt, case.context_lens, qs, case.heads, case.qk_scale, case.mask_type,
-                           case.calc_type, lse=lse, out=out)
+                           case.calc_type, lse=lse, out=out, mask=None if mask is None else mask.to(d))
     op()
     torch.cuda.synchronize()
     assert op.device_status() == 0, f"device status {op.device_status():#x}"
     return out, lse, op
 
 
-def _oracle(case, rows=None):
+def _oracle(case, rows=None, mask=None):
     return oracle.mla(case.q_nope, case.q_rope, case.ct_kv, case.k_rope, case.block_tables, case.block_size,
-                      case.context_lens, case.q_seq_len, case.heads, case.qk_scale, rows=rows)
+                      case.context_lens, case.q_seq_len, case.heads, case.qk_scale, rows=rows, mask=mask)
 
 
 @pytest.mark.parametrize("qs", [1, 4])
@@ -210,5 +210,69 @@ def test_mla_prefill_is_causal_within_each_batch():
     case.mask_type = synth.MLA_MASK_UNDEFINED
     out, lse, _ = _run(case)
     ref, lref = _oracle(case)
+    check_out(out.reshape(-1, 512), ref)
+    check_lse(lse.reshape(-1), lref)
+
+
+# ---------------------------------------------------------------------------- explicit MASK_TYPE_SPEC mask tensor
+
+def _random_mask(case, cols, seed, dtype, p_masked=0.3):
+    """[tokens, cols] additive mask: N(0, 2) values, a share of -inf, key 0 always open."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    m = (rng.standard_normal((case.n_tokens, cols)) * 2.0).astype(np.float32)
+    m[rng.random(m.shape) < p_masked] = -np.inf
+    m[:, 0] = 0.0
+    return torch.from_numpy(m).to(dtype)
+
+
+def _spec_mask(case, cols, dtype):
+    rows = []
+    for c, q in zip(case.context_lens.tolist(), case.q_seq_len.tolist()):
+        for t in range(q):
+            r = torch.full((cols,), torch.finfo(dtype).min, dtype=torch.float32)
+            r[:c - q + t + 1] = 0.0
+            rows.append(r)
+    return torch.stack(rows).to(dtype)
+
+
+def _with_mask(case):
+    case.calc_type = synth.MLA_CALC_SPEC
+    case.mask_type = synth.MLA_MASK_SPEC
+    return case
+
+
+@pytest.mark.parametrize("qs,block_size,cols", [(1, 128, 1104), (4, 16, 1100), ([1, 3, 4, 2], 64, 1107)])
+def test_mla_explicit_random_mask(qs, block_size, cols):
+    # a non-causal additive mask per token; key ranges long enough to be cut across CTAs (partials merged)
+    ctx = np.array([700, 1100, 65, 300], dtype=np.int32)
+    case = _with_mask(synth.make_mla("emask", ctx, qs, 128, 83, block_size=block_size))
+    mask = _random_mask(case, cols, 83, torch.bfloat16)
+    out, lse, _ = _run(case, mask)
+    ref, lref = _oracle(case, mask=mask)
+    check_out(out.reshape(-1, 512), ref)
+    check_lse(lse.reshape(-1), lref)
+
+
+def test_mla_explicit_mask_of_the_rule_matches_the_rule_fp16():
+    ctx = np.array([90, 640, 1500, 7], dtype=np.int32)
+    case = _with_mask(synth.make_mla("rule_mask", ctx, 4, 128, 85, block_size=32, dtype=torch.float16))
+    mask = _spec_mask(case, 1504, torch.float16)
+    out, lse, _ = _run(case, mask)
+    ref, lref = _oracle(case)  # the generated rule
+    check_out(out.reshape(-1, 512), ref)
+    check_lse(lse.reshape(-1), lref)
+
+
+def test_mla_explicit_mask_rows_without_an_allowed_key():
+    # token 1 is masked everywhere (output 0, lse -inf), token 2 only beyond key 900 (the row's whole key
+    # range is cut across CTAs, so empty partials meet in the merge)
+    ctx = np.array([1200], dtype=np.int32)
+    case = _with_mask(synth.make_mla("empty_rows", ctx, 4, 128, 87, block_size=64))
+    mask = _random_mask(case, 1200, 87, torch.bfloat16, p_masked=0.1)
+    mask[1, :] = -float("inf")
+    mask[2, :900] = -float("inf")
+    out, lse, _ = _run(case, mask)
+    ref, lref = _oracle(case, mask=mask)
+    assert (ref[128:256] == 0).all() and (lref[128:256] == -np.inf).all()
     check_out(out.reshape(-1, 512), ref)
     check_lse(lse.reshape(-1), lref)

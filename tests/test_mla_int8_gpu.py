@@ -24,7 +24,7 @@ def built():
     build.build()
 
 
-def _run(case, calc_type=None):
+def _run(case, calc_type=None, mask=None):
     d = "cuda"
     ct = case.calc_type if calc_type is None else calc_type
     qn, qr = case.q_nope.to(d), case.q_rope.to(d)
@@ -37,17 +37,18 @@ def _run(case, calc_type=None):
     qs = case.q_seq_len if (ct in (synth.MLA_CALC_SPEC, ala.MLA_CALC_PREFILL) or
                             (ct == ala.MLA_CALC_RING and (case.q_seq_len > 1).any())) else None
     op, out = ala.plan_mla(qn, qr, ck, kr, bt, case.context_lens, qs, case.heads, case.qk_scale, case.mask_type, ct,
-                           lse=lse, out=out, qk_descale=qkd, pv_descale=pvd)
+                           lse=lse, out=out, qk_descale=qkd, pv_descale=pvd,
+                           mask=None if mask is None else mask.to(d))
     op()
     torch.cuda.synchronize()
     assert op.device_status() == 0, f"device status {op.device_status():#x}"
     return out, lse, op
 
 
-def _oracle(case, rows=None):
+def _oracle(case, rows=None, mask=None):
     return oracle.mla_dequant(case.q_nope, case.q_rope, case.ct_kv, case.k_rope, case.qk_descale, case.pv_descale,
                               case.block_tables, case.block_size, case.context_lens, case.q_seq_len, case.heads,
-                              case.qk_scale, rows=rows)
+                              case.qk_scale, rows=rows, mask=mask)
 
 
 @pytest.mark.parametrize("qn_int8", [True, False])
@@ -159,5 +160,21 @@ def test_mla_int8_prefill_is_causal_within_each_batch():
     case = synth.make_mla_int8("prefill8", ctx, qs, 64, 57, block_size=64)
     out, lse, _ = _run(case, calc_type=ala.MLA_CALC_PREFILL)
     ref, lref = _oracle(case)
+    check_out(out.reshape(-1, 512), ref)
+    check_lse(lse.reshape(-1), lref)
+
+
+def test_mla_int8_explicit_mask():
+    # the MASK_TYPE_SPEC mask tensor over the int8 cache: a non-causal additive mask per token
+    ctx = np.array([700, 1100, 65], dtype=np.int32)
+    case = synth.make_mla_int8("mask8", ctx, 2, 128, 59, block_size=64)
+    case.calc_type, case.mask_type = synth.MLA_CALC_SPEC, synth.MLA_MASK_SPEC
+    rng = np.random.Generator(np.random.PCG64(59))
+    m = (rng.standard_normal((case.n_tokens, 1100)) * 2.0).astype(np.float32)
+    m[rng.random(m.shape) < 0.3] = -np.inf
+    m[:, 0] = 0.0
+    mask = torch.from_numpy(m).to(torch.float16)
+    out, lse, _ = _run(case, mask=mask)
+    ref, lref = _oracle(case, mask=mask)
     check_out(out.reshape(-1, 512), ref)
     check_lse(lse.reshape(-1), lref)
