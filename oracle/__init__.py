@@ -53,8 +53,10 @@ def _load():
         _lib.oracle_mla_dequant.argtypes = [P, ctypes.c_int, P, ctypes.c_int, P, ctypes.c_int, P, P, P, P, I64,
                                             I32, P, P, I32, I32, I32, I32, D, P, ctypes.c_int, I64, P, I64, P, P]
         _lib.oracle_lse_merge.argtypes = [I32, I64, I32, P, P, P, P]
+        _lib.oracle_decode.argtypes = [P, ctypes.c_int, I64, P]
         for f in ("oracle_attention", "oracle_build_mask", "oracle_attention_explicit",
-                  "oracle_expand_causal_compressed", "oracle_mla", "oracle_mla_dequant", "oracle_lse_merge"):
+                  "oracle_expand_causal_compressed", "oracle_mla", "oracle_mla_dequant", "oracle_lse_merge",
+                  "oracle_decode"):
             getattr(_lib, f).restype = ctypes.c_int
     return _lib
 
@@ -65,6 +67,17 @@ def _raw(t: torch.Tensor):
     code = _DTYPE_CODE[t.dtype]
     arr = t.view(torch.int16).numpy() if t.dtype in (torch.float16, torch.bfloat16) else t.numpy()
     return np.ascontiguousarray(arr), code
+
+
+_F64 = 4
+
+
+def _decoded(t: torch.Tensor):
+    """The stored elements of a CPU tensor decoded to float64 by oracle.c (exact), with the F64 code."""
+    raw, code = _raw(t)
+    out = np.empty(raw.size, dtype=np.float64)
+    _load().oracle_decode(raw.ctypes.data_as(ctypes.c_void_p), code, raw.size, out.ctypes.data_as(ctypes.c_void_p))
+    return out, _F64
 
 
 def _ptr(a):
@@ -85,10 +98,10 @@ def attention(q, k, v, seq_len, kv_seq_len, mask_type, heads, kv_heads, qk_scale
     nTokens*heads (row index = token*heads + head).
     """
     lib = _load()
-    qa, qc = _raw(q)
-    ka, kc = _raw(k)
-    va, vc = _raw(v)
-    assert kc == vc
+    assert k.dtype == v.dtype
+    qa, qc = _decoded(q)
+    ka, kc = _decoded(k)
+    va, vc = _decoded(v)
     d_qk, d_v = q.shape[-1], v.shape[-1]
     sl, kl = _i32(seq_len), _i32(kv_seq_len)
     bt = _i32(block_tables)
@@ -155,11 +168,11 @@ def mla(q_nope, q_rope, ct_kv, k_rope, block_tables, block_size, context_lens, q
         return mla_dequant(q_nope, q_rope, ct_kv, k_rope, None, None, block_tables, block_size, context_lens,
                            q_seq_len, heads, qk_scale, rows=rows, mask=mask)
     lib = _load()
-    qn, c1 = _raw(q_nope)
-    qr, c2 = _raw(q_rope)
-    ck, c3 = _raw(ct_kv)
-    kr, c4 = _raw(k_rope)
-    assert c1 == c2 == c3 == c4
+    assert q_nope.dtype == q_rope.dtype == ct_kv.dtype == k_rope.dtype
+    qn, c1 = _decoded(q_nope)
+    qr, _ = _decoded(q_rope)
+    ck, _ = _decoded(ct_kv)
+    kr, _ = _decoded(k_rope)
     bt = _i32(block_tables)
     cl = _i32(context_lens)
     qs = _i32(q_seq_len) if q_seq_len is not None else np.ones_like(cl)
@@ -182,11 +195,11 @@ def mla_dequant(q_nope, q_rope, ct_kv, k_rope, qk_descale, pv_descale, block_tab
     s = qkScale * (qkDescale[h] * qNope.ctKV + qRope.kRope), O = pvDescale[h] * softmax(s) ctKV,
     qNope and ctKV taken as stored (int8 or float); a None descale means 1.  ``mask`` as in ``mla``."""
     lib = _load()
-    qn, cq = _raw(q_nope)
-    qr, cr = _raw(q_rope)
-    ck, ckv = _raw(ct_kv)
-    kr, cr2 = _raw(k_rope)
-    assert cr == cr2
+    assert q_rope.dtype == k_rope.dtype
+    qn, cq = _decoded(q_nope)
+    qr, cr = _decoded(q_rope)
+    ck, ckv = _decoded(ct_kv)
+    kr, _ = _decoded(k_rope)
     qd = None if qk_descale is None else np.ascontiguousarray(np.asarray(qk_descale, dtype=np.float32))
     pd = None if pv_descale is None else np.ascontiguousarray(np.asarray(pv_descale, dtype=np.float32))
     for d in (qd, pd):

@@ -56,6 +56,7 @@
 #define ORC_BF16 1
 #define ORC_F32 2
 #define ORC_I8 3 /* two's-complement signed 8-bit integer */
+#define ORC_F64 4 /* already decoded (oracle_decode) */
 
 /* mask types, numbered as on the ATB PrefixEncoder page (maskType row) plus
  * 0 = no mask (all keys of the sequence allowed). */
@@ -95,8 +96,18 @@ static double orc_load(const void* base, int dtype, int64_t idx) {
     case ORC_F16: return orc_half_to_double(((const uint16_t*)base)[idx]);
     case ORC_BF16: return orc_bf16_to_double(((const uint16_t*)base)[idx]);
     case ORC_I8: return (double)((const int8_t*)base)[idx];
+    case ORC_F64: return ((const double*)base)[idx];
     default: return (double)((const float*)base)[idx];
   }
+}
+
+/* Decodes n stored elements into doubles once (exact for every type above),
+ * so that the attention loops, which read each key and value row once per
+ * query row, read plain doubles instead of decoding the same element again. */
+int oracle_decode(const void* src, int dtype, int64_t n, double* dst) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) dst[i] = orc_load(src, dtype, i);
+  return 0;
 }
 
 /* ---- the mask rule ------------------------------------------------------
