@@ -49,7 +49,8 @@ PROFILE = os.path.join(ROOT, "profiles", "prefill_varlen_causal_bf16.md")
 MLA_PROFILE = os.path.join(ROOT, "profiles", "mla_decode_qs1_bf16.md")
 MLA_INT8_PROFILE = os.path.join(ROOT, "profiles", "mla_decode_qs1_int8.md")
 KERNEL_SOURCES = ["paged_attention_varlen_b200/csrc/prefill.cu", "paged_attention_varlen_b200/csrc/ptx.cuh"]
-MLA_KERNEL_SOURCES = ["paged_attention_varlen_b200/csrc/mla.cu", "paged_attention_varlen_b200/csrc/ptx.cuh"]
+MLA_KERNEL_SOURCES = ["paged_attention_varlen_b200/csrc/mla.cu", "paged_attention_varlen_b200/csrc/mla_wide.cu",
+                      "paged_attention_varlen_b200/csrc/mla_common.cuh", "paged_attention_varlen_b200/csrc/ptx.cuh"]
 DEFAULT_WORKLOAD = "varlen_causal_bf16"
 WORKLOADS = {
     "varlen_causal_bf16": lambda: synth.varlen_causal_bf16(),
@@ -183,8 +184,8 @@ def mla_bytes(case) -> float:
     return kv + q + o
 
 
-def plan_case(ala, case, device):
-    """Device copies of the inputs and a planned op; returns (op, tensors dict)."""
+def device_inputs(case, device):
+    """Device copies of a workload's inputs (and fp32 lse / per-head descale buffers for MLA)."""
     if isinstance(case, synth.MlaCase):
         t = {"q_nope": case.q_nope.to(device), "q_rope": case.q_rope.to(device), "ct_kv": case.ct_kv.to(device),
              "k_rope": case.k_rope.to(device), "bt": torch.from_numpy(case.block_tables).to(device)}
@@ -192,23 +193,59 @@ def plan_case(ala, case, device):
         if case.qk_descale is not None:  # int8 latent cache
             t["qk_descale"] = torch.from_numpy(case.qk_descale).to(device)
             t["pv_descale"] = torch.from_numpy(case.pv_descale).to(device)
-        op, out = ala.plan_mla(t["q_nope"], t["q_rope"], t["ct_kv"], t["k_rope"], t["bt"], case.context_lens,
-                               case.q_seq_len if case.calc_type == synth.MLA_CALC_SPEC else None, case.heads,
-                               case.qk_scale, case.mask_type, case.calc_type, lse=t["lse"],
-                               qk_descale=t.get("qk_descale"), pv_descale=t.get("pv_descale"))
-        t["out"] = out
-        return op, t
+        return t
     t = {"q": case.q.to(device), "k": case.k.to(device), "v": case.v.to(device)}
-    slopes = None if case.slopes is None else torch.from_numpy(case.slopes).to(device)
+    t["slopes"] = None if case.slopes is None else torch.from_numpy(case.slopes).to(device)
     if case.paged:
         t["bt"] = torch.from_numpy(case.block_tables).to(device)
-        op, out = ala.plan_prefix_encoder(t["q"], t["k"], t["v"], t["bt"], case.seq_len, case.kv_seq_len,
-                                          case.mask_type, case.heads, case.kv_heads, case.qk_scale, slopes)
-    else:
-        op, out = ala.plan_varlen_attention(t["q"], t["k"], t["v"], case.seq_len, case.kv_seq_len, case.mask_type,
-                                            case.heads, case.kv_heads, case.qk_scale, slopes)
-    t["out"], t["slopes"] = out, slopes
+    return t
+
+
+def plan_on(ala, case, t, out=None):
+    """Plan the workload's call on device inputs `t` (the public *_get_workspace_size path); returns (op, out)."""
+    if isinstance(case, synth.MlaCase):
+        return ala.plan_mla(t["q_nope"], t["q_rope"], t["ct_kv"], t["k_rope"], t["bt"], case.context_lens,
+                            case.q_seq_len if case.calc_type == synth.MLA_CALC_SPEC else None, case.heads,
+                            case.qk_scale, case.mask_type, case.calc_type, lse=t["lse"], out=out,
+                            qk_descale=t.get("qk_descale"), pv_descale=t.get("pv_descale"))
+    if case.paged:
+        return ala.plan_prefix_encoder(t["q"], t["k"], t["v"], t["bt"], case.seq_len, case.kv_seq_len,
+                                       case.mask_type, case.heads, case.kv_heads, case.qk_scale, t["slopes"], out=out)
+    return ala.plan_varlen_attention(t["q"], t["k"], t["v"], case.seq_len, case.kv_seq_len, case.mask_type,
+                                     case.heads, case.kv_heads, case.qk_scale, t["slopes"], out=out)
+
+
+def plan_case(ala, case, device):
+    """Device copies of the inputs and a planned op; returns (op, tensors dict)."""
+    t = device_inputs(case, device)
+    op, t["out"] = plan_on(ala, case, t)
     return op, t
+
+
+def host_costs(ala, case, t, reps=15):
+    """Host-side cost of a call, reported apart from the kernel time (the schedule is host work):
+    plan = *_get_workspace_size (validation, per-sequence table, work units and their longest-first packing,
+    or the MLA lane plan) plus the output / workspace tensors from torch's caching allocator;
+    first_run_extra = the extra host time of an op's first execution (tensor-map encoding);
+    launch = host time of a later execution (schedule upload and kernel launches enqueued)."""
+    plan_ms, first_ms, later_ms = [], [], []
+    for _ in range(reps):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        op, _ = plan_on(ala, case, t, out=t["out"])
+        t1 = time.perf_counter()
+        op()
+        t2 = time.perf_counter()
+        op()
+        t3 = time.perf_counter()
+        torch.cuda.synchronize()
+        plan_ms.append((t1 - t0) * 1e3)
+        first_ms.append((t2 - t1) * 1e3)
+        later_ms.append((t3 - t2) * 1e3)
+        del op
+    med = statistics.median
+    return {"plan_ms": med(plan_ms), "first_run_extra_ms": max(0.0, med(first_ms) - med(later_ms)),
+            "launch_ms": med(later_ms), "reps": reps}
 
 
 def time_steps(op, steps, warmup, flush, stream, barrier=lambda: None):
@@ -250,8 +287,27 @@ def e2e_prefill(ala, case, tens, op, steps, stream):
         if i >= 2:
             times.append(e0.elapsed_time(e1))
     ms = statistics.mean(times)
+    # the same, with the call planned inside the timed region every step (a caller whose lengths change
+    # every step pays get_workspace_size and the tensor-map encoding each time); wall clock
+    wall = []
+    for i in range(steps + 2):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        with torch.cuda.stream(stream):
+            for k in ("q", "k", "v"):
+                tens[k].copy_(host[k], non_blocking=True)
+            op2, _ = plan_on(ala, case, tens, out=tens["out"])
+            op2(stream)
+            out_host.copy_(tens["out"], non_blocking=True)
+        torch.cuda.synchronize()
+        if i >= 2:
+            wall.append((time.perf_counter() - t0) * 1e3)
+        del op2
+    ms_plan = statistics.mean(wall)
     return {"value": prefill_flops(case) / (ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "with_plan": {"value": prefill_flops(case) / (ms_plan * 1e-3) / 1e12, "unit": "TFLOPS",
+                          "ms_per_step": ms_plan, "timing": "wall clock, synchronised on both sides"}}
 
 
 def cpu_baseline(case, sample_s=12.0):
@@ -282,6 +338,17 @@ def cpu_baseline(case, sample_s=12.0):
                       f"fp64 on the host (valid FLOPs of the sampled rows / time)"}
 
 
+def mla_kernel_name(case):
+    """The MLA kernel a workload runs on: 128 query rows per CTA (one token per row block, 16-bit cache,
+    heads a multiple of 128) or 64."""
+    int8 = case.qk_descale is not None
+    qs = case.q_seq_len
+    tpc = 4 if (qs % 4 == 0).all() else 2 if (qs % 2 == 0).all() else 1
+    if tpc == 1 and not int8 and case.heads % 128 == 0:
+        return "mla_wide_kernel<bf16>"
+    return "mla_kernel<bf16, int8 cache>" if int8 else "mla_kernel<bf16>"
+
+
 def case_dtype(case):
     return case.q_rope.dtype if isinstance(case, synth.MlaCase) else case.dtype
 
@@ -307,23 +374,76 @@ def base_config(case):
             "paged": case.paged, "parallelism": "replicas (independent sequences)", "l2": l2}
 
 
+def _row_flops(case, rows):
+    """Valid FLOPs of the given flattened (token * heads + head) rows."""
+    tok = rows // case.heads
+    if isinstance(case, synth.MlaCase):
+        cu = np.concatenate([[0], np.cumsum(case.q_seq_len)])
+        b = np.searchsorted(cu, tok, side="right") - 1
+        allowed = case.context_lens[b] - case.q_seq_len[b] + (tok - cu[b]) + 1
+        return float((allowed * (2 * 576 + 2 * 512)).sum())
+    cu = np.concatenate([[0], np.cumsum(case.seq_len)])
+    b = np.searchsorted(cu, tok, side="right") - 1
+    i = tok - cu[b]
+    if case.mask_type == synth.MASK_NONE:
+        allowed = case.kv_seq_len[b]
+    else:
+        allowed = np.minimum(i + (case.kv_seq_len[b] - case.seq_len[b]) + 1, case.kv_seq_len[b])
+    return float((4.0 * case.head_size * allowed).sum())
+
+
+def _oracle_rows(case, rows):
+    import oracle
+    if isinstance(case, synth.MlaCase):
+        oracle.mla(case.q_nope, case.q_rope, case.ct_kv, case.k_rope, case.block_tables, case.block_size,
+                   case.context_lens, case.q_seq_len, case.heads, case.qk_scale, rows=rows)
+    else:
+        oracle.attention(case.q, case.k, case.v, case.seq_len, case.kv_seq_len, case.mask_type, case.heads,
+                         case.kv_heads, case.qk_scale, slopes=case.slopes, block_tables=case.block_tables,
+                         block_size=case.block_size, rows=rows)
+
+
 def run_reference(args, rank, world):
+    """The oracle as it stands, timed on the host cores: every step computes the same fixed random sample
+    of the workload's (token, head) rows, sized so that warm-up plus timed steps take about a minute."""
     if rank != 0:
         return
-    case = synth.varlen_causal_bf16()
-    cb = cpu_baseline(case, sample_s=max(3.0, 10.0 / max(1, args.steps + args.warmup)))
-    vals = []
-    for _ in range(args.warmup + args.steps):
-        vals.append(cpu_baseline(case, sample_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)))["value"])
-    v = statistics.mean(vals[args.warmup:]) if len(vals) > args.warmup else vals[-1]
-    flops = prefill_flops(case)
-    line = {"impl": "reference", "metric": "attention TFLOPS on valid tokens (prefill)", "value": v,
-            "unit": "TFLOPS", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": flops / (v * 1e12) * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": base_config(case),
-            "cpu_baseline": {"value": v, "unit": "TFLOPS", "cores": cb["cores"], "kind": "oracle",
-                             "sample": "each step: a bounded random sample of rows; " + cb["sample"]},
-            "e2e": {"value": v, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    case = WORKLOADS[args.workload]()
+    is_mla = isinstance(case, synth.MlaCase)
+    n_total = case.n_tokens * case.heads
+    perm = np.random.Generator(np.random.PCG64(7)).permutation(n_total).astype(np.int64)
+    probe = np.sort(perm[:64])
+    t0 = time.perf_counter()
+    _oracle_rows(case, probe)
+    s_per_flop = (time.perf_counter() - t0) / max(_row_flops(case, probe), 1.0)
+    flops_per_row = _row_flops(case, perm[:4096]) / min(4096, n_total)  # the workload's mean row cost
+    step_s = min(10.0, max(0.5, 60.0 / (args.steps + args.warmup)))
+    n = int(min(n_total, max(64, step_s / (s_per_flop * flops_per_row))))
+    rows = np.sort(perm[:n])
+    flops = _row_flops(case, rows)
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        _oracle_rows(case, rows)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    ms = statistics.mean(times) * 1e3
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    if is_mla:
+        value, unit = mla_bytes(case) * n / n_total / (ms * 1e-3) / 1e9, "GB/s"
+        metric = "attention HBM GB/s (MLA decode)"
+    else:
+        value, unit = flops / (ms * 1e-3) / 1e12, "TFLOPS"
+        metric = "attention TFLOPS on valid tokens (prefill)"
+    sample = (f"each step: the same {n} random (token, head) rows of the {case.name} workload "
+              f"({n / n_total:.2%} of its rows, {flops / 1e9:.2f} valid GFLOP), fp64 oracle on the host")
+    config = base_config(case)
+    config["reference_sample_rows"] = n
+    line = {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
 
 
@@ -389,7 +509,7 @@ def main():
                         "traffic": profiled_traffic(MLA_INT8_PROFILE if int8 else MLA_PROFILE, src),
                         "algorithmic_bytes": nbytes, "peak_source": peaks["source"] + " (copy bandwidth)",
                         "tflops": flops / (mean_ms * 1e-3) / 1e12,
-                        "kernel": ("mla_kernel<bf16, int8 cache>" if int8 else "mla_kernel<bf16>") + " + mla_combine_kernel",
+                        "kernel": mla_kernel_name(case) + " + mla_combine_kernel",
                         "kernel_source_sha256": src}
             launches = args.steps * (2 if op_has_combine(op) else 1)
         else:
@@ -413,6 +533,7 @@ def main():
         args.no_extra = args.no_extra or args.workload != DEFAULT_WORKLOAD
         if not args.no_e2e:
             line["e2e"] = e2e_prefill(ala, case, tens, op, min(args.steps, 10), stream)
+        line["host"] = host_costs(ala, case, tens)
         if not args.no_extra:
             line["extra"] = extra_workloads(ala, device, flush, stream, peaks, case, args)
         if world == 1 and not args.no_cpu:
@@ -437,14 +558,15 @@ def extra_workloads(ala, device, flush, stream, peaks, main_case, args):
     del op
     for case in (synth.prefix_paged_alibi_fp16(), synth.long_alibi_bf16(synth.MASK_ALIBI_SQRT),
                  synth.long_alibi_bf16(synth.MASK_ALIBI_LEFT)):
-        op, _ = plan_case(ala, case, device)
+        op, t = plan_case(ala, case, device)
         ms = statistics.mean(time_steps(op, steps, 3, flush, stream))
         tf = prefill_flops(case) / (ms * 1e-3) / 1e12
-        out[case.name] = {"ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / peaks["bf16_tflops"]}
+        out[case.name] = {"ms": ms, "tflops": tf, "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
+                          "host": host_costs(ala, case, t, reps=5)}
         del op
     for case in (synth.mla_decode_bf16(1), synth.mla_decode_bf16(4), synth.mla_decode_int8()):
         try:
-            op, _ = plan_case(ala, case, device)
+            op, t = plan_case(ala, case, device)
             ms = statistics.mean(time_steps(op, steps, 3, flush, stream))
         except ala.AlaError as e:
             out[case.name] = {"unavailable": str(e)}
@@ -452,7 +574,8 @@ def extra_workloads(ala, device, flush, stream, peaks, main_case, args):
         gbs = mla_bytes(case) / (ms * 1e-3) / 1e9
         tf = mla_flops(case) / (ms * 1e-3) / 1e12
         out[case.name] = {"ms": ms, "hbm_gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"], "tflops": tf,
-                          "frac_of_bf16_peak": tf / peaks["bf16_tflops"]}
+                          "frac_of_bf16_peak": tf / peaks["bf16_tflops"], "kernel": mla_kernel_name(case),
+                          "host": host_costs(ala, case, t, reps=5)}
         del op
     return out
 
