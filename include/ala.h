@@ -107,7 +107,9 @@ ALA_API void ala_op_destroy(ala_op* op);
 
 /* Reads the device status word of `workspace` for `op` (synchronous copy on
  * the legacy stream after synchronising `stream`).  *code = 0 means every
- * kernel wait completed; nonzero identifies the wait that ran out. */
+ * kernel wait completed; 0x101..0x10A identifies the wait that ran out; 0x10B
+ * (range-checking build libala_debug.so only) means a block-table entry that
+ * was read lay outside [0, numBlocks): that page was read as zeros. */
 ALA_API int ala_workspace_status(const ala_op* op, const void* workspace, ala_stream_t stream, int32_t* code);
 
 /* ---------------------------------------------------------------------------

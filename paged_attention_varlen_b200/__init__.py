@@ -21,7 +21,8 @@ import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libala.so")
+# ALA_LIBRARY=debug selects libala_debug.so: the same kernels with every block-table entry range-checked
+LIB_PATH = os.path.join(_HERE, "libala_debug.so" if os.environ.get("ALA_LIBRARY") == "debug" else "libala.so")
 
 F16, BF16, F32, I32, I8 = 0, 1, 2, 3, 4
 MASK_NONE, MASK_ALIBI, MASK_ALIBI_SQRT, MASK_ALIBI_LEFT, MASK_CAUSAL = 0, 3, 4, 5, 9
@@ -55,7 +56,8 @@ def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m paged_attention_varlen_b200.build`")
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m paged_attention_varlen_b200.build`"
+                               " (add --debug-bounds for libala_debug.so)")
         L = ctypes.CDLL(LIB_PATH)
         P = ctypes.c_void_p
         T = ctypes.POINTER(AlaTensor)

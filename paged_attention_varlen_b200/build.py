@@ -1,9 +1,12 @@
 """Build libala.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m paged_attention_varlen_b200.build [--verbose-ptxas]
+    python -m paged_attention_varlen_b200.build [--verbose-ptxas] [--debug-bounds]
 
 Objects go to paged_attention_varlen_b200/_build/; the shared library lands
-next to this file so it travels with the source tree.
+next to this file so it travels with the source tree.  --debug-bounds builds
+libala_debug.so instead (objects in _build_debug/): the same library with
+ALA_DEBUG_BOUNDS=1, whose kernels range-check every block-table entry they
+read and report a bad one in the status word instead of reading it.
 """
 from __future__ import annotations
 
@@ -16,7 +19,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libala.so")
-SOURCES = ["api.cpp", "prefill.cu", "mla.cu", "noalloc.cu", "merge.cu"]
+BUILD_DEBUG = os.path.join(HERE, "_build_debug")
+LIB_DEBUG = os.path.join(HERE, "libala_debug.so")
+SOURCES = ["api.cpp", "prefill.cu", "mla.cu", "mla_wide.cu", "noalloc.cu", "merge.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
@@ -29,11 +34,13 @@ def _deps(src):
     return [os.path.join(CSRC, src)] + hdrs
 
 
-def _compile(src, verbose_ptxas):
-    obj = os.path.join(BUILD, src + ".o")
+def _compile(src, verbose_ptxas, debug_bounds=False):
+    obj = os.path.join(BUILD_DEBUG if debug_bounds else BUILD, src + ".o")
     if os.path.exists(obj) and all(os.path.getmtime(obj) >= os.path.getmtime(d) for d in _deps(src)):
         return obj, ""
     cmd = [NVCC, *ARCH, *FLAGS, "-c", os.path.join(CSRC, src), "-o", obj]
+    if debug_bounds:
+        cmd.insert(1, "-DALA_DEBUG_BOUNDS=1")
     if src.endswith(".cpp"):
         cmd[1:1] = ["-x", "cu"]
     if verbose_ptxas and src.endswith(".cu"):
@@ -44,23 +51,24 @@ def _compile(src, verbose_ptxas):
     return obj, r.stderr
 
 
-def build(verbose_ptxas: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(verbose_ptxas: bool = False, debug_bounds: bool = False) -> str:
+    out_dir, lib = (BUILD_DEBUG, LIB_DEBUG) if debug_bounds else (BUILD, LIB)
+    os.makedirs(out_dir, exist_ok=True)
     with cf.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
-        results = list(ex.map(lambda s: _compile(s, verbose_ptxas), SOURCES))
+        results = list(ex.map(lambda s: _compile(s, verbose_ptxas, debug_bounds), SOURCES))
     objs = [o for o, _ in results]
     if verbose_ptxas:
         for _, log in results:
             if log:
                 print(log, file=sys.stderr)
-    if not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        cmd = [NVCC, *ARCH, "-shared", "-Xcompiler", "-fPIC", *objs, "-o", LIB, "-lcudart_static", "-ldl", "-lrt",
+    if not os.path.exists(lib) or any(os.path.getmtime(o) > os.path.getmtime(lib) for o in objs):
+        cmd = [NVCC, *ARCH, "-shared", "-Xcompiler", "-fPIC", *objs, "-o", lib, "-lcudart_static", "-ldl", "-lrt",
                "-lpthread"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(verbose_ptxas="--verbose-ptxas" in sys.argv))
+    print(build(verbose_ptxas="--verbose-ptxas" in sys.argv, debug_bounds="--debug-bounds" in sys.argv))

@@ -161,14 +161,16 @@ void set_last_error(const char* msg) { g_last_error = msg; }
 extern "C" void ala_op_destroy(ala_op* op) { delete op; }
 
 extern "C" int ala_workspace_status(const ala_op* op, const void* workspace, ala_stream_t stream, int32_t* code) {
+  NvtxRange nvtx_range("ala_workspace_status");
   if (!op || !workspace || !code) return fail(ALA_NULL_REQUIRED, "ala_workspace_status: null argument");
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return fail(ALA_CUDA_ERROR, "ala_workspace_status: stream sync failed: %s",
                 cudaGetErrorString(cudaGetLastError()));
-  int32_t v = 0;
-  if (cudaMemcpy(&v, workspace, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess)
+  // word 0: a bounded wait that ran out; word 1: a bad block-table entry seen by a range-checking build
+  int32_t v[2] = {0, 0};
+  if (cudaMemcpy(v, workspace, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess)
     return fail(ALA_CUDA_ERROR, "ala_workspace_status: copy failed");
-  *code = v;
+  *code = v[0] != 0 ? v[0] : v[1];
   return ok();
 }
 
@@ -453,6 +455,7 @@ extern "C" int atb_like_prefix_encoder_get_workspace_size(
     const ala_tensor* mask, const ala_tensor* seqLen, const ala_tensor* kvSeqLen, const ala_tensor* slopes,
     int maskType, int32_t headNum, int32_t kvHeadNum, float qkScale, ala_tensor* attnOut, uint64_t* workspaceSize,
     ala_op** op) {
+  NvtxRange nvtx_range("atb_like_prefix_encoder_get_workspace_size");
   return plan_prefix_encoder(query, key, value, blockTables, mask, seqLen, kvSeqLen, slopes, maskType, headNum,
                              kvHeadNum, qkScale, attnOut, nullptr, workspaceSize, op,
                              "atb_like_prefix_encoder_get_workspace_size");
@@ -463,6 +466,7 @@ extern "C" int atb_like_prefix_encoder_lse_get_workspace_size(
     const ala_tensor* mask, const ala_tensor* seqLen, const ala_tensor* kvSeqLen, const ala_tensor* slopes,
     int maskType, int32_t headNum, int32_t kvHeadNum, float qkScale, ala_tensor* attnOut, ala_tensor* lse,
     uint64_t* workspaceSize, ala_op** op) {
+  NvtxRange nvtx_range("atb_like_prefix_encoder_lse_get_workspace_size");
   const char* fn = "atb_like_prefix_encoder_lse_get_workspace_size";
   if (!lse || !lse->data) return fail(ALA_NULL_REQUIRED, "%s: lse is required", fn);
   return plan_prefix_encoder(query, key, value, blockTables, mask, seqLen, kvSeqLen, slopes, maskType, headNum,
@@ -470,6 +474,7 @@ extern "C" int atb_like_prefix_encoder_lse_get_workspace_size(
 }
 
 extern "C" int atb_like_prefix_encoder(void* workspace, uint64_t workspaceSize, ala_op* op, ala_stream_t stream) {
+  NvtxRange nvtx_range("atb_like_prefix_encoder");
   return run_prefill(workspace, workspaceSize, op, stream, "atb_like_prefix_encoder");
 }
 
@@ -479,6 +484,7 @@ extern "C" int varlen_attention_get_workspace_size(const ala_tensor* query, cons
                                                    int32_t headNum, int32_t kvHeadNum, float qkScale,
                                                    ala_tensor* attnOut, ala_tensor* lse, uint64_t* workspaceSize,
                                                    ala_op** op) {
+  NvtxRange nvtx_range("varlen_attention_get_workspace_size");
   const char* fn = "varlen_attention_get_workspace_size";
   if (!workspaceSize || !op) return fail(ALA_NULL_REQUIRED, "%s: workspaceSize and op are required", fn);
   *op = nullptr;
@@ -495,6 +501,7 @@ extern "C" int varlen_attention_get_workspace_size(const ala_tensor* query, cons
 }
 
 extern "C" int varlen_attention(void* workspace, uint64_t workspaceSize, ala_op* op, ala_stream_t stream) {
+  NvtxRange nvtx_range("varlen_attention");
   return run_prefill(workspace, workspaceSize, op, stream, "varlen_attention");
 }
 
@@ -507,6 +514,7 @@ extern "C" int atb_like_mla_get_workspace_size(const ala_tensor* qNope, const al
                                                int32_t headNum, float qkScale, int32_t kvHeadNum, int maskType,
                                                int calcType, uint8_t cacheMode, ala_tensor* attenOut, ala_tensor* lse,
                                                uint64_t* workspaceSize, ala_op** op) {
+  NvtxRange nvtx_range("atb_like_mla_get_workspace_size");
   const char* fn = "atb_like_mla_get_workspace_size";
   if (!workspaceSize || !op) return fail(ALA_NULL_REQUIRED, "%s: workspaceSize and op are required", fn);
   *op = nullptr;
@@ -543,6 +551,7 @@ extern "C" int atb_like_mla_get_workspace_size(const ala_tensor* qNope, const al
 }
 
 extern "C" int atb_like_mla(void* workspace, uint64_t workspaceSize, ala_op* op, ala_stream_t stream) {
+  NvtxRange nvtx_range("atb_like_mla");
   const char* fn = "atb_like_mla";
   if (!op) return fail(ALA_NULL_REQUIRED, "%s: op is NULL", fn);
   if (op->kind != ala_op::kMla) return fail(ALA_INVALID_PARAM, "%s: op was not made by atb_like_mla_get_workspace_size", fn);
@@ -558,6 +567,7 @@ extern "C" int atb_like_mla(void* workspace, uint64_t workspaceSize, ala_op* op,
 
 extern "C" int ala_lse_merge(const ala_tensor* outA, const ala_tensor* lseA, const ala_tensor* outB,
                              const ala_tensor* lseB, ala_tensor* out, ala_tensor* lse, ala_stream_t stream) {
+  NvtxRange nvtx_range("ala_lse_merge");
   const char* fn = "ala_lse_merge";
   const ala_tensor* ts[6] = {outA, lseA, outB, lseB, out, lse};
   for (const ala_tensor* t : ts)

@@ -3,9 +3,19 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 namespace ala {
+
+// One NVTX range per C-ABI call (named after the entry point), visible in a profiler's timeline; without
+// a profiler attached the push and pop cost a function-pointer check.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Device status codes written by bounded waits (0 = no error).
 enum DeviceStatus : int {
@@ -20,7 +30,32 @@ enum DeviceStatus : int {
   kDevTimeoutPFull = 0x108,
   kDevTimeoutODone = 0x109,
   kDevTimeoutFinal = 0x10A,
+  kDevBadBlockIndex = 0x10B,  // ALA_DEBUG_BOUNDS builds: a block-table entry read lies outside [0, numBlocks)
 };
+
+#ifndef ALA_DEBUG_BOUNDS
+#define ALA_DEBUG_BOUNDS 0  // 1: kernels range-check every block-table entry they read (libala_debug.so)
+#endif
+
+// Cache row of key position `pos` of a sequence whose block-table row is `bt`: bt[pos / bs] * bs + pos % bs,
+// or `oob_row` (one past the cache: the TMA load fills zeros there) for pages at or past `n_pages`.  In an
+// ALA_DEBUG_BOUNDS build an entry outside [0, oob_row / bs) records kDevBadBlockIndex in the second status
+// word (status[1], which the pipeline's waits do not watch, so the kernel still runs to its end) and reads
+// the zero-filled row instead; otherwise such an entry still only ever feeds a bounds-checked TMA load.
+__device__ __forceinline__ int paged_row(const int32_t* bt, int pos, int bs, int n_pages, int oob_row, int* status) {
+  const int pg = pos / bs;
+  if (pg >= n_pages) return oob_row;
+  const int32_t blk = bt[pg];
+#if ALA_DEBUG_BOUNDS
+  if (blk < 0 || (int64_t)blk * bs >= oob_row) {
+    atomicCAS(status + 1, 0, kDevBadBlockIndex);
+    return oob_row;
+  }
+#else
+  (void)status;
+#endif
+  return blk * bs + (pos - pg * bs);
+}
 
 // Per-sequence metadata, built on the host from seqLen / kvSeqLen.
 struct SeqInfo {

@@ -88,6 +88,7 @@ extern "C" ALA_API int varlen_attention_noalloc(const ala_tensor* query, const a
                                                 const ala_tensor* kvSeqLen, const ala_tensor* slopes, int maskType,
                                                 int32_t headNum, int32_t kvHeadNum, float qkScale,
                                                 ala_tensor* attnOut, ala_tensor* lse, ala_stream_t stream) {
+  NvtxRange nvtx_range("varlen_attention_noalloc");
   const char* fn = "varlen_attention_noalloc";
   // ---- the same argument rules as varlen_attention
   if (!query || !key || !value || !seqLen || !kvSeqLen || !attnOut || !query->data || !key->data || !value->data ||
@@ -235,15 +236,16 @@ extern "C" ALA_API int varlen_attention_noalloc(const ala_tensor* query, const a
 }
 
 extern "C" ALA_API int varlen_attention_noalloc_status(ala_stream_t stream, int32_t* code) {
+  NvtxRange nvtx_range("varlen_attention_noalloc_status");
   const char* fn = "varlen_attention_noalloc_status";
   if (!code) return nfail(ALA_NULL_REQUIRED, "%s: code is NULL", fn);
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return nfail(ALA_CUDA_ERROR, "%s: stream sync failed: %s", fn, cudaGetErrorString(cudaGetLastError()));
-  int32_t v = 0;
-  // a copy out of the library's array by symbol: no allocation
-  const cudaError_t e = cudaMemcpyFromSymbol(&v, g_noalloc_scratch, sizeof v, 0, cudaMemcpyDeviceToHost);
+  int32_t v[2] = {0, 0};
+  // a copy out of the library's array by symbol: no allocation (word 1: a range-checking build's report)
+  const cudaError_t e = cudaMemcpyFromSymbol(v, g_noalloc_scratch, sizeof v, 0, cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return nfail(ALA_CUDA_ERROR, "%s: status read failed: %s", fn, cudaGetErrorString(e));
-  *code = v;
+  *code = v[0] != 0 ? v[0] : v[1];
   set_last_error("");
   return ALA_OK;
 }
