@@ -60,23 +60,20 @@
 
 #include "internal.h"
 #include "mla.h"
+#include "mla_common.cuh"
 #include "ptx.cuh"
 
 namespace ala {
 
 namespace {
 
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleThreshold = 8.0f;
+using namespace mlak;
 
 #ifndef ALA_MLA_PREFETCH_TILES
 #define ALA_MLA_PREFETCH_TILES 2  // the producer asks L2 for the tiles this far ahead of its loads
 #endif
 
 constexpr int kRows = 64;                  // attention rows per CTA: the M of every MMA
-constexpr int kTileKeys = 64;
-constexpr int kDNope = 512;
 constexpr int kBlk = kRows * 128;          // one 64-column block of 64 rows (query rows or keys): 8 KB
 constexpr int kQrBytes = kBlk;             // the 64 x 64 qRope rows (qNope lives in tensor memory)
 constexpr int kKvBytes = 9 * kBlk;         // 64 keys x 576 x 2 B: ctKV blocks 0..7, kRope block 8
@@ -97,93 +94,7 @@ constexpr uint32_t kSRCol = 320;           // int8 cache: the qRope kRope part o
 constexpr int kConvWarp0 = 6;              // int8 cache: warps 6..9 convert ctKV tiles
 constexpr uint32_t kOLane = 16;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kPlannedSms = 148;           // SMs of the part the schedule is cut for
-constexpr int kMinLaneTiles = 4;           // shortest key range worth a lane of its own
-constexpr unsigned kFull = 0xffffffffu;
 
-struct MlaPiece {
-  int32_t b;         // batch
-  int32_t token0;    // first packed query token of the chunk
-  int32_t kv_begin;  // first key of the range (a multiple of 32)
-  int32_t n_tiles;   // 32-key tiles in the range
-  int32_t last;      // last allowed key of the chunk's first token; token t of the chunk allows last + row_step*t
-  int32_t part;      // partial slot (rows part*tpc .. +tpc-1 of the partials), or -1: final output
-  int32_t n_keys;    // keys of the batch the chunk may read (its pages): last + tpc, or contextLens with a mask
-  int32_t row_step;  // 1: the speculative rule; 0: every token reads keys 0..n_keys-1 (explicit mask tensor)
-};
-
-struct MlaCombine {
-  int32_t token;       // packed query token
-  int32_t part_begin;  // its chunk's first partial slot
-  int32_t n_parts;
-  int32_t t_local;     // token index within the chunk
-};
-
-struct MlaParams {
-  const MlaPiece* pieces;
-  const int32_t* lane_off;  // [n_lanes + 1]: lane l walks pieces [lane_off[l], lane_off[l+1])
-  const int32_t* block_tables;
-  const uint8_t* q_nope;    // [tokens, heads, 512] (rows go to tensor memory through registers)
-  const uint8_t* ct_kv;     // [numBlocks * blockSize, 512] (the L2 prefetch reads raw rows)
-  const uint8_t* k_rope;    // [numBlocks * blockSize, 64]
-  void* out;                // [tokens, heads, 512] (written by TMA stores and by the combine)
-  float* lse;               // [tokens, heads] or null
-  float* part_o;            // [parts * tpc, heads, 512]
-  float* part_lse;          // [parts * tpc, heads]
-  int* status;
-  int32_t heads;
-  int32_t groups;           // heads / hpc
-  int32_t tpc;              // query tokens per CTA row block
-  int32_t hpc;              // heads per CTA row block (64 / tpc)
-  int32_t max_blocks;
-  int32_t block_size;
-  int32_t oob_row;
-  float scale_log2;
-  const float* qk_descale;  // [heads], int8 cache only
-  const float* pv_descale;  // [heads], int8 cache only
-  int32_t qn_int8;          // qNope holds int8 codes (int8 cache only)
-  const uint16_t* mask;     // [tokens, mask_cols] additive mask (fp16 or bf16 bits), or null: the rule
-  int64_t mask_cols;
-  int32_t mask_f16;         // the mask holds fp16 (else bf16)
-  int32_t mask_vec;         // rows start 16-byte aligned: 16-byte loads
-};
-
-// One fp16 or bf16 mask element (its 16 bits) as a float.
-__device__ __forceinline__ float mask_value(uint32_t bits, bool f16) {
-  return f16 ? __half2float(__ushort_as_half(static_cast<unsigned short>(bits))) : __uint_as_float(bits << 16);
-}
-
-// The additive mask of packed token `token` for keys j0 .. j0+63, in log2 units (times log2 e); keys at or
-// past the mask's row length read 0 (they lie past contextLens and are masked by the key limit).
-__device__ __forceinline__ void load_mask_log2(const MlaParams& p, int token, int j0, float (&mk)[64]) {
-  const uint16_t* row = p.mask + (size_t)token * p.mask_cols;
-  const bool f16 = p.mask_f16 != 0;
-  if (p.mask_vec && j0 + 64 <= p.mask_cols) {
-    const uint4* src = reinterpret_cast<const uint4*>(row + j0);
-#pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      const uint4 w = __ldg(src + v);
-      const uint32_t q[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        mk[8 * v + 2 * i] = mask_value(q[i] & 0xffffu, f16) * kLog2e;
-        mk[8 * v + 2 * i + 1] = mask_value(q[i] >> 16, f16) * kLog2e;
-      }
-    }
-  } else {
-#pragma unroll
-    for (int c = 0; c < 64; ++c) mk[c] = (j0 + c < p.mask_cols) ? mask_value(__ldg(row + j0 + c), f16) * kLog2e : 0.f;
-  }
-}
-
-__device__ __forceinline__ uint32_t pack2(float a, float b, __nv_bfloat16*) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-__device__ __forceinline__ uint32_t pack2(float a, float b, __half*) {
-  __half2 v = __floats2half2_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
 
 // Four int8 codes (one 32-bit word, the first code in the low byte) to four T values, exactly,
 // as two words of packed pairs.  The code v is biased to v + 128 in [0, 255] and placed in the low
@@ -215,11 +126,6 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
   return v;
-}
-
-// Warp-uniform wait on all lanes (each lane observes the phase itself).
-__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, int* status, int code) {
-  return __all_sync(kFull, mbar_wait(bar, parity, status, code));
 }
 
 // Loads one chunk's query into place: qNope rows into tensor memory (lanes 0..15 of the warp's
@@ -365,12 +271,11 @@ __global__ void __launch_bounds__(KV8 ? 320 : 192, 1)
             const int npf = (pf.n_keys + bs - 1) / bs;
             for (int r0 = 0; r0 < kTileKeys; r0 += box_rows) {
               const int pos = pf.kv_begin + jf * kTileKeys + r0;
-              const int pg = pos / bs;
-              const size_t row = pg < npf ? (size_t)btf[pg] * bs + (pos - pg * bs) : (size_t)p.oob_row;
-              if (row < (size_t)p.oob_row) {  // a block index outside the cache is never touched
+              const int row = paged_row(btf, pos, bs, npf, p.oob_row, p.status);
+              if (row >= 0 && row < p.oob_row) {  // a block index outside the cache is never touched
                 constexpr int kRowBytes = KV8 ? kDNope : 2 * kDNope;
-                bulk_prefetch_l2(p.ct_kv + row * kRowBytes, box_rows * kRowBytes);
-                bulk_prefetch_l2(p.k_rope + row * 128, box_rows * 128);
+                bulk_prefetch_l2(p.ct_kv + (size_t)row * kRowBytes, box_rows * kRowBytes);
+                bulk_prefetch_l2(p.k_rope + (size_t)row * 128, box_rows * 128);
               }
             }
             if (++jf == pf.n_tiles) {
@@ -388,8 +293,7 @@ __global__ void __launch_bounds__(KV8 ? 320 : 192, 1)
           const int j0 = pc.kv_begin + j * kTileKeys;
           for (int r0 = 0; r0 < kTileKeys; r0 += box_rows) {
             const int pos = j0 + r0;
-            const int pg = pos / bs;
-            const int row = pg < n_pages ? bt[pg] * bs + (pos - pg * bs) : p.oob_row;  // past the last page: zeros
+            const int row = paged_row(bt, pos, bs, n_pages, p.oob_row, p.status);  // past the last page: zeros
             if (KV8) {  // the codes, [4 blocks of 128 columns][key][128 B], into the upper half of the ctKV area
               if (whole) {
                 tma_load_3d(dst + kI8Off, &tmKV3, kv_full + s, 0, row, 0);
@@ -1025,8 +929,13 @@ int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, co
     for (int32_t b = 0; b < batch; ++b) divides = divides && plan->qs[b] % tpc == 0;
     if (divides) break;
   }
-  const int32_t hpc = kRows / tpc;
+  // one token per row block, 128-head groups and a 16-bit cache: the 128-row kernel, whose CTA pairs
+  // split the output columns (two CTAs per group); otherwise 64-row blocks
+  const bool wide = tpc == 1 && !kv8 && headNum % 128 == 0;
+  const int32_t hpc = wide ? 128 : kRows / tpc;
   const int32_t groups = headNum / hpc;
+  const int32_t ctas_per_lane = wide ? 2 * groups : groups;
+  plan->wide = wide;
   plan->tpc = tpc;
   plan->hpc = hpc;
   plan->groups = groups;
@@ -1049,7 +958,7 @@ int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, co
     }
   }
   // ---- lanes: equal contiguous ranges of that sequence, one CTA per lane and group
-  const int64_t lanes_max = std::max<int64_t>(1, kPlannedSms / groups);
+  const int64_t lanes_max = std::max<int64_t>(1, kPlannedSms / ctas_per_lane);
   const int64_t per_lane = std::max<int64_t>(kMinLaneTiles, (total_tiles + lanes_max - 1) / lanes_max);
   std::vector<MlaPiece> pieces;
   std::vector<int32_t> piece_lane;
@@ -1083,7 +992,7 @@ int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, co
     lane_off[l] = i;
   }
   plan->n_lanes = n_lanes;
-  plan->n_work = n_lanes * groups;
+  plan->n_work = n_lanes * ctas_per_lane;
   plan->n_splits_total = parts;
   plan->n_combine = (int32_t)comb.size();
   auto align = [](uint64_t x) { return (x + 255) / 256 * 256; };
@@ -1133,6 +1042,15 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
     cuuint64_t k83_dims[3] = {128, rows, 4};
     cuuint64_t k83_str[2] = {512, 128};
     cuuint32_t k83_box[3] = {128, (cuuint32_t)kTileKeys, 4};
+    if (plan->wide) {
+      // the 128-row kernel: query / output boxes of 64 columns x 128 heads of one token
+      cuuint32_t w_box[3] = {64, 128, 1};
+      if (!encode(&plan->tmQn, plan->q_nope, plan->dtype, 3, qn_dims, qn_str, w_box))
+        return mfail(err, n, ALA_CUDA_ERROR, "cuTensorMapEncodeTiled failed for qNope");
+      q_box[0] = 64;
+      q_box[1] = 128;
+      q_box[2] = 1;
+    }
     const bool kv_ok = plan->kv8 ? (encode(&plan->tmKV3, plan->ct_kv, ALA_I8, 3, k83_dims, k83_str, k83_box) &&
                                     encode(&plan->tmKV, plan->ct_kv, ALA_I8, 2, k8_dims, k8_str, k8_box))
                                  : (encode(&plan->tmKV3, plan->ct_kv, plan->dtype, 3, kv3_dims, kv3_str, kv3_box) &&
@@ -1148,7 +1066,7 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
   } else if (plan->tmPO_base != ws + plan->off_part_o) {
     cuuint64_t po_dims[3] = {512, (cuuint64_t)plan->heads, (cuuint64_t)plan->n_splits_total * tpc};
     cuuint64_t po_str[2] = {512 * 4, (cuuint64_t)plan->heads * 512 * 4};
-    cuuint32_t po_box[3] = {32, hpc, tpc};
+    cuuint32_t po_box[3] = {32, plan->wide ? 128u : hpc, tpc};
     if (!encode(&plan->tmPO, ws + plan->off_part_o, ALA_F32, 3, po_dims, po_str, po_box))
       return mfail(err, n, ALA_CUDA_ERROR, "cuTensorMapEncodeTiled failed for the partial-output map");
     plan->tmPO_base = ws + plan->off_part_o;
@@ -1192,6 +1110,18 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
   p.mask_f16 = plan->mask_f16 ? 1 : 0;
   p.mask_vec = (reinterpret_cast<uintptr_t>(plan->mask) % 16 == 0 && plan->mask_cols % 8 == 0) ? 1 : 0;
   const bool f16 = plan->dtype == ALA_F16;
+  if (plan->wide) {
+    cudaError_t e = launch_mla_wide(plan->dtype, (int)plan->n_work, plan->tmQn, plan->tmQr, plan->tmKV, plan->tmKV3,
+                                    plan->tmKR, plan->tmO, plan->tmPO, p, stream);
+    if (e == cudaSuccess && plan->n_combine > 0) {
+      auto ck = f16 ? mla_combine_kernel<__half> : mla_combine_kernel<__nv_bfloat16>;
+      dim3 grid(plan->n_combine, (plan->heads + 7) / 8);
+      ck<<<grid, 256, 0, stream>>>(reinterpret_cast<const MlaCombine*>(ws + plan->off_rows), p);
+      e = cudaGetLastError();
+    }
+    if (e != cudaSuccess) return mfail(err, n, ALA_CUDA_ERROR, cudaGetErrorString(e));
+    return ALA_OK;
+  }
   auto kern = plan->kv8 ? (f16 ? mla_kernel<__half, true> : mla_kernel<__nv_bfloat16, true>)
                         : (f16 ? mla_kernel<__half, false> : mla_kernel<__nv_bfloat16, false>);
   const int threads = plan->kv8 ? 320 : 192;

@@ -24,8 +24,13 @@
 //                the causal / prefix-offset rule in registers (the mask is
 //                never materialised), updates the running max and sum, rescales
 //                O_b in TMEM only when the max grew by more than 2^8, and writes
-//                P_b (16-bit, or fp32 for tf32) over S_b in TMEM.  At the end it
-//                normalises O_b and stores it.
+//                P_b (16-bit, or fp32 for tf32) over S_b in TMEM.  At the end of
+//                a unit it hands its row's max and sum to the epilogue warps and
+//                goes straight on to the next unit.
+//   warps 12..15 epilogue of both blocks: thread r reads row r of O_b from TMEM
+//                once the unit's last P_b V has completed, normalises it, stores
+//                it and the row's lse, and releases O_b for the next unit's
+//                first P_b V.
 //
 // Key tiles wholly above the prefix-shifted causal diagonal, or past the
 // sequence's kvSeqLen, are never visited: the host gives each block the number
@@ -76,8 +81,9 @@ struct Cfg {
   static constexpr int KV_BYTES = 128 * D * ES;
   static constexpr int TBL_FLOATS = 160;  // per-warp sqrt-bias table: lane - column + 127 in [0, 159)
   static constexpr int TBL_BYTES = 8 * 2 * TBL_FLOATS * 4;
-  static constexpr int N_BARS = 21;
-  static constexpr int SMEM = 1024 + 2 * Q_BYTES + 2 * STAGES * KV_BYTES + TBL_BYTES + N_BARS * 8 + 16;
+  static constexpr int ML_BYTES = 2 * 128 * 2 * 4;  // per block and row: the running max and sum at a unit's end
+  static constexpr int N_BARS = 27;
+  static constexpr int SMEM = 1024 + 2 * Q_BYTES + 2 * STAGES * KV_BYTES + TBL_BYTES + ML_BYTES + N_BARS * 8 + 16;
   static constexpr uint32_t IDESC_QK = instr_desc(ElemFmt<T>::fmt, false, false, 128, 128);
   static constexpr uint32_t IDESC_PV = instr_desc(ElemFmt<T>::fmt, false, true, 128, D);
   static constexpr uint32_t TMEM_COLS = 512;  // S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D, 256+2D)
@@ -170,14 +176,8 @@ __device__ __forceinline__ void load_kv_tile(const CUtensorMap* map, uint8_t* ds
   const int box_rows = paged ? (bs < 128 ? bs : 128) : 128;
   const int j0 = j * 128;
   for (int r0 = 0; r0 < 128; r0 += box_rows) {
-    int row;
-    if (!paged) {
-      row = si.cu_kv + j0 + r0;
-    } else {
-      const int pos = j0 + r0;
-      const int pg = pos / bs;
-      row = pg < n_pages ? bt[pg] * bs + (pos % bs) : p.oob_row;  // past the last page: zero fill
-    }
+    // contiguous rows, or the page's row through the block table (past the last page: zero fill)
+    const int row = paged ? paged_row(bt, j0 + r0, bs, n_pages, p.oob_row, p.status) : si.cu_kv + j0 + r0;
     if (leader) {
 #pragma unroll
       for (int cb = 0; cb < D / C::AW; ++cb) tma_load_3d(dst + cb * C::BLK + r0 * 128, map, full, cb * C::AW, kvh, row);
@@ -185,8 +185,83 @@ __device__ __forceinline__ void load_kv_tile(const CUtensorMap* map, uint8_t* ds
   }
 }
 
+// Epilogue warps (warps 12..15; warp 12 + w reads TMEM lanes 32w .. 32w+31, thread r row r of a block):
+// for every unit and block of the CTA, wait for the softmax warps' row max and sum and for the block's
+// last P V, read O_b in 32-column pieces, release O_b to the next unit's first P V, and store the
+// normalised row (32-byte pieces) and its lse.
 template <typename T, int D>
-__global__ void __launch_bounds__(384, 1)
+__device__ __forceinline__ void epilogue_warps(const PrefillParams& p, uint32_t tmem, int u_begin, int u_end,
+                                               const float2* sML, uint64_t* o_done, uint64_t* ml_full,
+                                               uint64_t* ml_empty, uint64_t* o_free) {
+  using C = Cfg<T, D>;
+  const int r = threadIdx.x & 127;
+  const uint32_t lane_base = static_cast<uint32_t>(((threadIdx.x >> 5) & 3) * 32) << 16;
+  const int mt = p.mask_type;
+  uint32_t up[2] = {0, 0};  // units each block took part in
+  bool ok = true;
+  for (int ui = u_begin; ui < u_end && ok; ++ui) {
+    const PrefillUnit u = p.units[ui];
+    const SeqInfo si = p.seqs[u.b];
+    for (int b = 0; b < u.n_blocks && ok; ++b) {
+      const uint32_t ph = up[b]++;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(ml_full + b, ph & 1, p.status, kDevTimeoutODone)))) break;
+      const float2 ml = sML[b * 128 + r];
+      mbar_arrive(ml_empty + b);
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(o_done + b, ph & 1, p.status, kDevTimeoutODone)))) break;
+      tc_fence_after();
+      const int head = b ? u.head[1] : u.head[0];
+      const int qi = (b ? u.q0[1] : u.q0[0]) + r;
+      const bool row_valid = qi < si.seq_len;
+      const float inv_l = 1.f / ml.y;
+      const uint32_t o_col = tmem + lane_base + 256 + b * D;
+      T* orow = reinterpret_cast<T*>(p.out) + ((size_t)(si.cu_q + qi) * p.heads + head) * D;
+#pragma unroll
+      for (int c32 = 0; c32 < D / 32; ++c32) {
+        uint32_t regs[32];
+        tmem_ld32(o_col + c32 * 32, regs);
+        tmem_ld_wait();
+        if (c32 == D / 32 - 1) {  // every read of O_b is done: the next unit's P_b V may overwrite it
+          tc_fence_before();
+          mbar_arrive(o_free + b);
+        }
+        if (row_valid) {
+          // rows start on 128-byte boundaries (D * element size), so every 32-byte store is aligned
+          if constexpr (C::ES == 2) {
+#pragma unroll
+            for (int v8 = 0; v8 < 2; ++v8) {
+              uint32_t w[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                w[i] = pack2(__uint_as_float(regs[v8 * 16 + 2 * i]) * inv_l,
+                             __uint_as_float(regs[v8 * 16 + 2 * i + 1]) * inv_l, (T*)nullptr);
+              st_global_v8(orow + c32 * 32 + v8 * 16, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+            }
+          } else {
+#pragma unroll
+            for (int v8 = 0; v8 < 4; ++v8) {
+              uint32_t w[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) w[i] = __float_as_uint(__uint_as_float(regs[v8 * 8 + i]) * inv_l);
+              st_global_v8(reinterpret_cast<float*>(orow) + c32 * 32 + v8 * 8, w[0], w[1], w[2], w[3], w[4], w[5],
+                           w[6], w[7]);
+            }
+          }
+        }
+      }
+      if (row_valid && p.lse) {
+        float lse = (ml.x == -INFINITY ? 0.f : ml.x) * kLn2 + logf(ml.y);
+        if (mt == 5) {  // left-aligned bias = right-aligned + slope * iabs
+          const int iabs = qi + si.kv_len - si.seq_len;
+          lse += p.slopes[head] * static_cast<float>(iabs);
+        }
+        p.lse[(size_t)(si.cu_q + qi) * p.heads + head] = lse;
+      }
+    }
+  }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(512, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
   using C = Cfg<T, D>;
@@ -196,7 +271,8 @@ __global__ void __launch_bounds__(384, 1)
   uint8_t* sK = sQ + 2 * C::Q_BYTES;         // [STAGES][KV_BYTES]
   uint8_t* sV = sK + C::STAGES * C::KV_BYTES;
   float* sTbl = reinterpret_cast<float*>(sV + C::STAGES * C::KV_BYTES);  // [8 warps][2][TBL_FLOATS]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sTbl) + C::TBL_BYTES);
+  float2* sML = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(sTbl) + C::TBL_BYTES);  // [2 blocks][128 rows]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sML) + C::ML_BYTES);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;    // [2]
   uint64_t* v_full = bars + 3;    // [2]
@@ -209,6 +285,9 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* fin = bars + 17;
   uint64_t* q_empty = bars + 18;
   uint64_t* p_lo = bars + 19;     // [2] per block: P of keys 0..63 written
+  uint64_t* ml_full = bars + 21;  // [2] per block: the rows' max and sum of a unit are in sML
+  uint64_t* ml_empty = bars + 23; // [2] per block: the epilogue has read them
+  uint64_t* o_free = bars + 25;   // [2] per block: the epilogue has read O_b
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::N_BARS);
 
   const int warp = threadIdx.x >> 5;
@@ -231,6 +310,9 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(p_lo + s, 128);
       mbar_init(pv_done + s, 1);
       mbar_init(o_done + s, 1);
+      mbar_init(ml_full + s, 128);
+      mbar_init(ml_empty + s, 128);
+      mbar_init(o_free + s, 128);
     }
     mbar_init(fin, 1);
     fence_mbar_init();
@@ -248,10 +330,13 @@ __global__ void __launch_bounds__(384, 1)
   // per-block S/P/PV barriers by each block's tile counter, q_full / q_empty and
   // o_done by unit counters.
   //
-  // register split: the softmax warpgroups take 216 per thread, warps 8..11 keep 72
-  // (256*216 + 128*72 = 64512 = 384*168, all the registers the block is launched with)
-  if (warp >= 8) {
-    regs_decrease<72>();
+  // register split: the softmax warpgroups take 200 per thread, warps 8..11 and the epilogue
+  // warpgroup 56 (256*200 + 256*56 = 65536 = 512*128, all the registers the block is launched with)
+  if (warp >= 12) {
+    regs_decrease<56>();
+    epilogue_warps<T, D>(p, tmem, u_begin, u_end, sML, o_done, ml_full, ml_empty, o_free);
+  } else if (warp >= 8) {
+    regs_decrease<56>();
     if (warp == 8) {
       // ------------------------------------------------------------ producer
       // the whole warp walks the schedule (warp-uniform values); one elected lane issues the copies
@@ -360,6 +445,7 @@ __global__ void __launch_bounds__(384, 1)
       bool ok = true;
       uint32_t kv_iter = 0;
       uint32_t sp0 = 0, sp1 = 0;  // tiles block 0 / 1 processed in earlier units
+      uint32_t ub0 = 0, ub1 = 0;  // earlier units block 0 / 1 took part in (o_free phases)
       for (int ui = u_begin; ui < u_end && ok; ++ui) {
         const int it = ui - u_begin;
         const PrefillUnit u = p.units[ui];
@@ -403,6 +489,12 @@ __global__ void __launch_bounds__(384, 1)
               break;
             }
             v_ready = true;
+            // the unit's first P_b V overwrites O_b: the epilogue warps must have read the previous unit's
+            const uint32_t ubb = b ? ub1 : ub0;
+            if (j == 0 && ubb > 0 && !wait_all(o_free + b, (ubb - 1) & 1, kDevTimeoutODone)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
             issue_pv(b, s, j > 0, 0);  // keys 0..63
             if (!wait_all(p_full + b, ph & 1, kDevTimeoutPFull)) {
@@ -442,6 +534,8 @@ __global__ void __launch_bounds__(384, 1)
         }
         sp0 += n0;
         sp1 += n1;
+        ub0 += 1;
+        ub1 += nb > 1 ? 1 : 0;
         kv_iter += nmax;
       }
       // all tensor-core work this thread issued has finished before TMEM is released
@@ -450,8 +544,8 @@ __global__ void __launch_bounds__(384, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax / epilogue of block b
-    regs_increase<216>();
+    // ------------------------------------------------------------ softmax of block b
+    regs_increase<200>();
     const int b = warp >> 2;
     const int r = threadIdx.x & 127;  // query row in the block == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -463,7 +557,7 @@ __global__ void __launch_bounds__(384, 1)
     const bool raw_max = !alibi && scale > 0.f;  // max of the raw scores, scale folded into the exponent
     float* tbl = sTbl + warp * 2 * C::TBL_FLOATS;
     uint32_t sp = 0;  // tiles this block processed in earlier units (barrier phases)
-    uint32_t up = 0;  // units this block took part in (o_done phases)
+    uint32_t up = 0;  // units this block took part in (ml_full / ml_empty phases)
     bool ok = true;
     for (int ui = u_begin; ui < u_end && ok; ++ui) {
       const PrefillUnit u = p.units[ui];
@@ -566,48 +660,13 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive(p_full + b);
       }
       sp += n;
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done + b, up & 1, status, kDevTimeoutODone));
-      ++up;
       if (!ok) break;
-      tc_fence_after();
-      const float inv_l = 1.f / l_run;
-      T* orow = reinterpret_cast<T*>(p.out) + ((size_t)(si.cu_q + qi) * p.heads + head) * D;
-      uint32_t orr[D / 32][32];
-#pragma unroll
-      for (int c32 = 0; c32 < D / 32; ++c32) tmem_ld32(o_col + c32 * 32, orr[c32]);
-      tmem_ld_wait();  // one wait for all loads of the row; the next unit's P_b * V may then overwrite O_b
-#pragma unroll
-      for (int c32 = 0; c32 < D / 32; ++c32) {
-        const uint32_t(&regs)[32] = orr[c32];
-        if (row_valid) {
-          // rows start on 128-byte boundaries (D * element size), so every 32-byte store is aligned
-          if constexpr (C::ES == 2) {
-#pragma unroll
-            for (int v8 = 0; v8 < 2; ++v8) {
-              uint32_t w[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                w[i] = pack2(__uint_as_float(regs[v8 * 16 + 2 * i]) * inv_l,
-                             __uint_as_float(regs[v8 * 16 + 2 * i + 1]) * inv_l, (T*)nullptr);
-              st_global_v8(orow + c32 * 32 + v8 * 16, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
-            }
-          } else {
-#pragma unroll
-            for (int v8 = 0; v8 < 4; ++v8) {
-              uint32_t w[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) w[i] = __float_as_uint(__uint_as_float(regs[v8 * 8 + i]) * inv_l);
-              st_global_v8(reinterpret_cast<float*>(orow) + c32 * 32 + v8 * 8, w[0], w[1], w[2], w[3], w[4], w[5],
-                           w[6], w[7]);
-            }
-          }
-        }
-      }
-      if (row_valid && p.lse) {
-        float lse = (m_run == -INFINITY ? 0.f : m_run) * kLn2 + logf(l_run);
-        if (mt == 5) lse += slope * static_cast<float>(iabs);  // left-aligned bias = right-aligned + slope*iabs
-        p.lse[(size_t)(si.cu_q + qi) * p.heads + head] = lse;
-      }
+      // hand the row's max and sum to the epilogue warps (once they have read the previous unit's)
+      if (up > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(ml_empty + b, (up - 1) & 1, status, kDevTimeoutODone))))
+        break;
+      sML[b * 128 + r] = make_float2(m_run, l_run);
+      mbar_arrive(ml_full + b);
+      ++up;
     }
   }
 
@@ -629,7 +688,7 @@ cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtenso
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   if (p.n_ctas == 0) return cudaSuccess;
-  kern<<<p.n_ctas, 384, kSmem, stream>>>(tmQ, tmK, tmV, p);
+  kern<<<p.n_ctas, 512, kSmem, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }
 

@@ -55,6 +55,18 @@ def test_mla_small_ragged(qs, block_size):
     check_lse(lse.reshape(-1), lref)
 
 
+@pytest.mark.parametrize("heads,dtype", [(64, torch.bfloat16), (128, torch.float16), (384, torch.bfloat16)])
+def test_mla_decode_row_kernels(heads, dtype):
+    # one token per batch: 64 heads run on the 64-row kernel, multiples of 128 on the 128-row kernel whose
+    # CTA pairs split the output columns (384 heads: three head groups, six CTAs per key range)
+    ctx = np.array([1, 64, 65, 700, 2500, 129], dtype=np.int32)
+    case = synth.make_mla(f"rows_{heads}", ctx, 1, heads, 89, block_size=64, dtype=dtype)
+    out, lse, _ = _run(case)
+    ref, lref = _oracle(case)
+    check_out(out.reshape(-1, 512), ref)
+    check_lse(lse.reshape(-1), lref)
+
+
 def test_mla_fp16_and_64_heads():
     ctx = np.array([300, 5, 900], dtype=np.int32)
     case = synth.make_mla("f16", ctx, 2, 64, 31, block_size=64, dtype=torch.float16)
