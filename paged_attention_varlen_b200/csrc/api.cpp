@@ -268,9 +268,10 @@ int build_prefill(ala_op* op, const ala_tensor* query, const ala_tensor* key, co
     if (!blockTables->data) return fail(ALA_NULL_REQUIRED, "%s: blockTables data is NULL", fn);
     if (blockTables->dtype != ALA_I32) return fail(ALA_INVALID_DTYPE, "%s: blockTables must be int32", fn);
     if (blockTables->ndim != 2) return fail(ALA_INVALID_SHAPE, "%s: blockTables must be [batch, maxBlockNum]", fn);
-    if (!(block_size > 0 && block_size % 16 == 0 && (128 % block_size == 0 || block_size % 128 == 0)))
-      return fail(ALA_UNSUPPORTED, "%s: blockSize %d must be a multiple of 16 dividing 128, or a multiple of 128", fn,
-                  block_size);
+    if (!(block_size > 0 && block_size % 16 == 0 &&
+          (kPrefillTileKeys % block_size == 0 || block_size % kPrefillTileKeys == 0)))
+      return fail(ALA_UNSUPPORTED, "%s: blockSize %d must be a multiple of 16 dividing %d, or a multiple of %d", fn,
+                  block_size, kPrefillTileKeys, kPrefillTileKeys);
     max_blocks = (int32_t)blockTables->dims[1];
   }
   if (kv_rows >= (int64_t)1 << 31 || n_tokens >= (int64_t)1 << 31)
@@ -302,9 +303,11 @@ int build_prefill(ala_op* op, const ala_tensor* query, const ala_tensor* key, co
     if (numel(lse) != n_tokens * headNum || lse->dims[0] != n_tokens)
       return fail(ALA_INVALID_SHAPE, "%s: lse must be [nTokens, headNum]", fn);
   }
-  if (prefill_smem_bytes(dt, (int32_t)head_size) == 0)
-    return fail(ALA_UNSUPPORTED, "%s: headSize %lld with this dtype is not built (bf16/f16: 64, 128; f32: 64)", fn,
-                (long long)head_size);
+  if (prefill_kernel_d(dt, head_size) == 0)
+    return fail(ALA_UNSUPPORTED,
+                "%s: headSize %lld with this dtype is not built (bf16/f16: a multiple of 16 up to 128; f32: a "
+                "multiple of 8 up to 64)",
+                fn, (long long)head_size);
 
   op->kind = ala_op::kPrefill;
   op->dtype = dt;
@@ -382,7 +385,7 @@ int run_prefill(void* workspace, uint64_t workspaceSize, ala_op* op, ala_stream_
   if (reinterpret_cast<uintptr_t>(workspace) % 16) return fail(ALA_INVALID_PARAM, "%s: workspace must be 16-byte aligned", fn);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (!op->maps_ready) {
-    const int kv_box = op->paged ? std::min(op->block_size, 128) : 128;
+    const int kv_box = op->paged ? std::min(op->block_size, kPrefillTileKeys) : kPrefillTileKeys;
     const int64_t q_rows = op->n_tokens;
     if (!encode_rows_heads_d(&op->tmQ, op->q, op->dtype, q_rows, op->heads, op->head_size, 128, false) ||
         !encode_rows_heads_d(&op->tmK, op->k, op->dtype, op->kv_rows, op->kv_heads, op->head_size, kv_box, false) ||
@@ -411,7 +414,8 @@ int run_prefill(void* workspace, uint64_t workspaceSize, ala_op* op, ala_stream_
   p.heads = op->heads;
   p.group = op->heads / op->kv_heads;
   p.scale_log2 = op->qk_scale * 1.4426950408889634f;
-  cudaError_t e = launch_prefill(op->dtype, op->head_size, op->tmQ, op->tmK, op->tmV, p, st);
+  p.d_out = op->head_size;
+  cudaError_t e = launch_prefill(op->dtype, prefill_kernel_d(op->dtype, op->head_size), op->tmQ, op->tmK, op->tmV, p, st);
   if (e != cudaSuccess) return fail(ALA_CUDA_ERROR, "%s: kernel launch failed: %s", fn, cudaGetErrorString(e));
   return ok();
 }

@@ -65,6 +65,9 @@ struct SeqInfo {
   int32_t cu_kv;    // first packed key row (contiguous layout only)
 };
 
+// Keys per K/V tile of the prefill kernel.
+constexpr int kPrefillTileKeys = 64;
+
 // One CTA's work: up to two blocks of 128 query rows of one sequence that read
 // the same kv head (two query heads of a group, or two consecutive row tiles of
 // one head), so every K/V tile the CTA loads serves both.
@@ -73,7 +76,7 @@ struct PrefillUnit {
   int32_t n_blocks;    // 1 or 2
   int32_t q0[2];       // first query row of each block (within the sequence)
   int32_t head[2];     // query head of each block
-  int32_t n_tiles[2];  // 128-key tiles each block visits: ceil(min(kv_len, last allowed key + 1) / 128);
+  int32_t n_tiles[2];  // key tiles each block visits: ceil(min(kv_len, last allowed key + 1) / kPrefillTileKeys);
                        // n_tiles[1] >= n_tiles[0] when n_blocks == 2
 };
 
@@ -95,6 +98,7 @@ struct PrefillParams {
   int32_t heads;
   int32_t group;                // heads / kvHeads
   float scale_log2;             // qkScale * log2(e)
+  int32_t d_out;                // head size of the tensors (<= the kernel's D; dims past it are zero-filled)
 };
 
 // Work units of one prefill request, in sequence order (every prefill entry point uses this list).
@@ -112,7 +116,7 @@ inline void prefill_units(int32_t batch, const int32_t* seq_len, const int32_t* 
       const int32_t last_row = (q0 + 127 < sl - 1) ? q0 + 127 : sl - 1;
       const int32_t causal_end = last_row + off + 1;
       const int32_t kv_end = (mask_type == 0 || kl < causal_end) ? kl : causal_end;
-      return (kv_end + 127) / 128;
+      return (kv_end + kPrefillTileKeys - 1) / kPrefillTileKeys;
     };
     if (group >= 2) {
       for (int32_t q0 = 0; q0 < sl; q0 += 128) {
@@ -155,11 +159,14 @@ bool encode_rows_heads_d(CUtensorMap* map, void* base, int32_t dtype, int64_t ro
 // dtype codes as in include/ala.h
 enum : int32_t { kF16 = 0, kBF16 = 1, kF32 = 2, kI32 = 3 };
 
-// Launches the prefill kernel for element type `dtype` and head size `d`.
-cudaError_t launch_prefill(int32_t dtype, int32_t d, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+// Head size D of the prefill kernel instance that serves head size `d` of element type `dtype` (0 if none
+// does): 16-bit types take d a multiple of 16 up to 128 (D = 64 or 128), fp32 a multiple of 8 up to 64
+// (D = 64).  The tensor maps are encoded over the real d, so the dimensions d..D-1 of every Q, K and V
+// tile are zero-filled by the TMA loads and contribute nothing; the epilogue stores the first d columns.
+int prefill_kernel_d(int32_t dtype, int64_t d);
+// Launches the prefill kernel for element type `dtype` and kernel head size `D` (prefill_kernel_d).
+cudaError_t launch_prefill(int32_t dtype, int32_t D, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                            const CUtensorMap& tmV, const PrefillParams& p, cudaStream_t stream);
-// Dynamic shared memory the prefill kernel needs (0 if the combination is unsupported).
-int prefill_smem_bytes(int32_t dtype, int32_t d);
 
 // Merges two partial results (rows x d, each normalised over its own keys) by their lse; out / lse may
 // alias the inputs.  d <= 1024.

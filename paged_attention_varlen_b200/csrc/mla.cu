@@ -1034,7 +1034,8 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
     // [column block][key][64 elements] as the 128B-swizzled K-major operand wants it
     cuuint64_t kv3_dims[3] = {64, rows, 8};
     cuuint64_t kv3_str[2] = {512 * es, 64 * es};
-    cuuint32_t kv3_box[3] = {64, (cuuint32_t)kTileKeys, 8};
+    // the 128-row kernel loads a tile in two parts of four column blocks each
+    cuuint32_t kv3_box[3] = {64, (cuuint32_t)kTileKeys, plan->wide ? 4u : 8u};
     // int8 codes: 512 bytes a row, seen as 128-byte column blocks (4 per row), same boxes of keys
     cuuint64_t k8_dims[2] = {512, rows};
     cuuint64_t k8_str[1] = {512};

@@ -20,7 +20,13 @@
 //                     P V MMAs (TS form);
 //   columns 256..511  this CTA's half of O.
 // Shared memory: qNope dims 256..511 and qRope (SS A operands, 80 KB) and a
-// two-deep ring of 64-key tiles (ctKV 64 KB + kRope 8 KB each).
+// two-deep ring of 64-key tiles (ctKV 64 KB + kRope 8 KB each).  A slot is
+// loaded and released in two parts: part A (the other half's ctKV columns and
+// kRope, 40 KB) is dead once the tile's QK has completed, part B (this CTA's
+// ctKV columns, the V of its P V, 32 KB) once the P V has.  The QK of tile
+// j+2 reuses the S buffer of tile j only after P(j) V has completed, so it
+// starts with the MMAs over part A, loaded long before, while part B is still
+// on its way.
 //
 //   warp 4      TMA producer (one thread): per piece the query's shared-memory
 //               part, then the tiles gathered through the block table, and
@@ -55,8 +61,11 @@ constexpr int kWQnBytes = 4 * kWBlkQ;    // qNope dims 256..511 of the 128 rows
 constexpr int kWQrBytes = kWBlkQ;        // qRope
 constexpr int kWKvBytes = 9 * kWBlkK;    // ctKV blocks 0..7 + kRope
 constexpr int kWStages = 2;
-// q_full, q_free, kv_full[2], kv_empty[2], s_full[2], p_full[2], pv_done[2], o_free, st_full, st_free, fin
-constexpr int kWNBars = 2 + 5 * kWStages + 4;
+// q_full, q_free, full_a[2], full_b[2], empty_a[2], empty_b[2], s_full[2], p_full[2], pv_done[2], o_free,
+// st_full, st_free, fin
+constexpr int kWNBars = 2 + 7 * kWStages + 4;
+constexpr int kWPartA = 5 * kWBlkK;  // part A bytes: four ctKV column blocks + kRope
+constexpr int kWPartB = 4 * kWBlkK;  // part B bytes: four ctKV column blocks
 constexpr int kWSmem = 1024 + kWQnBytes + kWQrBytes + kWStages * kWKvBytes + kWNBars * 8 + 16;
 static_assert(kWSmem <= 232448, "shared memory budget");
 static_assert(4 * kWBlkQ <= kWKvBytes, "the output staging (four 16 KB boxes) must fit in a ring slot");
@@ -83,19 +92,23 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + kWStages * kWKvBytes);
   uint64_t* q_full = bars;             // the piece's query is in place (128 TMEM stores + the TMA bytes)
   uint64_t* q_free = bars + 1;         // every QK of the piece has completed
-  uint64_t* kv_full = bars + 2;        // [2]
-  uint64_t* kv_empty = bars + 4;       // [2]
-  uint64_t* s_full = bars + 6;         // [2] per S buffer
-  uint64_t* p_full = bars + 8;         // [2] per S buffer: P written over S
-  uint64_t* pv_done = bars + 10;       // [2] per S buffer: the P V of that buffer's tile has completed
-  uint64_t* o_free = bars + 12;        // the epilogue has read O
-  uint64_t* st_full = bars + 13;
-  uint64_t* st_free = bars + 14;
-  uint64_t* fin = bars + 15;
+  uint64_t* full_a = bars + 2;         // [2] part A of the slot's tile has landed
+  uint64_t* full_b = bars + 4;         // [2] part B has landed
+  uint64_t* empty_a = bars + 6;        // [2] part A is free (the tile's QK has completed)
+  uint64_t* empty_b = bars + 8;        // [2] part B is free (the tile's P V has completed)
+  uint64_t* s_full = bars + 10;        // [2] per S buffer
+  uint64_t* p_full = bars + 12;        // [2] per S buffer: P written over S
+  uint64_t* pv_done = bars + 14;       // [2] per S buffer: the P V of that buffer's tile has completed
+  uint64_t* o_free = bars + 16;        // the epilogue has read O
+  uint64_t* st_full = bars + 17;
+  uint64_t* st_free = bars + 18;
+  uint64_t* fin = bars + 19;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kWNBars);
 
   const int warp = threadIdx.x >> 5;
   const int half = blockIdx.x & 1;                 // output columns [256 half, 256 half + 256)
+  const int cb_own = 4 * half;                     // the ctKV column blocks of this CTA's V (part B)
+  const int cb_other = 4 - cb_own;                 // the other half's column blocks (part A, with kRope)
   const int pair = blockIdx.x >> 1;
   const int ln = pair / p.groups;
   const int h0 = (pair - ln * p.groups) * kWRows;  // first head of this CTA's rows
@@ -107,8 +120,10 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(q_full, 129);
     mbar_init(q_free, 1);
     for (int s = 0; s < kWStages; ++s) {
-      mbar_init(kv_full + s, 1);
-      mbar_init(kv_empty + s, 1);
+      mbar_init(full_a + s, 1);
+      mbar_init(full_b + s, 1);
+      mbar_init(empty_a + s, 1);
+      mbar_init(empty_b + s, 1);
       mbar_init(s_full + s, 1);
       mbar_init(p_full + s, 128);
       mbar_init(pv_done + s, 1);
@@ -177,29 +192,39 @@ __global__ void __launch_bounds__(192, 1)
             }
           }
           const int s = G % kWStages;
-          if (G >= kWStages && !mbar_wait(kv_empty + s, ((G / kWStages) - 1) & 1, status, kDevTimeoutKEmpty)) {
-            ok = false;
-            break;
-          }
           uint8_t* dst = sKV + s * kWKvBytes;
-          mbar_expect_tx(kv_full + s, kWKvBytes);
           const int j0 = pc.kv_begin + j * kTileKeys;
-          for (int r0 = 0; r0 < kTileKeys; r0 += box_rows) {
-            const int pos = j0 + r0;
-            const int row = paged_row(bt, pos, bs, n_pages, p.oob_row, p.status);  // past the last page: zeros
-            if (whole) {
-              tma_load_3d(dst, &tmKV3, kv_full + s, 0, row, 0);  // [column block][key][64 elements]
-            } else {
-              for (int cb = 0; cb < 8; ++cb) tma_load_2d(dst + cb * kWBlkK + r0 * 128, &tmKV, kv_full + s, cb * 64, row);
+          // part A (other half's columns, kRope) once the previous tile in the slot has finished its QK; part B
+          // (this CTA's columns) once it has finished its P V
+          for (int part = 0; part < 2 && ok; ++part) {
+            uint64_t* empty = part == 0 ? empty_a : empty_b;
+            uint64_t* full = (part == 0 ? full_a : full_b) + s;
+            if (G >= kWStages && !mbar_wait(empty + s, ((G / kWStages) - 1) & 1, status, kDevTimeoutKEmpty)) {
+              ok = false;
+              break;
             }
-            tma_load_2d(dst + 8 * kWBlkK + r0 * 128, &tmKR, kv_full + s, 0, row);
+            mbar_expect_tx(full, part == 0 ? kWPartA : kWPartB);
+            const int cb0 = part == 0 ? cb_other : cb_own;
+            for (int r0 = 0; r0 < kTileKeys; r0 += box_rows) {
+              const int row = paged_row(bt, j0 + r0, bs, n_pages, p.oob_row, p.status);  // past the last page: zeros
+              if (whole) {
+                tma_load_3d(dst + cb0 * kWBlkK, &tmKV3, full, 0, row, cb0);  // [4 column blocks][key][64 elements]
+              } else {
+                for (int cb = cb0; cb < cb0 + 4; ++cb)
+                  tma_load_2d(dst + cb * kWBlkK + r0 * 128, &tmKV, full, cb * 64, row);
+              }
+              if (part == 0) tma_load_2d(dst + 8 * kWBlkK + r0 * 128, &tmKR, full, 0, row);
+            }
           }
+          if (!ok) break;
           ++G;
         }
       }
       // no copy may be in flight when the CTA exits
-      for (int t = G - kWStages < 0 ? 0 : G - kWStages; t < G; ++t)
-        mbar_wait(kv_full + (t % kWStages), (t / kWStages) & 1, status, kDevTimeoutKFull);
+      for (int t = G - kWStages < 0 ? 0 : G - kWStages; t < G; ++t) {
+        mbar_wait(full_a + (t % kWStages), (t / kWStages) & 1, status, kDevTimeoutKFull);
+        mbar_wait(full_b + (t % kWStages), (t / kWStages) & 1, status, kDevTimeoutKFull);
+      }
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer (one elected thread)
@@ -221,37 +246,59 @@ __global__ void __launch_bounds__(192, 1)
       uint64_t t_prog = global_timer_ns();
       uint32_t it = 0;
       bool progressed = false;
+      // the three groups of QK MMAs into S buffer d_s of slot offset so (the first one issued starts the sum)
+      auto qk_ts = [&](uint32_t d_s, uint64_t so, bool first) {  // qNope dims 0..255 from tensor memory
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk)
+          mma_ts(d_s, tmem + kWQnCol + kk * 8, dk + so + (uint64_t)(((kk >> 2) * kWBlkK + (kk & 3) * 32) >> 4),
+                 idesc_qk, (first && kk == 0) ? 0u : 1u, false);
+      };
+      auto qk_ss = [&](uint32_t d_s, uint64_t so, bool first) {  // qNope dims 256..511 from shared memory
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk)
+          mma_ss(d_s, dqn + (uint64_t)(((kk >> 2) * kWBlkQ + (kk & 3) * 32) >> 4),
+                 dk + so + (uint64_t)(((4 + (kk >> 2)) * kWBlkK + (kk & 3) * 32) >> 4), idesc_qk,
+                 (first && kk == 0) ? 0u : 1u, false);
+      };
+      auto qk_rope = [&](uint32_t d_s, uint64_t so) {  // qRope x kRope
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(d_s, dqr + (uint64_t)((kk * 32) >> 4), dk + so + (uint64_t)((8 * kWBlkK + kk * 32) >> 4), idesc_qk, 1u,
+                 false);
+      };
+      bool qk_a = false;  // the part-A MMAs of QK(Gq) are issued, the part-B ones not yet
       while (ok && Gp < total) {
-        // QK(Gq) needs its tile, its S buffer (PV(Gq-2), which read P over it, has completed) and, first in
-        // a piece, the query; it leads PV by at most one tile.  PV(Gp) needs P(Gp) and, first in a piece
-        // after the CTA's first, the previous epilogue's read of O.
+        // QK(Gq) needs its S buffer (PV(Gq-2), which read P over it, has completed), first in a piece the
+        // query, and leads PV by at most one tile; its MMAs over part A go first, those over part B once
+        // that part has landed.  PV(Gp) needs P(Gp) and, first in a piece after the CTA's first, the
+        // previous epilogue's read of O.
         const int bq = Gq & 1;
-        if (Gq < total && Gq - Gp < 2 && mbar_test_wait(kv_full + bq, (Gq >> 1) & 1) &&
-            (Gq < 2 || mbar_test_wait(pv_done + bq, ((Gq - 2) >> 1) & 1)) &&
-            (jq > 0 || mbar_test_wait(q_full, (kq - k0) & 1))) {
+        const uint32_t d_s = tmem + kWSCol + 64 * bq;
+        const uint64_t so_q = (uint64_t)((bq * kWKvBytes) >> 4);
+        if (qk_a && mbar_test_wait(full_b + bq, (Gq >> 1) & 1)) {
           tc_fence_after();
-          const uint32_t d_s = tmem + kWSCol + 64 * bq;
-          const uint64_t so = (uint64_t)((bq * kWKvBytes) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < 16; ++kk)  // qNope dims 0..255 from tensor memory (8 columns per 16 elements)
-            mma_ts(d_s, tmem + kWQnCol + kk * 8, dk + so + (uint64_t)(((kk >> 2) * kWBlkK + (kk & 3) * 32) >> 4),
-                   idesc_qk, kk > 0 ? 1u : 0u, false);
-#pragma unroll
-          for (int kk = 0; kk < 16; ++kk)  // qNope dims 256..511 from shared memory
-            mma_ss(d_s, dqn + (uint64_t)(((kk >> 2) * kWBlkQ + (kk & 3) * 32) >> 4),
-                   dk + so + (uint64_t)(((4 + (kk >> 2)) * kWBlkK + (kk & 3) * 32) >> 4), idesc_qk, 1u, false);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)  // qRope x kRope
-            mma_ss(d_s, dqr + (uint64_t)((kk * 32) >> 4), dk + so + (uint64_t)((8 * kWBlkK + kk * 32) >> 4), idesc_qk,
-                   1u, false);
+          if (half == 0) qk_ts(d_s, so_q, false);  // this CTA's column blocks: dims 0..255
+          else qk_ss(d_s, so_q, false);            // dims 256..511
           mma_commit(s_full + bq);
-          if (jq + 1 == nq) mma_commit(q_free);  // the piece's last QK: its query may be replaced
+          const bool last = jq + 1 == nq;
+          if (last) mma_commit(q_free);  // the piece's last QK: its query may be replaced
+          else mma_commit(empty_a + bq);  // a piece's last slot is the epilogue's staging area instead
+          qk_a = false;
           ++Gq;
           if (++jq == nq) {
             ++kq;
             jq = 0;
             nq = kq < k1 ? p.pieces[kq].n_tiles : 0;
           }
+          progressed = true;
+        } else if (!qk_a && Gq < total && Gq - Gp < 2 && mbar_test_wait(full_a + bq, (Gq >> 1) & 1) &&
+                   (Gq < 2 || mbar_test_wait(pv_done + bq, ((Gq - 2) >> 1) & 1)) &&
+                   (jq > 0 || mbar_test_wait(q_full, (kq - k0) & 1))) {
+          tc_fence_after();
+          if (half == 0) qk_ss(d_s, so_q, true);  // the other half's column blocks
+          else qk_ts(d_s, so_q, true);
+          qk_rope(d_s, so_q);
+          qk_a = true;
           progressed = true;
         } else if (Gp < Gq && mbar_test_wait(p_full + (Gp & 1), (Gp >> 1) & 1) &&
                    (jp > 0 || kp == k0 || mbar_test_wait(o_free, (kp - 1 - k0) & 1))) {
@@ -265,8 +312,8 @@ __global__ void __launch_bounds__(192, 1)
                    dv + so + (uint64_t)((4 * half * kWBlkK + kk * 16 * 128) >> 4), idesc_pv, (jp > 0 || kk > 0) ? 1u : 0u,
                    false);
           mma_commit(pv_done + bp);
-          // the slot returns to the producer; a piece's last slot is the epilogue's staging area instead
-          if (jp + 1 < np) mma_commit(kv_empty + bp);
+          // part B returns to the producer; a piece's last slot is the epilogue's staging area instead
+          if (jp + 1 < np) mma_commit(empty_b + bp);
           ++Gp;
           if (++jp == np) {
             ++kp;
@@ -507,7 +554,8 @@ __global__ void __launch_bounds__(192, 1)
       // the staging slot goes back to the producer once the stores have read it
       if (threadIdx.x == 0) {
         ok = mbar_wait(st_free, (R - 1) & 1, status, kDevTimeoutFinal);
-        mbar_arrive(kv_empty + s_last);
+        mbar_arrive(empty_a + s_last);
+        mbar_arrive(empty_b + s_last);
       }
       ok = __all_sync(kFull, ok);
     }

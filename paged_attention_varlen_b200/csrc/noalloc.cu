@@ -125,7 +125,7 @@ extern "C" ALA_API int varlen_attention_noalloc(const ala_tensor* query, const a
   if (!alibi && slopes && slopes->data) return nfail(ALA_INVALID_PARAM, "%s: slopes must be NULL for maskType %d", fn, maskType);
   if (alibi && (slopes->dtype != ALA_F32 || slopes->ndim != 1 || slopes->dims[0] != headNum))
     return nfail(ALA_INVALID_SHAPE, "%s: slopes must be fp32 [headNum]", fn);
-  if (prefill_smem_bytes(dt, (int32_t)d) == 0)
+  if (prefill_kernel_d(dt, d) == 0)
     return nfail(ALA_UNSUPPORTED, "%s: headSize %lld with this dtype is not built", fn, (long long)d);
   if (seqLen->ndim != 1 || kvSeqLen->ndim != 1 || seqLen->dims[0] != kvSeqLen->dims[0])
     return nfail(ALA_INVALID_SHAPE, "%s: seqLen and kvSeqLen must both be [batch]", fn);
@@ -201,8 +201,8 @@ extern "C" ALA_API int varlen_attention_noalloc(const ala_tensor* query, const a
 
   CUtensorMap tmQ, tmK, tmV;
   if (!encode_rows_heads_d(&tmQ, query->data, dt, n_tokens, headNum, d, 128, false) ||
-      !encode_rows_heads_d(&tmK, key->data, dt, key->dims[0], kvHeadNum, d, 128, false) ||
-      !encode_rows_heads_d(&tmV, value->data, dt, key->dims[0], kvHeadNum, d, 128, true))
+      !encode_rows_heads_d(&tmK, key->data, dt, key->dims[0], kvHeadNum, d, kPrefillTileKeys, false) ||
+      !encode_rows_heads_d(&tmV, value->data, dt, key->dims[0], kvHeadNum, d, kPrefillTileKeys, true))
     return nfail(ALA_CUDA_ERROR, "%s: cuTensorMapEncodeTiled failed (pointers must be 16-byte aligned)", fn);
 
   const size_t bytes = kStatusBytes + kSeqBytes + nu * sizeof(PrefillUnit);
@@ -229,7 +229,8 @@ extern "C" ALA_API int varlen_attention_noalloc(const ala_tensor* query, const a
   p.heads = headNum;
   p.group = group;
   p.scale_log2 = qkScale * 1.4426950408889634f;
-  const cudaError_t e = launch_prefill(dt, (int32_t)d, tmQ, tmK, tmV, p, st);
+  p.d_out = (int32_t)d;
+  const cudaError_t e = launch_prefill(dt, prefill_kernel_d(dt, d), tmQ, tmK, tmV, p, st);
   if (e != cudaSuccess) return nfail(ALA_CUDA_ERROR, "%s: kernel launch failed: %s", fn, cudaGetErrorString(e));
   set_last_error("");
   return ALA_OK;

@@ -76,10 +76,14 @@ def test_output_must_be_32_byte_aligned():
     (dict(slopes=np.ones(4, np.float32)), 4),                    # causal forbids slopes
     (dict(mask_type=3, slopes=np.ones(3, np.float32)), 2),       # slopes must be [headNum]
     (dict(k=torch.zeros(14, 2, 128, dtype=torch.float16)), 3),   # dtype mismatch
+    (dict(q=torch.zeros(10, 4, 72, dtype=torch.bfloat16), k=torch.zeros(14, 2, 72, dtype=torch.bfloat16),
+          v=torch.zeros(14, 2, 72, dtype=torch.bfloat16)), 5),     # headSize not a multiple of 16
+    (dict(q=torch.zeros(10, 4, 256, dtype=torch.bfloat16), k=torch.zeros(14, 2, 256, dtype=torch.bfloat16),
+          v=torch.zeros(14, 2, 256, dtype=torch.bfloat16)), 5),    # headSize > 128 is not built
+    (dict(q=torch.zeros(10, 4, 96, dtype=torch.float32), k=torch.zeros(14, 2, 96, dtype=torch.float32),
+          v=torch.zeros(14, 2, 96, dtype=torch.float32)), 5),      # fp32 up to 64
     (dict(q=torch.zeros(10, 4, 256, dtype=torch.bfloat16), k=torch.zeros(14, 2, 256, dtype=torch.bfloat16),
           v=torch.zeros(14, 2, 256, dtype=torch.bfloat16), mask_type=3, slopes=np.ones(4, np.float32)), 4),
-    (dict(q=torch.zeros(10, 4, 96, dtype=torch.bfloat16), k=torch.zeros(14, 2, 96, dtype=torch.bfloat16),
-          v=torch.zeros(14, 2, 96, dtype=torch.bfloat16)), 5),   # head size not built
     (dict(q=torch.zeros(10, 4, 128), k=torch.zeros(14, 2, 128), v=torch.zeros(14, 2, 128)), 5),  # f32 d=128
 ])
 def test_varlen_rejects(over, status):
@@ -344,3 +348,11 @@ def test_mla_explicit_mask_rejects(over, status):
     with pytest.raises(ala.AlaError) as e:
         _plan_mla(**over)
     assert e.value.status == status, str(e.value)
+
+
+@pytest.mark.parametrize("d,dtype", [(16, torch.bfloat16), (80, torch.float16), (96, torch.bfloat16),
+                                     (112, torch.bfloat16), (40, torch.float32)])
+def test_head_sizes_plan(d, dtype):
+    op, out = _plan_varlen(q=torch.zeros(10, 4, d, dtype=dtype), k=torch.zeros(14, 2, d, dtype=dtype),
+                           v=torch.zeros(14, 2, d, dtype=dtype))
+    assert out.shape == (10, 4, d)

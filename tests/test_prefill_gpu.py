@@ -94,6 +94,19 @@ def test_paged_prefix_encoder(block_size, mask_type):
     _full_check(case)
 
 
+@pytest.mark.parametrize("d,dtype,mask_type,paged", [
+    (16, torch.bfloat16, 9, False), (48, torch.float16, 3, False), (80, torch.bfloat16, 9, False),
+    (96, torch.bfloat16, 4, False), (112, torch.float16, 0, False), (96, torch.float16, 3, True),
+    (80, torch.float16, 5, True), (40, torch.float32, 9, False), (8, torch.float32, 0, False)])
+def test_head_sizes_between_the_kernel_sizes(d, dtype, mask_type, paged):
+    # head sizes run on the next kernel instance up (64 or 128) with the extra dimensions zero-filled
+    L = [1, 127, 128, 129, 300, 5]
+    pre = [0, 40, 0, 77, 129, 3]
+    case = synth.make_prefill(f"d{d}", L, [a + b for a, b in zip(L, pre)], 8, 2, d, dtype, mask_type, 95 + d,
+                              paged=paged, block_size=64)
+    _full_check(case)
+
+
 def test_paged_equals_contiguous_on_gpu():
     L, pre = [100, 250], [300, 17]
     kv = [a + b for a, b in zip(L, pre)]
