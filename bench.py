@@ -49,8 +49,8 @@ PROFILE = os.path.join(ROOT, "profiles", "prefill_varlen_causal_bf16.md")
 MLA_PROFILE = os.path.join(ROOT, "profiles", "mla_decode_qs1_bf16.md")
 MLA_INT8_PROFILE = os.path.join(ROOT, "profiles", "mla_decode_qs1_int8.md")
 KERNEL_SOURCES = ["paged_attention_varlen_b200/csrc/prefill.cu", "paged_attention_varlen_b200/csrc/ptx.cuh"]
-MLA_KERNEL_SOURCES = ["paged_attention_varlen_b200/csrc/mla.cu", "paged_attention_varlen_b200/csrc/mla_wide.cu",
-                      "paged_attention_varlen_b200/csrc/mla_common.cuh", "paged_attention_varlen_b200/csrc/ptx.cuh"]
+MLA_KERNEL_SOURCES = ["paged_attention_varlen_b200/csrc/mla.cu", "paged_attention_varlen_b200/csrc/mla_common.cuh",
+                      "paged_attention_varlen_b200/csrc/ptx.cuh"]
 DEFAULT_WORKLOAD = "varlen_causal_bf16"
 WORKLOADS = {
     "varlen_causal_bf16": lambda: synth.varlen_causal_bf16(),
@@ -339,14 +339,7 @@ def cpu_baseline(case, sample_s=12.0):
 
 
 def mla_kernel_name(case):
-    """The MLA kernel a workload runs on: 128 query rows per CTA (one token per row block, 16-bit cache,
-    heads a multiple of 128) or 64."""
-    int8 = case.qk_descale is not None
-    qs = case.q_seq_len
-    tpc = 4 if (qs % 4 == 0).all() else 2 if (qs % 2 == 0).all() else 1
-    if tpc == 1 and not int8 and case.heads % 128 == 0:
-        return "mla_wide_kernel<bf16>"
-    return "mla_kernel<bf16, int8 cache>" if int8 else "mla_kernel<bf16>"
+    return "mla_kernel<bf16, int8 cache>" if case.qk_descale is not None else "mla_kernel<bf16>"
 
 
 def case_dtype(case):

@@ -66,7 +66,7 @@ struct SeqInfo {
 };
 
 // Keys per K/V tile of the prefill kernel.
-constexpr int kPrefillTileKeys = 64;
+constexpr int kPrefillTileKeys = 128;
 
 // One CTA's work: up to two blocks of 128 query rows of one sequence that read
 // the same kv head (two query heads of a group, or two consecutive row tiles of

@@ -929,13 +929,9 @@ int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, co
     for (int32_t b = 0; b < batch; ++b) divides = divides && plan->qs[b] % tpc == 0;
     if (divides) break;
   }
-  // one token per row block, 128-head groups and a 16-bit cache: the 128-row kernel, whose CTA pairs
-  // split the output columns (two CTAs per group); otherwise 64-row blocks
-  const bool wide = tpc == 1 && !kv8 && headNum % 128 == 0;
-  const int32_t hpc = wide ? 128 : kRows / tpc;
+  const int32_t hpc = kRows / tpc;
   const int32_t groups = headNum / hpc;
-  const int32_t ctas_per_lane = wide ? 2 * groups : groups;
-  plan->wide = wide;
+  const int32_t ctas_per_lane = groups;
   plan->tpc = tpc;
   plan->hpc = hpc;
   plan->groups = groups;
@@ -1034,8 +1030,7 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
     // [column block][key][64 elements] as the 128B-swizzled K-major operand wants it
     cuuint64_t kv3_dims[3] = {64, rows, 8};
     cuuint64_t kv3_str[2] = {512 * es, 64 * es};
-    // the 128-row kernel loads a tile in two parts of four column blocks each
-    cuuint32_t kv3_box[3] = {64, (cuuint32_t)kTileKeys, plan->wide ? 4u : 8u};
+    cuuint32_t kv3_box[3] = {64, (cuuint32_t)kTileKeys, 8};
     // int8 codes: 512 bytes a row, seen as 128-byte column blocks (4 per row), same boxes of keys
     cuuint64_t k8_dims[2] = {512, rows};
     cuuint64_t k8_str[1] = {512};
@@ -1043,15 +1038,6 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
     cuuint64_t k83_dims[3] = {128, rows, 4};
     cuuint64_t k83_str[2] = {512, 128};
     cuuint32_t k83_box[3] = {128, (cuuint32_t)kTileKeys, 4};
-    if (plan->wide) {
-      // the 128-row kernel: query / output boxes of 64 columns x 128 heads of one token
-      cuuint32_t w_box[3] = {64, 128, 1};
-      if (!encode(&plan->tmQn, plan->q_nope, plan->dtype, 3, qn_dims, qn_str, w_box))
-        return mfail(err, n, ALA_CUDA_ERROR, "cuTensorMapEncodeTiled failed for qNope");
-      q_box[0] = 64;
-      q_box[1] = 128;
-      q_box[2] = 1;
-    }
     const bool kv_ok = plan->kv8 ? (encode(&plan->tmKV3, plan->ct_kv, ALA_I8, 3, k83_dims, k83_str, k83_box) &&
                                     encode(&plan->tmKV, plan->ct_kv, ALA_I8, 2, k8_dims, k8_str, k8_box))
                                  : (encode(&plan->tmKV3, plan->ct_kv, plan->dtype, 3, kv3_dims, kv3_str, kv3_box) &&
@@ -1067,7 +1053,7 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
   } else if (plan->tmPO_base != ws + plan->off_part_o) {
     cuuint64_t po_dims[3] = {512, (cuuint64_t)plan->heads, (cuuint64_t)plan->n_splits_total * tpc};
     cuuint64_t po_str[2] = {512 * 4, (cuuint64_t)plan->heads * 512 * 4};
-    cuuint32_t po_box[3] = {32, plan->wide ? 128u : hpc, tpc};
+    cuuint32_t po_box[3] = {32, hpc, tpc};
     if (!encode(&plan->tmPO, ws + plan->off_part_o, ALA_F32, 3, po_dims, po_str, po_box))
       return mfail(err, n, ALA_CUDA_ERROR, "cuTensorMapEncodeTiled failed for the partial-output map");
     plan->tmPO_base = ws + plan->off_part_o;
@@ -1111,18 +1097,6 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
   p.mask_f16 = plan->mask_f16 ? 1 : 0;
   p.mask_vec = (reinterpret_cast<uintptr_t>(plan->mask) % 16 == 0 && plan->mask_cols % 8 == 0) ? 1 : 0;
   const bool f16 = plan->dtype == ALA_F16;
-  if (plan->wide) {
-    cudaError_t e = launch_mla_wide(plan->dtype, (int)plan->n_work, plan->tmQn, plan->tmQr, plan->tmKV, plan->tmKV3,
-                                    plan->tmKR, plan->tmO, plan->tmPO, p, stream);
-    if (e == cudaSuccess && plan->n_combine > 0) {
-      auto ck = f16 ? mla_combine_kernel<__half> : mla_combine_kernel<__nv_bfloat16>;
-      dim3 grid(plan->n_combine, (plan->heads + 7) / 8);
-      ck<<<grid, 256, 0, stream>>>(reinterpret_cast<const MlaCombine*>(ws + plan->off_rows), p);
-      e = cudaGetLastError();
-    }
-    if (e != cudaSuccess) return mfail(err, n, ALA_CUDA_ERROR, cudaGetErrorString(e));
-    return ALA_OK;
-  }
   auto kern = plan->kv8 ? (f16 ? mla_kernel<__half, true> : mla_kernel<__nv_bfloat16, true>)
                         : (f16 ? mla_kernel<__half, false> : mla_kernel<__nv_bfloat16, false>);
   const int threads = plan->kv8 ? 320 : 192;

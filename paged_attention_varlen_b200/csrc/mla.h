@@ -14,7 +14,6 @@ struct MlaPlan {
   int32_t dtype = 0, heads = 0, batch = 0, block_size = 0, max_blocks = 0;
   int32_t calc_type = 0, mask_type = 0;
   bool kv8 = false, qn_int8 = false;  // int8 latent cache (cacheMode 2); qNope holds int8 codes
-  bool wide = false;                   // served by the 128-row kernel (mla_wide.cu): one token per row block
   const float *qk_descale = nullptr, *pv_descale = nullptr;
   float qk_scale = 1.f;
   int64_t tokens = 0, num_blocks = 0;
@@ -25,7 +24,7 @@ struct MlaPlan {
   int64_t mask_cols = 0;
   bool mask_f16 = false;
   std::vector<int32_t> ctx, qs;
-  // row blocks of tpc tokens x hpc heads; groups = heads / hpc (x 2 column halves with the 128-row kernel)
+  // row blocks of tpc tokens x hpc heads; groups = heads / hpc
   int32_t tpc = 1, hpc = 64, groups = 1;
   // schedule and workspace: [status | pieces | lane offsets | combine list | partial lse | partial O]
   int32_t n_lanes = 0, n_work = 0, n_splits_total = 0, n_combine = 0;
@@ -34,7 +33,7 @@ struct MlaPlan {
   std::vector<uint8_t> image;  // host copy of [status | pieces | lane offsets | combine list]
   void* pinned = nullptr;      // page-locked copy of `image`, made on first run
   bool maps_ready = false;
-  CUtensorMap tmQn, tmQr, tmKV, tmKV3, tmKR, tmO;
+  CUtensorMap tmQr, tmKV, tmKV3, tmKR, tmO;
   CUtensorMap tmPO;                // partial-output map, bound to the workspace it was encoded for
   const void* tmPO_base = nullptr;
   MlaPlan() = default;

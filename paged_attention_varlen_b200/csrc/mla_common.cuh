@@ -1,6 +1,5 @@
-// mla_common.cuh -- pieces shared by the two MLA decode kernels (mla.cu: 64 query rows per CTA;
-// mla_wide.cu: 128 query rows per CTA, the output columns split over a CTA pair): the schedule's
-// work records, the kernel parameters and small device helpers.  Internal to the library.
+// mla_common.cuh -- the MLA schedule's work records, the kernel parameters and small device helpers
+// (mla.cu).  Internal to the library.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -109,13 +108,6 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, __half*) {
 __device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, int* status, int code) {
   return __all_sync(kFull, mbar_wait(bar, parity, status, code));
 }
-
-// The 128-row kernel (mla_wide.cu): its dynamic shared memory and its launch (grid = lanes x head
-// groups of 128 x 2 column halves).
-int mla_wide_smem_bytes();
-cudaError_t launch_mla_wide(int32_t dtype, int grid, const CUtensorMap& tmQn, const CUtensorMap& tmQr,
-                            const CUtensorMap& tmKV, const CUtensorMap& tmKV3, const CUtensorMap& tmKR,
-                            const CUtensorMap& tmO, const CUtensorMap& tmPO, const MlaParams& p, cudaStream_t stream);
 
 }  // namespace mlak
 }  // namespace ala

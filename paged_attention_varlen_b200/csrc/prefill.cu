@@ -6,26 +6,25 @@
 //
 // One CTA computes up to two blocks of 128 query rows that read the same kv
 // head (two query heads of a GQA group, or two consecutive row tiles of one
-// head), so each K/V tile staged in shared memory serves 256 rows.  Keys come
-// in tiles of 64, and each block has two S buffers in tensor memory, so the
-// next tile's Q K^T runs on the tensor core while the softmax works on the
-// current one.
+// head), so each K/V tile staged in shared memory serves 256 rows.
 //
-//   warp 8       TMA producer: both Q tiles once per unit, then K and V tiles
-//                (64 keys) into 4-deep rings; paged rows are gathered page by
-//                page through the block table.
+//   warp 8       TMA producer: both Q tiles once, then K and V tiles (128 keys)
+//                into 2-deep rings; paged rows are gathered page by page
+//                through the block table.
 //   warp 9       tcgen05 issuer.  Per key tile j and block b:
-//                  S_b[j%2] = Q_b K_j^T    (SS MMA, M = 128, N = 64)
-//                  O_b     += P_b V_j      (TS MMA: P_b read from TMEM over S_b[j%2])
-//                in the order PV_0(j), PV_1(j), QK_0(j+2), QK_1(j+2): the S
-//                buffer of tile j is refilled with tile j+2 once P_b(j) V has
-//                completed, while the softmax works on tile j+1.
+//                  S_b = Q_b K_j^T        (SS MMA into TMEM columns of S_b)
+//                  O_b += P_b V_j         (TS MMA: P_b read from TMEM)
+//                in the order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so the
+//                tensor core works on one block while the other block's
+//                softmax runs.  P_b V_j goes in two halves of 64 keys: the
+//                first starts as soon as the softmax has written P for keys
+//                0..63, while it still computes the rest.
 //   warps 0..3,  softmax of block 0 / block 1: thread r owns row r (TMEM lane
 //   4..7         r).  It reads its S row, applies qkScale, the ALiBi bias and
 //                the causal / prefix-offset rule in registers (the mask is
 //                never materialised), updates the running max and sum, rescales
 //                O_b in TMEM only when the max grew by more than 2^8, and writes
-//                P_b (16-bit, or fp32 for tf32) over its S buffer.  At the end it
+//                P_b (16-bit, or fp32 for tf32) over S_b in TMEM.  At the end it
 //                normalises O_b and stores it.
 //
 // Key tiles wholly above the prefix-shifted causal diagonal, or past the
@@ -44,7 +43,6 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
-constexpr int KT = kPrefillTileKeys;       // keys per tile
 
 template <typename T>
 struct ElemFmt;
@@ -64,23 +62,19 @@ struct ElemFmt<float> {
 template <typename T, int D>
 struct Cfg {
   static constexpr int ES = sizeof(T);
-  static constexpr int AW = 128 / ES;      // elements in one 128-byte swizzled row
-  static constexpr int UK = 32 / ES;       // K extent of one MMA instruction
-  static constexpr int BLK_Q = 128 * 128;  // bytes of one 128-row x 128-byte swizzle column block
-  static constexpr int BLK_KV = KT * 128;  // bytes of one 64-key x 128-byte swizzle column block
-  static constexpr int STAGES = 4;
+  static constexpr int AW = 128 / ES;    // elements in one 128-byte swizzled row
+  static constexpr int UK = 32 / ES;     // K extent of one MMA instruction
+  static constexpr int BLK = 128 * 128;  // bytes of one 128-row x 128-byte swizzle column block
+  static constexpr int STAGES = 2;
   static constexpr int Q_BYTES = 128 * D * ES;
-  static constexpr int KV_BYTES = KT * D * ES;
-  static constexpr int TBL_FLOATS = 96;  // per-warp sqrt-bias table: lane - column + 63 in [0, 95)
+  static constexpr int KV_BYTES = 128 * D * ES;
+  static constexpr int TBL_FLOATS = 160;  // per-warp sqrt-bias table: lane - column + 127 in [0, 159)
   static constexpr int TBL_BYTES = 8 * 2 * TBL_FLOATS * 4;
-  // q_full, q_empty, fin, k_full[4], v_full[4], k_empty[4], v_empty[4], and per block:
-  // s_full[2], p_full[2], pv_done[2], o_done
-  static constexpr int N_BARS = 3 + 4 * STAGES + 2 * 7;
+  static constexpr int N_BARS = 21;
   static constexpr int SMEM = 1024 + 2 * Q_BYTES + 2 * STAGES * KV_BYTES + TBL_BYTES + N_BARS * 8 + 16;
-  static constexpr uint32_t IDESC_QK = instr_desc(ElemFmt<T>::fmt, false, false, 128, KT);
+  static constexpr uint32_t IDESC_QK = instr_desc(ElemFmt<T>::fmt, false, false, 128, 128);
   static constexpr uint32_t IDESC_PV = instr_desc(ElemFmt<T>::fmt, false, true, 128, D);
-  // block b: S_b[0] [128b, 128b+64), S_b[1] [128b+64, 128b+128); O_b [256 + b D, 256 + (b+1) D)
-  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t TMEM_COLS = 512;  // S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D, 256+2D)
   static_assert(D % AW == 0, "head size must fill whole swizzle rows");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(256 + 2 * D <= 512, "tensor memory budget");
@@ -103,16 +97,18 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, __half*) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// P = 2^(u) for one row's 64 scores, u = x*scale - m taken a pair of columns at a time with packed f32x2
-// arithmetic; writes P over S in TMEM (16-bit pairs, or fp32 for tf32) and returns the row sum.  Masked
-// keys hold -inf, which ex2 maps to exactly 0.
+// P = 2^(u) for one row's 128 scores, u = x*scale - m taken a pair of columns at a
+// time with packed f32x2 arithmetic; writes P over S in TMEM (16-bit pairs, or
+// fp32 for tf32) and returns the row sum.  Masked keys hold -inf, which ex2 maps
+// to exactly 0.
 template <typename T>
-__device__ __forceinline__ float exp_row(const float (&x)[KT], uint64_t scale2, uint64_t negm2, uint32_t s_col) {
+__device__ __forceinline__ float exp_rows(const float (&x)[128], uint64_t scale2, uint64_t negm2, uint32_t s_col,
+                                          uint64_t* p_lo) {
   constexpr bool kHalf = sizeof(T) == 2;
   constexpr int CHUNK = kHalf ? 64 : 32;  // columns per 32-register TMEM store
   uint64_t acc[4] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f), f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
 #pragma unroll
-  for (int h = 0; h < KT / CHUNK; ++h) {
+  for (int h = 0; h < 128 / CHUNK; ++h) {
     uint32_t pk[32];
 #pragma unroll
     for (int cc = 0; cc < CHUNK / 2; ++cc) {
@@ -130,6 +126,12 @@ __device__ __forceinline__ float exp_row(const float (&x)[KT], uint64_t scale2, 
       }
     }
     tmem_st32(s_col + h * 32, pk);
+    if (h == 128 / CHUNK / 2 - 1) {
+      // P of keys 0..63 is in place: the first half of P*V may start while the rest is computed
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_lo);
+    }
   }
   const uint64_t a = add_x2(add_x2(acc[0], acc[1]), add_x2(acc[2], acc[3]));
   float s0, s1;
@@ -144,15 +146,14 @@ __device__ __forceinline__ void load_kv_tile(const CUtensorMap* map, uint8_t* ds
   using C = Cfg<T, D>;
   const bool paged = bt != nullptr;
   const int bs = p.block_size;
-  const int box_rows = paged ? (bs < KT ? bs : KT) : KT;
-  const int j0 = j * KT;
-  for (int r0 = 0; r0 < KT; r0 += box_rows) {
+  const int box_rows = paged ? (bs < 128 ? bs : 128) : 128;
+  const int j0 = j * 128;
+  for (int r0 = 0; r0 < 128; r0 += box_rows) {
     // contiguous rows, or the page's row through the block table (past the last page: zero fill)
     const int row = paged ? paged_row(bt, j0 + r0, bs, n_pages, p.oob_row, p.status) : si.cu_kv + j0 + r0;
     if (leader) {
 #pragma unroll
-      for (int cb = 0; cb < D / C::AW; ++cb)
-        tma_load_3d(dst + cb * C::BLK_KV + r0 * 128, map, full, cb * C::AW, kvh, row);
+      for (int cb = 0; cb < D / C::AW; ++cb) tma_load_3d(dst + cb * C::BLK + r0 * 128, map, full, cb * C::AW, kvh, row);
     }
   }
 }
@@ -162,26 +163,25 @@ __global__ void __launch_bounds__(384, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
   using C = Cfg<T, D>;
-  constexpr int NS = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                   // [2][Q_BYTES]
-  uint8_t* sK = sQ + 2 * C::Q_BYTES;    // [STAGES][KV_BYTES]
-  uint8_t* sV = sK + NS * C::KV_BYTES;
-  float* sTbl = reinterpret_cast<float*>(sV + NS * C::KV_BYTES);  // [8 warps][2][TBL_FLOATS]
+  uint8_t* sQ = smem;                        // [2][Q_BYTES]
+  uint8_t* sK = sQ + 2 * C::Q_BYTES;         // [STAGES][KV_BYTES]
+  uint8_t* sV = sK + C::STAGES * C::KV_BYTES;
+  float* sTbl = reinterpret_cast<float*>(sV + C::STAGES * C::KV_BYTES);  // [8 warps][2][TBL_FLOATS]
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sTbl) + C::TBL_BYTES);
   uint64_t* q_full = bars;
-  uint64_t* q_empty = bars + 1;
-  uint64_t* fin = bars + 2;
-  uint64_t* k_full = bars + 3;            // [NS]
-  uint64_t* v_full = k_full + NS;         // [NS]
-  uint64_t* k_empty = v_full + NS;        // [NS]
-  uint64_t* v_empty = k_empty + NS;       // [NS]
-  uint64_t* blk_bars = v_empty + NS;      // per block b, at blk_bars + 7 b:
-  auto s_full = [&](int b, int s) { return blk_bars + 7 * b + s; };       // S_b[s] computed
-  auto p_full = [&](int b, int s) { return blk_bars + 7 * b + 2 + s; };   // P written over S_b[s]
-  auto pv_done = [&](int b, int s) { return blk_bars + 7 * b + 4 + s; };  // the P V of S_b[s]'s tile completed
-  auto o_done = [&](int b) { return blk_bars + 7 * b + 6; };              // the unit's last P_b V completed
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* v_full = bars + 3;    // [2]
+  uint64_t* k_empty = bars + 5;   // [2]
+  uint64_t* v_empty = bars + 7;   // [2]
+  uint64_t* s_full = bars + 9;    // [2] per block
+  uint64_t* p_full = bars + 11;   // [2] per block: P of keys 64..127 written (all of P)
+  uint64_t* pv_done = bars + 13;  // [2] per block
+  uint64_t* o_done = bars + 15;   // [2] per block
+  uint64_t* fin = bars + 17;
+  uint64_t* q_empty = bars + 18;
+  uint64_t* p_lo = bars + 19;     // [2] per block: P of keys 0..63 written
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::N_BARS);
 
   const int warp = threadIdx.x >> 5;
@@ -194,21 +194,18 @@ __global__ void __launch_bounds__(384, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    mbar_init(fin, 1);
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < 2; ++s) {
       mbar_init(k_full + s, 1);
       mbar_init(v_full + s, 1);
       mbar_init(k_empty + s, 1);
       mbar_init(v_empty + s, 1);
+      mbar_init(s_full + s, 1);
+      mbar_init(p_full + s, 128);
+      mbar_init(p_lo + s, 128);
+      mbar_init(pv_done + s, 1);
+      mbar_init(o_done + s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      for (int s = 0; s < 2; ++s) {
-        mbar_init(s_full(b, s), 1);
-        mbar_init(p_full(b, s), 128);
-        mbar_init(pv_done(b, s), 1);
-      }
-      mbar_init(o_done(b), 1);
-    }
+    mbar_init(fin, 1);
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -220,9 +217,9 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // Barrier phases run on across units: the K/V rings by a global tile counter g (slot g % 4, phase
-  // g / 4), the per-block S/P/PV barriers by each block's own tile counter t (buffer t % 2, phase
-  // t / 2), q_full / q_empty and o_done by unit counters.
+  // Barrier phases run on across units: the K/V ring by a global tile counter, the
+  // per-block S/P/PV barriers by each block's tile counter, q_full / q_empty and
+  // o_done by unit counters.
   //
   // register split: the softmax warpgroups take 216 per thread, warps 8..11 keep 72
   // (256*216 + 128*72 = 64512 = 384*168, all the registers the block is launched with)
@@ -238,7 +235,7 @@ __global__ void __launch_bounds__(384, 1)
         tma_prefetch_desc(&tmV);
       }
       bool ok = true;
-      uint32_t kv_iter = 0;                 // K/V tiles loaded so far (all units)
+      uint32_t kv_iter = 0;               // K/V tiles loaded so far (all units)
       uint32_t issued_k = 0, issued_v = 0;  // K / V loads issued
       int q_loads = 0;
       for (int ui = u_begin; ui < u_end && ok; ++ui) {
@@ -251,10 +248,10 @@ __global__ void __launch_bounds__(384, 1)
         const int n_pages = bt ? (si.kv_len + p.block_size - 1) / p.block_size : 0;
         for (int j = 0; j < nmax && ok; ++j) {
           const uint32_t g = kv_iter + j;
-          const int s = g % NS;
+          const int s = g & 1;
           for (int kv = 0; kv < 2; ++kv) {
-            if (g >= NS && !__all_sync(0xffffffffu, mbar_wait((kv ? v_empty : k_empty) + s, ((g / NS) - 1) & 1,
-                                                              status, kv ? kDevTimeoutVEmpty : kDevTimeoutKEmpty))) {
+            if (g >= 2 && !__all_sync(0xffffffffu, mbar_wait((kv ? v_empty : k_empty) + s, ((g >> 1) - 1) & 1, status,
+                                                              kv ? kDevTimeoutVEmpty : kDevTimeoutKEmpty))) {
               ok = false;
               break;
             }
@@ -278,7 +275,7 @@ __global__ void __launch_bounds__(384, 1)
                 if (b >= nb) break;
 #pragma unroll
                 for (int cb = 0; cb < D / C::AW; ++cb)
-                  tma_load_3d(sQ + b * C::Q_BYTES + cb * C::BLK_Q, &tmQ, q_full, cb * C::AW, b ? u.head[1] : u.head[0],
+                  tma_load_3d(sQ + b * C::Q_BYTES + cb * C::BLK, &tmQ, q_full, cb * C::AW, b ? u.head[1] : u.head[0],
                               si.cu_q + (b ? u.q0[1] : u.q0[0]));
               }
             }
@@ -288,10 +285,10 @@ __global__ void __launch_bounds__(384, 1)
         kv_iter += nmax;
       }
       // never leave the CTA while loads it issued are still landing in shared memory
-      for (uint32_t g = issued_k >= NS ? issued_k - NS : 0; g < issued_k; ++g)
-        mbar_wait(k_full + (g % NS), (g / NS) & 1, status, kDevTimeoutKFull);
-      for (uint32_t g = issued_v >= NS ? issued_v - NS : 0; g < issued_v; ++g)
-        mbar_wait(v_full + (g % NS), (g / NS) & 1, status, kDevTimeoutVFull);
+      for (uint32_t g = issued_k >= 2 ? issued_k - 2 : 0; g < issued_k; ++g)
+        mbar_wait(k_full + (g & 1), (g >> 1) & 1, status, kDevTimeoutKFull);
+      for (uint32_t g = issued_v >= 2 ? issued_v - 2 : 0; g < issued_v; ++g)
+        mbar_wait(v_full + (g & 1), (g >> 1) & 1, status, kDevTimeoutVFull);
       if (q_loads > 0) mbar_wait(q_full, (q_loads - 1) & 1, status, kDevTimeoutQ);
     } else if (warp == 9) {
       // ------------------------------------------------------------ MMA issuer
@@ -302,99 +299,121 @@ __global__ void __launch_bounds__(384, 1)
       const uint64_t dk = smem_desc_sw128(smem_addr(sK), 16, 1024);
       // V is the MN-major operand: 16-bit types use the 16-byte-chunk swizzle (8-row atoms),
       // tf32 the 32-byte-chunk swizzle (4-row atoms), matching how the V tensor map loads it
-      const uint64_t dv =
-          C::ES == 4 ? smem_desc(smem_addr(sV), C::BLK_KV, 512, 1) : smem_desc(smem_addr(sV), C::BLK_KV, 1024, 2);
+      const uint64_t dv = C::ES == 4 ? smem_desc(smem_addr(sV), C::BLK, 512, 1) : smem_desc(smem_addr(sV), C::BLK, 1024, 2);
       constexpr uint64_t kQStep = C::Q_BYTES >> 4, kKVStep = C::KV_BYTES >> 4;
-      auto wait_all = [&](uint64_t* bar, uint32_t parity, int code) {
-        return __all_sync(0xffffffffu, mbar_wait(bar, parity, status, code));
-      };
-      // S_b[t % 2] = Q_b K^T of the tile in ring slot s (t: the block's own tile counter)
-      auto issue_qk = [&](int b, uint32_t t, int s) {
+      auto issue_qk = [&](int b, int s) {
         if (leader) {
           const uint64_t a0 = dq + b * kQStep, b0 = dk + s * kKVStep;
 #pragma unroll
           for (int kk = 0; kk < D / C::UK; ++kk) {
             const int ke = kk * C::UK;
-            const uint64_t off_q = ((ke / C::AW) * C::BLK_Q + (ke % C::AW) * C::ES) >> 4;
-            const uint64_t off_k = ((ke / C::AW) * C::BLK_KV + (ke % C::AW) * C::ES) >> 4;
-            mma_ss(tmem + b * 128 + (t & 1) * KT, a0 + off_q, b0 + off_k, C::IDESC_QK, kk > 0, C::ES == 4);
+            const uint64_t off = ((ke / C::AW) * C::BLK + (ke % C::AW) * C::ES) >> 4;
+            mma_ss(tmem + b * 128, a0 + off, b0 + off, C::IDESC_QK, kk > 0, C::ES == 4);
           }
-          mma_commit(s_full(b, t & 1));
         }
       };
-      // O_b (+)= P_b V, P_b in TMEM over S_b[t % 2] (8 columns per K step: two 16-bit values, or 8 tf32)
-      auto issue_pv = [&](int b, uint32_t t, int s, bool acc) {
+      auto issue_pv = [&](int b, int s, bool acc, int half) {
         if (leader) {
           const uint64_t v0 = dv + s * kKVStep;
 #pragma unroll
-          for (int kk = 0; kk < KT / C::UK; ++kk)
-            mma_ts(tmem + 256 + b * D, tmem + b * 128 + (t & 1) * KT + kk * 8, v0 + ((kk * C::UK * 128) >> 4),
-                   C::IDESC_PV, (acc || kk > 0) ? 1u : 0u, C::ES == 4);
-          mma_commit(pv_done(b, t & 1));
+          for (int kk = half * 64 / C::UK; kk < (half + 1) * 64 / C::UK; ++kk) {
+            // P_b in TMEM over S_b: 8 columns per K step (two 16-bit values per column, or 8 tf32)
+            mma_ts(tmem + 256 + b * D, tmem + b * 128 + kk * 8, v0 + ((kk * C::UK * 128) >> 4), C::IDESC_PV,
+                   (acc || kk > 0) ? 1u : 0u, C::ES == 4);
+          }
         }
       };
       auto commit = [&](uint64_t* bar) {
         if (leader) mma_commit(bar);
       };
-      // QK_b at the block's tile counter t: its K tile is loaded and its S buffer is free (the P V of
-      // tile t - 2, whose P lies over it, has completed)
-      auto qk_ready = [&](int b, uint32_t t, uint32_t g) {
-        if (!wait_all(k_full + (g % NS), (g / NS) & 1, kDevTimeoutKFull)) return false;
-        if (t >= 2 && !wait_all(pv_done(b, t & 1), ((t - 2) >> 1) & 1, kDevTimeoutODone)) return false;
-        tc_fence_after();
-        return true;
+      auto wait_all = [&](uint64_t* bar, uint32_t parity, int code) {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, status, code));
       };
       bool ok = true;
       uint32_t kv_iter = 0;
-      uint32_t tb[2] = {0, 0};  // tiles each block processed in earlier units
+      uint32_t sp0 = 0, sp1 = 0;  // tiles block 0 / 1 processed in earlier units
       for (int ui = u_begin; ui < u_end && ok; ++ui) {
         const int it = ui - u_begin;
         const PrefillUnit u = p.units[ui];
         const int nb = u.n_blocks;
-        const int n[2] = {u.n_tiles[0], nb > 1 ? u.n_tiles[1] : 0};
-        const int nmax = n[0] > n[1] ? n[0] : n[1];
-        if (!wait_all(q_full, it & 1, kDevTimeoutQ)) {
+        const int n0 = u.n_tiles[0];
+        const int n1 = nb > 1 ? u.n_tiles[1] : 0;
+        const int nmax = n0 > n1 ? n0 : n1;
+        if (!wait_all(q_full, it & 1, kDevTimeoutQ) ||
+            !wait_all(k_full + (kv_iter & 1), (kv_iter >> 1) & 1, kDevTimeoutKFull)) {
           ok = false;
           break;
         }
-        // the last QK of tile j of this unit releases its K slot (and, for the unit's last tile, the Q buffers)
-        auto after_qk = [&](int j, int b) {
-          if (!(b == nb - 1 || j >= n[1])) return;
-          commit(k_empty + ((kv_iter + j) % NS));
-          if (j == nmax - 1) commit(q_empty);
-        };
-        // prologue: the first two tiles' QKs of both blocks
-        for (int j = 0; j < 2 && j < nmax && ok; ++j)
-          for (int b = 0; b < nb && ok; ++b) {
-            if (j >= n[b]) continue;
-            if (!(ok = qk_ready(b, tb[b] + j, kv_iter + j))) break;
-            issue_qk(b, tb[b] + j, (kv_iter + j) % NS);
-            after_qk(j, b);
+        for (int b = 0; b < nb; ++b) {
+          // S_b / P_b are free once the previous unit's last P_b * V has completed
+          const uint32_t spb = b ? sp1 : sp0;
+          if (spb > 0 && !wait_all(pv_done + b, (spb - 1) & 1, kDevTimeoutODone)) {
+            ok = false;
+            break;
           }
+          tc_fence_after();
+          issue_qk(b, kv_iter & 1);
+          commit(s_full + b);
+        }
+        if (!ok) break;
+        commit(k_empty + (kv_iter & 1));
+        if (nmax == 1) commit(q_empty);
         for (int j = 0; j < nmax && ok; ++j) {
           const uint32_t g = kv_iter + j;
-          const int s = g % NS;
-          if (!(ok = wait_all(v_full + s, (g / NS) & 1, kDevTimeoutVFull))) break;
+          const int s = g & 1;
+          bool v_ready = false;
           for (int b = 0; b < nb && ok; ++b) {
-            if (j >= n[b]) continue;
-            const uint32_t t = tb[b] + j;
-            if (!(ok = wait_all(p_full(b, t & 1), (t >> 1) & 1, kDevTimeoutPFull))) break;
+            const int nbt = b == 0 ? n0 : n1;
+            if (j >= nbt) continue;
+            const uint32_t ph = (b ? sp1 : sp0) + j;  // this block's barrier phase for tile j
+            if (!wait_all(p_lo + b, ph & 1, kDevTimeoutPFull)) {
+              ok = false;
+              break;
+            }
+            if (!v_ready && !wait_all(v_full + s, (g >> 1) & 1, kDevTimeoutVFull)) {
+              ok = false;
+              break;
+            }
+            v_ready = true;
             tc_fence_after();
-            issue_pv(b, t, s, j > 0);
-            if (j == n[b] - 1) commit(o_done(b));
-          }
-          if (!ok) break;
-          commit(v_empty + s);  // both blocks' P V of this tile are issued: the slot frees when they complete
-          // tile j + 2 into the S buffers tile j leaves (once its P V has completed)
-          for (int b = 0; b < nb && ok; ++b) {
-            if (j + 2 >= n[b]) continue;
-            if (!(ok = qk_ready(b, tb[b] + j + 2, g + 2))) break;
-            issue_qk(b, tb[b] + j + 2, (g + 2) % NS);
-            after_qk(j + 2, b);
+            issue_pv(b, s, j > 0, 0);  // keys 0..63
+            if (!wait_all(p_full + b, ph & 1, kDevTimeoutPFull)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_pv(b, s, true, 1);   // keys 64..127
+            commit(pv_done + b);
+            const bool last_pv = (b == nb - 1) || (j >= n1);
+            if (last_pv) commit(v_empty + s);
+            if (j == nbt - 1) {
+              commit(o_done + b);
+              continue;
+            }
+            // next key tile for this block; S_b / P_b are reused once P_b(j) * V has completed
+            const uint32_t g1 = g + 1;
+            const int s1 = g1 & 1;
+            const bool first_qk = (b == 0) || (j + 1 >= n0);
+            if (first_qk && !wait_all(k_full + s1, (g1 >> 1) & 1, kDevTimeoutKFull)) {
+              ok = false;
+              break;
+            }
+            if (!wait_all(pv_done + b, ph & 1, kDevTimeoutODone)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_qk(b, s1);
+            commit(s_full + b);
+            const bool last_qk = (b == nb - 1) || (j + 1 >= n1);
+            if (last_qk) {
+              commit(k_empty + s1);
+              if (j + 1 == nmax - 1) commit(q_empty);  // the unit's last QK: Q buffers free
+            }
           }
         }
-        tb[0] += n[0];
-        tb[1] += n[1];
+        sp0 += n0;
+        sp1 += n1;
         kv_iter += nmax;
       }
       // all tensor-core work this thread issued has finished before TMEM is released
@@ -408,13 +427,14 @@ __global__ void __launch_bounds__(384, 1)
     const int b = warp >> 2;
     const int r = threadIdx.x & 127;  // query row in the block == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_col = tmem + lane_base + b * 128;
     const uint32_t o_col = tmem + lane_base + 256 + b * D;
     const int mt = p.mask_type;
     const bool alibi = (mt == 3 || mt == 4 || mt == 5);
     const float scale = p.scale_log2;
     const bool raw_max = !alibi && scale > 0.f;  // max of the raw scores, scale folded into the exponent
     float* tbl = sTbl + warp * 2 * C::TBL_FLOATS;
-    uint32_t tp = 0;  // tiles this block processed in earlier units (barrier phases)
+    uint32_t sp = 0;  // tiles this block processed in earlier units (barrier phases)
     uint32_t up = 0;  // units this block took part in (o_done phases)
     bool ok = true;
     for (int ui = u_begin; ui < u_end && ok; ++ui) {
@@ -435,51 +455,50 @@ __global__ void __launch_bounds__(384, 1)
       float m_run = -INFINITY;  // running max in log2 units (the one P is computed against)
       float l_run = 0.f;
       for (int j = 0; j < n; ++j) {
-        const uint32_t t = tp + j;
-        const uint32_t s_col = tmem + lane_base + b * 128 + (t & 1) * KT;
-        const int j0 = j * KT;
-        float* tb = tbl + (t & 1) * C::TBL_FLOATS;
+        const uint32_t ph = sp + j;
+        const int j0 = j * 128;
+        float* t = tbl + (ph & 1) * C::TBL_FLOATS;
         if (mt == 4) {
-          // -slope*log2(e)*sqrt(distance) for distance = iabs_w + k - 63 - j0, k = lane - column + 63
+          // -slope*log2(e)*sqrt(distance) for distance = iabs_w + k - 127 - j0, k = lane - column + 127
           for (int k = lane; k < C::TBL_FLOATS; k += 32) {
-            const float dist = static_cast<float>(iabs_w - j0 + k - (KT - 1));
-            tb[k] = -slope_log2 * sqrtf(fmaxf(dist, 0.f));
+            const float dist = static_cast<float>(iabs_w - j0 + k - 127);
+            t[k] = -slope_log2 * sqrtf(fmaxf(dist, 0.f));
           }
           __syncwarp();
         }
-        ok = __all_sync(0xffffffffu, mbar_wait(s_full(b, t & 1), (t >> 1) & 1, status, kDevTimeoutSFull));
+        ok = __all_sync(0xffffffffu, mbar_wait(s_full + b, ph & 1, status, kDevTimeoutSFull));
         if (!ok) break;
         tc_fence_after();
-        float x[KT];
+        float x[128];
         {
-          uint32_t sr[2][32];
-          tmem_ld32(s_col, sr[0]);
-          tmem_ld32(s_col + 32, sr[1]);
-          tmem_ld_wait();  // one wait for both loads
+          uint32_t sr[4][32];
 #pragma unroll
-          for (int c = 0; c < KT; ++c) x[c] = __uint_as_float(sr[c >> 5][c & 31]);
+          for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(s_col + c4 * 32, sr[c4]);
+          tmem_ld_wait();  // one wait for all four loads
+#pragma unroll
+          for (int c = 0; c < 128; ++c) x[c] = __uint_as_float(sr[c >> 5][c & 31]);
         }
         const int lim = last_key - j0;  // columns c <= lim are allowed
         if (mt == 3 || mt == 5) {
           // right- and left-aligned bias differ by a per-row constant; both use (j - iabs)
           const float b0 = slope_log2 * static_cast<float>(j0 - iabs);
 #pragma unroll
-          for (int c = 0; c < KT; ++c) x[c] = fmaf(x[c], scale, fmaf(slope_log2, static_cast<float>(c), b0));
+          for (int c = 0; c < 128; ++c) x[c] = fmaf(x[c], scale, fmaf(slope_log2, static_cast<float>(c), b0));
         } else if (mt == 4) {
-          const float* tl = tb + lane + (KT - 1);
+          const float* tl = t + lane + 127;
 #pragma unroll
-          for (int c = 0; c < KT; ++c) x[c] = fmaf(x[c], scale, tl[-c]);
+          for (int c = 0; c < 128; ++c) x[c] = fmaf(x[c], scale, tl[-c]);
         } else if (!raw_max) {
 #pragma unroll
-          for (int c = 0; c < KT; ++c) x[c] *= scale;
+          for (int c = 0; c < 128; ++c) x[c] *= scale;
         }
-        if (lim < KT - 1) {
+        if (lim < 127) {
 #pragma unroll
-          for (int c = 0; c < KT; ++c) x[c] = (c > lim) ? -INFINITY : x[c];
+          for (int c = 0; c < 128; ++c) x[c] = (c > lim) ? -INFINITY : x[c];
         }
         float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < KT; c += 8) {
+        for (int c = 0; c < 128; c += 8) {
           mx0 = max3(mx0, x[c], x[c + 1]);
           mx1 = max3(mx1, x[c + 2], x[c + 3]);
           mx2 = max3(mx2, x[c + 4], x[c + 5]);
@@ -494,12 +513,8 @@ __global__ void __launch_bounds__(384, 1)
           m_run = m_new;
         }
         const float m_base = (m_run == -INFINITY) ? 0.f : m_run;
+        // O_b is quiescent here: P_b(j-1) * V completed before S_b(j) was written
         if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
-          // O_b must hold P_b(j-1) V(j-1) before it is scaled; P_b(j) V cannot start before P_b(j) below
-          ok = __all_sync(0xffffffffu,
-                          mbar_wait(pv_done(b, (t - 1) & 1), ((t - 1) >> 1) & 1, status, kDevTimeoutODone));
-          if (!ok) break;
-          tc_fence_after();
 #pragma unroll
           for (int c32 = 0; c32 < D / 32; ++c32) {
             uint32_t regs[32];
@@ -513,14 +528,14 @@ __global__ void __launch_bounds__(384, 1)
         // P = 2^(x*scale - m) (raw scores) or 2^(x - m) (biased scores), written over S in TMEM
         const uint64_t scale2 = f2pack(raw_max ? scale : 1.f, raw_max ? scale : 1.f);
         const uint64_t negm2 = f2pack(-m_base, -m_base);
-        const float row_sum = exp_row<T>(x, scale2, negm2, s_col);
+        const float row_sum = exp_rows<T>(x, scale2, negm2, s_col, p_lo + b);
         l_run = l_run * alpha + row_sum;
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(p_full(b, t & 1));
+        mbar_arrive(p_full + b);
       }
-      tp += n;
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done(b), up & 1, status, kDevTimeoutODone));
+      sp += n;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done + b, up & 1, status, kDevTimeoutODone));
       ++up;
       if (!ok) break;
       tc_fence_after();

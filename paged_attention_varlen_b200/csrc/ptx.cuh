@@ -109,25 +109,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
-// Same contract as mbar_wait, but the thread polls without being suspended, so
-// it resumes within a few cycles of the phase completing (for waits on the
-// critical path of a pipeline; each poll takes an issue slot of the warp's
-// scheduler).  The status word and the clock are checked every 1024 polls.
-__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* status, int code) {
-  if (mbar_test_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_test_wait(bar, parity)) return true;
-    if ((it & 1023u) == 0) {
-      if (*status != 0) return false;
-      if (global_timer_ns() - t0 > ALA_WAIT_LIMIT_NS) {
-        atomicCAS((int*)status, 0, code);
-        return false;
-      }
-    }
-  }
-}
-
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
@@ -369,28 +350,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
-}
-
-// 2^x for two values on the FMA pipe instead of the MUFU unit.  x = n + f with
-// n = round(x) taken with the 1.5*2^23 shifter, f in [-1/2, 1/2]; 2^f from a
-// degree-3 minimax polynomial (relative error 7.5e-5 in float32, coefficients
-// from csrc/exp2_poly_fit.py); 2^n added into the exponent field.  Inputs must
-// be >= -125 (the caller clamps), so the result stays a normal float.
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
-  const uint64_t shifter = f2pack(12582912.f, 12582912.f);
-  const uint64_t neg_shifter = f2pack(-12582912.f, -12582912.f);
-  const uint64_t t = add_x2(x, shifter);
-  const uint64_t n = add_x2(t, neg_shifter);
-  const uint64_t f = fma_x2(n, f2pack(-1.f, -1.f), x);
-  uint64_t p = fma_x2(f2pack(5.517166853e-02f, 5.517166853e-02f), f, f2pack(2.426111251e-01f, 2.426111251e-01f));
-  p = fma_x2(p, f, f2pack(6.932609677e-01f, 6.932609677e-01f));
-  p = fma_x2(p, f, f2pack(9.999280572e-01f, 9.999280572e-01f));
-  float t0, t1, p0, p1;
-  f2unpack(t, t0, t1);
-  f2unpack(p, p0, p1);
-  p0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  p1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-  return f2pack(p0, p1);
 }
 
 }  // namespace ala

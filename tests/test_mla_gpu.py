@@ -57,8 +57,7 @@ def test_mla_small_ragged(qs, block_size):
 
 @pytest.mark.parametrize("heads,dtype", [(64, torch.bfloat16), (128, torch.float16), (384, torch.bfloat16)])
 def test_mla_decode_row_kernels(heads, dtype):
-    # one token per batch: 64 heads run on the 64-row kernel, multiples of 128 on the 128-row kernel whose
-    # CTA pairs split the output columns (384 heads: three head groups, six CTAs per key range)
+    # one token per batch: 64-row blocks of one token's heads (384 heads: six head groups per key range)
     ctx = np.array([1, 64, 65, 700, 2500, 129], dtype=np.int32)
     case = synth.make_mla(f"rows_{heads}", ctx, 1, heads, 89, block_size=64, dtype=dtype)
     out, lse, _ = _run(case)
