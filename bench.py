@@ -22,7 +22,8 @@ Also reported on rank 0:
   * cpu_baseline: the fp64 oracle on the host cores over a bounded sample of
     the same workload's rows;
   * extra: the other workloads (paged ALiBi prefix encoder fp16, long ALiBi
-    bf16 in both variants, MLA decode/spec when built) measured the same way.
+    bf16 in both variants, the causal batch at head size 256, MLA decode/spec
+    when built) measured the same way.
 """
 from __future__ import annotations
 
@@ -48,7 +49,9 @@ import synth  # noqa: E402
 PROFILE = os.path.join(ROOT, "profiles", "prefill_varlen_causal_bf16.md")
 MLA_PROFILE = os.path.join(ROOT, "profiles", "mla_decode_qs1_bf16.md")
 MLA_INT8_PROFILE = os.path.join(ROOT, "profiles", "mla_decode_qs1_int8.md")
+PROFILE_D256 = os.path.join(ROOT, "profiles", "prefill_d256_varlen_causal_bf16.md")
 KERNEL_SOURCES = ["paged_attention_varlen_b200/csrc/prefill.cu", "paged_attention_varlen_b200/csrc/ptx.cuh"]
+D256_KERNEL_SOURCES = ["paged_attention_varlen_b200/csrc/prefill_d256.cu", "paged_attention_varlen_b200/csrc/ptx.cuh"]
 MLA_KERNEL_SOURCES = ["paged_attention_varlen_b200/csrc/mla.cu", "paged_attention_varlen_b200/csrc/mla_common.cuh",
                       "paged_attention_varlen_b200/csrc/ptx.cuh"]
 DEFAULT_WORKLOAD = "varlen_causal_bf16"
@@ -57,6 +60,7 @@ WORKLOADS = {
     "prefix_paged_alibi_fp16": lambda: synth.prefix_paged_alibi_fp16(),
     "long_alibi_sqrt_bf16": lambda: synth.long_alibi_bf16(synth.MASK_ALIBI_SQRT),
     "long_alibi_left_bf16": lambda: synth.long_alibi_bf16(synth.MASK_ALIBI_LEFT),
+    "varlen_causal_bf16_d256": lambda: synth.varlen_causal_bf16(heads=16, kv_heads=4, head_size=256),
     "mla_decode_qs1_bf16": lambda: synth.mla_decode_bf16(1),
     "mla_spec_qs4_bf16": lambda: synth.mla_decode_bf16(4),
     "mla_decode_qs1_int8": lambda: synth.mla_decode_int8(),
@@ -506,12 +510,14 @@ def main():
                         "kernel_source_sha256": src}
             launches = args.steps * (2 if op_has_combine(op) else 1)
         else:
-            src = kernel_source_hash()
+            d256 = case.head_size > 128
+            src = kernel_source_hash(D256_KERNEL_SOURCES if d256 else KERNEL_SOURCES)
             achieved = flops / (mean_ms * 1e-3) / 1e12
             roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                        "frac": achieved / peaks["bf16_tflops"], "traffic": profiled_traffic(PROFILE, src),
+                        "frac": achieved / peaks["bf16_tflops"],
+                        "traffic": profiled_traffic(PROFILE_D256 if d256 else PROFILE, src),
                         "algorithmic_bytes": nbytes, "peak_source": peaks["source"] + " (burst bf16)",
-                        "kernel": "prefill_kernel", "kernel_source_sha256": src}
+                        "kernel": "prefill_d256_kernel" if d256 else "prefill_kernel", "kernel_source_sha256": src}
             launches = args.steps
         line = {"metric": metric, "value": value, "unit": unit,
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -550,7 +556,8 @@ def extra_workloads(ala, device, flush, stream, peaks, main_case, args):
         "valid_tflops": prefill_flops(main_case) / (ms * 1e-3) / 1e12}
     del op
     for case in (synth.prefix_paged_alibi_fp16(), synth.long_alibi_bf16(synth.MASK_ALIBI_SQRT),
-                 synth.long_alibi_bf16(synth.MASK_ALIBI_LEFT)):
+                 synth.long_alibi_bf16(synth.MASK_ALIBI_LEFT),
+                 synth.varlen_causal_bf16(heads=16, kv_heads=4, head_size=256)):
         op, t = plan_case(ala, case, device)
         ms = statistics.mean(time_steps(op, steps, 3, flush, stream))
         tf = prefill_flops(case) / (ms * 1e-3) / 1e12

@@ -122,7 +122,7 @@ ALA_API int ala_workspace_status(const ala_op* op, const void* workspace, ala_st
  *             [numBlocks, blockSize, kvHeadNum, headSize], same dtype, device.
  *             Key position j of sequence b is slot j % blockSize of block
  *             blockTables[b][j / blockSize].  blockSize must be a multiple
- *             of 16 that divides 64, or a multiple of 64.
+ *             of 16 that divides 128, or a multiple of 128.
  * blockTables [batch, maxBlockNum] int32, device.  Entries past
  *             ceil(kvSeqLen_b / blockSize) are never read; entries read must
  *             be in [0, numBlocks).
@@ -138,9 +138,10 @@ ALA_API int ala_workspace_status(const ala_op* op, const void* workspace, ala_st
  * headNum     > 0; kvHeadNum > 0 and divides headNum (query head h reads kv
  *             head h / (headNum/kvHeadNum)).
  * qkScale     multiplies Q K^T before the bias is added.
- * headSize    a multiple of 16 up to 128 (ALiBi masks: <= 128, per the
- *             compressed-mask page's constraints); 64 and 128 run natively,
- *             others on the next of those with zero-filled extra dimensions.
+ * headSize    a multiple of 16 up to 256 (ALiBi masks: <= 128, per the
+ *             compressed-mask page's constraints); 64, 128 and 256 run
+ *             natively, others on the next of those with zero-filled extra
+ *             dimensions.
  * attnOut     same shape and dtype as query, device, 32-byte aligned.
  * ------------------------------------------------------------------------- */
 ALA_API int atb_like_prefix_encoder_get_workspace_size(

@@ -21,7 +21,7 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libala.so")
 BUILD_DEBUG = os.path.join(HERE, "_build_debug")
 LIB_DEBUG = os.path.join(HERE, "libala_debug.so")
-SOURCES = ["api.cpp", "prefill.cu", "mla.cu", "noalloc.cu", "merge.cu"]
+SOURCES = ["api.cpp", "prefill.cu", "prefill_d256.cu", "mla.cu", "noalloc.cu", "merge.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

@@ -305,7 +305,7 @@ int build_prefill(ala_op* op, const ala_tensor* query, const ala_tensor* key, co
   }
   if (prefill_kernel_d(dt, head_size) == 0)
     return fail(ALA_UNSUPPORTED,
-                "%s: headSize %lld with this dtype is not built (bf16/f16: a multiple of 16 up to 128; f32: a "
+                "%s: headSize %lld with this dtype is not built (bf16/f16: a multiple of 16 up to 256; f32: a "
                 "multiple of 8 up to 64)",
                 fn, (long long)head_size);
 
@@ -334,9 +334,10 @@ int build_prefill(ala_op* op, const ala_tensor* query, const ala_tensor* key, co
   // its last allowed key (prefill_units)
   std::vector<SeqInfo> seqs(batch);
   for (int32_t b = 0, cq = 0, ckv = 0; b < batch; cq += sl[b], ckv += kl[b], ++b) seqs[b] = SeqInfo{cq, sl[b], kl[b], ckv};
+  const PrefillShape shape = prefill_shape(prefill_kernel_d(dt, head_size));
   std::vector<PrefillUnit> units;
-  units.reserve(prefill_unit_count(batch, sl, headNum, kvHeadNum));
-  prefill_units(batch, sl, kl, maskType, headNum, kvHeadNum, [&](const PrefillUnit& u) { units.push_back(u); });
+  units.reserve(prefill_unit_count(batch, sl, headNum, kvHeadNum, shape));
+  prefill_units(batch, sl, kl, maskType, headNum, kvHeadNum, shape, [&](const PrefillUnit& u) { units.push_back(u); });
   // Persistent grid: one CTA per SM, each running a list of units.  Units are
   // assigned longest first to the least loaded CTA (greedy LPT); a unit costs
   // its key tiles plus about one tile of fixed work (Q load, epilogue).
@@ -385,7 +386,8 @@ int run_prefill(void* workspace, uint64_t workspaceSize, ala_op* op, ala_stream_
   if (reinterpret_cast<uintptr_t>(workspace) % 16) return fail(ALA_INVALID_PARAM, "%s: workspace must be 16-byte aligned", fn);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (!op->maps_ready) {
-    const int kv_box = op->paged ? std::min(op->block_size, kPrefillTileKeys) : kPrefillTileKeys;
+    const int tk = prefill_shape(prefill_kernel_d(op->dtype, op->head_size)).tile_keys;
+    const int kv_box = op->paged ? std::min(op->block_size, tk) : tk;
     const int64_t q_rows = op->n_tokens;
     if (!encode_rows_heads_d(&op->tmQ, op->q, op->dtype, q_rows, op->heads, op->head_size, 128, false) ||
         !encode_rows_heads_d(&op->tmK, op->k, op->dtype, op->kv_rows, op->kv_heads, op->head_size, kv_box, false) ||

@@ -101,24 +101,38 @@ struct PrefillParams {
   int32_t d_out;                // head size of the tensors (<= the kernel's D; dims past it are zero-filled)
 };
 
+// Tiling of the prefill kernel instance that serves kernel head size D (prefill_kernel_d): keys per K/V
+// tile and whether a unit holds one block of 128 query rows (D = 256, whose O takes half of tensor memory)
+// or up to two.
+struct PrefillShape {
+  int32_t tile_keys;
+  bool one_block;
+};
+inline PrefillShape prefill_shape(int32_t D) { return D > 128 ? PrefillShape{64, true} : PrefillShape{kPrefillTileKeys, false}; }
+
 // Work units of one prefill request, in sequence order (every prefill entry point uses this list).
 // Per sequence b, blocks of 128 query rows; two blocks that read the same kv head form a unit: two
 // query heads of a GQA group on the same rows, or, without grouping, two consecutive row tiles of one
-// head.  Each block visits the key tiles up to its last allowed key (the causal rule with the prefix
-// offset kvSeqLen - seqLen; every key for mask type 0).  `emit(const PrefillUnit&)` receives them.
+// head (one block per unit with shape.one_block).  Each block visits the key tiles up to its last
+// allowed key (the causal rule with the prefix offset kvSeqLen - seqLen; every key for mask type 0).
+// `emit(const PrefillUnit&)` receives them.
 template <class Emit>
 inline void prefill_units(int32_t batch, const int32_t* seq_len, const int32_t* kv_len, int mask_type,
-                          int32_t heads, int32_t kv_heads, Emit&& emit) {
+                          int32_t heads, int32_t kv_heads, PrefillShape shape, Emit&& emit) {
   const int32_t group = heads / kv_heads;
+  const int32_t tk = shape.tile_keys;
   for (int32_t b = 0; b < batch; ++b) {
     const int32_t sl = seq_len[b], kl = kv_len[b], off = kl - sl;
     auto tiles_for = [&](int32_t q0) {
       const int32_t last_row = (q0 + 127 < sl - 1) ? q0 + 127 : sl - 1;
       const int32_t causal_end = last_row + off + 1;
       const int32_t kv_end = (mask_type == 0 || kl < causal_end) ? kl : causal_end;
-      return (kv_end + kPrefillTileKeys - 1) / kPrefillTileKeys;
+      return (kv_end + tk - 1) / tk;
     };
-    if (group >= 2) {
+    if (shape.one_block) {
+      for (int32_t h = 0; h < heads; ++h)
+        for (int32_t q0 = 0; q0 < sl; q0 += 128) emit(PrefillUnit{b, 1, {q0, q0}, {h, h}, {tiles_for(q0), 0}});
+    } else if (group >= 2) {
       for (int32_t q0 = 0; q0 < sl; q0 += 128) {
         const int32_t nt = tiles_for(q0);
         for (int32_t g = 0; g < kv_heads; ++g)
@@ -139,12 +153,14 @@ inline void prefill_units(int32_t batch, const int32_t* seq_len, const int32_t* 
 }
 
 // Number of units prefill_units emits (no list is built).
-inline int64_t prefill_unit_count(int32_t batch, const int32_t* seq_len, int32_t heads, int32_t kv_heads) {
+inline int64_t prefill_unit_count(int32_t batch, const int32_t* seq_len, int32_t heads, int32_t kv_heads,
+                                  PrefillShape shape) {
   const int32_t group = heads / kv_heads;
   int64_t n = 0;
   for (int32_t b = 0; b < batch; ++b)
-    n += group >= 2 ? (int64_t)((seq_len[b] + 127) / 128) * kv_heads * ((group + 1) / 2)
-                    : (int64_t)heads * ((seq_len[b] + 255) / 256);
+    n += shape.one_block ? (int64_t)heads * ((seq_len[b] + 127) / 128)
+         : group >= 2    ? (int64_t)((seq_len[b] + 127) / 128) * kv_heads * ((group + 1) / 2)
+                         : (int64_t)heads * ((seq_len[b] + 255) / 256);
   return n;
 }
 
@@ -160,10 +176,13 @@ bool encode_rows_heads_d(CUtensorMap* map, void* base, int32_t dtype, int64_t ro
 enum : int32_t { kF16 = 0, kBF16 = 1, kF32 = 2, kI32 = 3 };
 
 // Head size D of the prefill kernel instance that serves head size `d` of element type `dtype` (0 if none
-// does): 16-bit types take d a multiple of 16 up to 128 (D = 64 or 128), fp32 a multiple of 8 up to 64
-// (D = 64).  The tensor maps are encoded over the real d, so the dimensions d..D-1 of every Q, K and V
+// does): 16-bit types take d a multiple of 16 up to 256 (D = 64, 128 or 256), fp32 a multiple of 8 up to
+// 64 (D = 64).  The tensor maps are encoded over the real d, so the dimensions d..D-1 of every Q, K and V
 // tile are zero-filled by the TMA loads and contribute nothing; the epilogue stores the first d columns.
 int prefill_kernel_d(int32_t dtype, int64_t d);
+// The D = 256 instance (prefill_d256.cu): one block of 128 rows per unit, 64-key tiles.
+cudaError_t launch_prefill_d256(int32_t dtype, const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                const PrefillParams& p, cudaStream_t stream);
 // Launches the prefill kernel for element type `dtype` and kernel head size `D` (prefill_kernel_d).
 cudaError_t launch_prefill(int32_t dtype, int32_t D, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                            const CUtensorMap& tmV, const PrefillParams& p, cudaStream_t stream);

@@ -155,7 +155,8 @@ extern "C" ALA_API int varlen_attention_noalloc(const ala_tensor* query, const a
 
   // ---- count the work units first, so an oversized call is rejected before anything is written
   const int32_t group = headNum / kvHeadNum;
-  const int64_t n_units = prefill_unit_count(batch, sl, headNum, kvHeadNum);
+  const PrefillShape shape = prefill_shape(prefill_kernel_d(dt, d));
+  const int64_t n_units = prefill_unit_count(batch, sl, headNum, kvHeadNum, shape);
   if (n_units > (int64_t)kMaxUnits)
     return nfail(ALA_UNSUPPORTED, "%s: the call needs %lld work units; the fixed %zu-byte scratch holds at most %zu", fn,
                  (long long)n_units, kNoAllocScratchBytes, kMaxUnits);
@@ -189,7 +190,7 @@ extern "C" ALA_API int varlen_attention_noalloc(const ala_tensor* query, const a
   PrefillUnit* units = reinterpret_cast<PrefillUnit*>(g_stage + kStatusBytes + kSeqBytes);
   size_t nu = 0;
   for (int32_t b = 0, cq = 0, ckv = 0; b < batch; cq += sl[b], ckv += kl[b], ++b) seqs[b] = SeqInfo{cq, sl[b], kl[b], ckv};
-  prefill_units(batch, sl, kl, maskType, headNum, kvHeadNum, [&](const PrefillUnit& u) { units[nu++] = u; });
+  prefill_units(batch, sl, kl, maskType, headNum, kvHeadNum, shape, [&](const PrefillUnit& u) { units[nu++] = u; });
   // longest first; ties in a fixed order so every call gets the same schedule
   std::sort(units, units + nu, [](const PrefillUnit& a, const PrefillUnit& c) {
     const int64_t ca = prefill_unit_cost(a), cc = prefill_unit_cost(c);
@@ -201,8 +202,8 @@ extern "C" ALA_API int varlen_attention_noalloc(const ala_tensor* query, const a
 
   CUtensorMap tmQ, tmK, tmV;
   if (!encode_rows_heads_d(&tmQ, query->data, dt, n_tokens, headNum, d, 128, false) ||
-      !encode_rows_heads_d(&tmK, key->data, dt, key->dims[0], kvHeadNum, d, kPrefillTileKeys, false) ||
-      !encode_rows_heads_d(&tmV, value->data, dt, key->dims[0], kvHeadNum, d, kPrefillTileKeys, true))
+      !encode_rows_heads_d(&tmK, key->data, dt, key->dims[0], kvHeadNum, d, shape.tile_keys, false) ||
+      !encode_rows_heads_d(&tmV, value->data, dt, key->dims[0], kvHeadNum, d, shape.tile_keys, true))
     return nfail(ALA_CUDA_ERROR, "%s: cuTensorMapEncodeTiled failed (pointers must be 16-byte aligned)", fn);
 
   const size_t bytes = kStatusBytes + kSeqBytes + nu * sizeof(PrefillUnit);

@@ -609,8 +609,8 @@ cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtenso
 
 int prefill_kernel_d(int32_t dtype, int64_t d) {
   if (dtype == kBF16 || dtype == kF16) {
-    if (d <= 0 || d % 16 != 0 || d > 128) return 0;
-    return d <= 64 ? 64 : 128;
+    if (d <= 0 || d % 16 != 0 || d > 256) return 0;
+    return d <= 64 ? 64 : d <= 128 ? 128 : 256;
   }
   if (dtype == kF32) return (d > 0 && d % 8 == 0 && d <= 64) ? 64 : 0;
   return 0;
@@ -618,6 +618,7 @@ int prefill_kernel_d(int32_t dtype, int64_t d) {
 
 cudaError_t launch_prefill(int32_t dtype, int32_t d, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                            const CUtensorMap& tmV, const PrefillParams& p, cudaStream_t stream) {
+  if (d == 256) return launch_prefill_d256(dtype, tmQ, tmK, tmV, p, stream);
   if (dtype == kBF16) {
     if (d == 128) return launch<__nv_bfloat16, 128>(tmQ, tmK, tmV, p, stream);
     if (d == 64) return launch<__nv_bfloat16, 64>(tmQ, tmK, tmV, p, stream);

@@ -142,12 +142,13 @@ def tiny_causal_fp32(seed=1000) -> PrefillCase:
                         seed, qk_scale=1.0 / 8.0)
 
 
-def varlen_causal_bf16(seed=1001, batch=8, lo=64, hi=2048) -> PrefillCase:
-    """batch 8, seqLen ~ U{64..2048}, H=32, Hkv=8, d=128, bf16, causal, contiguous."""
+def varlen_causal_bf16(seed=1001, batch=8, lo=64, hi=2048, heads=32, kv_heads=8, head_size=128) -> PrefillCase:
+    """batch 8, seqLen ~ U{64..2048}, H=32, Hkv=8, d=128, bf16, causal, contiguous (heads and head size
+    adjustable: the d=256 variant keeps the lengths and takes H=16, Hkv=4)."""
     rng = np.random.Generator(np.random.PCG64(seed))
     L = rng.integers(lo, hi + 1, size=batch).astype(np.int32)
-    return make_prefill(f"varlen_causal_bf16_b{batch}_h32kv8_d128", L, L, 32, 8, 128, torch.bfloat16,
-                        MASK_CAUSAL, seed, rng=rng)
+    return make_prefill(f"varlen_causal_bf16_b{batch}_h{heads}kv{kv_heads}_d{head_size}", L, L, heads, kv_heads,
+                        head_size, torch.bfloat16, MASK_CAUSAL, seed, rng=rng)
 
 
 def padded_from(case: PrefillCase) -> PrefillCase:

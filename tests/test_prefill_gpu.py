@@ -107,6 +107,18 @@ def test_head_sizes_between_the_kernel_sizes(d, dtype, mask_type, paged):
     _full_check(case, LSE_REL_TF32 if dtype == torch.float32 else LSE_REL)
 
 
+@pytest.mark.parametrize("d,dtype,mask_type,paged,block_size", [
+    (256, torch.bfloat16, 9, False, 128), (256, torch.float16, 0, False, 128), (256, torch.bfloat16, 9, True, 16),
+    (256, torch.float16, 9, True, 128), (192, torch.bfloat16, 9, True, 64), (144, torch.float16, 0, False, 128)])
+def test_large_head_sizes(d, dtype, mask_type, paged, block_size):
+    # head sizes above 128 run on the D = 256 kernel (one 128-row block per CTA, 64-key tiles); GQA group 4
+    L = [1, 63, 64, 65, 128, 129, 400, 7]
+    pre = [0, 0, 1, 200, 64, 77, 129, 3]
+    case = synth.make_prefill(f"d{d}", L, [a + b for a, b in zip(L, pre)], 8, 2, d, dtype, mask_type, 311 + d,
+                              paged=paged, block_size=block_size)
+    _full_check(case)
+
+
 def test_paged_equals_contiguous_on_gpu():
     L, pre = [100, 250], [300, 17]
     kv = [a + b for a, b in zip(L, pre)]

@@ -10,9 +10,9 @@ workloads, and compare each result element by element with the fp64 oracle
 and with the regular varlen_attention entry point on the same inputs, within
 the parity tolerance; the status word read back through
 varlen_attention_noalloc_status must be 0 after each call.  They also cover a
-call without lse (mask type 0, fp32 inputs on tf32), and the refusals: a
-schedule larger than the fixed scratch, an lse of the wrong shape, and a
-stream that is being captured.  This file is collected last so that, if it
+call without lse (mask type 0, fp32 inputs on tf32), a head size of 256, and
+the refusals: a schedule larger than the fixed scratch, an lse of the wrong
+shape, and a stream that is being captured.  This file is collected last so that, if it
 fails, a run that stops at the first failure has already run every other
 test; it passes alone in a fresh process as well.
 """
@@ -89,6 +89,15 @@ def test_noalloc_without_lse_fp32_no_mask():
     out, _ = _noalloc(case, with_lse=False)
     ref, _ = _oracle(case)
     check_out(out.reshape(-1, 64), ref)
+
+
+def test_noalloc_head_size_256_causal():
+    # the D = 256 kernel: one 128-row block per unit, 64-key K/V tiles
+    case = synth.make_prefill("na6", [1, 200, 129], [30, 200, 300], 4, 2, 256, torch.bfloat16, synth.MASK_CAUSAL, 76)
+    out, lse = _noalloc(case)
+    ref, lref = _oracle(case)
+    check_out(out.reshape(-1, 256), ref)
+    check_lse(lse.reshape(-1), lref)
 
 
 def test_noalloc_refuses_a_schedule_larger_than_its_scratch():
