@@ -5,19 +5,23 @@
 //
 // O of one 128-row block takes 256 of the 512 tensor-memory columns, so a CTA
 // computes one block of 128 query rows (not two, as the D <= 128 kernel does)
-// and keeps two S buffers of 64 keys in the other half:
+// and keeps four S buffers of 64 keys in the other half:
 //
-//   TMEM columns [0, 64) S[0], [64, 128) S[1], [256, 512) O
-//   shared memory Q 64 KB, K and V rings of 2 x 32 KB each (64-key tiles)
+//   TMEM columns [64 s, 64 s + 64) S[s] for s = 0..3, [256, 512) O
+//   shared memory Q 64 KB, a K ring of 3 x 32 KB and a V ring of 2 x 32 KB
+//                (64-key tiles)
 //
-//   warp 4       TMA producer: the Q tile once per unit, then K and V tiles;
-//                paged rows are gathered page by page through the block table.
+//   warps 4, 6   TMA producers: warp 4 the K tiles and each unit's Q tile,
+//                warp 6 the V tiles; paged rows are gathered page by page
+//                through the block table.
 //   warp 5       tcgen05 issuer.  Per key tile j:
-//                  S[j%2] = Q K_j^T       (SS MMA, M = 128, N = 64)
-//                  O     += P V_j         (TS MMA, N = 256: P read from TMEM over S[j%2])
-//                in the order PV(j), QK(j+2): the S buffer of tile j is refilled
-//                with tile j+2 once P(j) V has completed, while the softmax
-//                works on tile j+1.
+//                  S[j%4] = Q K_j^T       (SS MMA, M = 128, N = 64)
+//                  O     += P V_j         (TS MMA, N = 256: P read from TMEM over S[j%4])
+//                in the order PV(j), QK(j+2).  QK(j+2) refills the buffer of
+//                tile j-2, whose P V completed well before, so the issuer never
+//                waits for the P V it has just issued and the tensor pipe gets
+//                PV(j) and QK(j+2) back to back while the softmax works on
+//                tile j+1.
 //   warps 0..3   softmax: thread r owns row r (TMEM lane r).  It reads its S
 //                row, applies qkScale and the causal / prefix-offset rule in
 //                registers, updates the running max and sum, rescales O in TMEM
@@ -45,18 +49,20 @@ constexpr int AW = 64;                     // 16-bit elements in one 128-byte sw
 constexpr int UK = 16;                     // K extent of one MMA instruction (16-bit types)
 constexpr int BLK_Q = 128 * 128;           // bytes of one 128-row x 128-byte swizzle column block
 constexpr int BLK_KV = KT * 128;           // bytes of one 64-key x 128-byte swizzle column block
-constexpr int NS = 2;                      // K and V ring depth
+constexpr int NSK = 3;                     // K ring depth
+constexpr int NSV = 2;                     // V ring depth
+constexpr int NSB = 4;                     // S buffers in tensor memory
 constexpr int Q_BYTES = 128 * D * 2;
 constexpr int KV_BYTES = KT * D * 2;
-// q_full, q_empty, fin, k_full[NS], v_full[NS], k_empty[NS], v_empty[NS], s_full[2], p_full[2], pv_done[2],
-// o_done
-constexpr int N_BARS = 3 + 4 * NS + 7;
-constexpr int SMEM = 1024 + Q_BYTES + 2 * NS * KV_BYTES + N_BARS * 8 + 16;
+// q_full, q_empty, fin, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], s_full[NSB], p_full[NSB],
+// pv_done[NSB], o_done
+constexpr int N_BARS = 3 + 2 * NSK + 2 * NSV + 3 * NSB + 1;
+constexpr int SMEM = 1024 + Q_BYTES + (NSK + NSV) * KV_BYTES + N_BARS * 8 + 16;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t O_COL = 256;
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
 static_assert(SMEM <= 232448, "shared memory budget");
-static_assert(O_COL + D <= TMEM_COLS && 2 * KT <= O_COL, "tensor memory budget");
+static_assert(O_COL + D <= TMEM_COLS && NSB * KT <= O_COL, "tensor memory budget");
 
 template <typename T>
 struct Fmt;
@@ -132,20 +138,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sK = sQ + Q_BYTES;  // [NS][KV_BYTES]
-  uint8_t* sV = sK + NS * KV_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + NS * KV_BYTES);
+  uint8_t* sK = sQ + Q_BYTES;  // [NSK][KV_BYTES]
+  uint8_t* sV = sK + NSK * KV_BYTES;  // [NSV][KV_BYTES]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + NSV * KV_BYTES);
   uint64_t* q_full = bars;
   uint64_t* q_empty = bars + 1;
   uint64_t* fin = bars + 2;
-  uint64_t* k_full = bars + 3;       // [NS]
-  uint64_t* v_full = k_full + NS;    // [NS]
-  uint64_t* k_empty = v_full + NS;   // [NS]
-  uint64_t* v_empty = k_empty + NS;  // [NS]
-  uint64_t* s_full = v_empty + NS;   // [2] S[s] computed
-  uint64_t* p_full = s_full + 2;     // [2] P written over S[s]
-  uint64_t* pv_done = p_full + 2;    // [2] the P V of S[s]'s tile completed
-  uint64_t* o_done = pv_done + 2;    // the unit's last P V completed
+  uint64_t* k_full = bars + 3;         // [NSK]
+  uint64_t* k_empty = k_full + NSK;    // [NSK]
+  uint64_t* v_full = k_empty + NSK;    // [NSV]
+  uint64_t* v_empty = v_full + NSV;    // [NSV]
+  uint64_t* s_full = v_empty + NSV;    // [NSB] S[s] computed
+  uint64_t* p_full = s_full + NSB;     // [NSB] P written over S[s]
+  uint64_t* pv_done = p_full + NSB;    // [NSB] the P V of S[s]'s tile completed
+  uint64_t* o_done = pv_done + NSB;    // the unit's last P V completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + N_BARS);
 
   const int warp = threadIdx.x >> 5;
@@ -158,13 +164,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     mbar_init(fin, 1);
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < NSK; ++s) {
       mbar_init(k_full + s, 1);
-      mbar_init(v_full + s, 1);
       mbar_init(k_empty + s, 1);
+    }
+    for (int s = 0; s < NSV; ++s) {
+      mbar_init(v_full + s, 1);
       mbar_init(v_empty + s, 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NSB; ++s) {
       mbar_init(s_full + s, 1);
       mbar_init(p_full + s, 128);
       mbar_init(pv_done + s, 1);
@@ -182,20 +190,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   (void)lane;
 
-  // Barrier phases run on across units: the K/V rings by a global tile counter g (slot g % NS, phase
-  // g / NS), the S/P/PV barriers by the same counter (buffer g % 2, phase g / 2), q_full / q_empty and
-  // o_done by unit counters.
-  if (warp == 4) {
-    // ------------------------------------------------------------ producer
+  // Barrier phases run on across units: the K and V rings by a global tile counter g (slot g % depth,
+  // phase g / depth), the S/P/PV barriers by the same counter (buffer g % NSB, phase g / NSB), q_full /
+  // q_empty and o_done by unit counters.
+  if (warp == 4 || warp == 6) {
+    // ------------------------------------------------------------ producers
+    // warp 4 loads K (3-deep ring) and each unit's Q; warp 6 loads V (2-deep ring).  Two warps, so a K
+    // load never waits behind a V slot: K(j+3) can start as soon as QK(j) has completed.
+    const bool is_k = warp == 4;
+    const int depth = is_k ? NSK : NSV;
+    uint8_t* ring = is_k ? sK : sV;
+    uint64_t* full_bar = is_k ? k_full : v_full;
+    uint64_t* empty_bar = is_k ? k_empty : v_empty;
+    const CUtensorMap* map = is_k ? &tmK : &tmV;
     const bool leader = elect_one();
     if (leader) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(map);
+      if (is_k) tma_prefetch_desc(&tmQ);
     }
     bool ok = true;
     uint32_t kv_iter = 0;
-    uint32_t issued_k = 0, issued_v = 0;
+    uint32_t issued = 0;
     int q_loads = 0;
     for (int ui = u_begin; ui < u_end && ok; ++ui) {
       const PrefillUnit u = p.units[ui];
@@ -206,20 +221,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n_pages = bt ? (si.kv_len + p.block_size - 1) / p.block_size : 0;
       for (int j = 0; j < n && ok; ++j) {
         const uint32_t g = kv_iter + j;
-        const int s = g % NS;
-        for (int kv = 0; kv < 2; ++kv) {
-          if (g >= NS && !__all_sync(0xffffffffu, mbar_wait((kv ? v_empty : k_empty) + s, ((g / NS) - 1) & 1, status,
-                                                            kv ? kDevTimeoutVEmpty : kDevTimeoutKEmpty))) {
-            ok = false;
-            break;
-          }
-          uint64_t* full = (kv ? v_full : k_full) + s;
-          if (leader) mbar_expect_tx(full, KV_BYTES);
-          load_kv_tile(kv ? &tmV : &tmK, (kv ? sV : sK) + s * KV_BYTES, full, j, si, p, bt, n_pages, kvh, leader);
-          if (kv) issued_v = g + 1; else issued_k = g + 1;
+        const int s = g % depth;
+        if (g >= (uint32_t)depth &&
+            !__all_sync(0xffffffffu, mbar_wait(empty_bar + s, ((g / depth) - 1) & 1, status,
+                                               is_k ? kDevTimeoutKEmpty : kDevTimeoutVEmpty))) {
+          ok = false;
+          break;
         }
-        if (j == 0 && ok) {
-          // Q after the first K/V tile, so both latencies overlap; the Q buffer is free once the
+        if (leader) mbar_expect_tx(full_bar + s, KV_BYTES);
+        load_kv_tile(map, ring + s * KV_BYTES, full_bar + s, j, si, p, bt, n_pages, kvh, leader);
+        issued = g + 1;
+        if (is_k && j == 0) {
+          // Q after the unit's first K tile, so both latencies overlap; the Q buffer is free once the
           // previous unit's last QK has finished
           if (q_loads > 0 && !__all_sync(0xffffffffu, mbar_wait(q_empty, (q_loads - 1) & 1, status, kDevTimeoutQ))) {
             ok = false;
@@ -236,11 +249,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       kv_iter += n;
     }
-    // never leave the CTA while loads it issued are still landing in shared memory
-    for (uint32_t g = issued_k >= NS ? issued_k - NS : 0; g < issued_k; ++g)
-      mbar_wait(k_full + (g % NS), (g / NS) & 1, status, kDevTimeoutKFull);
-    for (uint32_t g = issued_v >= NS ? issued_v - NS : 0; g < issued_v; ++g)
-      mbar_wait(v_full + (g % NS), (g / NS) & 1, status, kDevTimeoutVFull);
+    // never leave the CTA while loads this warp issued are still landing in shared memory
+    for (uint32_t g = issued >= (uint32_t)depth ? issued - depth : 0; g < issued; ++g)
+      mbar_wait(full_bar + (g % depth), (g / depth) & 1, status, is_k ? kDevTimeoutKFull : kDevTimeoutVFull);
     if (q_loads > 0) mbar_wait(q_full, (q_loads - 1) & 1, status, kDevTimeoutQ);
     __syncwarp();
   } else if (warp == 5) {
@@ -256,38 +267,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto wait_all = [&](uint64_t* bar, uint32_t parity, int code) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, status, code));
     };
-    // S[g % 2] = Q K^T of the tile in ring slot g % NS
+    // S[g % NSB] = Q K^T of the tile in K ring slot g % NSK
     auto issue_qk = [&](uint32_t g) {
       if (leader) {
-        const uint64_t b0 = dk + (g % NS) * kKVStep;
+        const uint64_t b0 = dk + (g % NSK) * kKVStep;
 #pragma unroll
         for (int kk = 0; kk < D / UK; ++kk) {
           const int ke = kk * UK;
           const uint64_t off_q = ((ke / AW) * BLK_Q + (ke % AW) * 2) >> 4;
           const uint64_t off_k = ((ke / AW) * BLK_KV + (ke % AW) * 2) >> 4;
-          mma_ss(tmem + (g & 1) * KT, dq + off_q, b0 + off_k, kIdescQK, kk > 0, false);
+          mma_ss(tmem + (g % NSB) * KT, dq + off_q, b0 + off_k, kIdescQK, kk > 0, false);
         }
-        mma_commit(s_full + (g & 1));
+        mma_commit(s_full + (g % NSB));
       }
     };
-    // O (+)= P V, P in TMEM over S[g % 2] (8 columns of packed 16-bit pairs per K step of 16 keys)
+    // O (+)= P V, P in TMEM over S[g % NSB] (8 columns of packed 16-bit pairs per K step of 16 keys)
     auto issue_pv = [&](uint32_t g, bool acc) {
       if (leader) {
-        const uint64_t v0 = dv + (g % NS) * kKVStep;
+        const uint64_t v0 = dv + (g % NSV) * kKVStep;
 #pragma unroll
         for (int kk = 0; kk < KT / UK; ++kk)
-          mma_ts(tmem + O_COL, tmem + (g & 1) * KT + kk * 8, v0 + ((kk * UK * 128) >> 4), kIdescPV,
+          mma_ts(tmem + O_COL, tmem + (g % NSB) * KT + kk * 8, v0 + ((kk * UK * 128) >> 4), kIdescPV,
                  (acc || kk > 0) ? 1u : 0u, false);
-        mma_commit(pv_done + (g & 1));
+        mma_commit(pv_done + (g % NSB));
       }
     };
     auto commit = [&](uint64_t* bar) {
       if (leader) mma_commit(bar);
     };
-    // QK of tile g: its K tile is loaded and its S buffer is free (the P V of tile g - 2 has completed)
+    // QK of tile g: its K tile is loaded and its S buffer is free (the P V of tile g - NSB has completed)
     auto qk_ready = [&](uint32_t g) {
-      if (!wait_all(k_full + (g % NS), (g / NS) & 1, kDevTimeoutKFull)) return false;
-      if (g >= 2 && !wait_all(pv_done + (g & 1), ((g - 2) >> 1) & 1, kDevTimeoutODone)) return false;
+      if (!wait_all(k_full + (g % NSK), (g / NSK) & 1, kDevTimeoutKFull)) return false;
+      if (g >= NSB && !wait_all(pv_done + (g % NSB), ((g / NSB) - 1) & 1, kDevTimeoutODone)) return false;
       tc_fence_after();
       return true;
     };
@@ -304,19 +315,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto qk = [&](int j) {
         if (!qk_ready(kv_iter + j)) return false;
         issue_qk(kv_iter + j);
-        commit(k_empty + ((kv_iter + j) % NS));
+        commit(k_empty + ((kv_iter + j) % NSK));
         if (j == n - 1) commit(q_empty);
         return true;
       };
       for (int j = 0; j < 2 && j < n && ok; ++j) ok = qk(j);
       for (int j = 0; j < n && ok; ++j) {
         const uint32_t g = kv_iter + j;
-        if (!(ok = wait_all(v_full + (g % NS), (g / NS) & 1, kDevTimeoutVFull))) break;
-        if (!(ok = wait_all(p_full + (g & 1), (g >> 1) & 1, kDevTimeoutPFull))) break;
+        if (!(ok = wait_all(v_full + (g % NSV), (g / NSV) & 1, kDevTimeoutVFull))) break;
+        if (!(ok = wait_all(p_full + (g % NSB), (g / NSB) & 1, kDevTimeoutPFull))) break;
         tc_fence_after();
         issue_pv(g, j > 0);
         if (j == n - 1) commit(o_done);
-        commit(v_empty + (g % NS));
+        commit(v_empty + (g % NSV));
         if (j + 2 < n) ok = qk(j + 2);
       }
       kv_iter += n;
@@ -349,9 +360,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       float l_run = 0.f;
       for (int j = 0; j < n; ++j) {
         const uint32_t t = tp + j;
-        const uint32_t s_col = tmem + lane_base + (t & 1) * KT;
+        const uint32_t s_col = tmem + lane_base + (t % NSB) * KT;
         const int j0 = j * KT;
-        ok = __all_sync(0xffffffffu, mbar_wait(s_full + (t & 1), (t >> 1) & 1, status, kDevTimeoutSFull));
+        ok = __all_sync(0xffffffffu, mbar_wait(s_full + (t % NSB), (t / NSB) & 1, status, kDevTimeoutSFull));
         if (!ok) break;
         tc_fence_after();
         float x[KT];
@@ -391,7 +402,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_base = (m_run == -INFINITY) ? 0.f : m_run;
         if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
           // O must hold P(j-1) V(j-1) before it is scaled; P(j) V cannot start before P(j) below
-          ok = __all_sync(0xffffffffu, mbar_wait(pv_done + ((t - 1) & 1), ((t - 1) >> 1) & 1, status, kDevTimeoutODone));
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(pv_done + ((t - 1) % NSB), ((t - 1) / NSB) & 1, status, kDevTimeoutODone));
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
@@ -414,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_run = l_run * alpha + row_sum;
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(p_full + (t & 1));
+        mbar_arrive(p_full + (t % NSB));
       }
       tp += n;
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, up & 1, status, kDevTimeoutODone));
