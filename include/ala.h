@@ -122,7 +122,8 @@ ALA_API int ala_workspace_status(const ala_op* op, const void* workspace, ala_st
  *             [numBlocks, blockSize, kvHeadNum, headSize], same dtype, device.
  *             Key position j of sequence b is slot j % blockSize of block
  *             blockTables[b][j / blockSize].  blockSize must be a multiple
- *             of 16 that divides 128, or a multiple of 128.
+ *             of 16 (the kernels gather each key tile in boxes of
+ *             gcd(blockSize, keys per tile) rows, each inside one page).
  * blockTables [batch, maxBlockNum] int32, device.  Entries past
  *             ceil(kvSeqLen_b / blockSize) are never read; entries read must
  *             be in [0, numBlocks).
@@ -226,7 +227,7 @@ ALA_API int varlen_attention_noalloc_status(ala_stream_t stream, int32_t* code);
  * qRope       [tokens, headNum, 64] bf16/f16, device: the compute and output type.
  * ctKV        [numBlocks, blockSize, kvHeadNum, 512], device (ND layout), qRope's
  *             dtype, or int8 codes with cacheMode 2 (16-byte aligned);
- *             blockSize a multiple of 16 dividing 64, or a multiple of 64.
+ *             blockSize a multiple of 16.
  * kRope       [numBlocks, blockSize, kvHeadNum, 64], device.
  * blockTables [batch, maxBlocks] int32, device (entries read must be valid).
  * contextLens [batch] int32, HOST: keys per batch, including the new tokens.

@@ -268,10 +268,8 @@ int build_prefill(ala_op* op, const ala_tensor* query, const ala_tensor* key, co
     if (!blockTables->data) return fail(ALA_NULL_REQUIRED, "%s: blockTables data is NULL", fn);
     if (blockTables->dtype != ALA_I32) return fail(ALA_INVALID_DTYPE, "%s: blockTables must be int32", fn);
     if (blockTables->ndim != 2) return fail(ALA_INVALID_SHAPE, "%s: blockTables must be [batch, maxBlockNum]", fn);
-    if (!(block_size > 0 && block_size % 16 == 0 &&
-          (kPrefillTileKeys % block_size == 0 || block_size % kPrefillTileKeys == 0)))
-      return fail(ALA_UNSUPPORTED, "%s: blockSize %d must be a multiple of 16 dividing %d, or a multiple of %d", fn,
-                  block_size, kPrefillTileKeys, kPrefillTileKeys);
+    if (!(block_size > 0 && block_size % 16 == 0))
+      return fail(ALA_UNSUPPORTED, "%s: blockSize %d must be a multiple of 16", fn, block_size);
     max_blocks = (int32_t)blockTables->dims[1];
   }
   if (kv_rows >= (int64_t)1 << 31 || n_tokens >= (int64_t)1 << 31)
@@ -387,7 +385,7 @@ int run_prefill(void* workspace, uint64_t workspaceSize, ala_op* op, ala_stream_
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (!op->maps_ready) {
     const int tk = prefill_shape(prefill_kernel_d(op->dtype, op->head_size)).tile_keys;
-    const int kv_box = op->paged ? std::min(op->block_size, tk) : tk;
+    const int kv_box = op->paged ? kv_box_rows(op->block_size, tk) : tk;
     const int64_t q_rows = op->n_tokens;
     if (!encode_rows_heads_d(&op->tmQ, op->q, op->dtype, q_rows, op->heads, op->head_size, 128, false) ||
         !encode_rows_heads_d(&op->tmK, op->k, op->dtype, op->kv_rows, op->kv_heads, op->head_size, kv_box, false) ||
@@ -417,6 +415,8 @@ int run_prefill(void* workspace, uint64_t workspaceSize, ala_op* op, ala_stream_
   p.group = op->heads / op->kv_heads;
   p.scale_log2 = op->qk_scale * 1.4426950408889634f;
   p.d_out = op->head_size;
+  const int tile_keys = prefill_shape(prefill_kernel_d(op->dtype, op->head_size)).tile_keys;
+  p.kv_box_rows = op->paged ? kv_box_rows(op->block_size, tile_keys) : tile_keys;
   cudaError_t e = launch_prefill(op->dtype, prefill_kernel_d(op->dtype, op->head_size), op->tmQ, op->tmK, op->tmV, p, st);
   if (e != cudaSuccess) return fail(ALA_CUDA_ERROR, "%s: kernel launch failed: %s", fn, cudaGetErrorString(e));
   return ok();

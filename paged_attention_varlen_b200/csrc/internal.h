@@ -99,7 +99,20 @@ struct PrefillParams {
   int32_t group;                // heads / kvHeads
   float scale_log2;             // qkScale * log2(e)
   int32_t d_out;                // head size of the tensors (<= the kernel's D; dims past it are zero-filled)
+  int32_t kv_box_rows;          // paged caches: rows per K/V TMA box, gcd(blockSize, keys per tile)
 };
+
+// Rows per K/V TMA box for a paged cache: the largest count that divides both the key tile and blockSize,
+// so every box lies inside one page (blockSize a multiple of 16 gives at least 16).
+inline int kv_box_rows(int block_size, int tile_keys) {
+  int a = block_size, b = tile_keys;
+  while (b) {
+    const int t = a % b;
+    a = b;
+    b = t;
+  }
+  return a;
+}
 
 // Tiling of the prefill kernel instance that serves kernel head size D (prefill_kernel_d): keys per K/V
 // tile and whether a unit holds one block of 128 query rows (D = 256, whose O takes half of tensor memory)

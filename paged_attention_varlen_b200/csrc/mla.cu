@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(KV8 ? 320 : 192, 1)
       tma_prefetch_desc(&tmKR);
       const int bs = p.block_size;
       const bool whole = bs % kTileKeys == 0;  // a tile lies in one page: one 3-D box holds its ctKV part
-      const int box_rows = bs < kTileKeys ? bs : kTileKeys;
+      const int box_rows = p.kv_box_rows;  // every box lies inside one page
       int G = 0;  // tiles issued so far by this CTA
       // L2 prefetch cursor (piece kf, tile jf, CTA tile Gf), kept ALA_MLA_PREFETCH_TILES tiles ahead of the loads
       int kf = k0, jf = 0, Gf = 0;
@@ -842,8 +842,7 @@ int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, co
       kRope->dims[3] != 64)
     return mfail(err, n, ALA_INVALID_SHAPE, "kRope must be [numBlocks, blockSize, 1, 64]");
   const int64_t bs = ctKV->dims[1];
-  if (!(bs > 0 && bs % 16 == 0 && (64 % bs == 0 || bs % 64 == 0)))  // also tiles both 32- and 64-key rings
-    return mfail(err, n, ALA_UNSUPPORTED, "blockSize must be a multiple of 16 dividing 64, or a multiple of 64");
+  if (!(bs > 0 && bs % 16 == 0)) return mfail(err, n, ALA_UNSUPPORTED, "blockSize must be a multiple of 16");
   if (attenOut->ndim != 3 || attenOut->dims[0] != tokens || attenOut->dims[1] != headNum || attenOut->dims[2] != 512)
     return mfail(err, n, ALA_INVALID_SHAPE, "attenOut must be [tokens, headNum, 512]");
   if (contextLens->ndim != 1) return mfail(err, n, ALA_INVALID_SHAPE, "contextLens must be [batch]");
@@ -1015,7 +1014,7 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
   if (!plan->maps_ready) {
     const int es = 2;
     const cuuint64_t rows = (cuuint64_t)plan->num_blocks * plan->block_size;
-    const cuuint32_t kv_box_rows = (cuuint32_t)std::min(plan->block_size, kTileKeys);
+    const cuuint32_t box_rows = (cuuint32_t)kv_box_rows(plan->block_size, kTileKeys);
     cuuint64_t qn_dims[3] = {512, (cuuint64_t)plan->heads, (cuuint64_t)plan->tokens};
     cuuint64_t qn_str[2] = {512 * es, (cuuint64_t)plan->heads * 512 * es};
     cuuint64_t qr_dims[3] = {64, (cuuint64_t)plan->heads, (cuuint64_t)plan->tokens};
@@ -1025,7 +1024,7 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
     cuuint64_t kv_str[1] = {512 * es};
     cuuint64_t kr_dims[2] = {64, rows};
     cuuint64_t kr_str[1] = {64 * es};
-    cuuint32_t kv_box[2] = {64, kv_box_rows};
+    cuuint32_t kv_box[2] = {64, box_rows};
     // ctKV seen as (64 elements, rows, 8 column blocks): one box is a whole 64-key tile, laid out
     // [column block][key][64 elements] as the 128B-swizzled K-major operand wants it
     cuuint64_t kv3_dims[3] = {64, rows, 8};
@@ -1034,7 +1033,7 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
     // int8 codes: 512 bytes a row, seen as 128-byte column blocks (4 per row), same boxes of keys
     cuuint64_t k8_dims[2] = {512, rows};
     cuuint64_t k8_str[1] = {512};
-    cuuint32_t k8_box[2] = {128, kv_box_rows};
+    cuuint32_t k8_box[2] = {128, box_rows};
     cuuint64_t k83_dims[3] = {128, rows, 4};
     cuuint64_t k83_str[2] = {512, 128};
     cuuint32_t k83_box[3] = {128, (cuuint32_t)kTileKeys, 4};
@@ -1087,6 +1086,7 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
   p.hpc = plan->hpc;
   p.max_blocks = plan->max_blocks;
   p.block_size = plan->block_size;
+  p.kv_box_rows = kv_box_rows(plan->block_size, kTileKeys);
   p.oob_row = (int32_t)(plan->num_blocks * plan->block_size);
   p.scale_log2 = plan->qk_scale * kLog2e;
   p.qk_descale = plan->qk_descale;

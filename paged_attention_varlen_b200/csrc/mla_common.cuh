@@ -56,6 +56,7 @@ struct MlaParams {
   int32_t hpc;              // heads per CTA row block (64 / tpc)
   int32_t max_blocks;
   int32_t block_size;
+  int32_t kv_box_rows;      // rows per cache TMA box when a tile spans pages: gcd(blockSize, kTileKeys)
   int32_t oob_row;
   float scale_log2;
   const float* qk_descale;  // [heads], int8 cache only

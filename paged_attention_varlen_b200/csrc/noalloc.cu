@@ -231,6 +231,7 @@ extern "C" ALA_API int varlen_attention_noalloc(const ala_tensor* query, const a
   p.group = group;
   p.scale_log2 = qkScale * 1.4426950408889634f;
   p.d_out = (int32_t)d;
+  p.kv_box_rows = shape.tile_keys;  // contiguous K/V: one box per tile
   const cudaError_t e = launch_prefill(dt, prefill_kernel_d(dt, d), tmQ, tmK, tmV, p, st);
   if (e != cudaSuccess) return nfail(ALA_CUDA_ERROR, "%s: kernel launch failed: %s", fn, cudaGetErrorString(e));
   set_last_error("");

@@ -146,7 +146,7 @@ __device__ __forceinline__ void load_kv_tile(const CUtensorMap* map, uint8_t* ds
   using C = Cfg<T, D>;
   const bool paged = bt != nullptr;
   const int bs = p.block_size;
-  const int box_rows = paged ? (bs < 128 ? bs : 128) : 128;
+  const int box_rows = paged ? p.kv_box_rows : 128;  // paged: every box lies inside one page
   const int j0 = j * 128;
   for (int r0 = 0; r0 < 128; r0 += box_rows) {
     // contiguous rows, or the page's row through the block table (past the last page: zero fill)

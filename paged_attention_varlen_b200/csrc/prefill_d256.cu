@@ -119,7 +119,7 @@ __device__ __forceinline__ void load_kv_tile(const CUtensorMap* map, uint8_t* ds
                                              int n_pages, int kvh, bool leader) {
   const bool paged = bt != nullptr;
   const int bs = p.block_size;
-  const int box_rows = paged ? (bs < KT ? bs : KT) : KT;
+  const int box_rows = paged ? p.kv_box_rows : KT;  // paged: every box lies inside one page
   const int j0 = j * KT;
   for (int r0 = 0; r0 < KT; r0 += box_rows) {
     // contiguous rows, or the page's row through the block table (past the last page: zero fill)

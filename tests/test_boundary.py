@@ -109,6 +109,8 @@ def _plan_prefix(**over):
 
 def test_prefix_plan_ok_and_mask_tensor_accepted():
     _plan_prefix()
+    for bs in (48, 80, 144):  # any multiple of 16 (K/V boxes of gcd(blockSize, 128) rows)
+        _plan_prefix(k=torch.zeros(8, bs, 2, 128, dtype=torch.float16), v=torch.zeros(8, bs, 2, 128, dtype=torch.float16))
     _plan_prefix(mask=torch.zeros(256, 256, dtype=torch.float16))
     _plan_prefix(mask=torch.zeros(4, 4, 128, dtype=torch.float16), mask_type=4)
 
@@ -158,6 +160,9 @@ def _int8_cache(**over):
 
 def test_mla_plan_ok():
     _plan_mla()
+    for bs in (80, 112, 144):  # any multiple of 16 (cache boxes of gcd(blockSize, 64) rows)
+        _plan_mla(ct_kv=torch.zeros(6, bs, 1, 512, dtype=torch.bfloat16),
+                  k_rope=torch.zeros(6, bs, 1, 64, dtype=torch.bfloat16))
     _plan_mla(q_nope=torch.zeros(6, 128, 512, dtype=torch.bfloat16), q_rope=torch.zeros(6, 128, 64, dtype=torch.bfloat16),
               q_seq_len=[2, 2, 2], mask_type=1, calc_type=1)
 

@@ -45,7 +45,7 @@ def _oracle(case, rows=None, mask=None):
 
 
 @pytest.mark.parametrize("qs", [1, 4])
-@pytest.mark.parametrize("block_size", [16, 32, 64, 128])
+@pytest.mark.parametrize("block_size", [16, 32, 48, 64, 80, 128, 192])
 def test_mla_small_ragged(qs, block_size):
     ctx = np.array([qs, 63, 64, 65, 700, 1100], dtype=np.int32)
     case = synth.make_mla("small", ctx, qs, 128, 5 + qs, block_size=block_size)

@@ -84,9 +84,10 @@ def test_prefix_offset_masks_contiguous(mask_type):
     _full_check(case)
 
 
-@pytest.mark.parametrize("block_size", [16, 32, 64, 128, 256])
+@pytest.mark.parametrize("block_size", [16, 32, 48, 64, 96, 128, 160, 256])
 @pytest.mark.parametrize("mask_type", [3, 4, 5, 9])
 def test_paged_prefix_encoder(block_size, mask_type):
+    # block sizes that neither divide nor are multiples of the 128-key tile gather in gcd-high boxes
     L = [64, 1, 333, 129]
     pre = [256, 40, 512, 0]
     case = synth.make_prefill("paged", L, [a + b for a, b in zip(L, pre)], 8, 2, 128, torch.float16, mask_type, 13,
@@ -109,7 +110,8 @@ def test_head_sizes_between_the_kernel_sizes(d, dtype, mask_type, paged):
 
 @pytest.mark.parametrize("d,dtype,mask_type,paged,block_size", [
     (256, torch.bfloat16, 9, False, 128), (256, torch.float16, 0, False, 128), (256, torch.bfloat16, 9, True, 16),
-    (256, torch.float16, 9, True, 128), (192, torch.bfloat16, 9, True, 64), (144, torch.float16, 0, False, 128)])
+    (256, torch.float16, 9, True, 128), (192, torch.bfloat16, 9, True, 64), (144, torch.float16, 0, False, 128),
+    (256, torch.bfloat16, 9, True, 48), (160, torch.float16, 9, True, 80)])
 def test_large_head_sizes(d, dtype, mask_type, paged, block_size):
     # head sizes above 128 run on the D = 256 kernel (one 128-row block per CTA, 64-key tiles); GQA group 4
     L = [1, 63, 64, 65, 128, 129, 400, 7]
