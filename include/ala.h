@@ -139,7 +139,7 @@ ALA_API int ala_workspace_status(const ala_op* op, const void* workspace, ala_st
  * headNum     > 0; kvHeadNum > 0 and divides headNum (query head h reads kv
  *             head h / (headNum/kvHeadNum)).
  * qkScale     multiplies Q K^T before the bias is added.
- * headSize    a multiple of 16 up to 256 (ALiBi masks: <= 128, per the
+ * headSize    a multiple of 8 up to 256 (ALiBi masks: <= 128, per the
  *             compressed-mask page's constraints); 64, 128 and 256 run
  *             natively, others on the next of those with zero-filled extra
  *             dimensions.

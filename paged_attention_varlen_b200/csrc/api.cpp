@@ -303,7 +303,7 @@ int build_prefill(ala_op* op, const ala_tensor* query, const ala_tensor* key, co
   }
   if (prefill_kernel_d(dt, head_size) == 0)
     return fail(ALA_UNSUPPORTED,
-                "%s: headSize %lld with this dtype is not built (bf16/f16: a multiple of 16 up to 256; f32: a "
+                "%s: headSize %lld with this dtype is not built (bf16/f16: a multiple of 8 up to 256; f32: a "
                 "multiple of 8 up to 64)",
                 fn, (long long)head_size);
 

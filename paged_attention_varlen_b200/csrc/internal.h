@@ -189,7 +189,7 @@ bool encode_rows_heads_d(CUtensorMap* map, void* base, int32_t dtype, int64_t ro
 enum : int32_t { kF16 = 0, kBF16 = 1, kF32 = 2, kI32 = 3 };
 
 // Head size D of the prefill kernel instance that serves head size `d` of element type `dtype` (0 if none
-// does): 16-bit types take d a multiple of 16 up to 256 (D = 64, 128 or 256), fp32 a multiple of 8 up to
+// does): 16-bit types take d a multiple of 8 up to 256 (D = 64, 128 or 256), fp32 a multiple of 8 up to
 // 64 (D = 64).  The tensor maps are encoded over the real d, so the dimensions d..D-1 of every Q, K and V
 // tile are zero-filled by the TMA loads and contribute nothing; the epilogue stores the first d columns.
 int prefill_kernel_d(int32_t dtype, int64_t d);

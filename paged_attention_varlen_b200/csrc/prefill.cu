@@ -88,6 +88,11 @@ __device__ __forceinline__ void st_global_v8(void* p, uint32_t a0, uint32_t a1, 
                : "memory");
 }
 
+// One 16-byte store (address 16-byte aligned): rows of a 16-bit head size that is an odd multiple of 8.
+__device__ __forceinline__ void st_global_v4(void* p, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
+  asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a0), "r"(a1), "r"(a2), "r"(a3) : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack2(float a, float b, __nv_bfloat16*) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -541,6 +546,7 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       const float inv_l = 1.f / l_run;
       const int d_out = p.d_out;  // columns d_out..D-1 hold zeros (zero-filled Q, K and V dimensions)
+      const bool wide_rows = d_out % 16 == 0;  // 16-bit rows 32-byte aligned: 32-byte stores
       T* orow = reinterpret_cast<T*>(p.out) + ((size_t)(si.cu_q + qi) * p.heads + head) * d_out;
       uint32_t orr[D / 32][32];
 #pragma unroll
@@ -552,15 +558,24 @@ __global__ void __launch_bounds__(384, 1)
         if (row_valid) {
           // rows are d_out * element size apart, a multiple of 32 bytes: every 32-byte store is aligned
           if constexpr (C::ES == 2) {
+            uint32_t w[16];
 #pragma unroll
-            for (int v8 = 0; v8 < 2; ++v8) {
-              if (c32 * 32 + v8 * 16 >= d_out) break;
-              uint32_t w[8];
+            for (int i = 0; i < 16; ++i)
+              w[i] = pack2(__uint_as_float(regs[2 * i]) * inv_l, __uint_as_float(regs[2 * i + 1]) * inv_l, (T*)nullptr);
+            if (wide_rows) {
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
-                w[i] = pack2(__uint_as_float(regs[v8 * 16 + 2 * i]) * inv_l,
-                             __uint_as_float(regs[v8 * 16 + 2 * i + 1]) * inv_l, (T*)nullptr);
-              st_global_v8(orow + c32 * 32 + v8 * 16, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+              for (int v8 = 0; v8 < 2; ++v8) {
+                if (c32 * 32 + v8 * 16 >= d_out) break;
+                st_global_v8(orow + c32 * 32 + v8 * 16, w[8 * v8], w[8 * v8 + 1], w[8 * v8 + 2], w[8 * v8 + 3],
+                             w[8 * v8 + 4], w[8 * v8 + 5], w[8 * v8 + 6], w[8 * v8 + 7]);
+              }
+            } else {
+              // rows 16 bytes apart only (d_out an odd multiple of 8): 16-byte stores
+#pragma unroll
+              for (int v4 = 0; v4 < 4; ++v4) {
+                if (c32 * 32 + v4 * 8 >= d_out) break;
+                st_global_v4(orow + c32 * 32 + v4 * 8, w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+              }
             }
           } else {
 #pragma unroll
@@ -609,7 +624,7 @@ cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtenso
 
 int prefill_kernel_d(int32_t dtype, int64_t d) {
   if (dtype == kBF16 || dtype == kF16) {
-    if (d <= 0 || d % 16 != 0 || d > 256) return 0;
+    if (d <= 0 || d % 8 != 0 || d > 256) return 0;
     return d <= 64 ? 64 : d <= 128 ? 128 : 256;
   }
   if (dtype == kF32) return (d > 0 && d % 8 == 0 && d <= 64) ? 64 : 0;

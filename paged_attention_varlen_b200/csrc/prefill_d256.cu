@@ -84,6 +84,11 @@ __device__ __forceinline__ uint32_t pack2(float a, float b, __half*) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// One 16-byte store (address 16-byte aligned): rows of a 16-bit head size that is an odd multiple of 8.
+__device__ __forceinline__ void st_global_v4(void* p, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
+  asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a0), "r"(a1), "r"(a2), "r"(a3) : "memory");
+}
+
 // One 32-byte store (address 32-byte aligned).
 __device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[8]) {
   asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
@@ -445,7 +450,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 4; ++c) tmem_ld32(o_col + half * 128 + c * 32, orr[c]);
         tmem_ld_wait();
         if (row_valid) {
-          // rows are d_out * 2 bytes apart, a multiple of 32 bytes: every 32-byte store is aligned
 #pragma unroll
           for (int v16 = 0; v16 < 8; ++v16) {
             const int col = half * 128 + v16 * 16;
@@ -455,7 +459,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 8; ++i)
               w[i] = pack2(__uint_as_float(orr[v16 >> 1][(v16 & 1) * 16 + 2 * i]) * inv_l,
                            __uint_as_float(orr[v16 >> 1][(v16 & 1) * 16 + 2 * i + 1]) * inv_l, (T*)nullptr);
-            st_global_v8(orow + col, w);
+            if (d_out % 16 == 0) {
+              st_global_v8(orow + col, w);  // rows d_out * 2 bytes apart, a multiple of 32 bytes
+            } else {
+              // rows 16 bytes apart only (d_out an odd multiple of 8): 16-byte stores
+              st_global_v4(orow + col, w[0], w[1], w[2], w[3]);
+              if (col + 8 < d_out) st_global_v4(orow + col + 8, w[4], w[5], w[6], w[7]);
+            }
           }
         }
       }

@@ -76,8 +76,8 @@ def test_output_must_be_32_byte_aligned():
     (dict(slopes=np.ones(4, np.float32)), 4),                    # causal forbids slopes
     (dict(mask_type=3, slopes=np.ones(3, np.float32)), 2),       # slopes must be [headNum]
     (dict(k=torch.zeros(14, 2, 128, dtype=torch.float16)), 3),   # dtype mismatch
-    (dict(q=torch.zeros(10, 4, 72, dtype=torch.bfloat16), k=torch.zeros(14, 2, 72, dtype=torch.bfloat16),
-          v=torch.zeros(14, 2, 72, dtype=torch.bfloat16)), 5),     # headSize not a multiple of 16
+    (dict(q=torch.zeros(10, 4, 68, dtype=torch.bfloat16), k=torch.zeros(14, 2, 68, dtype=torch.bfloat16),
+          v=torch.zeros(14, 2, 68, dtype=torch.bfloat16)), 5),     # headSize not a multiple of 8
     (dict(q=torch.zeros(10, 4, 272, dtype=torch.bfloat16), k=torch.zeros(14, 2, 272, dtype=torch.bfloat16),
           v=torch.zeros(14, 2, 272, dtype=torch.bfloat16)), 5),    # headSize > 256 is not built
     (dict(q=torch.zeros(10, 4, 96, dtype=torch.float32), k=torch.zeros(14, 2, 96, dtype=torch.float32),
@@ -357,7 +357,8 @@ def test_mla_explicit_mask_rejects(over, status):
 
 @pytest.mark.parametrize("d,dtype", [(16, torch.bfloat16), (80, torch.float16), (96, torch.bfloat16),
                                      (112, torch.bfloat16), (40, torch.float32), (144, torch.float16),
-                                     (192, torch.bfloat16), (256, torch.bfloat16)])
+                                     (192, torch.bfloat16), (256, torch.bfloat16), (8, torch.bfloat16),
+                                     (72, torch.float16), (200, torch.bfloat16)])
 def test_head_sizes_plan(d, dtype):
     op, out = _plan_varlen(q=torch.zeros(10, 4, d, dtype=dtype), k=torch.zeros(14, 2, d, dtype=dtype),
                            v=torch.zeros(14, 2, d, dtype=dtype))

@@ -98,7 +98,9 @@ def test_paged_prefix_encoder(block_size, mask_type):
 @pytest.mark.parametrize("d,dtype,mask_type,paged", [
     (16, torch.bfloat16, 9, False), (48, torch.float16, 3, False), (80, torch.bfloat16, 9, False),
     (96, torch.bfloat16, 4, False), (112, torch.float16, 0, False), (96, torch.float16, 3, True),
-    (80, torch.float16, 5, True), (40, torch.float32, 9, False), (8, torch.float32, 0, False)])
+    (80, torch.float16, 5, True), (40, torch.float32, 9, False), (8, torch.float32, 0, False),
+    (8, torch.bfloat16, 9, False), (40, torch.float16, 3, False), (72, torch.bfloat16, 9, True),
+    (120, torch.float16, 4, False)])
 def test_head_sizes_between_the_kernel_sizes(d, dtype, mask_type, paged):
     # head sizes run on the next kernel instance up (64 or 128) with the extra dimensions zero-filled
     L = [1, 127, 128, 129, 300, 5]
@@ -111,7 +113,8 @@ def test_head_sizes_between_the_kernel_sizes(d, dtype, mask_type, paged):
 @pytest.mark.parametrize("d,dtype,mask_type,paged,block_size", [
     (256, torch.bfloat16, 9, False, 128), (256, torch.float16, 0, False, 128), (256, torch.bfloat16, 9, True, 16),
     (256, torch.float16, 9, True, 128), (192, torch.bfloat16, 9, True, 64), (144, torch.float16, 0, False, 128),
-    (256, torch.bfloat16, 9, True, 48), (160, torch.float16, 9, True, 80)])
+    (256, torch.bfloat16, 9, True, 48), (160, torch.float16, 9, True, 80), (200, torch.bfloat16, 0, False, 128),
+    (136, torch.float16, 9, True, 16)])
 def test_large_head_sizes(d, dtype, mask_type, paged, block_size):
     # head sizes above 128 run on the D = 256 kernel (one 128-row block per CTA, 64-key tiles); GQA group 4
     L = [1, 63, 64, 65, 128, 129, 400, 7]
