@@ -1,7 +1,8 @@
-// prefill_d256.cu -- the prefill kernel for head sizes 144..256 (kernel head
-// size D = 256; ATB "PrefixEncoder" page, parameter table: headDim up to 256,
-// no ALiBi above 128), 16-bit types, no mask or the causal rule with the prefix
-// offset kvSeqLen - seqLen.
+// prefill_d256.cu -- the prefill kernel for head sizes 136..256 (kernel head
+// size D = 256), 16-bit types, no mask or the causal rule with the prefix offset
+// kvSeqLen - seqLen.  The pages bound headSize only for ALiBi compressed masks
+// (at most 128: the compressed-mask page, constraints), so head sizes above 128
+// take the causal rule or no mask.
 //
 // O of one 128-row block takes 256 of the 512 tensor-memory columns, so a CTA
 // computes one block of 128 query rows (not two, as the D <= 128 kernel does)
