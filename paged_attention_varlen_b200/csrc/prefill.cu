@@ -8,9 +8,11 @@
 // head (two query heads of a GQA group, or two consecutive row tiles of one
 // head), so each K/V tile staged in shared memory serves 256 rows.
 //
-//   warp 8       TMA producer: both Q tiles once, then K and V tiles (128 keys)
-//                into 2-deep rings; paged rows are gathered page by page
-//                through the block table.
+//   warps 8, 10  TMA producers: warp 8 both Q tiles of each unit and the K
+//                tiles (128 keys, 2-deep ring), warp 10 the V tiles (3-deep
+//                ring, 2-deep for sqrt ALiBi, whose bias tables take that
+//                room); paged rows are gathered page by page through the
+//                block table.
 //   warp 9       tcgen05 issuer.  Per key tile j and block b:
 //                  S_b = Q_b K_j^T        (SS MMA into TMEM columns of S_b)
 //                  O_b += P_b V_j         (TS MMA: P_b read from TMEM)
@@ -59,19 +61,25 @@ struct ElemFmt<float> {
   static constexpr uint32_t fmt = 2;  // tf32 tensor-core inputs
 };
 
-template <typename T, int D>
+// SQ: the instance carries the per-warp tables of the sqrt-ALiBi bias (maskType 4).  Their 10 KB take the
+// room of a third V slot, so the other mask types run on an instance with a 3-deep V ring: a K or V tile
+// arrives ~5000 cycles after its TMA load is issued, and two slots leave the MMA warp waiting for it.
+template <typename T, int D, bool SQ>
 struct Cfg {
   static constexpr int ES = sizeof(T);
   static constexpr int AW = 128 / ES;    // elements in one 128-byte swizzled row
   static constexpr int UK = 32 / ES;     // K extent of one MMA instruction
   static constexpr int BLK = 128 * 128;  // bytes of one 128-row x 128-byte swizzle column block
-  static constexpr int STAGES = 2;
+  static constexpr int NSK = 2;           // K ring depth
+  static constexpr int NSV = SQ ? 2 : 3;  // V ring depth
   static constexpr int Q_BYTES = 128 * D * ES;
   static constexpr int KV_BYTES = 128 * D * ES;
   static constexpr int TBL_FLOATS = 160;  // per-warp sqrt-bias table: lane - column + 127 in [0, 159)
-  static constexpr int TBL_BYTES = 8 * 2 * TBL_FLOATS * 4;
-  static constexpr int N_BARS = 21;
-  static constexpr int SMEM = 1024 + 2 * Q_BYTES + 2 * STAGES * KV_BYTES + TBL_BYTES + N_BARS * 8 + 16;
+  static constexpr int TBL_BYTES = SQ ? 8 * 2 * TBL_FLOATS * 4 : 0;
+  // q_full, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], and per block s_full, p_full, pv_done, o_done,
+  // p_lo; fin, q_empty
+  static constexpr int N_BARS = 1 + 2 * NSK + 2 * NSV + 2 * 5 + 2;
+  static constexpr int SMEM = 1024 + 2 * Q_BYTES + (NSK + NSV) * KV_BYTES + TBL_BYTES + N_BARS * 8 + 16;
   static constexpr uint32_t IDESC_QK = instr_desc(ElemFmt<T>::fmt, false, false, 128, 128);
   static constexpr uint32_t IDESC_PV = instr_desc(ElemFmt<T>::fmt, false, true, 128, D);
   static constexpr uint32_t TMEM_COLS = 512;  // S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D, 256+2D)
@@ -148,7 +156,7 @@ template <typename T, int D>
 __device__ __forceinline__ void load_kv_tile(const CUtensorMap* map, uint8_t* dst, uint64_t* full, int j,
                                              const SeqInfo& si, const PrefillParams& p, const int32_t* bt,
                                              int n_pages, int kvh, bool leader) {
-  using C = Cfg<T, D>;
+  using C = Cfg<T, D, false>;
   const bool paged = bt != nullptr;
   const int bs = p.block_size;
   const int box_rows = paged ? p.kv_box_rows : 128;  // paged: every box lies inside one page
@@ -163,30 +171,31 @@ __device__ __forceinline__ void load_kv_tile(const CUtensorMap* map, uint8_t* ds
   }
 }
 
-template <typename T, int D>
+template <typename T, int D, bool SQ>
 __global__ void __launch_bounds__(384, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
-  using C = Cfg<T, D>;
+  using C = Cfg<T, D, SQ>;
+  constexpr int NSK = C::NSK, NSV = C::NSV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                        // [2][Q_BYTES]
-  uint8_t* sK = sQ + 2 * C::Q_BYTES;         // [STAGES][KV_BYTES]
-  uint8_t* sV = sK + C::STAGES * C::KV_BYTES;
-  float* sTbl = reinterpret_cast<float*>(sV + C::STAGES * C::KV_BYTES);  // [8 warps][2][TBL_FLOATS]
+  uint8_t* sK = sQ + 2 * C::Q_BYTES;         // [NSK][KV_BYTES]
+  uint8_t* sV = sK + NSK * C::KV_BYTES;      // [NSV][KV_BYTES]
+  float* sTbl = reinterpret_cast<float*>(sV + NSV * C::KV_BYTES);  // SQ: [8 warps][2][TBL_FLOATS]
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sTbl) + C::TBL_BYTES);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;    // [2]
-  uint64_t* v_full = bars + 3;    // [2]
-  uint64_t* k_empty = bars + 5;   // [2]
-  uint64_t* v_empty = bars + 7;   // [2]
-  uint64_t* s_full = bars + 9;    // [2] per block
-  uint64_t* p_full = bars + 11;   // [2] per block: P of keys 64..127 written (all of P)
-  uint64_t* pv_done = bars + 13;  // [2] per block
-  uint64_t* o_done = bars + 15;   // [2] per block
-  uint64_t* fin = bars + 17;
-  uint64_t* q_empty = bars + 18;
-  uint64_t* p_lo = bars + 19;     // [2] per block: P of keys 0..63 written
+  uint64_t* k_full = bars + 1;          // [NSK]
+  uint64_t* k_empty = k_full + NSK;     // [NSK]
+  uint64_t* v_full = k_empty + NSK;     // [NSV]
+  uint64_t* v_empty = v_full + NSV;     // [NSV]
+  uint64_t* s_full = v_empty + NSV;     // [2] per block
+  uint64_t* p_full = s_full + 2;        // [2] per block: P of keys 64..127 written (all of P)
+  uint64_t* pv_done = p_full + 2;       // [2] per block
+  uint64_t* o_done = pv_done + 2;       // [2] per block
+  uint64_t* p_lo = o_done + 2;          // [2] per block: P of keys 0..63 written
+  uint64_t* fin = p_lo + 2;
+  uint64_t* q_empty = fin + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::N_BARS);
 
   const int warp = threadIdx.x >> 5;
@@ -199,11 +208,15 @@ __global__ void __launch_bounds__(384, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NSK; ++s) {
       mbar_init(k_full + s, 1);
-      mbar_init(v_full + s, 1);
       mbar_init(k_empty + s, 1);
+    }
+    for (int s = 0; s < NSV; ++s) {
+      mbar_init(v_full + s, 1);
       mbar_init(v_empty + s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(s_full + s, 1);
       mbar_init(p_full + s, 128);
       mbar_init(p_lo + s, 128);
@@ -222,26 +235,32 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // Barrier phases run on across units: the K/V ring by a global tile counter, the
-  // per-block S/P/PV barriers by each block's tile counter, q_full / q_empty and
+  // Barrier phases run on across units: the K and V rings by a global tile counter g (slot g % depth,
+  // phase g / depth), the per-block S/P/PV barriers by each block's tile counter, q_full / q_empty and
   // o_done by unit counters.
   //
   // register split: the softmax warpgroups take 216 per thread, warps 8..11 keep 72
   // (256*216 + 128*72 = 64512 = 384*168, all the registers the block is launched with)
   if (warp >= 8) {
     regs_decrease<72>();
-    if (warp == 8) {
-      // ------------------------------------------------------------ producer
-      // the whole warp walks the schedule (warp-uniform values); one elected lane issues the copies
+    if (warp == 8 || warp == 10) {
+      // ------------------------------------------------------------ producers
+      // warp 8 loads the K tiles and each unit's Q tiles, warp 10 the V tiles, so a K load never waits
+      // behind a V slot.  Each walks the schedule (warp-uniform values); one elected lane issues the copies.
+      const bool is_k = warp == 8;
+      const int depth = is_k ? NSK : NSV;
+      uint8_t* ring = is_k ? sK : sV;
+      uint64_t* full_bar = is_k ? k_full : v_full;
+      uint64_t* empty_bar = is_k ? k_empty : v_empty;
+      const CUtensorMap* map = is_k ? &tmK : &tmV;
       const bool leader = elect_one();
       if (leader) {
-        tma_prefetch_desc(&tmQ);
-        tma_prefetch_desc(&tmK);
-        tma_prefetch_desc(&tmV);
+        tma_prefetch_desc(map);
+        if (is_k) tma_prefetch_desc(&tmQ);
       }
       bool ok = true;
-      uint32_t kv_iter = 0;               // K/V tiles loaded so far (all units)
-      uint32_t issued_k = 0, issued_v = 0;  // K / V loads issued
+      uint32_t kv_iter = 0;  // K/V tiles loaded so far (all units)
+      uint32_t issued = 0;   // loads this warp issued
       int q_loads = 0;
       for (int ui = u_begin; ui < u_end && ok; ++ui) {
         const PrefillUnit u = p.units[ui];
@@ -253,21 +272,18 @@ __global__ void __launch_bounds__(384, 1)
         const int n_pages = bt ? (si.kv_len + p.block_size - 1) / p.block_size : 0;
         for (int j = 0; j < nmax && ok; ++j) {
           const uint32_t g = kv_iter + j;
-          const int s = g & 1;
-          for (int kv = 0; kv < 2; ++kv) {
-            if (g >= 2 && !__all_sync(0xffffffffu, mbar_wait((kv ? v_empty : k_empty) + s, ((g >> 1) - 1) & 1, status,
-                                                              kv ? kDevTimeoutVEmpty : kDevTimeoutKEmpty))) {
-              ok = false;
-              break;
-            }
-            uint64_t* full = (kv ? v_full : k_full) + s;
-            if (leader) mbar_expect_tx(full, C::KV_BYTES);
-            load_kv_tile<T, D>(kv ? &tmV : &tmK, (kv ? sV : sK) + s * C::KV_BYTES, full, j, si, p, bt, n_pages, kvh,
-                               leader);
-            if (kv) issued_v = g + 1; else issued_k = g + 1;
+          const int s = g % depth;
+          if (g >= (uint32_t)depth &&
+              !__all_sync(0xffffffffu, mbar_wait(empty_bar + s, ((g / depth) - 1) & 1, status,
+                                                 is_k ? kDevTimeoutKEmpty : kDevTimeoutVEmpty))) {
+            ok = false;
+            break;
           }
-          if (j == 0 && ok) {
-            // Q after the first K/V tile, so both latencies overlap; the Q buffers are free
+          if (leader) mbar_expect_tx(full_bar + s, C::KV_BYTES);
+          load_kv_tile<T, D>(map, ring + s * C::KV_BYTES, full_bar + s, j, si, p, bt, n_pages, kvh, leader);
+          issued = g + 1;
+          if (is_k && j == 0) {
+            // Q after the unit's first K tile, so both latencies overlap; the Q buffers are free
             // once the previous unit's last QK has finished
             if (q_loads > 0 && !__all_sync(0xffffffffu, mbar_wait(q_empty, (q_loads - 1) & 1, status, kDevTimeoutQ))) {
               ok = false;
@@ -289,11 +305,9 @@ __global__ void __launch_bounds__(384, 1)
         }
         kv_iter += nmax;
       }
-      // never leave the CTA while loads it issued are still landing in shared memory
-      for (uint32_t g = issued_k >= 2 ? issued_k - 2 : 0; g < issued_k; ++g)
-        mbar_wait(k_full + (g & 1), (g >> 1) & 1, status, kDevTimeoutKFull);
-      for (uint32_t g = issued_v >= 2 ? issued_v - 2 : 0; g < issued_v; ++g)
-        mbar_wait(v_full + (g & 1), (g >> 1) & 1, status, kDevTimeoutVFull);
+      // never leave the CTA while loads this warp issued are still landing in shared memory
+      for (uint32_t g = issued >= (uint32_t)depth ? issued - depth : 0; g < issued; ++g)
+        mbar_wait(full_bar + (g % depth), (g / depth) & 1, status, is_k ? kDevTimeoutKFull : kDevTimeoutVFull);
       if (q_loads > 0) mbar_wait(q_full, (q_loads - 1) & 1, status, kDevTimeoutQ);
     } else if (warp == 9) {
       // ------------------------------------------------------------ MMA issuer
@@ -345,7 +359,7 @@ __global__ void __launch_bounds__(384, 1)
         const int n1 = nb > 1 ? u.n_tiles[1] : 0;
         const int nmax = n0 > n1 ? n0 : n1;
         if (!wait_all(q_full, it & 1, kDevTimeoutQ) ||
-            !wait_all(k_full + (kv_iter & 1), (kv_iter >> 1) & 1, kDevTimeoutKFull)) {
+            !wait_all(k_full + (kv_iter % NSK), (kv_iter / NSK) & 1, kDevTimeoutKFull)) {
           ok = false;
           break;
         }
@@ -357,15 +371,15 @@ __global__ void __launch_bounds__(384, 1)
             break;
           }
           tc_fence_after();
-          issue_qk(b, kv_iter & 1);
+          issue_qk(b, kv_iter % NSK);
           commit(s_full + b);
         }
         if (!ok) break;
-        commit(k_empty + (kv_iter & 1));
+        commit(k_empty + (kv_iter % NSK));
         if (nmax == 1) commit(q_empty);
         for (int j = 0; j < nmax && ok; ++j) {
           const uint32_t g = kv_iter + j;
-          const int s = g & 1;
+          const int sv = g % NSV;  // V ring slot of tile j
           bool v_ready = false;
           for (int b = 0; b < nb && ok; ++b) {
             const int nbt = b == 0 ? n0 : n1;
@@ -375,31 +389,31 @@ __global__ void __launch_bounds__(384, 1)
               ok = false;
               break;
             }
-            if (!v_ready && !wait_all(v_full + s, (g >> 1) & 1, kDevTimeoutVFull)) {
+            if (!v_ready && !wait_all(v_full + sv, (g / NSV) & 1, kDevTimeoutVFull)) {
               ok = false;
               break;
             }
             v_ready = true;
             tc_fence_after();
-            issue_pv(b, s, j > 0, 0);  // keys 0..63
+            issue_pv(b, sv, j > 0, 0);  // keys 0..63
             if (!wait_all(p_full + b, ph & 1, kDevTimeoutPFull)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            issue_pv(b, s, true, 1);   // keys 64..127
+            issue_pv(b, sv, true, 1);   // keys 64..127
             commit(pv_done + b);
             const bool last_pv = (b == nb - 1) || (j >= n1);
-            if (last_pv) commit(v_empty + s);
+            if (last_pv) commit(v_empty + sv);
             if (j == nbt - 1) {
               commit(o_done + b);
               continue;
             }
             // next key tile for this block; S_b / P_b are reused once P_b(j) * V has completed
             const uint32_t g1 = g + 1;
-            const int s1 = g1 & 1;
+            const int s1 = g1 % NSK;  // K ring slot of tile j + 1
             const bool first_qk = (b == 0) || (j + 1 >= n0);
-            if (first_qk && !wait_all(k_full + s1, (g1 >> 1) & 1, kDevTimeoutKFull)) {
+            if (first_qk && !wait_all(k_full + s1, (g1 / NSK) & 1, kDevTimeoutKFull)) {
               ok = false;
               break;
             }
@@ -463,7 +477,7 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t ph = sp + j;
         const int j0 = j * 128;
         float* t = tbl + (ph & 1) * C::TBL_FLOATS;
-        if (mt == 4) {
+        if (SQ && mt == 4) {
           // -slope*log2(e)*sqrt(distance) for distance = iabs_w + k - 127 - j0, k = lane - column + 127
           for (int k = lane; k < C::TBL_FLOATS; k += 32) {
             const float dist = static_cast<float>(iabs_w - j0 + k - 127);
@@ -489,7 +503,7 @@ __global__ void __launch_bounds__(384, 1)
           const float b0 = slope_log2 * static_cast<float>(j0 - iabs);
 #pragma unroll
           for (int c = 0; c < 128; ++c) x[c] = fmaf(x[c], scale, fmaf(slope_log2, static_cast<float>(c), b0));
-        } else if (mt == 4) {
+        } else if (SQ && mt == 4) {
           const float* tl = t + lane + 127;
 #pragma unroll
           for (int c = 0; c < 128; ++c) x[c] = fmaf(x[c], scale, tl[-c]);
@@ -606,18 +620,27 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-template <typename T, int D>
-cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const PrefillParams& p,
-                   cudaStream_t stream) {
-  using C = Cfg<T, D>;
+template <typename T, int D, bool SQ>
+cudaError_t launch_instance(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                            const PrefillParams& p, cudaStream_t stream) {
+  using C = Cfg<T, D, SQ>;
   // at least 120 KB so a second CTA never shares the SM (each CTA allocates all 512 TMEM columns)
   constexpr int kSmem = C::SMEM > 120 * 1024 ? C::SMEM : 120 * 1024;
-  auto kern = prefill_kernel<T, D>;
+  auto kern = prefill_kernel<T, D, SQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
   if (e != cudaSuccess) return e;
   if (p.n_ctas == 0) return cudaSuccess;
   kern<<<p.n_ctas, 384, kSmem, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
+}
+
+// maskType 4 (sqrt ALiBi) runs on the instance with the bias tables, every other mask type on the one with
+// the deeper V ring
+template <typename T, int D>
+cudaError_t launch(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV, const PrefillParams& p,
+                   cudaStream_t stream) {
+  return p.mask_type == 4 ? launch_instance<T, D, true>(tmQ, tmK, tmV, p, stream)
+                          : launch_instance<T, D, false>(tmQ, tmK, tmV, p, stream);
 }
 
 }  // namespace
