@@ -173,7 +173,7 @@ ALA_API int atb_like_prefix_encoder_lse_get_workspace_size(
  * key, value  [nKvTokens, kvHeadNum, headSize], same dtype, device; keys of
  *             sequence b are packed at [sum_{c<b} kvSeqLen_c, + kvSeqLen_b).
  * seqLen, kvSeqLen, slopes, headNum, kvHeadNum, qkScale, headSize as above;
- *             maskType 0, 3, 4, 5 or 9 (above 128, headSize takes 0 or 9).
+ *             maskType 0, 3, 4, 5 or 9 (0 or 9 when headSize > 128).
  *             f32 inputs run on tf32 tensor cores (headSize a multiple of 8
  *             up to 64).
  * attnOut     like query, 32-byte aligned.
