@@ -22,7 +22,8 @@
 // tiles (ctKV 64 KB + kRope 8 KB each).  Once S(j) is computed, the softmax
 // writes P(j) over tile j's kRope block; the PV of the tile reads P and V from
 // the same slot.  Tensor memory: lanes 0..15 of each 32-lane quarter hold qNope
-// (columns 0..255) and S (256..319); lanes 16..31 hold O (columns 0..511).
+// (columns 0..255) and two S buffers (256..319, 384..447); lanes 16..31 hold O
+// (columns 0..511).
 //
 //   warp 4      TMA producer (one thread): ctKV + kRope tiles gathered through
 //               the block table (one 3-D box per tile when a tile lies in one
@@ -30,8 +31,9 @@
 //               the tiles after.
 //   warp 5      tcgen05 issuer (one thread): S = qNope K^T (TS, A in tensor
 //               memory) + qRope kRope^T (SS), and O += P V with V the ctKV part
-//               of the tile (two N = 256 halves); it issues whichever of the
-//               next QK and the next PV is ready.
+//               of the tile (two N = 256 halves); it issues the next PV when
+//               its P is ready, else the next QK when its tile and S buffer
+//               are (QK may lead PV by two tiles).
 //   warps 0..3  softmax: lane l < 16 of warp w owns S row 16w + l (scale, mask,
 //               online max / sum, P); lane 16 + l owns the O row and rescales
 //               it when the max grew by more than 2^8.  At the end of a piece
@@ -79,18 +81,21 @@ constexpr int kQrBytes = kBlk;             // the 64 x 64 qRope rows (qNope live
 constexpr int kKvBytes = 9 * kBlk;         // 64 keys x 576 x 2 B: ctKV blocks 0..7, kRope block 8
 constexpr int kPOff = 8 * kBlk;            // P(j) overwrites tile j's kRope block once S(j) is computed
 constexpr int kStages = 3;
-// q_full, kv_full[3], kv_empty[3], p_full[3], pv_last, s_full, s_free, fin, st_full, st_free, cv_full[3], cv_read
-constexpr int kNBars = 1 + 3 * kStages + 6 + kStages + 1;
+// q_full, kv_full[3], kv_empty[3], p_full[3], pv_last, s_full(0), s_free(0), fin, st_full, st_free, cv_full[3],
+// cv_read, s_full(1), s_free(1)
+constexpr int kNBars = 1 + 3 * kStages + 6 + kStages + 1 + 2;
 constexpr int kI8Off = 4 * kBlk;           // int8 cache: the tile's codes ([4][64 keys][128 B], 128B swizzle)
 constexpr int kSmem = 1024 + kQrBytes + kStages * kKvBytes + kNBars * 8 + 16;
 static_assert(kSmem <= 232448, "shared memory budget");
 static_assert(8 * kBlk <= kKvBytes, "the output staging (eight 8 KB boxes) must fit in a ring slot");
 // tensor memory: lanes 0..15 of each 32-lane quarter hold qNope (columns 0..255, the A operand of the
-// QK MMAs, which must accumulate at lane offset 0) and S (columns 256..319); lanes 16..31 hold O
-// (columns 0..511: output columns 0..255 and 256..511 as two N = 256 accumulators)
+// QK MMAs, which must accumulate at lane offset 0) and two S buffers (columns 256..319 and 384..447, so
+// that QK(j+1) runs while the softmax works on S(j)); lanes 16..31 hold O (columns 0..511: output
+// columns 0..255 and 256..511 as two N = 256 accumulators)
 constexpr uint32_t kQnCol = 0;
 constexpr uint32_t kSCol = 256;
 constexpr uint32_t kSRCol = 320;           // int8 cache: the qRope kRope part of S, lanes 0..15
+constexpr uint32_t kSBuf = 128;            // column offset of the second S buffer (and its qRope kRope part)
 constexpr int kConvWarp0 = 6;              // int8 cache: warps 6..9 convert ctKV tiles
 constexpr uint32_t kOLane = 16;
 constexpr uint32_t kTmemCols = 512;
@@ -195,8 +200,13 @@ __global__ void __launch_bounds__(KV8 ? 320 : 192, 1)
   uint64_t* kv_empty = bars + 1 + kStages;    // [kStages] slot free again
   uint64_t* p_full = bars + 1 + 2 * kStages;  // [kStages] P of the slot's tile written
   uint64_t* pv_last = bars + 1 + 3 * kStages; // the last PV of a piece is complete
-  uint64_t* s_full = pv_last + 1;
-  uint64_t* s_free = pv_last + 2;
+  // S buffer b (tile G uses b = G % 2): computed / read by all 128 softmax threads
+  uint64_t* const s_full0 = pv_last + 1;
+  uint64_t* const s_full1 = pv_last + 7 + kStages;
+  uint64_t* const s_free0 = pv_last + 2;
+  uint64_t* const s_free1 = pv_last + 8 + kStages;
+  auto s_full = [=](int b) { return b ? s_full1 : s_full0; };
+  auto s_free = [=](int b) { return b ? s_free1 : s_free0; };
   uint64_t* fin = pv_last + 3;
   uint64_t* st_full = pv_last + 4;  // the 128 softmax threads have written a round of output boxes
   uint64_t* st_free = pv_last + 5;  // the stores of a round have read their boxes
@@ -220,8 +230,10 @@ __global__ void __launch_bounds__(KV8 ? 320 : 192, 1)
       mbar_init(p_full + s, 128);
     }
     mbar_init(pv_last, 1);
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(s_full(b), 1);
+      mbar_init(s_free(b), 128);
+    }
     mbar_init(fin, 1);
     mbar_init(st_full, 128);
     mbar_init(st_free, 1);
@@ -336,31 +348,11 @@ __global__ void __launch_bounds__(KV8 ? 320 : 192, 1)
       uint32_t it = 0;
       bool progressed = false;
       while (ok && Gp < total) {
-        // QK(Gq) needs its tile, the S buffer (softmax is done with S(Gq-1)) and, first in a piece, the
-        // query; it may lead PV by one tile (S is single-buffered).  PV(Gp) needs P(Gp).
+        // PV(Gp) needs P(Gp) and goes first when ready: it frees its ring slot for the producer.
+        // QK(Gq) needs its tile, its S buffer (softmax is done with S(Gq-2)) and, first in a piece, the
+        // query; it may lead PV by two tiles (two S buffers, three ring slots).
         const int sq = Gq % kStages;
-        if (Gq < total && Gq - Gp < 2 && mbar_test_wait(kv_full + sq, (Gq / kStages) & 1) &&
-            (!KV8 || mbar_test_wait(cv_full + sq, (Gq / kStages) & 1)) &&
-            (Gq == 0 || mbar_test_wait(s_free, (Gq - 1) & 1)) && (jq > 0 || mbar_test_wait(q_full, (kq - k0) & 1))) {
-          tc_fence_after();
-          const uint64_t so = (uint64_t)((sq * kKvBytes) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < kDNope / 16; ++kk)  // qNope from tensor memory (8 columns per 16 elements)
-            mma_ts(tmem + kSCol, tmem + kQnCol + kk * 8, dk + so + (uint64_t)(((kk >> 2) * kBlk + (kk & 3) * 32) >> 4),
-                   idesc_qk, kk > 0 ? 1u : 0u, false);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)  // qRope x kRope from shared memory (own accumulator with an int8 cache)
-            mma_ss(tmem + (KV8 ? kSRCol : kSCol), dqr + (uint64_t)((kk * 32) >> 4),
-                   dk + so + (uint64_t)((8 * kBlk + kk * 32) >> 4), idesc_qk, (!KV8 || kk > 0) ? 1u : 0u, false);
-          mma_commit(s_full);
-          ++Gq;
-          if (++jq == nq) {
-            ++kq;
-            jq = 0;
-            nq = kq < k1 ? p.pieces[kq].n_tiles : 0;
-          }
-          progressed = true;
-        } else if (Gp < Gq && mbar_test_wait(p_full + (Gp % kStages), (Gp / kStages) & 1)) {
+        if (Gp < Gq && mbar_test_wait(p_full + (Gp % kStages), (Gp / kStages) & 1)) {
           tc_fence_after();
           const uint64_t so = (uint64_t)(((Gp % kStages) * kKvBytes) >> 4);
 #pragma unroll
@@ -379,6 +371,29 @@ __global__ void __launch_bounds__(KV8 ? 320 : 192, 1)
             ++kp;
             jp = 0;
             np = kp < k1 ? p.pieces[kp].n_tiles : 0;
+          }
+          progressed = true;
+        } else if (Gq < total && Gq - Gp < 3 && mbar_test_wait(kv_full + sq, (Gq / kStages) & 1) &&
+            (!KV8 || mbar_test_wait(cv_full + sq, (Gq / kStages) & 1)) &&
+            (Gq < 2 || mbar_test_wait(s_free(Gq & 1), ((Gq - 2) >> 1) & 1)) &&
+            (jq > 0 || mbar_test_wait(q_full, (kq - k0) & 1))) {
+          const uint32_t sb = (Gq & 1) * kSBuf;
+          tc_fence_after();
+          const uint64_t so = (uint64_t)((sq * kKvBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kDNope / 16; ++kk)  // qNope from tensor memory (8 columns per 16 elements)
+            mma_ts(tmem + kSCol + sb, tmem + kQnCol + kk * 8,
+                   dk + so + (uint64_t)(((kk >> 2) * kBlk + (kk & 3) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u, false);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // qRope x kRope from shared memory (own accumulator with an int8 cache)
+            mma_ss(tmem + (KV8 ? kSRCol : kSCol) + sb, dqr + (uint64_t)((kk * 32) >> 4),
+                   dk + so + (uint64_t)((8 * kBlk + kk * 32) >> 4), idesc_qk, (!KV8 || kk > 0) ? 1u : 0u, false);
+          mma_commit(s_full(Gq & 1));
+          ++Gq;
+          if (++jq == nq) {
+            ++kq;
+            jq = 0;
+            nq = kq < k1 ? p.pieces[kq].n_tiles : 0;
           }
           progressed = true;
         } else if ((++it & 1023u) == 0) {
@@ -477,19 +492,20 @@ __global__ void __launch_bounds__(KV8 ? 320 : 192, 1)
       float m_run = -INFINITY;
       float l_run = 0.f;
       for (int j = 0; j < pc.n_tiles; ++j, ++G) {
-        ok = wait_all(s_full, G & 1, status, kDevTimeoutSFull);
+        ok = wait_all(s_full(G & 1), (G >> 1) & 1, status, kDevTimeoutSFull);
         if (!ok) break;
         tc_fence_after();
+        const uint32_t sb = (G & 1) * kSBuf;
         float x[kTileKeys];
         {
           uint32_t regs[2][32];
-          tmem_ld32(tmem_warp + kSCol, regs[0]);
-          tmem_ld32(tmem_warp + kSCol + 32, regs[1]);
+          tmem_ld32(tmem_warp + kSCol + sb, regs[0]);
+          tmem_ld32(tmem_warp + kSCol + sb + 32, regs[1]);
           if constexpr (KV8) {
             // score = qkDescale * (qNope . ctKV) + qRope . kRope
             uint32_t rr[2][32];
-            tmem_ld32(tmem_warp + kSRCol, rr[0]);
-            tmem_ld32(tmem_warp + kSRCol + 32, rr[1]);
+            tmem_ld32(tmem_warp + kSRCol + sb, rr[0]);
+            tmem_ld32(tmem_warp + kSRCol + sb + 32, rr[1]);
             tmem_ld_wait();
 #pragma unroll
             for (int c = 0; c < kTileKeys; ++c)
@@ -540,9 +556,13 @@ __global__ void __launch_bounds__(KV8 ? 320 : 192, 1)
         const float a_row = __shfl_sync(kFull, alpha, lane & 15);
         if (j >= 1 && __any_sync(kFull, a_row != 1.f)) {
           // O must hold P(j-1) V(j-1) before it is scaled, and no MMA may run while the warp-wide
-          // tensor-memory stores rewrite this quarter (lanes 0..15 store back qNope and S unchanged):
-          // S(j+1) is not computed before s_free below, and PV(j) waits for P(j)
+          // tensor-memory stores rewrite this quarter (lanes 0..15 store back qNope and both S buffers
+          // unchanged): QK(j+1) of this piece, which may already be running into the other S buffer, is
+          // waited for; QK(j+2) is not issued before s_free below, and PV(j) waits for P(j).  (A next
+          // piece's first QK waits for its query, which is loaded after this piece.)
           ok = wait_all(kv_empty + ((G - 1) % kStages), ((G - 1) / kStages) & 1, status, kDevTimeoutODone);
+          if (ok && j + 1 < pc.n_tiles)
+            ok = wait_all(s_full((G + 1) & 1), ((G + 1) >> 1) & 1, status, kDevTimeoutSFull);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll 2
@@ -558,7 +578,7 @@ __global__ void __launch_bounds__(KV8 ? 320 : 192, 1)
           tmem_st_wait();
         }
         tc_fence_before();
-        mbar_arrive(s_free);
+        mbar_arrive(s_free(G & 1));
         const float m_base = (m_run == -INFINITY) ? 0.f : m_run;
         // P = 2^(x*scale - m), a pair of columns at a time (-inf masked keys give exactly 0)
         const uint64_t scale2 = f2pack(raw_max ? scale : 1.f, raw_max ? scale : 1.f);
