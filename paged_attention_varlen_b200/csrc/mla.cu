@@ -251,6 +251,9 @@ __global__ void __launch_bounds__(KV8 ? 320 : 192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the combine grid (launched as a programmatic dependent) may be scheduled from now on; it waits for this
+  // grid's completion before it reads the partials
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer (one elected thread)
@@ -722,6 +725,9 @@ __global__ void __launch_bounds__(KV8 ? 320 : 192, 1)
 // One CTA per (token, 8 heads); one warp per head, 16 output columns per lane.
 template <typename T>
 __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaCombine* work, const MlaParams p) {
+  // launched as a programmatic dependent of mla_kernel: wait until that grid has completed and its writes
+  // (the partials) are visible
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const MlaCombine w = work[blockIdx.x];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int head = blockIdx.y * 8 + warp;
@@ -1128,9 +1134,19 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
   }
   if (e == cudaSuccess && plan->n_combine > 0) {
     auto ck = plan->dtype == ALA_F16 ? mla_combine_kernel<__half> : mla_combine_kernel<__nv_bfloat16>;
-    dim3 grid(plan->n_combine, (plan->heads + 7) / 8);
-    ck<<<grid, 256, 0, stream>>>(reinterpret_cast<const MlaCombine*>(ws + plan->off_rows), p);
-    e = cudaGetLastError();
+    // a programmatic dependent launch: the combine grid is scheduled during mla_kernel's tail instead of
+    // after it, and griddepcontrol.wait holds it until mla_kernel has completed
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(plan->n_combine, (plan->heads + 7) / 8);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, ck, reinterpret_cast<const MlaCombine*>(ws + plan->off_rows), p);
   }
   if (e != cudaSuccess) return mfail(err, n, ALA_CUDA_ERROR, cudaGetErrorString(e));
   return ALA_OK;
