@@ -105,6 +105,18 @@ ALA_API const char* ala_last_error(void);
 /* Frees an op (NULL is allowed). */
 ALA_API void ala_op_destroy(ala_op* op);
 
+/* Binds `workspace` to `op`: copies the op's schedule (the host metadata the
+ * planning call built) into it and waits for that copy on `stream`.  Later
+ * executions of `op` into this same workspace pointer skip the schedule copy
+ * (~10 us of host-to-device latency per call) and only clear the status words
+ * with a 16-byte memset on their stream; executions into any other workspace
+ * copy the schedule as before.  While bound, the caller guarantees that
+ * nothing else writes to the workspace and that it stays allocated; binding a
+ * NULL workspace unbinds.  Status: ALA_NULL_REQUIRED (op NULL),
+ * ALA_WORKSPACE_TOO_SMALL, ALA_INVALID_PARAM (misaligned: 16 bytes for the
+ * prefill ops, 256 for MLA), ALA_CUDA_ERROR. */
+ALA_API int ala_op_bind_workspace(ala_op* op, void* workspace, uint64_t workspaceSize, ala_stream_t stream);
+
 /* Reads the device status word of `workspace` for `op` (synchronous copy on
  * the legacy stream after synchronising `stream`).  *code = 0 means every
  * kernel wait completed; 0x101..0x10A identifies the wait that ran out; 0x10B

@@ -83,6 +83,8 @@ def lib() -> ctypes.CDLL:
                                                                      ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
                                                                      T, T, U64P, OPP]
         L.atb_like_prefix_encoder_lse_get_workspace_size.restype = ctypes.c_int
+        L.ala_op_bind_workspace.argtypes = [P, P, ctypes.c_uint64, P]
+        L.ala_op_bind_workspace.restype = ctypes.c_int
         L.ala_lse_merge.argtypes = [T, T, T, T, T, T, P]
         L.ala_lse_merge.restype = ctypes.c_int
         for f in ("atb_like_prefix_encoder", "varlen_attention", "atb_like_mla"):
@@ -136,14 +138,19 @@ class Op:
     def __init__(self, handle, ws_size, execute_fn, device, keep):
         self._handle = handle
         self._execute = execute_fn
-        self.workspace = torch.empty(max(int(ws_size), 16), dtype=torch.uint8, device=device)
+        self.workspace = torch.empty(max(int(ws_size), 256), dtype=torch.uint8, device=device)
         self.workspace_size = int(ws_size)
         self._keep = keep
+        self._bound = False
 
     def __call__(self, stream: torch.cuda.Stream | None = None):
         s = stream if stream is not None else torch.cuda.current_stream(self.workspace.device)
-        _check(self._execute(ctypes.c_void_p(self.workspace.data_ptr()), self.workspace_size, self._handle,
-                             ctypes.c_void_p(s.cuda_stream)))
+        ws = ctypes.c_void_p(self.workspace.data_ptr())
+        if not self._bound:
+            # the workspace belongs to this Op alone: the schedule is copied into it once (ala_op_bind_workspace)
+            _check(lib().ala_op_bind_workspace(self._handle, ws, self.workspace_size, ctypes.c_void_p(s.cuda_stream)))
+            self._bound = True
+        _check(self._execute(ws, self.workspace_size, self._handle, ctypes.c_void_p(s.cuda_stream)))
         return self
 
     def device_status(self) -> int:

@@ -147,6 +147,7 @@ struct ala_op {
   PinnedImage pinned;
   bool maps_ready = false;
   CUtensorMap tmQ, tmK, tmV;
+  const void* bound_ws = nullptr;  // a workspace that holds this op's schedule (ala_op_bind_workspace)
   // mla
   MlaPlan mla;
 };
@@ -159,6 +160,41 @@ void set_last_error(const char* msg) { g_last_error = msg; }
 }  // namespace ala
 
 extern "C" void ala_op_destroy(ala_op* op) { delete op; }
+
+extern "C" int ala_op_bind_workspace(ala_op* op, void* workspace, uint64_t workspaceSize, ala_stream_t stream) {
+  NvtxRange nvtx_range("ala_op_bind_workspace");
+  const char* fn = "ala_op_bind_workspace";
+  if (!op) return fail(ALA_NULL_REQUIRED, "%s: op is NULL", fn);
+  if (!workspace) {  // unbind
+    op->bound_ws = nullptr;
+    op->mla.bound_ws = nullptr;
+    return ok();
+  }
+  const bool mla = op->kind == ala_op::kMla;
+  const uint64_t need = mla ? op->mla.ws_size : op->ws_size;
+  if (workspaceSize < need)
+    return fail(ALA_WORKSPACE_TOO_SMALL, "%s: workspace %llu < required %llu", fn, (unsigned long long)workspaceSize,
+                (unsigned long long)need);
+  if (reinterpret_cast<uintptr_t>(workspace) % (mla ? 256 : 16))
+    return fail(ALA_INVALID_PARAM, "%s: workspace must be %d-byte aligned", fn, mla ? 256 : 16);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  op->bound_ws = nullptr;
+  op->mla.bound_ws = nullptr;
+  if (mla) {
+    char err[512] = {0};
+    const int s = mla_upload(&op->mla, workspace, st, err, sizeof err);
+    if (s != ALA_OK) return fail(s, "%s: %s", fn, err);
+  } else if (cudaMemcpyAsync(workspace, op->pinned.get(op->image), op->ws_size, cudaMemcpyHostToDevice, st) !=
+             cudaSuccess) {
+    return fail(ALA_CUDA_ERROR, "%s: schedule upload failed: %s", fn, cudaGetErrorString(cudaGetLastError()));
+  }
+  // complete before returning, so that executions on any stream find the schedule in place
+  if (cudaStreamSynchronize(st) != cudaSuccess)
+    return fail(ALA_CUDA_ERROR, "%s: stream sync failed: %s", fn, cudaGetErrorString(cudaGetLastError()));
+  if (mla) op->mla.bound_ws = workspace;
+  else op->bound_ws = workspace;
+  return ok();
+}
 
 extern "C" int ala_workspace_status(const ala_op* op, const void* workspace, ala_stream_t stream, int32_t* code) {
   NvtxRange nvtx_range("ala_workspace_status");
@@ -393,8 +429,14 @@ int run_prefill(void* workspace, uint64_t workspaceSize, ala_op* op, ala_stream_
       return fail(ALA_CUDA_ERROR, "%s: cuTensorMapEncodeTiled failed (pointers must be 16-byte aligned)", fn);
     op->maps_ready = true;
   }
-  if (cudaMemcpyAsync(workspace, op->pinned.get(op->image), op->ws_size, cudaMemcpyHostToDevice, st) != cudaSuccess)
+  if (workspace == op->bound_ws) {
+    // the workspace already holds the schedule (ala_op_bind_workspace): only the status words are cleared
+    if (cudaMemsetAsync(workspace, 0, 16, st) != cudaSuccess)
+      return fail(ALA_CUDA_ERROR, "%s: status reset failed: %s", fn, cudaGetErrorString(cudaGetLastError()));
+  } else if (cudaMemcpyAsync(workspace, op->pinned.get(op->image), op->ws_size, cudaMemcpyHostToDevice, st) !=
+             cudaSuccess) {
     return fail(ALA_CUDA_ERROR, "%s: schedule upload failed: %s", fn, cudaGetErrorString(cudaGetLastError()));
+  }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   PrefillParams p{};
   p.units = reinterpret_cast<const PrefillUnit*>(ws + op->off_units);

@@ -1032,6 +1032,21 @@ int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, co
   return ALA_OK;
 }
 
+int mla_upload(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size_t n) {
+  if (!plan->pinned) {
+    if (cudaHostAlloc(&plan->pinned, plan->image_size, cudaHostAllocDefault) == cudaSuccess)
+      std::memcpy(plan->pinned, plan->image.data(), plan->image_size);
+    else {
+      plan->pinned = nullptr;
+      cudaGetLastError();
+    }
+  }
+  if (cudaMemcpyAsync(workspace, plan->pinned ? plan->pinned : plan->image.data(), plan->image_size,
+                      cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return mfail(err, n, ALA_CUDA_ERROR, "schedule upload failed");
+  return ALA_OK;
+}
+
 int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size_t n) {
   if (reinterpret_cast<uintptr_t>(workspace) % 256) return mfail(err, n, ALA_INVALID_PARAM, "workspace must be 256-byte aligned");
   if (plan->n_work == 0) return ALA_OK;
@@ -1083,17 +1098,14 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
       return mfail(err, n, ALA_CUDA_ERROR, "cuTensorMapEncodeTiled failed for the partial-output map");
     plan->tmPO_base = ws + plan->off_part_o;
   }
-  if (!plan->pinned) {
-    if (cudaHostAlloc(&plan->pinned, plan->image_size, cudaHostAllocDefault) == cudaSuccess)
-      std::memcpy(plan->pinned, plan->image.data(), plan->image_size);
-    else {
-      plan->pinned = nullptr;
-      cudaGetLastError();
-    }
+  if (workspace == plan->bound_ws) {
+    // the workspace already holds the schedule (ala_op_bind_workspace): only the status words are cleared
+    if (cudaMemsetAsync(workspace, 0, 16, stream) != cudaSuccess)
+      return mfail(err, n, ALA_CUDA_ERROR, "status reset failed");
+  } else {
+    const int st = mla_upload(plan, workspace, stream, err, n);
+    if (st != ALA_OK) return st;
   }
-  if (cudaMemcpyAsync(workspace, plan->pinned ? plan->pinned : plan->image.data(), plan->image_size,
-                      cudaMemcpyHostToDevice, stream) != cudaSuccess)
-    return mfail(err, n, ALA_CUDA_ERROR, "schedule upload failed");
   MlaParams p{};
   p.pieces = reinterpret_cast<const MlaPiece*>(ws + plan->off_work);
   p.lane_off = reinterpret_cast<const int32_t*>(ws + plan->off_lanes);

@@ -36,6 +36,7 @@ struct MlaPlan {
   CUtensorMap tmQr, tmKV, tmKV3, tmKR, tmO;
   CUtensorMap tmPO;                // partial-output map, bound to the workspace it was encoded for
   const void* tmPO_base = nullptr;
+  const void* bound_ws = nullptr;  // a workspace that holds this plan's schedule (ala_op_bind_workspace)
   MlaPlan() = default;
   MlaPlan(const MlaPlan&) = delete;
   MlaPlan& operator=(const MlaPlan&) = delete;
@@ -49,5 +50,7 @@ int mla_plan(MlaPlan* plan, const ala_tensor* qNope, const ala_tensor* qRope, co
              int calcType, uint8_t cacheMode, ala_tensor* attenOut, ala_tensor* lse, char* err, size_t errlen);
 
 int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size_t errlen);
+// Copies the plan's schedule image into `workspace` (stream-ordered).
+int mla_upload(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size_t errlen);
 
 }  // namespace ala

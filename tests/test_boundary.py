@@ -52,6 +52,16 @@ def test_valid_plan_needs_no_gpu():
     assert op.workspace_size > 0 and out.shape == (10, 4, 128)
 
 
+def test_bind_workspace_refusals_need_no_gpu():
+    op, _ = _plan_varlen()
+    L = ala.lib()
+    fake = ctypes.c_void_p(1 << 20)
+    assert L.ala_op_bind_workspace(None, fake, op.workspace_size, None) == 1           # op NULL
+    assert L.ala_op_bind_workspace(op._handle, fake, op.workspace_size - 1, None) == 6  # too small
+    assert L.ala_op_bind_workspace(op._handle, ctypes.c_void_p((1 << 20) + 8), op.workspace_size, None) == 4
+    assert L.ala_op_bind_workspace(op._handle, None, 0, None) == 0                     # unbinding is host-only
+
+
 def test_output_must_be_32_byte_aligned():
     # the kernel writes output rows in 32-byte pieces: a 16-byte-aligned output is refused on the host
     a = _varlen_args()

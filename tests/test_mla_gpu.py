@@ -3,6 +3,8 @@ the fp64 oracle on the same seeded inputs: small ragged cases element by
 element (key ranges long enough to be split, so the lse merge runs), and the
 full-size decode and speculative workloads, every element of the output and
 the lse.  Output buffers start out as NaN, so an unwritten row fails."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -42,6 +44,25 @@ def _run(case, mask=None):
 def _oracle(case, rows=None, mask=None):
     return oracle.mla(case.q_nope, case.q_rope, case.ct_kv, case.k_rope, case.block_tables, case.block_size,
                       case.context_lens, case.q_seq_len, case.heads, case.qk_scale, rows=rows, mask=mask)
+
+
+def test_mla_bound_workspace_equals_fresh_upload():
+    # the Op binds its workspace (schedule copied once); an execution into another workspace copies it again,
+    # with split key ranges so the partials and the combine are exercised, and must give the same bits
+    ctx = np.array([1, 700, 3000, 65], dtype=np.int32)
+    case = synth.make_mla("bind", ctx, 1, 128, 31, block_size=64)
+    out, lse, op = _run(case)
+    op()
+    torch.cuda.synchronize()
+    ref_out, ref_lse = out.clone(), lse.clone()
+    other = torch.full((max(op.workspace_size, 256),), 0xFF, dtype=torch.uint8, device="cuda")
+    out.fill_(float("nan"))
+    lse.fill_(float("nan"))
+    s = torch.cuda.current_stream()
+    assert ala.lib().atb_like_mla(ctypes.c_void_p(other.data_ptr()), op.workspace_size, op._handle,
+                                  ctypes.c_void_p(s.cuda_stream)) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(ref_out, out) and torch.equal(ref_lse, lse)
 
 
 @pytest.mark.parametrize("qs", [1, 4])

@@ -5,6 +5,8 @@ Every test compares every output element and every lse value with the
 oracle, the full-size workloads included.  Outputs and lse buffers start out
 as NaN, so a row the kernel never writes fails the comparison.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -144,6 +146,34 @@ def test_padded_run_matches_packed_on_valid_rows():
     for b, L in enumerate(case.seq_len.tolist()):
         assert torch.equal(out[pos:pos + L], outp[b * Lmax:b * Lmax + L])
         pos += L
+
+
+def test_bound_workspace_equals_fresh_upload():
+    # Op executions bind their own workspace (the schedule is copied once, later calls clear the status only);
+    # an execution into a second, unbound workspace copies the schedule and must give the same bits
+    case = synth.make_prefill("bind", [300, 1, 129], [400, 1, 200], 8, 2, 128, torch.bfloat16, 9, 29)
+    q, k, v, slopes, _ = _dev(case)
+    op, out = ala.plan_varlen_attention(q, k, v, case.seq_len, case.kv_seq_len, 9, 8, 2, case.qk_scale, slopes)
+    for _ in range(3):
+        op()
+    torch.cuda.synchronize()
+    assert op.device_status() == 0
+    bound = out.clone()
+    other = torch.full((max(op.workspace_size, 256),), 0xFF, dtype=torch.uint8, device="cuda")
+    out.fill_(float("nan"))
+    s = torch.cuda.current_stream()
+    L = ala.lib()
+    assert L.varlen_attention(ctypes.c_void_p(other.data_ptr()), op.workspace_size, op._handle,
+                              ctypes.c_void_p(s.cuda_stream)) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(bound, out)
+    # unbinding makes the Op's own workspace take the copying path again
+    assert L.ala_op_bind_workspace(op._handle, None, 0, None) == 0
+    out.fill_(float("nan"))
+    assert L.varlen_attention(ctypes.c_void_p(op.workspace.data_ptr()), op.workspace_size, op._handle,
+                              ctypes.c_void_p(s.cuda_stream)) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(bound, out)
 
 
 def test_repeat_is_deterministic_and_status_clean():
