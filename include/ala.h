@@ -106,13 +106,17 @@ ALA_API const char* ala_last_error(void);
 ALA_API void ala_op_destroy(ala_op* op);
 
 /* Binds `workspace` to `op`: copies the op's schedule (the host metadata the
- * planning call built) into it and waits for that copy on `stream`.  Later
- * executions of `op` into this same workspace pointer skip the schedule copy
- * (~10 us of host-to-device latency per call) and only clear the status words
- * with a 16-byte memset on their stream; executions into any other workspace
- * copy the schedule as before.  While bound, the caller guarantees that
- * nothing else writes to the workspace and that it stays allocated; binding a
- * NULL workspace unbinds.  Status: ALA_NULL_REQUIRED (op NULL),
+ * planning call built, with cleared status words) into it and waits for that
+ * copy on `stream`.  Later executions of `op` into this same workspace pointer
+ * skip the copy (~10 us of host-to-device latency per call) and launch their
+ * kernels only; executions into any other workspace copy the schedule as
+ * before.  The status words of a bound workspace are not cleared between
+ * executions: a code that an execution records there stays until the
+ * workspace is bound again (ala_workspace_status reports it), and a wait
+ * timeout's code makes later executions return at once without writing their
+ * outputs.  While bound,
+ * the caller guarantees that nothing else writes to the workspace and that it
+ * stays allocated; binding a NULL workspace unbinds.  Status: ALA_NULL_REQUIRED (op NULL),
  * ALA_WORKSPACE_TOO_SMALL, ALA_INVALID_PARAM (misaligned: 16 bytes for the
  * prefill ops, 256 for MLA), ALA_CUDA_ERROR. */
 ALA_API int ala_op_bind_workspace(ala_op* op, void* workspace, uint64_t workspaceSize, ala_stream_t stream);

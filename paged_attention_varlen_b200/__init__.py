@@ -158,6 +158,8 @@ class Op:
         s = torch.cuda.current_stream(self.workspace.device)
         _check(lib().ala_workspace_status(self._handle, ctypes.c_void_p(self.workspace.data_ptr()),
                                           ctypes.c_void_p(s.cuda_stream), ctypes.byref(code)))
+        if code.value != 0:
+            self._bound = False  # a recorded failure stays in a bound workspace: the next call binds it afresh
         return code.value
 
     def __del__(self):

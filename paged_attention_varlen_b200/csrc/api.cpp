@@ -429,14 +429,11 @@ int run_prefill(void* workspace, uint64_t workspaceSize, ala_op* op, ala_stream_
       return fail(ALA_CUDA_ERROR, "%s: cuTensorMapEncodeTiled failed (pointers must be 16-byte aligned)", fn);
     op->maps_ready = true;
   }
-  if (workspace == op->bound_ws) {
-    // the workspace already holds the schedule (ala_op_bind_workspace): only the status words are cleared
-    if (cudaMemsetAsync(workspace, 0, 16, st) != cudaSuccess)
-      return fail(ALA_CUDA_ERROR, "%s: status reset failed: %s", fn, cudaGetErrorString(cudaGetLastError()));
-  } else if (cudaMemcpyAsync(workspace, op->pinned.get(op->image), op->ws_size, cudaMemcpyHostToDevice, st) !=
-             cudaSuccess) {
+  // a bound workspace already holds the schedule and status words that only a failed execution sets
+  // (ala_op_bind_workspace); any other workspace gets both copied in
+  if (workspace != op->bound_ws &&
+      cudaMemcpyAsync(workspace, op->pinned.get(op->image), op->ws_size, cudaMemcpyHostToDevice, st) != cudaSuccess)
     return fail(ALA_CUDA_ERROR, "%s: schedule upload failed: %s", fn, cudaGetErrorString(cudaGetLastError()));
-  }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   PrefillParams p{};
   p.units = reinterpret_cast<const PrefillUnit*>(ws + op->off_units);

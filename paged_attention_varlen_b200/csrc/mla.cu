@@ -1098,11 +1098,9 @@ int mla_run(MlaPlan* plan, void* workspace, cudaStream_t stream, char* err, size
       return mfail(err, n, ALA_CUDA_ERROR, "cuTensorMapEncodeTiled failed for the partial-output map");
     plan->tmPO_base = ws + plan->off_part_o;
   }
-  if (workspace == plan->bound_ws) {
-    // the workspace already holds the schedule (ala_op_bind_workspace): only the status words are cleared
-    if (cudaMemsetAsync(workspace, 0, 16, stream) != cudaSuccess)
-      return mfail(err, n, ALA_CUDA_ERROR, "status reset failed");
-  } else {
+  // a bound workspace already holds the schedule and status words that only a failed execution sets
+  // (ala_op_bind_workspace); any other workspace gets both copied in
+  if (workspace != plan->bound_ws) {
     const int st = mla_upload(plan, workspace, stream, err, n);
     if (st != ALA_OK) return st;
   }
