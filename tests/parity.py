@@ -1,4 +1,4 @@
-"""Shared parity helpers: tolerances and row sampling (test infrastructure).
+"""Shared parity helpers: tolerances and NaN-filled output buffers (test infrastructure).
 
 Tolerances (GPU result vs the fp64 oracle on the same stored inputs):
   * attention output (bf16 / fp16 / fp32 stored): max |err| <= 2e-2 and
