@@ -4,9 +4,10 @@
 
 One step = one call of the library's varlen_attention over the packed-varlen
 causal prefill workload (batch 8, seqLen ~ U[64, 2048] seeded, headNum 32,
-kvHeadNum 8, headSize 128, bf16, qkScale 1/sqrt(128)): host-side schedule
-upload plus one prefill kernel launch.  The metric is attention TFLOPS on
-valid tokens: 4 * headSize * headNum * (allowed query/key pairs) per step.
+kvHeadNum 8, headSize 128, bf16, qkScale 1/sqrt(128)): one prefill kernel
+launch into the op's workspace, which holds the op's schedule since its first
+execution (ala_op_bind_workspace).  The metric is attention TFLOPS on valid
+tokens: 4 * headSize * headNum * (allowed query/key pairs) per step.
 
 Timing: W untimed warm-up steps, then K timed steps bracketed by a barrier
 and a device synchronise; each step is timed with CUDA events on the launch
