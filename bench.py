@@ -55,6 +55,9 @@ KERNEL_SOURCES = ["paged_attention_varlen_b200/csrc/prefill.cu", "paged_attentio
 D256_KERNEL_SOURCES = ["paged_attention_varlen_b200/csrc/prefill_d256.cu", "paged_attention_varlen_b200/csrc/ptx.cuh"]
 MLA_KERNEL_SOURCES = ["paged_attention_varlen_b200/csrc/mla.cu", "paged_attention_varlen_b200/csrc/mla_common.cuh",
                       "paged_attention_varlen_b200/csrc/ptx.cuh"]
+# the workload each committed ncu summary was captured on: its dram bytes describe that workload's launch only
+PROFILED_WORKLOADS = {"varlen_causal_bf16": PROFILE, "varlen_causal_bf16_d256": PROFILE_D256,
+                      "mla_decode_qs1_bf16": MLA_PROFILE, "mla_decode_qs1_int8": MLA_INT8_PROFILE}
 DEFAULT_WORKLOAD = "varlen_causal_bf16"
 WORKLOADS = {
     "varlen_causal_bf16": lambda: synth.varlen_causal_bf16(),
@@ -101,9 +104,11 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def profiled_traffic(path, src_hash):
-    """dram bytes per launch from the committed ncu summary, if it was taken on the current kernel source."""
-    if not os.path.exists(path):
+def profiled_traffic(workload, src_hash):
+    """dram bytes per launch from the committed ncu summary of this workload, if there is one and it was taken
+    on the current kernel source (None otherwise)."""
+    path = PROFILED_WORKLOADS.get(workload)
+    if path is None or not os.path.exists(path):
         return None
     vals = {}
     for line in open(path):
@@ -501,10 +506,9 @@ def main():
         if is_mla:
             src = kernel_source_hash(MLA_KERNEL_SOURCES)
             achieved = nbytes / (mean_ms * 1e-3) / 1e9
-            int8 = case.qk_descale is not None
             roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                         "frac": achieved / peaks["hbm_gbs"],
-                        "traffic": profiled_traffic(MLA_INT8_PROFILE if int8 else MLA_PROFILE, src),
+                        "traffic": profiled_traffic(args.workload, src),
                         "algorithmic_bytes": nbytes, "peak_source": peaks["source"] + " (copy bandwidth)",
                         "tflops": flops / (mean_ms * 1e-3) / 1e12,
                         "kernel": mla_kernel_name(case) + " + mla_combine_kernel",
@@ -516,7 +520,7 @@ def main():
             achieved = flops / (mean_ms * 1e-3) / 1e12
             roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                         "frac": achieved / peaks["bf16_tflops"],
-                        "traffic": profiled_traffic(PROFILE_D256 if d256 else PROFILE, src),
+                        "traffic": profiled_traffic(args.workload, src),
                         "algorithmic_bytes": nbytes, "peak_source": peaks["source"] + " (burst bf16)",
                         "kernel": "prefill_d256_kernel" if d256 else "prefill_kernel", "kernel_source_sha256": src}
             launches = args.steps
