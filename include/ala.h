@@ -114,9 +114,10 @@ ALA_API void ala_op_destroy(ala_op* op);
  * executions: a code that an execution records there stays until the
  * workspace is bound again (ala_workspace_status reports it), and a wait
  * timeout's code makes later executions return at once without writing their
- * outputs.  While bound,
- * the caller guarantees that nothing else writes to the workspace and that it
- * stays allocated; binding a NULL workspace unbinds.  Status: ALA_NULL_REQUIRED (op NULL),
+ * outputs.  While bound, the caller guarantees that nothing else writes to
+ * the workspace (an execution of another op into it included: that would
+ * replace the schedule this op's executions read) and that it stays
+ * allocated; binding a NULL workspace unbinds.  Status: ALA_NULL_REQUIRED (op NULL),
  * ALA_WORKSPACE_TOO_SMALL, ALA_INVALID_PARAM (misaligned: 16 bytes for the
  * prefill ops, 256 for MLA), ALA_CUDA_ERROR. */
 ALA_API int ala_op_bind_workspace(ala_op* op, void* workspace, uint64_t workspaceSize, ala_stream_t stream);
