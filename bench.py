@@ -57,6 +57,7 @@ MLA_KERNEL_SOURCES = ["paged_attention_varlen_b200/csrc/mla.cu", "paged_attentio
                       "paged_attention_varlen_b200/csrc/ptx.cuh"]
 # the workload each committed ncu summary was captured on: its dram bytes describe that workload's launch only
 PROFILED_WORKLOADS = {"varlen_causal_bf16": PROFILE, "varlen_causal_bf16_d256": PROFILE_D256,
+                      "long_alibi_sqrt_bf16": os.path.join(ROOT, "profiles", "prefill_long_alibi_sqrt_bf16.md"),
                       "mla_decode_qs1_bf16": MLA_PROFILE, "mla_decode_qs1_int8": MLA_INT8_PROFILE}
 DEFAULT_WORKLOAD = "varlen_causal_bf16"
 WORKLOADS = {

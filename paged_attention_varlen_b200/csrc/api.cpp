@@ -390,6 +390,16 @@ int build_prefill(ala_op* op, const ala_tensor* query, const ala_tensor* key, co
       load.push({l + cost(units[i]), c});
     }
   }
+  // Each CTA then runs its units in (sequence, kv head) order, longest first within one head: every CTA
+  // walks the heads in the same order, so the units running at one time read the K/V of a few heads,
+  // which stay in L2 (in longest-first order every head's K/V is read at once, and over long sequences
+  // that overflows L2).  A CTA's load is its units' sum, so the order leaves the balance as it is.
+  const int32_t group = headNum / kvHeadNum;
+  for (auto& list : lists)
+    std::stable_sort(list.begin(), list.end(), [&](int32_t x, int32_t y) {
+      const PrefillUnit &a = units[x], &c = units[y];
+      return a.b != c.b ? a.b < c.b : a.head[0] / group < c.head[0] / group;
+    });
   std::vector<PrefillUnit> ordered;
   std::vector<int32_t> offsets(n_ctas + 1, 0);
   ordered.reserve(units.size());

@@ -27,7 +27,7 @@ def test_each_summary_is_keyed_by_the_workload_its_commands_run():
 
 def test_traffic_is_null_for_a_workload_without_its_own_summary():
     src = bench.kernel_source_hash()
-    for workload in ("prefix_paged_alibi_fp16", "long_alibi_sqrt_bf16", "long_alibi_left_bf16"):
+    for workload in ("prefix_paged_alibi_fp16", "long_alibi_left_bf16"):
         assert bench.profiled_traffic(workload, src) is None
     assert bench.profiled_traffic("mla_spec_qs4_bf16", bench.kernel_source_hash(bench.MLA_KERNEL_SOURCES)) is None
 
