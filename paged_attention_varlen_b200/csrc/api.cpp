@@ -1,6 +1,7 @@
 // api.cpp -- host side of the C ABI declared in include/ala.h: argument
-// validation, the per-call schedule (work units sorted longest first), the
-// workspace layout, TMA descriptor encoding and the kernel launches.
+// validation, the per-call schedule (work units packed longest first onto
+// the CTAs, each CTA's list in (sequence, kv head) order), the workspace
+// layout, TMA descriptor encoding and the kernel launches.
 //
 // Validation never touches the GPU, so every error path is testable on a
 // machine without one.
